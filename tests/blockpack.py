@@ -1,0 +1,140 @@
+"""Test-side block ENCODER and a second, bit-string DECODER (no oracle code).
+
+The encoder places chosen integer fields into block bytes following the GGUF
+layout statement (the inverse direction of the oracle's decoders), so a round
+trip through the oracle pins each field's position.  The second decoder reads
+the same fields by absolute bit index over the block viewed as one
+little-endian bit string; it shares no structure with the oracle's loops.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def f16_bits(v: float) -> int:
+    return int(np.array([v], dtype=np.float16).view(np.uint16)[0])
+
+
+# ------------------------------------------------------------------ encoders
+
+def pack_q8_0(d_bits: int, q) -> np.ndarray:
+    q = [int(v) for v in q]
+    assert len(q) == 32 and all(-128 <= v <= 127 for v in q)
+    out = np.zeros(34, dtype=np.uint8)
+    out[0], out[1] = d_bits & 0xFF, d_bits >> 8
+    for i, v in enumerate(q):
+        out[2 + i] = v & 0xFF
+    return out
+
+
+def pack_q4_k(d_bits: int, dmin_bits: int, sc, m, q) -> np.ndarray:
+    sc, m, q = [int(v) for v in sc], [int(v) for v in m], [int(v) for v in q]
+    assert len(sc) == 8 and len(m) == 8 and len(q) == 256
+    assert all(0 <= v < 64 for v in sc + m) and all(0 <= v < 16 for v in q)
+    out = np.zeros(144, dtype=np.uint8)
+    out[0], out[1] = d_bits & 0xFF, d_bits >> 8
+    out[2], out[3] = dmin_bits & 0xFF, dmin_bits >> 8
+    s = [0] * 12
+    for j in range(4):
+        s[j] |= sc[j]
+        s[j + 4] |= m[j]
+    for j in range(4, 8):
+        s[j + 4] |= (sc[j] & 15) | ((m[j] & 15) << 4)
+        s[j - 4] |= (sc[j] >> 4) << 6
+        s[j] |= (m[j] >> 4) << 6
+    out[4:16] = s
+    for c in range(4):
+        for l in range(32):
+            out[16 + 32 * c + l] = q[64 * c + l] | (q[64 * c + 32 + l] << 4)
+    return out
+
+
+def pack_q6_k(d_bits: int, scales, q) -> np.ndarray:
+    scales, q = [int(v) for v in scales], [int(v) for v in q]
+    assert len(scales) == 16 and len(q) == 256
+    assert all(-128 <= v <= 127 for v in scales) and all(0 <= v < 64 for v in q)
+    out = np.zeros(210, dtype=np.uint8)
+    for h in range(2):
+        for t in range(4):
+            for l in range(32):
+                v = q[128 * h + 32 * t + l]
+                k = 64 * h + l + 32 * (t & 1)
+                out[k] |= (v & 15) << (0 if t < 2 else 4)
+                out[128 + 32 * h + l] |= (v >> 4) << (2 * t)
+    for i, v in enumerate(scales):
+        out[192 + i] = v & 0xFF
+    out[208], out[209] = d_bits & 0xFF, d_bits >> 8
+    return out
+
+
+# ----------------------------------------------------------- second decoder
+
+def _bits(blk: np.ndarray, start: int, n: int) -> int:
+    """Unsigned integer from n bits starting at absolute bit `start` (bit k of
+    the block is bit k % 8 of byte k // 8)."""
+    v = 0
+    for k in range(n):
+        b = start + k
+        v |= ((int(blk[b // 8]) >> (b % 8)) & 1) << k
+    return v
+
+
+def _signed(v: int, n: int) -> int:
+    return v - (1 << n) if v >= 1 << (n - 1) else v
+
+
+def _half(bits: int) -> float:
+    return float(np.array([bits], dtype=np.uint16).view(np.float16)[0])
+
+
+def fields_q8_0(blk):
+    return {"d": _half(_bits(blk, 0, 16)),
+            "q": [_signed(_bits(blk, 16 + 8 * i, 8), 8) for i in range(32)]}
+
+
+def fields_q4_k(blk):
+    sc, m = [], []
+    for j in range(8):
+        if j < 4:
+            sc.append(_bits(blk, 32 + 8 * j, 6))
+            m.append(_bits(blk, 32 + 8 * (j + 4), 6))
+        else:
+            # low 4 bits from the low / high nibble of scale byte j+4, top 2 bits
+            # from bits 6..7 of scale byte j-4 (sc) or j (m)
+            sc.append(_bits(blk, 32 + 8 * (j + 4), 4) | (_bits(blk, 32 + 8 * (j - 4) + 6, 2) << 4))
+            m.append(_bits(blk, 32 + 8 * (j + 4) + 4, 4) | (_bits(blk, 32 + 8 * j + 6, 2) << 4))
+    q = []
+    for i in range(256):
+        c, r = divmod(i, 64)
+        hi, l = divmod(r, 32)
+        q.append(_bits(blk, 8 * (16 + 32 * c + l) + 4 * hi, 4))
+    return {"d": _half(_bits(blk, 0, 16)), "dmin": _half(_bits(blk, 16, 16)),
+            "sc": sc, "m": m, "q": q}
+
+
+def fields_q6_k(blk):
+    q = []
+    for i in range(256):
+        h, r = divmod(i, 128)
+        t, l = divmod(r, 32)
+        low = _bits(blk, 8 * (64 * h + l + 32 * (t % 2)) + (4 if t >= 2 else 0), 4)
+        high = _bits(blk, 8 * (128 + 32 * h + l) + 2 * t, 2)
+        q.append(low + 16 * high)
+    return {"d": _half(_bits(blk, 8 * 208, 16)),
+            "scales": [_signed(_bits(blk, 8 * (192 + k), 8), 8) for k in range(16)],
+            "q": q}
+
+
+def decode2(fmt: int, blk) -> np.ndarray:
+    """Second decoder: fields by bit index, then the weight formula evaluated in
+    f64 and rounded once to f32 (the products are exact, see the oracle)."""
+    if fmt == 0:
+        f = fields_q8_0(blk)
+        return np.array([f["d"] * q for q in f["q"]], dtype=np.float64).astype(np.float32)
+    if fmt == 1:
+        f = fields_q4_k(blk)
+        return np.array([f["d"] * f["sc"][i // 32] * f["q"][i] - f["dmin"] * f["m"][i // 32]
+                         for i in range(256)], dtype=np.float64).astype(np.float32)
+    f = fields_q6_k(blk)
+    return np.array([f["d"] * f["scales"][i // 16] * (f["q"][i] - 32) for i in range(256)],
+                    dtype=np.float64).astype(np.float32)
