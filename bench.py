@@ -1,0 +1,550 @@
+#!/usr/bin/env python
+"""Benchmark of the quantized decode-step matvec on B200.
+
+Headline step: the full decode-step matvec sweep of a 16-layer dense stack
+(hidden 2048, intermediate 8192, 32 query / 8 KV heads of head_dim 64), all
+weights Q8_0, one token: per layer the fused QKV 3072x2048, O 2048x2048, fused
+gate/up 16384x2048 and down 2048x8192 matvecs -- 64 launches, 1.034 GB of
+weights per step (larger than the 126 MB L2, so no flush is needed).  The step
+is captured once as a CUDA graph of the library's C-ABI calls and replayed.
+Metric: weight bytes streamed per second (GB/s), with the fraction of the
+measured HBM peak.  The other workloads (Q8_0 1024^2, Q4_K fused QKV, Q6_K
+vocab projection at 1 and 4 tokens, the MoE FFN step, the sweep at 2/4/8
+tokens) are measured in the same run and reported under "per_config".
+
+  python bench.py [--gpus N --steps K --warmup W]      # our CUDA path
+  python bench.py --impl reference ...                   # the oracle on host cores
+  python bench.py --profile-case q8_0|q4_k|q6_k          # one large matvec, for ncu
+
+Multi-GPU: replicas only (the sweep does not shard across GPUs in this build):
+each rank runs the same step on its own GPU, timed on the device, max over
+ranks; value = all ranks' bytes / that time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from quantized_decode_superblocks_b200 import synth  # noqa: E402
+
+Q8_0, Q4_K, Q6_K = synth.Q8_0, synth.Q4_K, synth.Q6_K
+L2_BYTES = 126 * 1024 * 1024
+METRIC = "quantized matvec µs and weight GB/s as % of B200 HBM peak (batch 1)"
+WORKLOAD = ("16-layer Q8_0 decode-step matvec sweep, batch 1: per layer fused QKV 3072x2048, "
+            "O 2048x2048, fused gate/up 16384x2048, down 2048x8192")
+
+
+def bpw(fmt):
+    return synth.BLOCK_BYTES[fmt] / synth.BLOCK_WEIGHTS[fmt]
+
+
+def algo_bytes(fmt, rows, cols, n_tok):
+    """Algorithmic bytes of one matvec: packed weights + x read + y written."""
+    return synth.matrix_bytes(fmt, rows, cols) + 4 * n_tok * (cols + rows)
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "quantized_decode_superblocks_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def sweep_layers():
+    return [(l, m, name, rows, cols) for l in range(synth.CFG4_LAYERS)
+            for m, (name, rows, cols) in enumerate(synth.workload_cfg4_layer())]
+
+
+# ------------------------------------------------------------------ clocks --
+
+class ClockSampler:
+    """nvidia-smi samples of this GPU's clocks and throttle reasons."""
+    FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, pci_bus_id):
+        self.bus = (pci_bus_id or "").lower()
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
+                                          "-lms", "200"], stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) < 9:
+                        continue
+                    bus = parts[0].lower()
+                    if self.bus and not (bus.endswith(self.bus[-12:]) or self.bus.endswith(bus[-12:])):
+                        continue
+                    rows.append(parts)
+            os.unlink(self.path)
+        except OSError:
+            pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+
+        def num(v):
+            try:
+                return float(v.split()[0])
+            except (ValueError, IndexError):
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------- device helpers --
+
+class Dist:
+    def __init__(self, n_gpus):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if n_gpus > 1 and self.world != n_gpus:
+            raise SystemExit(f"--gpus {n_gpus} needs torchrun with {n_gpus} ranks (WORLD_SIZE={self.world})")
+
+    def init(self, torch):
+        torch.cuda.set_device(self.local)
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+
+    def barrier(self, torch):
+        if self.pg is not None:
+            self.pg.barrier(device_ids=[self.local])
+
+    def max(self, torch, v):
+        if self.pg is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+def time_graph(torch, graph, reps, stream):
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end) / 1e3   # seconds
+
+
+def capture(torch, fn, stream):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        fn()                        # warm: plans, attributes, lazy module loading
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+    torch.cuda.synchronize()
+    return g
+
+
+# ----------------------------------------------------------- the sweep step --
+
+class Sweep:
+    """Device-resident weights / activations of the 16-layer Q8_0 sweep."""
+
+    def __init__(self, torch, q, n_tok, host_cache):
+        self.q, self.torch, self.n_tok = q, torch, n_tok
+        self.mats = []
+        x_off = y_off = 0
+        for (l, m, name, rows, cols) in sweep_layers():
+            key = (l, m)
+            if key not in host_cache:
+                host_cache[key] = synth.gen_blocks(Q8_0, rows, cols, synth.CFG4_SEED, 16 * l + m)
+            self.mats.append(dict(rows=rows, cols=cols, W=torch.from_numpy(host_cache[key]).cuda(),
+                                  x_off=x_off, y_off=y_off))
+            x_off += n_tok * cols
+            y_off += n_tok * rows
+        xs = np.concatenate([synth.gen_x(n_tok, mm["cols"], synth.CFG4_SEED, 5000 + i).reshape(-1)
+                             for i, mm in enumerate(self.mats)])
+        self.x_host = torch.from_numpy(xs).pin_memory()
+        self.x = self.x_host.cuda()
+        self.y = torch.empty(y_off, device="cuda")
+        self.y_host = torch.empty(y_off, dtype=torch.float32).pin_memory()
+        self.weight_bytes = sum(synth.matrix_bytes(Q8_0, mm["rows"], mm["cols"]) for mm in self.mats)
+        self.algo = sum(algo_bytes(Q8_0, mm["rows"], mm["cols"], n_tok) for mm in self.mats)
+        self.launches = len(self.mats)
+
+    def launch(self, i, stream=None):
+        mm = self.mats[i]
+        x = self.x.data_ptr() + 4 * mm["x_off"]
+        y = self.y.data_ptr() + 4 * mm["y_off"]
+        if self.n_tok == 1:
+            self.q.qmv_f32(Q8_0, mm["W"], mm["rows"], mm["cols"], x, y, stream)
+        else:
+            self.q.qmv_batched(Q8_0, mm["W"], mm["rows"], mm["cols"], x, y, self.n_tok, stream)
+
+    def step(self, stream=None):
+        for i in range(len(self.mats)):
+            self.launch(i, stream)
+
+
+def per_launch_durations(torch, sweep, stream, reps=3):
+    """CUDA-event duration of every launch of the step, on its stream."""
+    n = sweep.launches
+    tot = [0.0] * n
+    for _ in range(reps):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            for i in range(n):
+                evs[i][0].record(stream)
+                sweep.launch(i, stream)
+                evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        for i in range(n):
+            tot[i] += evs[i][0].elapsed_time(evs[i][1]) / 1e3
+    return [t / reps for t in tot]
+
+
+# --------------------------------------------------------- per-config runs --
+
+def rotating_pool(torch, fmt, rows, cols, seed, min_total):
+    host = synth.gen_blocks(fmt, rows, cols, seed, 0)
+    base = torch.from_numpy(host).cuda()
+    copies = max(1, -(-min_total // host.nbytes))
+    return [base] + [base.clone() for _ in range(copies - 1)]
+
+
+def measure_matvec(torch, q, stream, fmt, rows, cols, n_tok, seed, reps=200):
+    """µs per matvec over a pool of weight copies larger than L2 (replayed graph)."""
+    pool = rotating_pool(torch, fmt, rows, cols, seed, 2 * L2_BYTES)
+    x = torch.from_numpy(synth.gen_x(n_tok, cols, seed, 1)).cuda()
+    y = torch.empty((n_tok, rows), device="cuda")
+    per_graph = min(len(pool) * max(1, 64 // len(pool)), 256)
+
+    def body():
+        for i in range(per_graph):
+            W = pool[i % len(pool)]
+            if n_tok == 1:
+                q.qmv_f32(fmt, W, rows, cols, x, y)
+            else:
+                q.qmv_batched(fmt, W, rows, cols, x, y, n_tok)
+    g = capture(torch, body, stream)
+    time_graph(torch, g, 3, stream)
+    n_rep = max(2, reps // per_graph)
+    sec = time_graph(torch, g, n_rep, stream) / (n_rep * per_graph)
+    wb = synth.matrix_bytes(fmt, rows, cols)
+    return {"fmt": synth.FORMAT_NAMES[fmt], "rows": rows, "cols": cols, "n_tok": n_tok,
+            "us": sec * 1e6, "weight_gbs": wb / sec / 1e9, "copies": len(pool)}
+
+
+def measure_moe(torch, q, stream, reps=200):
+    w = synth.workload_cfg3()
+    E, hidden, inter, seed = w["n_expert"], w["hidden"], w["inter"], w["seed"]
+    gus = synth.matrix_bytes(Q4_K, inter, hidden)
+    ds = synth.matrix_bytes(Q4_K, hidden, inter)
+    host = [synth.gen_blocks(Q4_K, inter * E, hidden, seed, 1), synth.gen_blocks(Q4_K, inter * E, hidden, seed, 2),
+            synth.gen_blocks(Q4_K, hidden * E, inter, seed, 3)]
+    base = [torch.from_numpy(h).cuda() for h in host]
+    n_copies = 6      # each step touches 24.8 MB; six copies keep reuse distance > L2
+    sets = [base] + [[t.clone() for t in base] for _ in range(n_copies - 1)]
+    logits, bias = synth.gen_router(E, seed, 5)
+    lg, bs = torch.from_numpy(logits).cuda(), torch.from_numpy(bias).cuda()
+    x = torch.from_numpy(synth.gen_x(1, hidden, seed, 4)[0]).cuda()
+    ids = torch.empty(4, dtype=torch.int32, device="cuda")
+    g = torch.empty(4, device="cuda")
+    h = torch.empty((4, inter), device="cuda")
+    y = torch.empty(hidden, device="cuda")
+    per_graph = 4 * n_copies
+
+    def body():
+        for i in range(per_graph):
+            G, U, D = sets[i % n_copies]
+            q.moe_route(lg, bs, E, 4, ids, g)
+            q.moe_ffn(Q4_K, G, U, gus, Q4_K, D, ds, E, ids, g, 4, hidden, inter, x, h, y)
+    gr = capture(torch, body, stream)
+    time_graph(torch, gr, 3, stream)
+    n_rep = max(2, reps // per_graph)
+    sec = time_graph(torch, gr, n_rep, stream) / (n_rep * per_graph)
+    touched = 4 * (2 * gus + ds)
+    return {"workload": "MoE FFN step: route top-4 of 32 + Q4_K gate/up 1792x2048 + down 2048x1792",
+            "us": sec * 1e6, "weight_gbs": touched / sec / 1e9, "launches_per_step": 3,
+            "weight_bytes_touched": touched}
+
+
+# ----------------------------------------------------------- reference arm --
+
+def oracle_rate(seconds, cache):
+    """The oracle on the host cores over a bounded sample of the sweep: GB/s of
+    weight bytes, the threads it used, and the sample description."""
+    import oracle
+    threads = os.cpu_count() or 1
+    mats = [(l, m, name, rows, cols) for (l, m, name, rows, cols) in sweep_layers() if l == 0]
+    data = []
+    for (l, m, name, rows, cols) in mats:
+        key = (l, m)
+        if key not in cache:
+            cache[key] = synth.gen_blocks(Q8_0, rows, cols, synth.CFG4_SEED, 16 * l + m)
+        data.append((cache[key], rows, cols, synth.gen_x(1, cols, synth.CFG4_SEED, 5000 + m)))
+    done_bytes, t0, passes = 0, time.perf_counter(), 0
+    while True:
+        for W, rows, cols, x in data:
+            oracle.qmv(Q8_0, W, rows, cols, x, nthreads=threads)
+            done_bytes += W.nbytes
+        passes += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return done_bytes / dt / 1e9, threads, f"{passes} passes over layer 0's four Q8_0 matvecs ({dt:.1f} s)"
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    cache = {}
+    # calibrate, then size each step's sample so warm-up + timed steps take ~60 s
+    rate, threads, _ = oracle_rate(1.0, cache)
+    per_step_bytes = max(1, int(rate * 1e9 * 60.0 / max(1, args.steps + args.warmup)))
+    W0, rows0, cols0 = cache[(0, 2)], 16384, 2048
+    row_bytes = W0.nbytes // rows0
+    n_rows = max(1, min(rows0, per_step_bytes // row_bytes))
+    x = synth.gen_x(1, cols0, synth.CFG4_SEED, 5002)
+    sub = W0[: n_rows * row_bytes]
+    for _ in range(args.warmup):
+        oracle.qmv(Q8_0, sub, n_rows, cols0, x, nthreads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.qmv(Q8_0, sub, n_rows, cols0, x, nthreads=threads)
+    dt = time.perf_counter() - t0
+    value = n_rows * row_bytes * args.steps / dt / 1e9
+    sample = f"each step: {n_rows} rows of the 16384x2048 Q8_0 gate/up matvec ({n_rows * row_bytes} B)"
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "n_tok": 1, "parallelism": "host cores (oracle)"},
+            "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------ profile case --
+
+def run_profile_case(args):
+    """A few launches of one large matvec (weights larger than L2, < 1 GB on the
+    device) -- the small case that ncu captures."""
+    import torch
+    import quantized_decode_superblocks_b200 as q
+    fmt = {"q8_0": Q8_0, "q4_k": Q4_K, "q6_k": Q6_K}[args.profile_case]
+    rows, cols = {Q8_0: (65536, 2048), Q4_K: (131072, 2048), Q6_K: (96000, 2048)}[fmt]
+    torch.cuda.set_device(0)
+    W = torch.from_numpy(synth.gen_blocks(fmt, rows, cols, 77, 0)).cuda()
+    x = torch.from_numpy(synth.gen_x(args.n_tok, cols, 77, 1)).cuda()
+    y = torch.empty((args.n_tok, rows), device="cuda")
+    for _ in range(max(1, args.steps)):
+        q.qmv_batched(fmt, W, rows, cols, x, y, args.n_tok)
+    torch.cuda.synchronize()
+    assert q.qmv_check() == 0
+    print(json.dumps({"profile_case": args.profile_case, "rows": rows, "cols": cols, "n_tok": args.n_tok,
+                      "weight_bytes": synth.matrix_bytes(fmt, rows, cols)}))
+    return 0
+
+
+# --------------------------------------------------------------------- main --
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--n-tok", type=int, default=1)
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip the per-config measurements and the CPU baseline")
+    ap.add_argument("--profile-case", choices=["q8_0", "q4_k", "q6_k"])
+    args = ap.parse_args()
+    if args.warmup < 3 and not args.profile_case:
+        raise SystemExit("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.profile_case:
+        return run_profile_case(args)
+
+    import torch
+    import quantized_decode_superblocks_b200 as q
+    dist = Dist(args.gpus)
+    dist.init(torch)
+    q.lib()                                  # fails loudly if the library is missing
+    stream = torch.cuda.Stream()
+    hbm_peak, peak_kind = peaks()
+    props = torch.cuda.get_device_properties(torch.cuda.current_device())
+    cache = {}
+
+    sweep = Sweep(torch, q, args.n_tok, cache)
+    graph = capture(torch, lambda: sweep.step(), stream)
+    assert q.qmv_check(stream) == 0
+
+    per_config = {}
+    with ClockSampler(getattr(props, "pci_bus_id", "")) as clk:
+        # warm-up, then the timed steps (device time, barrier + sync on both sides)
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+        dist.barrier(torch)
+        torch.cuda.synchronize()
+        sec = time_graph(torch, graph, args.steps, stream)
+        torch.cuda.synchronize()
+        dist.barrier(torch)
+        sec = dist.max(torch, sec)
+        # the dominant kernel: every launch of the step, event-timed on its stream
+        durs = per_launch_durations(torch, sweep, stream)
+        # end to end: pinned x -> device, the step's library calls, y -> pinned host
+        e2e_reps = max(3, min(200, args.steps // 5))
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(e2e_reps):
+                sweep.x.copy_(sweep.x_host, non_blocking=True)
+                graph.replay()
+                sweep.y_host.copy_(sweep.y, non_blocking=True)
+        ev1.record(stream)
+        ev1.synchronize()
+        e2e_sec = dist.max(torch, ev0.elapsed_time(ev1) / 1e3 / e2e_reps)
+        if not args.headline_only and dist.rank == 0:
+            per_config["cfg0_q8_0_1024x1024"] = measure_matvec(torch, q, stream, Q8_0, 1024, 1024, 1, 0)
+            per_config["cfg1_q4_k_fused_qkv_3072x2048"] = measure_matvec(torch, q, stream, Q4_K, 3072, 2048, 1, 1)
+            for nt in (1, 4):
+                per_config[f"cfg2_q6_k_vocab_128000x2048_ntok{nt}"] = measure_matvec(
+                    torch, q, stream, Q6_K, 128000, 2048, nt, 2, reps=20)
+            per_config["cfg3_moe_ffn_step"] = measure_moe(torch, q, stream)
+            for nt in (1, 2, 4, 8):
+                if nt == args.n_tok:
+                    continue
+                sw = Sweep(torch, q, nt, cache)
+                gr = capture(torch, lambda: sw.step(), stream)
+                s2 = time_graph(torch, gr, max(3, args.steps // 10), stream) / max(3, args.steps // 10)
+                per_config[f"cfg4_sweep_ntok{nt}"] = {"us": s2 * 1e6, "weight_gbs": sw.weight_bytes / s2 / 1e9,
+                                                      "launches": sw.launches}
+                del gr, sw
+    clocks = clk.summary()
+    assert q.qmv_check(stream) == 0
+
+    total_bytes = sweep.weight_bytes * dist.world
+    value = total_bytes / sec / 1e9 * 1.0 if False else sweep.weight_bytes * dist.world / (sec / args.steps) / 1e9
+    ms_per_step = sec / args.steps * 1e3
+    achieved = sweep.algo / sum(durs) / 1e9
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            t = json.load(f)
+        if t.get("source_hash") == source_hash() and t.get("n_tok") == args.n_tok:
+            traffic = t.get("step_traffic_bytes_per_launch")
+    cfg4_key = f"cfg4_sweep_ntok{args.n_tok}"
+    per_config[cfg4_key] = {"us": ms_per_step * 1e3, "weight_gbs": sweep.weight_bytes / (sec / args.steps) / 1e9,
+                            "launches": sweep.launches}
+    for v in per_config.values():
+        if "weight_gbs" in v:
+            v["frac_of_hbm_peak"] = round(v["weight_gbs"] / hbm_peak, 4)
+            v["us"] = round(v["us"], 3)
+            v["weight_gbs"] = round(v["weight_gbs"], 1)
+
+    cpu = None
+    if dist.rank == 0 and args.gpus == 1 and not args.headline_only:
+        rate, threads, sample = oracle_rate(10.0, cache)
+        cpu = {"value": round(rate, 3), "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample}
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "n_tok": args.n_tok, "layers": synth.CFG4_LAYERS,
+                   "weight_bytes_per_step": sweep.weight_bytes, "launches_per_step": sweep.launches,
+                   "l2": "inputs larger than L2 (1.03 GB of weights per step, L2 126 MB)",
+                   "timing": "CUDA graph of the step's C-ABI calls, replayed; CUDA events on the launch stream",
+                   "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"},
+        "frac_of_hbm_peak": round(value / dist.world / hbm_peak, 4),
+        "us_per_step": round(ms_per_step * 1e3, 2),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6.65 TB/s",
+                     "kernel": "qmv_pipeline_kernel (Q8_0, every launch of the step)",
+                     "algorithmic_bytes_per_step": sweep.algo,
+                     "mean_launch_us": round(sum(durs) / len(durs) * 1e6, 3)},
+        "e2e": {"value": round(sweep.weight_bytes * dist.world / e2e_sec / 1e9, 1), "unit": "GB/s",
+                "h2d_bytes_per_step": int(sweep.x_host.numel() * 4),
+                "d2h_bytes_per_step": int(sweep.y_host.numel() * 4)},
+        "gpu_launches": sweep.launches * args.steps,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+        "per_config": per_config,
+    }
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    del graph
+    dist.close()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

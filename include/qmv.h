@@ -1,0 +1,170 @@
+/*
+ * qmv.h -- C ABI of libqmv.so: the decode-step matrix-vector product of a
+ * GGUF block-quantized weight matrix (Q8_0, Q4_K, Q6_K) with f32 activations,
+ * dequantized on the fly, on one NVIDIA B200 (sm_100a).
+ *
+ * Sources (page title, section):
+ *   BebeLM：纯Rust实现的端侧大模型推理引擎
+ *     §量化格式支持 -- Q4_K: 256 weights per superblock in 144 bytes; Q6_K for
+ *       sensitive tensors; dequantization happens at run time and activations
+ *       stay f32.
+ *     §核心算子 (MoE前馈网络) -- sigmoid router, top-k = 4 of 32 experts, the
+ *       expert bias takes part in the selection only, weights normalised.
+ *     §性能表现 -- decode is bound by memory bandwidth.
+ *   FlareLLM：纯Rust打造的浏览器端LLM推理引擎
+ *     §推理层面的深度优化 -- fused QKV and gate/up matvecs (43% fewer matvec
+ *       calls per layer); n-gram speculative decoding (several tokens checked
+ *       in one pass over the weights); zero-allocation forward pass.
+ *     §计算路径的智能选择, §量化技术的全面支持 -- Q8_0 and the K-quants.
+ *     §生态对比与定位 -- standard GGUF files.
+ *
+ * Block layouts (GGUF, little-endian, fp16 = IEEE binary16):
+ *   Q8_0  32 weights / 34 B : d | q[32] int8                 w = d*q
+ *   Q4_K 256 weights / 144 B: d | dmin | scales[12] | qs[128]
+ *                             w = d*sc_j*q - dmin*m_j, j = sub-block of 32
+ *   Q6_K 256 weights / 210 B: ql[128] | qh[64] | scales[16] int8 | d
+ *                             w = d*scales[i/16]*(q - 32), q = 6 bits
+ * A matrix is rows x cols weights stored densely row-major: row r starts at
+ * byte r * (cols / block_weights) * block_bytes; no padding.
+ *
+ * Conventions shared by every entry point:
+ *   - Every array pointer is a DEVICE pointer owned by the caller (for
+ *     example torch.empty(..., device="cuda").data_ptr()); the library keeps
+ *     no reference after the call returns.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
+ *     enqueued asynchronously on it; outputs are complete in stream order.
+ *   - The library allocates no memory during any call; intermediates (the
+ *     SwiGLU activations of moe_ffn) live in caller-provided buffers.
+ *   - Outputs are fully overwritten, never accumulated into.
+ *   - Argument errors are detected on the host and returned before anything
+ *     is enqueued; outputs are then left untouched.  No call aborts.
+ *   - Alignment: W (every expert base and expert stride) 16 B, x 16 B,
+ *     y / out 4 B.
+ *   - The arithmetic is f32: dequantized weights are exact f32 values, dot
+ *     products accumulate in f32 (order unspecified, deterministic for a
+ *     given shape).  There is no CPU fallback and no other backend.
+ *   - Thread safety: calls may be made from several host threads; the only
+ *     global state is a per-device properties cache and the sticky device
+ *     error word read by qmv_check().
+ */
+#ifndef QMV_H
+#define QMV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, without including the CUDA headers. */
+typedef struct CUstream_st *qmv_stream_t;
+
+typedef enum { QMV_Q8_0 = 0, QMV_Q4_K = 1, QMV_Q6_K = 2 } qmv_fmt;
+
+typedef enum {
+    QMV_OK = 0,
+    QMV_ERR_NULL = -1,    /* a required pointer is NULL                         */
+    QMV_ERR_FMT = -2,     /* fmt is not one of qmv_fmt                           */
+    QMV_ERR_SHAPE = -3,   /* rows < 1, cols < 1, cols % block_weights != 0, or a
+                             size above the limits below                        */
+    QMV_ERR_ALIGN = -4,   /* a pointer or stride breaks the alignment rules      */
+    QMV_ERR_NTOK = -5,    /* n_tok outside [1, QMV_MAX_NTOK]                     */
+    QMV_ERR_NSEL = -6,    /* n_sel / top_k outside [1, min(n_expert, 8)], or
+                             n_expert outside [1, QMV_MAX_EXPERTS]              */
+    QMV_ERR_CUDA = -7,    /* a CUDA call or a kernel launch failed               */
+    QMV_ERR_DEVICE = -8,  /* no usable CUDA device, or a device-side error was
+                             recorded (see qmv_check)                            */
+} qmv_status;
+
+#define QMV_MAX_NTOK 8
+#define QMV_MAX_SEL 8
+#define QMV_MAX_EXPERTS 1024
+#define QMV_MAX_ROWS 2147483647LL   /* rows of one matrix                       */
+#define QMV_MAX_COLS 1048576LL      /* weights per row                          */
+
+/* Device error bits reported by qmv_check(). */
+#define QMV_DEVERR_EXPERT_ID 1      /* an expert id was outside [0, n_expert); that
+                                       expert's contribution was dropped        */
+#define QMV_DEVERR_TIMEOUT 2        /* a pipeline wait gave up (bounded wait)   */
+
+/* y[rows] = W x.  x: f32 [cols]; y: f32 [rows].
+ * One launch covers a whole fused projection: pass the row-concatenation of
+ * Q, K and V (or of gate and up) as W (FlareLLM page, §推理层面的深度优化).
+ * Returns QMV_OK or a qmv_status error. */
+int qmv_f32(int fmt, const void *W_blocks, int64_t rows, int64_t cols,
+            const float *x, float *y, qmv_stream_t stream);
+
+/* Multi-token variant for speculative verification (FlareLLM page,
+ * §推理层面的深度优化: n-gram speculative decoding): every weight is read once
+ * and applied to n_tok activation vectors.
+ * x: f32 [n_tok][cols] (token-major); y: f32 [n_tok][rows]; 1 <= n_tok <= 8. */
+int qmv_batched(int fmt, const void *W_blocks, int64_t rows, int64_t cols,
+                const float *x, float *y, int n_tok, qmv_stream_t stream);
+
+/* MoE router on the device, no host round trip (BebeLM page, §核心算子):
+ *   s_e = sigmoid(logits[e]),  b_e = s_e + bias[e]   (f32)
+ *   ids_out[k] = the top_k experts by b, in descending b (ties to the lower
+ *                index);  g_out[k] = s_{ids[k]} / sum_j s_{ids[j]}.
+ * logits, bias: f32 [n_expert]; ids_out: int32 [top_k]; g_out: f32 [top_k].
+ * 1 <= top_k <= min(n_expert, 8), n_expert <= QMV_MAX_EXPERTS. */
+int moe_route(const float *logits, const float *bias, int n_expert, int top_k,
+              int32_t *ids_out, float *g_out, qmv_stream_t stream);
+
+/* Expert-indexed grouped matvec.  Expert e's matrix (rows x cols, format fmt)
+ * starts at expert_blocks + e * expert_stride_bytes; the n_sel expert ids are
+ * read on the device from expert_ids (int32 [n_sel]), so the call can follow
+ * moe_route without a host synchronisation.
+ * x_k = x + k * x_stride (x_stride in floats; 0 = one shared x [cols]).
+ *   gate_w == NULL: y[k][r] = (W_{ids[k]} x_k)[r]           y: f32 [n_sel][rows]
+ *   gate_w != NULL: y[r] = sum_k gate_w[k] * (W_{ids[k]} x_k)[r]  y: f32 [rows]
+ *                   (gate_w: device f32 [n_sel]; summed in k order)
+ * An id outside [0, n_expert) contributes zero and sets QMV_DEVERR_EXPERT_ID.
+ * 1 <= n_sel <= min(n_expert, 8).  expert_stride_bytes must be a multiple of
+ * 16 and at least the matrix size. */
+int moe_qmv(int fmt, const void *expert_blocks, int64_t expert_stride_bytes, int n_expert,
+            const int32_t *expert_ids, int n_sel, int64_t rows, int64_t cols,
+            const float *x, int64_t x_stride, const float *gate_w, float *y,
+            qmv_stream_t stream);
+
+/* One MoE SwiGLU FFN step for the n_sel routed experts (BebeLM page, §核心算子):
+ *   h_k = silu(G_{ids[k]} x) * (U_{ids[k]} x)        -> h_scratch f32 [n_sel][inter]
+ *   y   = sum_k g[k] * D_{ids[k]} h_k                 -> y f32 [hidden]
+ * G and U of expert e: [inter x hidden] in fmt_gu at gate_blocks / up_blocks
+ * + e * gu_stride_bytes; D of expert e: [hidden x inter] in fmt_down at
+ * down_blocks + e * down_stride_bytes.  x: f32 [hidden]; g: f32 [n_sel]
+ * (e.g. from moe_route).  silu(z) = z / (1 + exp(-z)).  Two launches, no host
+ * synchronisation; h_scratch is caller-owned scratch and is overwritten. */
+int moe_ffn(int fmt_gu, const void *gate_blocks, const void *up_blocks,
+            int64_t gu_stride_bytes, int fmt_down, const void *down_blocks,
+            int64_t down_stride_bytes, int n_expert, const int32_t *expert_ids,
+            const float *g, int n_sel, int64_t hidden, int64_t inter,
+            const float *x, float *h_scratch, float *y, qmv_stream_t stream);
+
+/* Dequantize the whole matrix to f32: out[rows][cols].  The values are
+ * bit-exact f32 evaluations of the block formulas above (every product in
+ * them is exact in f32; Q4_K rounds once, in the subtraction). */
+int qmv_dequant(int fmt, const void *W_blocks, int64_t rows, int64_t cols,
+                float *out, qmv_stream_t stream);
+
+/* Synchronises `stream`, then reads and clears the sticky device error word
+ * of the current device.  Returns QMV_OK, QMV_ERR_CUDA if the synchronisation
+ * failed, or QMV_ERR_DEVICE if an error bit was set (the bits are stored in
+ * *dev_err_out when it is not NULL). */
+int qmv_check(qmv_stream_t stream, int *dev_err_out);
+
+/* Static, never-NULL description of a qmv_status value. */
+const char *qmv_strerror(int status);
+
+/* Bytes and weights per block of a format; 0 for an unknown format. */
+size_t qmv_block_bytes(int fmt);
+int qmv_block_weights(int fmt);
+
+/* Test hook for host-side failure handling: the next `count` launches made by
+ * this library fail with QMV_ERR_CUDA without reaching the GPU. */
+void qmv_debug_fail_next_launches(int count);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QMV_H */

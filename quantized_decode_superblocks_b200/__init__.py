@@ -1,0 +1,155 @@
+"""quantized_decode_superblocks_b200 -- Python binding of libqmv.so.
+
+The decode-step matvec of GGUF block-quantized weights (Q8_0, Q4_K, Q6_K) with
+f32 activations, dequantized on the fly, on an NVIDIA B200 (sm_100a).  Every
+step runs in the library's CUDA kernels; this module only marshals arguments
+(tensor data pointers, sizes, the current CUDA stream) through ctypes to the C
+ABI declared in ``include/qmv.h``, with the same function names.  PyTorch
+provides device memory and streams.  There is no CPU fallback: if the library
+is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+from .synth import Q4_K, Q6_K, Q8_0  # noqa: F401  (format ids)
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqmv.so")
+
+QMV_OK = 0
+STATUS_NAMES = {0: "QMV_OK", -1: "QMV_ERR_NULL", -2: "QMV_ERR_FMT", -3: "QMV_ERR_SHAPE",
+                -4: "QMV_ERR_ALIGN", -5: "QMV_ERR_NTOK", -6: "QMV_ERR_NSEL", -7: "QMV_ERR_CUDA",
+                -8: "QMV_ERR_DEVICE"}
+DEVERR_EXPERT_ID = 1
+DEVERR_TIMEOUT = 2
+
+EXPORTED = ("qmv_f32", "qmv_batched", "moe_route", "moe_qmv", "moe_ffn", "qmv_dequant",
+            "qmv_check", "qmv_strerror", "qmv_block_bytes", "qmv_block_weights",
+            "qmv_debug_fail_next_launches")
+
+
+class QmvError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({strerror(status)})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libqmv.so (built by ``build()``); raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built: run quantized_decode_superblocks_b200.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, c_int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        L.qmv_f32.argtypes = [c_int, vp, i64, i64, vp, vp, vp]
+        L.qmv_batched.argtypes = [c_int, vp, i64, i64, vp, vp, c_int, vp]
+        L.moe_route.argtypes = [vp, vp, c_int, c_int, vp, vp, vp]
+        L.moe_qmv.argtypes = [c_int, vp, i64, c_int, vp, c_int, i64, i64, vp, i64, vp, vp, vp]
+        L.moe_ffn.argtypes = [c_int, vp, vp, i64, c_int, vp, i64, c_int, vp, vp, c_int, i64, i64,
+                              vp, vp, vp, vp]
+        L.qmv_dequant.argtypes = [c_int, vp, i64, i64, vp, vp]
+        L.qmv_check.argtypes = [vp, ctypes.POINTER(c_int)]
+        L.qmv_strerror.argtypes = [c_int]
+        L.qmv_strerror.restype = ctypes.c_char_p
+        L.qmv_block_bytes.argtypes = [c_int]
+        L.qmv_block_bytes.restype = ctypes.c_size_t
+        L.qmv_block_weights.argtypes = [c_int]
+        L.qmv_debug_fail_next_launches.argtypes = [c_int]
+        L.qmv_debug_fail_next_launches.restype = None
+        for name in EXPORTED:
+            if name not in ("qmv_strerror", "qmv_block_bytes", "qmv_debug_fail_next_launches"):
+                getattr(L, name).restype = c_int
+        _lib = L
+    return _lib
+
+
+def build(verbose: bool = False) -> str:
+    from .build import build as _build
+    return _build(verbose=verbose)
+
+
+def strerror(status: int) -> str:
+    return lib().qmv_strerror(status).decode()
+
+
+def _ptr(t) -> int:
+    """Device (or host) address of a tensor, an int address, or None -> NULL."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc: int, where: str):
+    if rc != QMV_OK:
+        raise QmvError(rc, where)
+
+
+def qmv_block_bytes(fmt: int) -> int:
+    return lib().qmv_block_bytes(fmt)
+
+
+def qmv_block_weights(fmt: int) -> int:
+    return lib().qmv_block_weights(fmt)
+
+
+def qmv_f32(fmt, W, rows, cols, x, y, stream=None):
+    """y[rows] = W x (see include/qmv.h)."""
+    _check(lib().qmv_f32(fmt, _ptr(W), rows, cols, _ptr(x), _ptr(y), _stream(stream)), "qmv_f32")
+
+
+def qmv_batched(fmt, W, rows, cols, x, y, n_tok, stream=None):
+    """y[n_tok][rows] = W x[n_tok][cols]^T, 1 <= n_tok <= 8."""
+    _check(lib().qmv_batched(fmt, _ptr(W), rows, cols, _ptr(x), _ptr(y), n_tok, _stream(stream)),
+           "qmv_batched")
+
+
+def moe_route(logits, bias, n_expert, top_k, ids_out, g_out, stream=None):
+    _check(lib().moe_route(_ptr(logits), _ptr(bias), n_expert, top_k, _ptr(ids_out), _ptr(g_out),
+                           _stream(stream)), "moe_route")
+
+
+def moe_qmv(fmt, expert_blocks, expert_stride_bytes, n_expert, expert_ids, n_sel, rows, cols,
+            x, x_stride, gate_w, y, stream=None):
+    _check(lib().moe_qmv(fmt, _ptr(expert_blocks), expert_stride_bytes, n_expert, _ptr(expert_ids),
+                         n_sel, rows, cols, _ptr(x), x_stride, _ptr(gate_w), _ptr(y),
+                         _stream(stream)), "moe_qmv")
+
+
+def moe_ffn(fmt_gu, gate_blocks, up_blocks, gu_stride_bytes, fmt_down, down_blocks,
+            down_stride_bytes, n_expert, expert_ids, g, n_sel, hidden, inter, x, h_scratch, y,
+            stream=None):
+    _check(lib().moe_ffn(fmt_gu, _ptr(gate_blocks), _ptr(up_blocks), gu_stride_bytes, fmt_down,
+                         _ptr(down_blocks), down_stride_bytes, n_expert, _ptr(expert_ids), _ptr(g),
+                         n_sel, hidden, inter, _ptr(x), _ptr(h_scratch), _ptr(y), _stream(stream)),
+           "moe_ffn")
+
+
+def qmv_dequant(fmt, W, rows, cols, out, stream=None):
+    _check(lib().qmv_dequant(fmt, _ptr(W), rows, cols, _ptr(out), _stream(stream)), "qmv_dequant")
+
+
+def qmv_check(stream=None) -> int:
+    """Synchronises the stream; returns the device error bits (0 = none).
+    Raises QmvError only when the synchronisation itself fails."""
+    word = ctypes.c_int(0)
+    rc = lib().qmv_check(_stream(stream), ctypes.byref(word))
+    if rc not in (QMV_OK, -8):
+        raise QmvError(rc, "qmv_check")
+    return word.value

@@ -1,0 +1,386 @@
+// qmv_api.cu -- the C ABI of libqmv.so (declared in include/qmv.h): host-side
+// argument validation, launch planning and the launches themselves.  Nothing
+// here allocates device memory; every buffer is the caller's.
+#include <atomic>
+#include <mutex>
+
+#include "../../include/qmv.h"
+#include "qmv_misc.cuh"
+
+namespace {
+
+using namespace qmv;
+
+// Sticky device error word (QMV_DEVERR_* bits), read and cleared by qmv_check.
+__device__ int g_dev_err;
+
+constexpr int STAGE_MAX = 32 * 1024;      // bytes of one pipeline stage
+constexpr int STAGES_BUDGET = 96 * 1024;  // all stages of one CTA (two CTAs per SM)
+
+struct DevInfo {
+    int sm_count = 0;
+    int smem_optin = 0;
+    int *err = nullptr;
+    bool ok = false;
+};
+
+std::mutex g_mu;
+DevInfo g_dev[64];
+std::atomic<int> g_fail_launches{0};
+
+int block_weights(int fmt) { return fmt == QMV_Q8_0 ? 32 : (fmt == QMV_Q4_K || fmt == QMV_Q6_K) ? 256 : 0; }
+int block_bytes(int fmt) { return fmt == QMV_Q8_0 ? 34 : fmt == QMV_Q4_K ? 144 : fmt == QMV_Q6_K ? 210 : 0; }
+bool fmt_ok(int fmt) { return fmt == QMV_Q8_0 || fmt == QMV_Q4_K || fmt == QMV_Q6_K; }
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+int pow2ceil(int v) { int p = 1; while (p < v) p <<= 1; return p; }
+
+bool injected_failure()
+{
+    int n = g_fail_launches.load();
+    while (n > 0) {
+        if (g_fail_launches.compare_exchange_weak(n, n - 1)) return true;
+    }
+    return false;
+}
+
+int get_dev(DevInfo &out)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        (void)cudaGetLastError();
+        return QMV_ERR_DEVICE;
+    }
+    std::lock_guard<std::mutex> lk(g_mu);
+    DevInfo &d = g_dev[dev];
+    if (!d.ok) {
+        int major = 0;
+        if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaGetSymbolAddress(reinterpret_cast<void **>(&d.err), g_dev_err) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return QMV_ERR_DEVICE;
+        }
+        if (major < 10) return QMV_ERR_DEVICE;   // built for sm_100a only
+        d.ok = true;
+    }
+    out = d;
+    return QMV_OK;
+}
+
+// Launch shape of one pipeline launch: how many rows a warp and a tile take,
+// whether rows are split into K-chunks, the stage ring, and the grid.
+struct Plan {
+    KernelChoice kc;
+    Params p;
+    dim3 grid;
+    size_t smem;
+};
+
+int make_plan(int fmt, int64_t rows, int64_t cols, int n_tok, int G, int n_jobs, bool shared_x,
+              const DevInfo &di, Plan &pl)
+{
+    const int bw = block_weights(fmt), bb = block_bytes(fmt);
+    const int64_t rb = cols / bw * bb;
+    const int ntp = pow2ceil(n_tok);
+    const int gp = pow2ceil(G);
+    const bool tma = (rb % 16) == 0;
+    const int target_ctas = 2 * di.sm_count;
+    const int64_t ctas_job0 = std::max<int64_t>(1, target_ctas / n_jobs);
+    const int64_t rows_cta0 = ceil_div(rows, ctas_job0);
+
+    int R = gp;
+    const int rmax = std::min(8, 32 / ntp);
+    for (int cand = rmax; cand >= gp; cand >>= 1) {
+        const int64_t t = (int64_t)NC * cand / gp;
+        if (t <= std::max<int64_t>(rows_cta0, NC / gp) && (int64_t)G * t * rb <= STAGE_MAX) {
+            R = cand;
+            break;
+        }
+    }
+    if (R * ntp > 32 || R < gp) return QMV_ERR_SHAPE;
+    const int T = NC * R / gp;
+
+    int64_t chunk_cols = cols, chunk_bytes = rb;
+    if ((int64_t)G * T * rb > STAGE_MAX) {
+        const int64_t align = tma ? (fmt == QMV_Q6_K ? 2048 : 256) : bw;
+        const int64_t per_row = STAGE_MAX / ((int64_t)G * T);
+        int64_t n_ch = ceil_div(rb, per_row);
+        chunk_cols = ceil_div(ceil_div(cols, n_ch), align) * align;
+        if (chunk_cols >= cols) chunk_cols = cols;
+        chunk_bytes = chunk_cols / bw * bb;
+    }
+    const int64_t n_chunks = ceil_div(cols, chunk_cols);
+    const int64_t last_cols = cols - (n_chunks - 1) * chunk_cols;
+    const int64_t stage_bytes = (int64_t)G * T * chunk_bytes;
+    const int64_t stage_pitch = ceil_div(stage_bytes + 16, 128) * 128;
+    int n_stage = (int)std::min<int64_t>(MAX_STAGES, std::max<int64_t>(2, STAGES_BUDGET / stage_pitch));
+    while (n_stage > 2 && 128 + SMEM_HDR + n_stage * stage_pitch > di.smem_optin) --n_stage;
+    const int64_t smem = 128 + SMEM_HDR + n_stage * stage_pitch;   // 128: base alignment slack
+    if (smem > di.smem_optin) return QMV_ERR_SHAPE;
+
+    const int64_t rows_per_cta = std::max<int64_t>(1, rows_cta0);
+    const int64_t ctas_per_job = ceil_div(rows, rows_per_cta);
+
+    Params &p = pl.p;
+    p = Params{};
+    p.rows = rows;
+    p.row_bytes = rb;
+    p.cols = (int32_t)cols;
+    p.chunk_cols = (int32_t)chunk_cols;
+    p.chunk_bytes = (int32_t)chunk_bytes;
+    p.n_chunks = (int32_t)n_chunks;
+    p.last_chunk_cols = (int32_t)last_cols;
+    p.last_chunk_bytes = (int32_t)(last_cols / bw * bb);
+    p.tile_rows = T;
+    p.G = G;
+    p.Gp = gp;
+    p.n_stage = n_stage;
+    p.stage_pitch = (int32_t)stage_pitch;
+    p.row_pitch = (int32_t)chunk_bytes;
+    p.rows_per_cta = (int32_t)rows_per_cta;
+    p.tma = tma ? 1 : 0;
+    p.err = di.err;
+    pl.kc.ntok = n_tok;
+    pl.kc.R = R;
+    pl.kc.xreg = (n_tok == 1 && n_chunks == 1 && shared_x && cols <= 2048);
+    pl.grid = dim3((unsigned)ctas_per_job, (unsigned)n_jobs);
+    pl.smem = (size_t)smem;
+    return QMV_OK;
+}
+
+int launch_plan(int fmt, const Plan &pl, cudaStream_t stream)
+{
+    cudaError_t e;
+    switch (fmt) {
+    case QMV_Q8_0: e = launch_pipeline<FMT_Q8_0>(pl.p, pl.kc, pl.grid, pl.smem, stream); break;
+    case QMV_Q4_K: e = launch_pipeline<FMT_Q4_K>(pl.p, pl.kc, pl.grid, pl.smem, stream); break;
+    default: e = launch_pipeline<FMT_Q6_K>(pl.p, pl.kc, pl.grid, pl.smem, stream); break;
+    }
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return QMV_ERR_CUDA;
+    }
+    return QMV_OK;
+}
+
+int check_matrix(int fmt, int64_t rows, int64_t cols)
+{
+    if (!fmt_ok(fmt)) return QMV_ERR_FMT;
+    if (rows < 1 || cols < 1 || rows > QMV_MAX_ROWS || cols > QMV_MAX_COLS || cols % block_weights(fmt) != 0)
+        return QMV_ERR_SHAPE;
+    return QMV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t qmv_block_bytes(int fmt) { return (size_t)block_bytes(fmt); }
+int qmv_block_weights(int fmt) { return block_weights(fmt); }
+
+void qmv_debug_fail_next_launches(int count) { g_fail_launches.store(count > 0 ? count : 0); }
+
+const char *qmv_strerror(int status)
+{
+    switch (status) {
+    case QMV_OK: return "success";
+    case QMV_ERR_NULL: return "a required pointer is NULL";
+    case QMV_ERR_FMT: return "unknown block format";
+    case QMV_ERR_SHAPE: return "bad shape (rows/cols < 1, cols not a multiple of the block size, or too large)";
+    case QMV_ERR_ALIGN: return "misaligned pointer or stride (W and x need 16 bytes, y 4 bytes)";
+    case QMV_ERR_NTOK: return "n_tok outside [1, 8]";
+    case QMV_ERR_NSEL: return "n_sel / top_k / n_expert outside the supported range";
+    case QMV_ERR_CUDA: return "a CUDA call or kernel launch failed";
+    case QMV_ERR_DEVICE: return "no usable sm_100 device, or a device-side error was recorded";
+    default: return "unknown status";
+    }
+}
+
+int qmv_batched(int fmt, const void *W_blocks, int64_t rows, int64_t cols, const float *x, float *y,
+                int n_tok, qmv_stream_t stream)
+{
+    if (!W_blocks || !x || !y) return QMV_ERR_NULL;
+    int rc = check_matrix(fmt, rows, cols);
+    if (rc) return rc;
+    if (n_tok < 1 || n_tok > QMV_MAX_NTOK) return QMV_ERR_NTOK;
+    if (!aligned(W_blocks, 16) || !aligned(x, 16) || !aligned(y, 4)) return QMV_ERR_ALIGN;
+    if (injected_failure()) return QMV_ERR_CUDA;
+    DevInfo di;
+    if ((rc = get_dev(di))) return rc;
+    Plan pl;
+    if ((rc = make_plan(fmt, rows, cols, n_tok, 1, 1, true, di, pl))) return rc;
+    pl.p.mode = MODE_SEPARATE;
+    pl.p.base0 = static_cast<const uint8_t *>(W_blocks);
+    pl.p.x = x;
+    pl.p.x_tok_stride = cols;
+    pl.p.y = y;
+    pl.p.y_tok_stride = rows;
+    return launch_plan(fmt, pl, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int qmv_f32(int fmt, const void *W_blocks, int64_t rows, int64_t cols, const float *x, float *y,
+            qmv_stream_t stream)
+{
+    return qmv_batched(fmt, W_blocks, rows, cols, x, y, 1, stream);
+}
+
+int moe_route(const float *logits, const float *bias, int n_expert, int top_k, int32_t *ids_out,
+              float *g_out, qmv_stream_t stream)
+{
+    if (!logits || !bias || !ids_out || !g_out) return QMV_ERR_NULL;
+    if (n_expert < 1 || n_expert > QMV_MAX_EXPERTS || top_k < 1 || top_k > QMV_MAX_SEL || top_k > n_expert)
+        return QMV_ERR_NSEL;
+    if (!aligned(logits, 4) || !aligned(bias, 4) || !aligned(ids_out, 4) || !aligned(g_out, 4))
+        return QMV_ERR_ALIGN;
+    if (injected_failure()) return QMV_ERR_CUDA;
+    DevInfo di;
+    int rc = get_dev(di);
+    if (rc) return rc;
+    moe_route_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(logits, bias, n_expert, top_k,
+                                                                          ids_out, g_out);
+    if (cudaGetLastError() != cudaSuccess) return QMV_ERR_CUDA;
+    return QMV_OK;
+}
+
+int moe_qmv(int fmt, const void *expert_blocks, int64_t expert_stride_bytes, int n_expert,
+            const int32_t *expert_ids, int n_sel, int64_t rows, int64_t cols, const float *x,
+            int64_t x_stride, const float *gate_w, float *y, qmv_stream_t stream)
+{
+    if (!expert_blocks || !expert_ids || !x || !y) return QMV_ERR_NULL;
+    int rc = check_matrix(fmt, rows, cols);
+    if (rc) return rc;
+    if (n_expert < 1 || n_expert > QMV_MAX_EXPERTS || n_sel < 1 || n_sel > QMV_MAX_SEL || n_sel > n_expert)
+        return QMV_ERR_NSEL;
+    const int64_t mat_bytes = rows * (cols / block_weights(fmt)) * block_bytes(fmt);
+    if (expert_stride_bytes < mat_bytes || x_stride < 0) return QMV_ERR_SHAPE;
+    if (!aligned(expert_blocks, 16) || expert_stride_bytes % 16 != 0 || !aligned(x, 16) ||
+        x_stride % 4 != 0 || !aligned(y, 4) || !aligned(expert_ids, 4) || (gate_w && !aligned(gate_w, 4)))
+        return QMV_ERR_ALIGN;
+    if (injected_failure()) return QMV_ERR_CUDA;
+    DevInfo di;
+    if ((rc = get_dev(di))) return rc;
+    Plan pl;
+    const bool weighted = gate_w != nullptr;
+    if ((rc = make_plan(fmt, rows, cols, 1, weighted ? n_sel : 1, weighted ? 1 : n_sel,
+                        weighted ? (x_stride == 0) : true, di, pl)))
+        return rc;
+    Params &p = pl.p;
+    p.mode = weighted ? MODE_WEIGHTED : MODE_SEPARATE;
+    p.base0 = static_cast<const uint8_t *>(expert_blocks);
+    p.expert_stride = expert_stride_bytes;
+    p.ids = expert_ids;
+    p.n_expert = n_expert;
+    p.x = x;
+    p.x_stride = x_stride;
+    p.x_tok_stride = cols;
+    p.gw = gate_w;
+    p.y = y;
+    p.y_job_stride = rows;
+    p.y_tok_stride = rows;
+    return launch_plan(fmt, pl, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_ffn(int fmt_gu, const void *gate_blocks, const void *up_blocks, int64_t gu_stride_bytes,
+            int fmt_down, const void *down_blocks, int64_t down_stride_bytes, int n_expert,
+            const int32_t *expert_ids, const float *g, int n_sel, int64_t hidden, int64_t inter,
+            const float *x, float *h_scratch, float *y, qmv_stream_t stream)
+{
+    if (!gate_blocks || !up_blocks || !down_blocks || !expert_ids || !g || !x || !h_scratch || !y)
+        return QMV_ERR_NULL;
+    int rc = check_matrix(fmt_gu, inter, hidden);
+    if (rc) return rc;
+    if ((rc = check_matrix(fmt_down, hidden, inter))) return rc;
+    if (n_expert < 1 || n_expert > QMV_MAX_EXPERTS || n_sel < 1 || n_sel > QMV_MAX_SEL || n_sel > n_expert)
+        return QMV_ERR_NSEL;
+    const int64_t gu_bytes = inter * (hidden / block_weights(fmt_gu)) * block_bytes(fmt_gu);
+    const int64_t dn_bytes = hidden * (inter / block_weights(fmt_down)) * block_bytes(fmt_down);
+    if (gu_stride_bytes < gu_bytes || down_stride_bytes < dn_bytes) return QMV_ERR_SHAPE;
+    if (!aligned(gate_blocks, 16) || !aligned(up_blocks, 16) || !aligned(down_blocks, 16) ||
+        gu_stride_bytes % 16 != 0 || down_stride_bytes % 16 != 0 || !aligned(x, 16) ||
+        !aligned(h_scratch, 16) || !aligned(y, 4) || !aligned(expert_ids, 4) || !aligned(g, 4))
+        return QMV_ERR_ALIGN;
+    if (injected_failure()) return QMV_ERR_CUDA;
+    DevInfo di;
+    if ((rc = get_dev(di))) return rc;
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+    // h_k = silu(G_k x) * (U_k x): two groups (gate, up) per routed expert
+    Plan a;
+    if ((rc = make_plan(fmt_gu, inter, hidden, 1, 2, n_sel, true, di, a))) return rc;
+    a.p.mode = MODE_SWIGLU;
+    a.p.base0 = static_cast<const uint8_t *>(gate_blocks);
+    a.p.base1 = static_cast<const uint8_t *>(up_blocks);
+    a.p.expert_stride = gu_stride_bytes;
+    a.p.ids = expert_ids;
+    a.p.n_expert = n_expert;
+    a.p.x = x;
+    a.p.x_stride = 0;
+    a.p.x_tok_stride = hidden;
+    a.p.y = h_scratch;
+    a.p.y_job_stride = inter;
+    a.p.y_tok_stride = inter;
+    if ((rc = launch_plan(fmt_gu, a, st))) return rc;
+
+    // y = sum_k g_k D_k h_k: one group per routed expert, weighted in k order
+    Plan b;
+    if ((rc = make_plan(fmt_down, hidden, inter, 1, n_sel, 1, false, di, b))) return rc;
+    b.p.mode = MODE_WEIGHTED;
+    b.p.base0 = static_cast<const uint8_t *>(down_blocks);
+    b.p.expert_stride = down_stride_bytes;
+    b.p.ids = expert_ids;
+    b.p.n_expert = n_expert;
+    b.p.x = h_scratch;
+    b.p.x_stride = inter;
+    b.p.x_tok_stride = inter;
+    b.p.gw = g;
+    b.p.y = y;
+    b.p.y_tok_stride = hidden;
+    return launch_plan(fmt_down, b, st);
+}
+
+int qmv_dequant(int fmt, const void *W_blocks, int64_t rows, int64_t cols, float *out, qmv_stream_t stream)
+{
+    if (!W_blocks || !out) return QMV_ERR_NULL;
+    int rc = check_matrix(fmt, rows, cols);
+    if (rc) return rc;
+    if (!aligned(W_blocks, 16) || !aligned(out, 4)) return QMV_ERR_ALIGN;
+    if (injected_failure()) return QMV_ERR_CUDA;
+    DevInfo di;
+    if ((rc = get_dev(di))) return rc;
+    const int64_t bpr = cols / block_weights(fmt);
+    const int64_t nblk = rows * bpr;
+    const unsigned grid = (unsigned)std::min<int64_t>(ceil_div(nblk, 256), (int64_t)di.sm_count * 16);
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const uint8_t *W = static_cast<const uint8_t *>(W_blocks);
+    switch (fmt) {
+    case QMV_Q8_0: dequant_kernel<FMT_Q8_0><<<grid, 256, 0, st>>>(W, nblk, bpr, cols, out); break;
+    case QMV_Q4_K: dequant_kernel<FMT_Q4_K><<<grid, 256, 0, st>>>(W, nblk, bpr, cols, out); break;
+    default: dequant_kernel<FMT_Q6_K><<<grid, 256, 0, st>>>(W, nblk, bpr, cols, out); break;
+    }
+    if (cudaGetLastError() != cudaSuccess) return QMV_ERR_CUDA;
+    return QMV_OK;
+}
+
+int qmv_check(qmv_stream_t stream, int *dev_err_out)
+{
+    if (dev_err_out) *dev_err_out = 0;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return QMV_ERR_CUDA;
+    }
+    DevInfo di;
+    int rc = get_dev(di);
+    if (rc) return rc;
+    int word = 0;
+    if (cudaMemcpy(&word, di.err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
+        cudaMemset(di.err, 0, sizeof(int)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+        (void)cudaGetLastError();
+        return QMV_ERR_CUDA;
+    }
+    if (dev_err_out) *dev_err_out = word;
+    return word ? QMV_ERR_DEVICE : QMV_OK;
+}
+
+}  // extern "C"

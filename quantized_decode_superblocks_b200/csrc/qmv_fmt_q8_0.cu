@@ -1,0 +1,6 @@
+// Kernel instances of the quantized matvec pipeline for one block format.
+#include "qmv_dispatch.cuh"
+
+namespace qmv {
+template cudaError_t launch_pipeline<FMT_Q8_0>(const Params &, const KernelChoice &, dim3, size_t, cudaStream_t);
+}  // namespace qmv

@@ -1,0 +1,375 @@
+"""Parity of the CUDA path (through the C ABI) with the oracle.
+
+Bars: dequantization bit-exact; every matvec output within
+|y - y_ref| <= 1e-4 * sum_i |w_i x_i| + 1e-6 (y_ref, the bound: f64 oracle);
+router ids exact (a margin at the top-k cut is asserted first), weights within
+1e-6 relative; the MoE FFN by the composite rule written in each test.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+import oracle
+import quantized_decode_superblocks_b200 as q
+from quantized_decode_superblocks_b200 import synth
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+Q8_0, Q4_K, Q6_K = synth.Q8_0, synth.Q4_K, synth.Q6_K
+REL, ABS = 1e-4, 1e-6
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    q.build()
+    q.lib()
+    yield
+    assert q.qmv_check() == 0
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def within(y, ref, bound, rel=REL, abs_=ABS):
+    y = np.asarray(y, dtype=np.float64)
+    err = np.abs(y - ref)
+    lim = rel * bound + abs_
+    bad = err > lim
+    assert not bad.any(), (f"{bad.sum()} of {bad.size} outside tolerance; worst err/lim "
+                           f"{(err / lim).max():.3g} at {np.unravel_index((err / lim).argmax(), err.shape)}")
+    return float((err / lim).max())
+
+
+def run_qmv(fmt, W, rows, cols, x):
+    x = np.atleast_2d(x)
+    n_tok = x.shape[0]
+    Wd, xd = dev(W), dev(x)
+    yd = torch.full((n_tok, rows), float("nan"), device="cuda")
+    if n_tok == 1:
+        q.qmv_f32(fmt, Wd, rows, cols, xd, yd)
+    else:
+        q.qmv_batched(fmt, Wd, rows, cols, xd, yd, n_tok)
+    torch.cuda.synchronize()
+    return yd.cpu().numpy()
+
+
+# ----------------------------------------------------------------- dequant --
+
+@pytest.mark.parametrize("fmt,rows,cols", [(Q8_0, 37, 96), (Q8_0, 5, 2048), (Q4_K, 37, 512),
+                                           (Q4_K, 3, 1792), (Q6_K, 37, 768), (Q6_K, 2, 2048)])
+def test_dequant_bit_exact(fmt, rows, cols):
+    W = synth.gen_blocks(fmt, rows, cols, seed=31, tensor_id=fmt)
+    out = torch.empty((rows, cols), device="cuda")
+    q.qmv_dequant(fmt, dev(W), rows, cols, out)
+    ref = oracle.dequant(fmt, W, rows, cols)
+    assert np.array_equal(out.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+def test_fp16_decode_every_pattern_on_gpu():
+    # one Q8_0 block per fp16 pattern: d = pattern, q[0] = 1  ->  w[0] = f32(d)
+    n = 65536
+    W = np.zeros((n, 34), np.uint8)
+    W[:, 0] = np.arange(n) & 0xFF
+    W[:, 1] = np.arange(n) >> 8
+    W[:, 2] = 1
+    out = torch.empty((n, 32), device="cuda")
+    q.qmv_dequant(Q8_0, dev(W.reshape(-1)), n, 32, out)
+    got = out[:, 0].cpu().numpy()
+    ref = np.array([oracle.half_to_float(b) for b in range(n)], np.float32)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan].view(np.uint32), ref[~nan].view(np.uint32))
+
+
+def test_dequant_rejects_with_status_and_leaves_output():
+    out = torch.full((4, 256), 7.0, device="cuda")
+    with pytest.raises(q.QmvError):
+        q.qmv_dequant(Q4_K, dev(np.zeros(4 * 144, np.uint8)), 4, 200, out)
+    assert bool((out == 7.0).all())
+
+
+# ------------------------------------------------------------------ matvec --
+
+SMALL = [
+    (Q8_0, 1, 32), (Q8_0, 3, 96), (Q8_0, 37, 1024), (Q8_0, 257, 2048), (Q8_0, 70, 4096),
+    (Q4_K, 1, 256), (Q4_K, 3, 512), (Q4_K, 37, 1792), (Q4_K, 257, 2048), (Q4_K, 20, 4096),
+    (Q6_K, 1, 256), (Q6_K, 3, 768), (Q6_K, 37, 1792), (Q6_K, 257, 2048), (Q6_K, 20, 4096),
+]
+
+
+@pytest.mark.parametrize("fmt,rows,cols", SMALL)
+@pytest.mark.parametrize("n_tok", [1, 2, 3, 5, 8])
+def test_qmv_small_shapes(fmt, rows, cols, n_tok):
+    W = synth.gen_blocks(fmt, rows, cols, seed=7, tensor_id=100 + fmt)
+    x = synth.gen_x(n_tok, cols, seed=7, tensor_id=200 + n_tok)
+    y = run_qmv(fmt, W, rows, cols, x)
+    ref, bound = oracle.qmv(fmt, W, rows, cols, x)
+    within(y, ref, bound)
+
+
+@pytest.mark.parametrize("fmt,rows,cols", [(Q8_0, 300, 8192), (Q8_0, 9, 16384), (Q4_K, 40, 16384),
+                                           (Q6_K, 33, 8192), (Q8_0, 17, 8224), (Q6_K, 5, 4352)])
+@pytest.mark.parametrize("n_tok", [1, 4, 8])
+def test_qmv_long_rows_k_chunked(fmt, rows, cols, n_tok):
+    W = synth.gen_blocks(fmt, rows, cols, seed=8, tensor_id=300 + fmt)
+    x = synth.gen_x(n_tok, cols, seed=8, tensor_id=400 + n_tok)
+    y = run_qmv(fmt, W, rows, cols, x)
+    ref, bound = oracle.qmv(fmt, W, rows, cols, x)
+    within(y, ref, bound)
+
+
+@pytest.mark.parametrize("n_tok", [1, 4, 8])
+def test_every_n_tok_agrees_with_single_token_calls(n_tok):
+    fmt, rows, cols = Q6_K, 129, 2048
+    W = synth.gen_blocks(fmt, rows, cols, seed=9, tensor_id=1)
+    x = synth.gen_x(n_tok, cols, seed=9, tensor_id=2)
+    yb = run_qmv(fmt, W, rows, cols, x)
+    ref, bound = oracle.qmv(fmt, W, rows, cols, x)
+    for t in range(n_tok):
+        within(run_qmv(fmt, W, rows, cols, x[t]), ref[t:t + 1], bound[t:t + 1])
+    within(yb, ref, bound)
+
+
+def test_closed_form_constant_blocks_on_gpu():
+    # Q4_K with every field constant: y = (d*S*Q - dmin*M) * sum(x) for every row
+    from blockpack import f16_bits, pack_q4_k, pack_q8_0
+    d, dmin, S, Q, M = 0.0078125, 0.00390625, 37, 11, 5
+    rows, cols = 64, 2048
+    blk = pack_q4_k(f16_bits(d), f16_bits(dmin), [S] * 8, [M] * 8, [Q] * 256)
+    x = synth.gen_x(1, cols, 13, 0)
+    y = run_qmv(Q4_K, np.tile(blk, rows * cols // 256), rows, cols, x)
+    exact = (d * S * Q - dmin * M) * float(np.sum(x.astype(np.float64)))
+    bound = (abs(d * S * Q - dmin * M)) * float(np.sum(np.abs(x.astype(np.float64))))
+    within(y, np.full_like(y, exact, dtype=np.float64), np.full(y.shape, bound))
+    # Q8_0 with d = 1 and small integer x: the dot is an exact integer
+    g = np.random.default_rng(5)
+    qv = g.integers(-127, 128, size=(8, 1024))
+    W8 = np.concatenate([pack_q8_0(f16_bits(1.0), qv[r, 32 * b:32 * b + 32])
+                         for r in range(8) for b in range(32)])
+    xi = g.integers(-8, 9, size=(1, 1024)).astype(np.float32)
+    y8 = run_qmv(Q8_0, W8, 8, 1024, xi)
+    assert y8[0].tolist() == [float(v) for v in (qv @ xi[0].astype(np.int64))]
+
+
+def test_results_are_deterministic():
+    fmt, rows, cols = Q4_K, 3072, 2048
+    W = synth.gen_blocks(fmt, rows, cols, seed=1, tensor_id=0)
+    x = synth.gen_x(1, cols, seed=1, tensor_id=1)
+    ys = [run_qmv(fmt, W, rows, cols, x) for _ in range(5)]
+    for y in ys[1:]:
+        assert np.array_equal(y.view(np.uint32), ys[0].view(np.uint32))
+
+
+# ---------------------------------------------------- full-size workloads --
+
+def test_cfg0_q8_0_1024x1024():
+    w = synth.workload_cfg0()
+    W = synth.gen_blocks(w["fmt"], w["rows"], w["cols"], w["seed"], 0)
+    x = synth.gen_x(1, w["cols"], w["seed"], 1)
+    y = run_qmv(w["fmt"], W, w["rows"], w["cols"], x)
+    ref, bound = oracle.qmv(w["fmt"], W, w["rows"], w["cols"], x)
+    within(y, ref, bound)
+
+
+def test_cfg1_fused_qkv_equals_the_three_projections():
+    w = synth.workload_cfg1()
+    fmt, rows, cols = w["fmt"], w["rows"], w["cols"]
+    W = synth.gen_blocks(fmt, rows, cols, w["seed"], 0)
+    x = synth.gen_x(1, cols, w["seed"], 1)
+    y = run_qmv(fmt, W, rows, cols, x)
+    ref, bound = oracle.qmv(fmt, W, rows, cols, x)
+    within(y, ref, bound)
+    rb = synth.matrix_bytes(fmt, 1, cols)
+    parts = [run_qmv(fmt, W[a * rb:b * rb], b - a, cols, x) for _, a, b in w["segments"]]
+    within(np.concatenate(parts, axis=1), ref, bound)
+
+
+@pytest.mark.parametrize("n_tok", [1, 4])
+def test_cfg2_q6_k_vocab_projection_sampled_rows(n_tok):
+    w = synth.workload_cfg2(n_tok)
+    fmt, rows, cols = w["fmt"], w["rows"], w["cols"]
+    W = synth.gen_blocks(fmt, rows, cols, w["seed"], 0)
+    x = synth.gen_x(n_tok, cols, w["seed"], 1)
+    y = run_qmv(fmt, W, rows, cols, x)
+    idx = np.unique(np.concatenate([np.arange(64), np.arange(rows - 64, rows),
+                                    np.random.default_rng(n_tok).integers(0, rows, 4000)]))
+    ref, bound = oracle.qmv_rows(fmt, W, rows, cols, idx, x)
+    within(y[:, idx], ref, bound)
+
+
+@pytest.mark.parametrize("n_tok", [1, 2, 4, 8])
+def test_cfg4_q8_0_layer_matvecs(n_tok):
+    # layer 0 of the 16-layer Q8_0 stack: every row; the bench times the same calls
+    for m, (name, rows, cols) in enumerate(synth.workload_cfg4_layer()):
+        W = synth.gen_blocks(Q8_0, rows, cols, synth.CFG4_SEED, m)
+        x = synth.gen_x(n_tok, cols, synth.CFG4_SEED, 1000 + m)
+        y = run_qmv(Q8_0, W, rows, cols, x)
+        if rows * cols <= 3072 * 2048 or n_tok == 1:
+            ref, bound = oracle.qmv(Q8_0, W, rows, cols, x, nthreads=8)
+            within(y, ref, bound)
+        else:
+            idx = np.random.default_rng(m).integers(0, rows, 1024)
+            ref, bound = oracle.qmv_rows(Q8_0, W, rows, cols, idx, x)
+            within(y[:, idx], ref, bound)
+
+
+# --------------------------------------------------------------------- MoE --
+
+def _router_case(seed):
+    logits, bias = synth.gen_router(32, seed, 5)
+    ids, g, biased = oracle.route(logits, bias, 4)
+    srt = np.sort(biased.astype(np.float64))[::-1]
+    assert srt[3] - srt[4] > 1e-5, "ambiguous top-4 cut for this seed"
+    return logits, bias, ids, g
+
+
+@pytest.mark.parametrize("seed", [3, 4, 5, 6, 7, 8, 9, 10])
+def test_router_matches_oracle(seed):
+    logits, bias, ids, g = _router_case(seed)
+    ids_d = torch.empty(4, dtype=torch.int32, device="cuda")
+    g_d = torch.empty(4, device="cuda")
+    q.moe_route(dev(logits), dev(bias), 32, 4, ids_d, g_d)
+    torch.cuda.synchronize()
+    assert ids_d.cpu().tolist() == ids.tolist()
+    assert np.allclose(g_d.cpu().numpy(), g, rtol=1e-6, atol=0)
+
+
+def test_router_other_sizes_and_ties():
+    logits = np.zeros(40, np.float32)
+    bias = np.zeros(40, np.float32)
+    bias[[3, 17, 39]] = 1.0
+    ids_d = torch.empty(5, dtype=torch.int32, device="cuda")
+    g_d = torch.empty(5, device="cuda")
+    q.moe_route(dev(logits), dev(bias), 40, 5, ids_d, g_d)
+    torch.cuda.synchronize()
+    ids, g, _ = oracle.route(logits, bias, 5)
+    assert ids_d.cpu().tolist() == ids.tolist() == [3, 17, 39, 0, 1]
+    assert np.allclose(g_d.cpu().numpy(), 0.2, rtol=1e-6)
+
+
+def _moe_weights(n_expert, hidden, inter, seed):
+    gus = synth.matrix_bytes(Q4_K, inter, hidden)
+    ds = synth.matrix_bytes(Q4_K, hidden, inter)
+    gate = synth.gen_blocks(Q4_K, inter * n_expert, hidden, seed, 1)
+    up = synth.gen_blocks(Q4_K, inter * n_expert, hidden, seed, 2)
+    down = synth.gen_blocks(Q4_K, hidden * n_expert, inter, seed, 3)
+    x = synth.gen_x(1, hidden, seed, 4)[0]
+    return gate, up, down, gus, ds, x
+
+
+def test_moe_qmv_separate_and_weighted():
+    n_expert, rows, cols = 8, 300, 1792
+    mb = synth.matrix_bytes(Q4_K, rows, cols)
+    E = synth.gen_blocks(Q4_K, rows * n_expert, cols, 40, 1)
+    ids = np.array([5, 0, 7, 2], np.int32)
+    xs = synth.gen_x(4, cols, 40, 2)
+    gw = np.array([0.1, 0.2, 0.3, 0.4], np.float32)
+    # separate: y[k] = W_{ids[k]} x_k
+    y = torch.empty((4, rows), device="cuda")
+    q.moe_qmv(Q4_K, dev(E), mb, n_expert, dev(ids), 4, rows, cols, dev(xs), cols, None, y)
+    yw = torch.empty(rows, device="cuda")
+    q.moe_qmv(Q4_K, dev(E), mb, n_expert, dev(ids), 4, rows, cols, dev(xs), cols, dev(gw), yw)
+    # shared x (x_stride 0), weighted
+    ys = torch.empty(rows, device="cuda")
+    q.moe_qmv(Q4_K, dev(E), mb, n_expert, dev(ids[:3]), 3, rows, cols, dev(xs[0]), 0, dev(gw[:3]), ys)
+    torch.cuda.synchronize()
+    refs, bounds = [], []
+    for k, e in enumerate(ids):
+        r, b = oracle.qmv(Q4_K, E[e * mb:(e + 1) * mb], rows, cols, xs[k])
+        refs.append(r[0]); bounds.append(b[0])
+    within(y.cpu().numpy(), np.array(refs), np.array(bounds))
+    wsum = sum(float(gw[k]) * refs[k] for k in range(4))
+    wb = sum(abs(float(gw[k])) * bounds[k] for k in range(4))
+    within(yw.cpu().numpy(), wsum, wb)
+    r3 = [oracle.qmv(Q4_K, E[e * mb:(e + 1) * mb], rows, cols, xs[0]) for e in ids[:3]]
+    within(ys.cpu().numpy(), sum(float(gw[k]) * r3[k][0][0] for k in range(3)),
+           sum(abs(float(gw[k])) * r3[k][1][0] for k in range(3)))
+
+
+def test_moe_bad_expert_id_is_dropped_and_reported():
+    n_expert, rows, cols = 4, 64, 256
+    mb = synth.matrix_bytes(Q4_K, rows, cols)
+    E = synth.gen_blocks(Q4_K, rows * n_expert, cols, 41, 1)
+    x = synth.gen_x(1, cols, 41, 2)
+    y = torch.full((2, rows), 5.0, device="cuda")
+    q.moe_qmv(Q4_K, dev(E), mb, n_expert, dev(np.array([1, 9], np.int32)), 2, rows, cols,
+              dev(x), 0, None, y)
+    err = q.qmv_check()
+    assert err & q.DEVERR_EXPERT_ID
+    assert q.qmv_check() == 0                      # cleared by the read
+    ref, bound = oracle.qmv(Q4_K, E[mb:2 * mb], rows, cols, x)
+    yh = y.cpu().numpy()
+    within(yh[:1], ref, bound)
+    assert np.array_equal(yh[1], np.zeros(rows, np.float32))
+
+
+def _check_moe_ffn(n_expert, hidden, inter, seed, ids, g32):
+    gate, up, down, gus, ds, x = _moe_weights(n_expert, hidden, inter, seed)
+    n_sel = len(ids)
+    h = torch.empty((n_sel, inter), device="cuda")
+    y = torch.empty(hidden, device="cuda")
+    q.moe_ffn(Q4_K, dev(gate), dev(up), gus, Q4_K, dev(down), ds, n_expert,
+              dev(np.asarray(ids, np.int32)), dev(g32), n_sel, hidden, inter, dev(x), h, y)
+    torch.cuda.synchronize()
+    hg, yg = h.cpu().numpy(), y.cpu().numpy()
+    g64 = g32.astype(np.float64)
+    full = oracle.moe_ffn(Q4_K, gate, up, gus, Q4_K, down, ds, n_expert, ids, g64, hidden, inter, x)
+    # (i) h_k = silu(u_k) v_k, with u_k and v_k each held to the single-matvec rule
+    y_ref2 = np.zeros(hidden)
+    b2 = np.zeros(hidden)
+    prop = np.zeros(hidden)
+    for k, e in enumerate(ids):
+        _, bu = oracle.qmv(Q4_K, gate[e * gus:(e + 1) * gus], inter, hidden, x)
+        _, bv = oracle.qmv(Q4_K, up[e * gus:(e + 1) * gus], inter, hidden, x)
+        du, dv = REL * bu[0] + ABS, REL * bv[0] + ABS
+        u, v = full["u"][k], full["v"][k]
+        su = u / (1 + np.exp(-u))
+        dh = 1.1 * du * np.abs(v) + np.abs(su) * dv + 1.1 * du * dv + 1e-6 * np.abs(full["h"][k])
+        err = np.abs(hg[k] - full["h"][k])
+        assert (err <= dh + ABS).all(), f"h_{k}: worst {(err / (dh + ABS)).max():.3g}"
+        # (ii) the down stage fed the GPU's own h_k
+        Dk = down[e * ds:(e + 1) * ds]
+        r, b = oracle.qmv(Q4_K, Dk, hidden, inter, hg[k])
+        y_ref2 += g64[k] * r[0]
+        b2 += abs(g64[k]) * b[0]
+        prop += abs(g64[k]) * (np.abs(oracle.dequant(Q4_K, Dk, hidden, inter).astype(np.float64)) @ dh)
+    within(yg, y_ref2, b2)
+    # (iii) end to end against the all-f64 oracle, the bound widened by the h error
+    err = np.abs(yg - full["y"])
+    assert (err <= REL * b2 + ABS + prop).all()
+
+
+def test_moe_ffn_cfg3_routed_on_device():
+    w = synth.workload_cfg3()
+    n_expert, hidden, inter, seed = w["n_expert"], w["hidden"], w["inter"], w["seed"]
+    logits, bias, ids, g = _router_case(seed)
+    # route on the device, then the FFN step from the device ids / weights
+    gate, up, down, gus, ds, x = _moe_weights(n_expert, hidden, inter, seed)
+    ids_d = torch.empty(4, dtype=torch.int32, device="cuda")
+    g_d = torch.empty(4, device="cuda")
+    q.moe_route(dev(logits), dev(bias), n_expert, 4, ids_d, g_d)
+    h = torch.empty((4, inter), device="cuda")
+    y = torch.empty(hidden, device="cuda")
+    q.moe_ffn(Q4_K, dev(gate), dev(up), gus, Q4_K, dev(down), ds, n_expert, ids_d, g_d, 4,
+              hidden, inter, dev(x), h, y)
+    torch.cuda.synchronize()
+    assert ids_d.cpu().tolist() == ids.tolist()
+    y_dev = y.cpu().numpy()
+    # the same step with the oracle's ids and the device's weights, checked in full
+    _check_moe_ffn(n_expert, hidden, inter, seed, ids.tolist(), g_d.cpu().numpy())
+    h2 = torch.empty((4, inter), device="cuda")
+    y2 = torch.empty(hidden, device="cuda")
+    q.moe_ffn(Q4_K, dev(gate), dev(up), gus, Q4_K, dev(down), ds, n_expert, dev(ids), g_d, 4,
+              hidden, inter, dev(x), h2, y2)
+    torch.cuda.synchronize()
+    assert np.array_equal(y2.cpu().numpy().view(np.uint32), y_dev.view(np.uint32))
+
+
+@pytest.mark.parametrize("ids", [[2], [0, 3], [1, 2, 3], [4, 0, 6, 1, 5, 7, 3, 2]])
+def test_moe_ffn_other_expert_counts(ids):
+    g = np.random.default_rng(len(ids)).uniform(0.1, 1.0, len(ids)).astype(np.float32)
+    _check_moe_ffn(8, 512, 768, 50 + len(ids), ids, g)
