@@ -87,8 +87,14 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, pci_bus_id):
-        self.bus = (pci_bus_id or "").lower()
+    def __init__(self, props):
+        b = getattr(props, "pci_bus_id", "")
+        if not isinstance(b, str):
+            try:
+                b = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            except (AttributeError, TypeError, ValueError):
+                b = ""
+        self.bus = b.lower()
         self.proc = None
         self.path = None
 
@@ -182,10 +188,11 @@ def time_graph(torch, graph, reps, stream):
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
-    start.record(stream)
-    for _ in range(reps):
-        graph.replay()
-    end.record(stream)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        end.record(stream)
     end.synchronize()
     return start.elapsed_time(end) / 1e3   # seconds
 
@@ -443,10 +450,11 @@ def main():
     assert q.qmv_check(stream) == 0
 
     per_config = {}
-    with ClockSampler(getattr(props, "pci_bus_id", "")) as clk:
+    with ClockSampler(props) as clk:
         # warm-up, then the timed steps (device time, barrier + sync on both sides)
-        for _ in range(args.warmup):
-            graph.replay()
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                graph.replay()
         torch.cuda.synchronize()
         dist.barrier(torch)
         torch.cuda.synchronize()
@@ -488,8 +496,7 @@ def main():
     clocks = clk.summary()
     assert q.qmv_check(stream) == 0
 
-    total_bytes = sweep.weight_bytes * dist.world
-    value = total_bytes / sec / 1e9 * 1.0 if False else sweep.weight_bytes * dist.world / (sec / args.steps) / 1e9
+    value = sweep.weight_bytes * dist.world / (sec / args.steps) / 1e9
     ms_per_step = sec / args.steps * 1e3
     achieved = sweep.algo / sum(durs) / 1e9
     traffic = None

@@ -70,7 +70,7 @@ def lib() -> ctypes.CDLL:
 
 
 def build(verbose: bool = False) -> str:
-    from .build import build as _build
+    from .buildlib import build as _build
     return _build(verbose=verbose)
 
 
