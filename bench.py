@@ -400,8 +400,9 @@ def run_profile_case(args):
     device) -- the small case that ncu captures."""
     import torch
     import quantized_decode_superblocks_b200 as q
-    fmt = {"q8_0": Q8_0, "q4_k": Q4_K, "q6_k": Q6_K}[args.profile_case]
-    rows, cols = {Q8_0: (65536, 2048), Q4_K: (131072, 2048), Q6_K: (96000, 2048)}[fmt]
+    fmt = {"q8_0": Q8_0, "q4_k": Q4_K, "q6_k": Q6_K, "q8_0_down": Q8_0, "q8_0_o": Q8_0}[args.profile_case]
+    rows, cols = {"q8_0": (65536, 2048), "q4_k": (131072, 2048), "q6_k": (96000, 2048),
+                  "q8_0_down": (16384, 8192), "q8_0_o": (2048, 2048)}[args.profile_case]
     torch.cuda.set_device(0)
     W = torch.from_numpy(synth.gen_blocks(fmt, rows, cols, 77, 0)).cuda()
     x = torch.from_numpy(synth.gen_x(args.n_tok, cols, 77, 1)).cuda()
@@ -426,7 +427,7 @@ def main():
     ap.add_argument("--n-tok", type=int, default=1)
     ap.add_argument("--headline-only", action="store_true",
                     help="skip the per-config measurements and the CPU baseline")
-    ap.add_argument("--profile-case", choices=["q8_0", "q4_k", "q6_k"])
+    ap.add_argument("--profile-case", choices=["q8_0", "q4_k", "q6_k", "q8_0_down", "q8_0_o"])
     args = ap.parse_args()
     if args.warmup < 3 and not args.profile_case:
         raise SystemExit("--warmup must be at least 3")

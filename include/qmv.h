@@ -156,9 +156,24 @@ int qmv_check(qmv_stream_t stream, int *dev_err_out);
 /* Static, never-NULL description of a qmv_status value. */
 const char *qmv_strerror(int status);
 
+/* Description of the CUDA error behind the last QMV_ERR_CUDA returned on the
+ * calling host thread ("no error" if there was none). */
+const char *qmv_last_cuda_error(void);
+
 /* Bytes and weights per block of a format; 0 for an unknown format. */
 size_t qmv_block_bytes(int fmt);
 int qmv_block_weights(int fmt);
+
+/* Programmatic dependent launch for the matvec launches (process-wide, off by
+ * default).  When enabled, a matvec launch may start -- and begin streaming
+ * its weight blocks into shared memory -- while the previous kernel in the
+ * stream is still running; it waits for that kernel to finish before it reads
+ * x, expert ids or gate weights and before it writes any output.  This hides
+ * the launch gap between back-to-back matvecs of a decode step.  Enable it
+ * only when no kernel still in flight on the stream writes the weight blocks
+ * (true for inference weights loaded once).  qmv_get_pdl returns the setting. */
+void qmv_set_pdl(int enable);
+int qmv_get_pdl(void);
 
 /* Test hook for host-side failure handling: the next `count` launches made by
  * this library fail with QMV_ERR_CUDA without reaching the GPU. */

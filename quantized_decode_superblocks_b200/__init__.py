@@ -27,13 +27,16 @@ DEVERR_TIMEOUT = 2
 
 EXPORTED = ("qmv_f32", "qmv_batched", "moe_route", "moe_qmv", "moe_ffn", "qmv_dequant",
             "qmv_check", "qmv_strerror", "qmv_block_bytes", "qmv_block_weights",
-            "qmv_debug_fail_next_launches")
+            "qmv_debug_fail_next_launches", "qmv_set_pdl", "qmv_get_pdl", "qmv_last_cuda_error")
 
 
 class QmvError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({strerror(status)})")
+        detail = strerror(status)
+        if status == -7:
+            detail += ": " + lib().qmv_last_cuda_error().decode()
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({detail})")
 
 
 _lib = None
@@ -62,8 +65,14 @@ def lib() -> ctypes.CDLL:
         L.qmv_block_weights.argtypes = [c_int]
         L.qmv_debug_fail_next_launches.argtypes = [c_int]
         L.qmv_debug_fail_next_launches.restype = None
+        L.qmv_set_pdl.argtypes = [c_int]
+        L.qmv_set_pdl.restype = None
+        L.qmv_get_pdl.argtypes = []
+        L.qmv_last_cuda_error.argtypes = []
+        L.qmv_last_cuda_error.restype = ctypes.c_char_p
         for name in EXPORTED:
-            if name not in ("qmv_strerror", "qmv_block_bytes", "qmv_debug_fail_next_launches"):
+            if name not in ("qmv_strerror", "qmv_block_bytes", "qmv_debug_fail_next_launches", "qmv_set_pdl",
+                            "qmv_last_cuda_error"):
                 getattr(L, name).restype = c_int
         _lib = L
     return _lib
@@ -99,6 +108,15 @@ def _stream(stream):
 def _check(rc: int, where: str):
     if rc != QMV_OK:
         raise QmvError(rc, where)
+
+
+def qmv_set_pdl(enable: bool) -> None:
+    """Programmatic dependent launch for matvec launches (see include/qmv.h)."""
+    lib().qmv_set_pdl(1 if enable else 0)
+
+
+def qmv_get_pdl() -> bool:
+    return bool(lib().qmv_get_pdl())
 
 
 def qmv_block_bytes(fmt: int) -> int:

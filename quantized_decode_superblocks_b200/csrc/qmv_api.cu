@@ -14,8 +14,13 @@ using namespace qmv;
 // Sticky device error word (QMV_DEVERR_* bits), read and cleared by qmv_check.
 __device__ int g_dev_err;
 
-constexpr int STAGE_MAX = 32 * 1024;      // bytes of one pipeline stage
-constexpr int STAGES_BUDGET = 96 * 1024;  // all stages of one CTA (two CTAs per SM)
+constexpr int STAGE_MAX = 36 * 1024;       // bytes of one pipeline stage
+constexpr int STAGES_BUDGET2 = 105 * 1024; // all stages of one CTA, two CTAs per SM (1-2 tokens)
+constexpr int STAGES_BUDGET1 = 192 * 1024; // one CTA per SM (3-8 tokens: more registers per thread)
+#ifndef QMV_SMALL_CTA_BYTES
+#define QMV_SMALL_CTA_BYTES (96 * 1024)
+#endif
+constexpr int64_t SMALL_CTA_BYTES = QMV_SMALL_CTA_BYTES;
 
 struct DevInfo {
     int sm_count = 0;
@@ -27,6 +32,15 @@ struct DevInfo {
 std::mutex g_mu;
 DevInfo g_dev[64];
 std::atomic<int> g_fail_launches{0};
+std::atomic<int> g_pdl{0};
+thread_local cudaError_t t_last_cuda = cudaSuccess;
+
+int cuda_fail(cudaError_t e)
+{
+    t_last_cuda = e;
+    (void)cudaGetLastError();
+    return QMV_ERR_CUDA;
+}
 
 int block_weights(int fmt) { return fmt == QMV_Q8_0 ? 32 : (fmt == QMV_Q4_K || fmt == QMV_Q6_K) ? 256 : 0; }
 int block_bytes(int fmt) { return fmt == QMV_Q8_0 ? 34 : fmt == QMV_Q4_K ? 144 : fmt == QMV_Q6_K ? 210 : 0; }
@@ -78,35 +92,60 @@ struct Plan {
     size_t smem;
 };
 
-int make_plan(int fmt, int64_t rows, int64_t cols, int n_tok, int G, int n_jobs, bool shared_x,
+int make_plan(int fmt, int64_t rows, int64_t cols, int n_tok, int G, int n_jobs, bool /*shared_x*/,
               const DevInfo &di, Plan &pl)
 {
     const int bw = block_weights(fmt), bb = block_bytes(fmt);
     const int64_t rb = cols / bw * bb;
     const int ntp = pow2ceil(n_tok);
     const int gp = pow2ceil(G);
+    const int sw = fmt == QMV_Q8_0 ? 32 : 64;          // weights per lane slice
+    const int64_t xcap = fmt == QMV_Q8_0 ? 64 : 32;    // register-resident slices per lane x 32
+    const int64_t n1 = cols / sw;
     const bool tma = (rb % 16) == 0;
-    const int target_ctas = 2 * di.sm_count;
+    // Two CTAs per SM hide memory latency for large matrices.  A small matrix
+    // (under SMALL_CTA_BYTES of weights per CTA at two per SM) instead takes
+    // one CTA per SM, leaving the second slot free: with programmatic
+    // dependent launch the next kernel's CTAs then start on it and prefetch
+    // their weights while this kernel finishes.
+    int ctas_per_sm = n_tok <= 2 ? 2 : 1;
+    if (ctas_per_sm == 2) {
+        const int64_t per_cta = ceil_div((int64_t)n_jobs * rows, 2LL * di.sm_count) * rb * G;
+        if (per_cta < SMALL_CTA_BYTES) ctas_per_sm = 1;
+    }
+    const int target_ctas = ctas_per_sm * di.sm_count;
+    const int64_t budget = n_tok <= 2 ? STAGES_BUDGET2 : STAGES_BUDGET1;
     const int64_t ctas_job0 = std::max<int64_t>(1, target_ctas / n_jobs);
     const int64_t rows_cta0 = ceil_div(rows, ctas_job0);
 
-    int R = gp;
-    const int rmax = std::min(8, 32 / ntp);
-    for (int cand = rmax; cand >= gp; cand >>= 1) {
-        const int64_t t = (int64_t)NC * cand / gp;
-        if (t <= std::max<int64_t>(rows_cta0, NC / gp) && (int64_t)G * t * rb <= STAGE_MAX) {
+    // warps per row (K-segments): one token -> the fewest that keep a warp's x
+    // in registers; several tokens -> segments of at most 2048 columns
+    const int maxw = NW / gp;
+    int wpr = 1;
+    if (n_tok == 1) {
+        while (wpr < maxw && ceil_div(n1, wpr) > xcap) wpr *= 2;
+    } else {
+        while (wpr < maxw && cols / wpr > 2048) wpr *= 2;
+    }
+    const int nrs = NW / (gp * wpr);
+
+    const int rmax = n_tok == 1 ? 8 : std::min(4, 32 / ntp);
+    int R = 1;
+    for (int cand = rmax; cand >= 1; cand >>= 1) {
+        const int64_t t = (int64_t)nrs * cand;
+        if (t <= std::max<int64_t>(rows_cta0, nrs) && (int64_t)G * t * rb <= STAGE_MAX) {
             R = cand;
             break;
         }
     }
-    if (R * ntp > 32 || R < gp) return QMV_ERR_SHAPE;
-    const int T = NC * R / gp;
+    if (R * ntp > 32) return QMV_ERR_SHAPE;
+    const int T = nrs * R;
 
     int64_t chunk_cols = cols, chunk_bytes = rb;
     if ((int64_t)G * T * rb > STAGE_MAX) {
-        const int64_t align = tma ? (fmt == QMV_Q6_K ? 2048 : 256) : bw;
+        const int64_t align = tma ? (fmt == QMV_Q6_K ? 2048 : 256) : (fmt == QMV_Q8_0 ? 32 : 256);
         const int64_t per_row = STAGE_MAX / ((int64_t)G * T);
-        int64_t n_ch = ceil_div(rb, per_row);
+        const int64_t n_ch = ceil_div(rb, per_row);
         chunk_cols = ceil_div(ceil_div(cols, n_ch), align) * align;
         if (chunk_cols >= cols) chunk_cols = cols;
         chunk_bytes = chunk_cols / bw * bb;
@@ -115,7 +154,7 @@ int make_plan(int fmt, int64_t rows, int64_t cols, int n_tok, int G, int n_jobs,
     const int64_t last_cols = cols - (n_chunks - 1) * chunk_cols;
     const int64_t stage_bytes = (int64_t)G * T * chunk_bytes;
     const int64_t stage_pitch = ceil_div(stage_bytes + 16, 128) * 128;
-    int n_stage = (int)std::min<int64_t>(MAX_STAGES, std::max<int64_t>(2, STAGES_BUDGET / stage_pitch));
+    int n_stage = (int)std::min<int64_t>(MAX_STAGES, std::max<int64_t>(2, budget / stage_pitch));
     while (n_stage > 2 && 128 + SMEM_HDR + n_stage * stage_pitch > di.smem_optin) --n_stage;
     const int64_t smem = 128 + SMEM_HDR + n_stage * stage_pitch;   // 128: base alignment slack
     if (smem > di.smem_optin) return QMV_ERR_SHAPE;
@@ -133,9 +172,11 @@ int make_plan(int fmt, int64_t rows, int64_t cols, int n_tok, int G, int n_jobs,
     p.n_chunks = (int32_t)n_chunks;
     p.last_chunk_cols = (int32_t)last_cols;
     p.last_chunk_bytes = (int32_t)(last_cols / bw * bb);
-    p.tile_rows = T;
     p.G = G;
     p.Gp = gp;
+    p.wpr = wpr;
+    p.nrs = nrs;
+    p.tile_rows = T;
     p.n_stage = n_stage;
     p.stage_pitch = (int32_t)stage_pitch;
     p.row_pitch = (int32_t)chunk_bytes;
@@ -144,7 +185,8 @@ int make_plan(int fmt, int64_t rows, int64_t cols, int n_tok, int G, int n_jobs,
     p.err = di.err;
     pl.kc.ntok = n_tok;
     pl.kc.R = R;
-    pl.kc.xreg = (n_tok == 1 && n_chunks == 1 && shared_x && cols <= 2048);
+    pl.kc.xreg = n_tok == 1 && n_chunks == 1 && ceil_div(n1, wpr) <= xcap;
+    pl.kc.pdl = g_pdl.load() != 0;
     pl.grid = dim3((unsigned)ctas_per_job, (unsigned)n_jobs);
     pl.smem = (size_t)smem;
     return QMV_OK;
@@ -158,10 +200,7 @@ int launch_plan(int fmt, const Plan &pl, cudaStream_t stream)
     case QMV_Q4_K: e = launch_pipeline<FMT_Q4_K>(pl.p, pl.kc, pl.grid, pl.smem, stream); break;
     default: e = launch_pipeline<FMT_Q6_K>(pl.p, pl.kc, pl.grid, pl.smem, stream); break;
     }
-    if (e != cudaSuccess) {
-        (void)cudaGetLastError();
-        return QMV_ERR_CUDA;
-    }
+    if (e != cudaSuccess) return cuda_fail(e);
     return QMV_OK;
 }
 
@@ -181,6 +220,15 @@ size_t qmv_block_bytes(int fmt) { return (size_t)block_bytes(fmt); }
 int qmv_block_weights(int fmt) { return block_weights(fmt); }
 
 void qmv_debug_fail_next_launches(int count) { g_fail_launches.store(count > 0 ? count : 0); }
+
+void qmv_set_pdl(int enable) { g_pdl.store(enable ? 1 : 0); }
+
+int qmv_get_pdl(void) { return g_pdl.load(); }
+
+const char *qmv_last_cuda_error(void)
+{
+    return t_last_cuda == cudaSuccess ? "no error" : cudaGetErrorString(t_last_cuda);
+}
 
 const char *qmv_strerror(int status)
 {
@@ -240,7 +288,8 @@ int moe_route(const float *logits, const float *bias, int n_expert, int top_k, i
     if (rc) return rc;
     moe_route_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(logits, bias, n_expert, top_k,
                                                                           ids_out, g_out);
-    if (cudaGetLastError() != cudaSuccess) return QMV_ERR_CUDA;
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e);
     return QMV_OK;
 }
 
@@ -359,17 +408,16 @@ int qmv_dequant(int fmt, const void *W_blocks, int64_t rows, int64_t cols, float
     case QMV_Q4_K: dequant_kernel<FMT_Q4_K><<<grid, 256, 0, st>>>(W, nblk, bpr, cols, out); break;
     default: dequant_kernel<FMT_Q6_K><<<grid, 256, 0, st>>>(W, nblk, bpr, cols, out); break;
     }
-    if (cudaGetLastError() != cudaSuccess) return QMV_ERR_CUDA;
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e);
     return QMV_OK;
 }
 
 int qmv_check(qmv_stream_t stream, int *dev_err_out)
 {
     if (dev_err_out) *dev_err_out = 0;
-    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
-        (void)cudaGetLastError();
-        return QMV_ERR_CUDA;
-    }
+    const cudaError_t se = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (se != cudaSuccess) return cuda_fail(se);
     DevInfo di;
     int rc = get_dev(di);
     if (rc) return rc;

@@ -8,7 +8,7 @@
 namespace qmv {
 
 template <int FMT, int NTOK, int R, bool XREG>
-static cudaError_t launch_one(const Params &p, dim3 grid, size_t smem, cudaStream_t stream)
+static cudaError_t launch_one(const Params &p, dim3 grid, size_t smem, cudaStream_t stream, bool pdl)
 {
     auto kern = qmv_pipeline_kernel<FMT, NTOK, R, XREG>;
     // Raise the dynamic shared-memory limit once per (kernel, device).
@@ -22,11 +22,16 @@ static cudaError_t launch_one(const Params &p, dim3 grid, size_t smem, cudaStrea
         if (e != cudaSuccess) return e;
         configured[dev] = (int)smem;
     }
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = dim3(NTHREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
@@ -34,25 +39,24 @@ template <int FMT, int NTOK>
 static cudaError_t launch_ntok(const Params &p, const KernelChoice &kc, dim3 grid, size_t smem,
                                cudaStream_t stream)
 {
-    constexpr int NTP = Pow2Ceil<NTOK>::v;
     if (kc.xreg) {
         if constexpr (NTOK == 1) {
             switch (kc.R) {
-            case 1: return launch_one<FMT, 1, 1, true>(p, grid, smem, stream);
-            case 2: return launch_one<FMT, 1, 2, true>(p, grid, smem, stream);
-            case 4: return launch_one<FMT, 1, 4, true>(p, grid, smem, stream);
-            case 8: return launch_one<FMT, 1, 8, true>(p, grid, smem, stream);
+            case 1: return launch_one<FMT, 1, 1, true>(p, grid, smem, stream, kc.pdl);
+            case 2: return launch_one<FMT, 1, 2, true>(p, grid, smem, stream, kc.pdl);
+            case 4: return launch_one<FMT, 1, 4, true>(p, grid, smem, stream, kc.pdl);
+            case 8: return launch_one<FMT, 1, 8, true>(p, grid, smem, stream, kc.pdl);
             default: return cudaErrorInvalidValue;
             }
         }
         return cudaErrorInvalidValue;
     }
     switch (kc.R) {
-    case 1: return launch_one<FMT, NTOK, 1, false>(p, grid, smem, stream);
-    case 2: return launch_one<FMT, NTOK, 2, false>(p, grid, smem, stream);
-    case 4: return launch_one<FMT, NTOK, 4, false>(p, grid, smem, stream);
+    case 1: return launch_one<FMT, NTOK, 1, false>(p, grid, smem, stream, kc.pdl);
+    case 2: return launch_one<FMT, NTOK, 2, false>(p, grid, smem, stream, kc.pdl);
+    case 4: return launch_one<FMT, NTOK, 4, false>(p, grid, smem, stream, kc.pdl);
     case 8:
-        if constexpr (8 * NTP <= 32) return launch_one<FMT, NTOK, 8, false>(p, grid, smem, stream);
+        if constexpr (NTOK == 1) return launch_one<FMT, NTOK, 8, false>(p, grid, smem, stream, kc.pdl);
         return cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
     }

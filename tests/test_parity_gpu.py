@@ -112,7 +112,9 @@ def test_qmv_small_shapes(fmt, rows, cols, n_tok):
 
 
 @pytest.mark.parametrize("fmt,rows,cols", [(Q8_0, 300, 8192), (Q8_0, 9, 16384), (Q4_K, 40, 16384),
-                                           (Q6_K, 33, 8192), (Q8_0, 17, 8224), (Q6_K, 5, 4352)])
+                                           (Q6_K, 33, 8192), (Q8_0, 17, 8224), (Q6_K, 5, 4352),
+                                           (Q8_0, 5, 65536), (Q4_K, 3, 65536), (Q6_K, 4, 34816),
+                                           (Q8_0, 2, 40992)])
 @pytest.mark.parametrize("n_tok", [1, 4, 8])
 def test_qmv_long_rows_k_chunked(fmt, rows, cols, n_tok):
     W = synth.gen_blocks(fmt, rows, cols, seed=8, tensor_id=300 + fmt)
