@@ -152,36 +152,53 @@ class ClockSampler:
 # ---------------------------------------------------------- device helpers --
 
 class Dist:
+    """Ranks of a torchrun launch: NCCL on GPUs (gloo for host-only tests).
+    Only the timing is exchanged (barriers and a max over ranks): the sweep runs
+    as an independent replica on every GPU."""
+
     def __init__(self, n_gpus):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = None
+        self.device = "cuda"
         if n_gpus > 1 and self.world != n_gpus:
             raise SystemExit(f"--gpus {n_gpus} needs torchrun with {n_gpus} ranks (WORLD_SIZE={self.world})")
 
-    def init(self, torch):
-        torch.cuda.set_device(self.local)
+    def init(self, torch, backend="nccl"):
+        if backend == "nccl":
+            torch.cuda.set_device(self.local)
+        else:
+            self.device = "cpu"
         if self.world > 1:
             import datetime
             import torch.distributed as dist
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
             self.pg = dist
 
     def barrier(self, torch):
         if self.pg is not None:
-            self.pg.barrier(device_ids=[self.local])
+            if self.device == "cuda":
+                self.pg.barrier(device_ids=[self.local])
+            else:
+                self.pg.barrier()
 
     def max(self, torch, v):
         if self.pg is None:
             return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        t = torch.tensor([v], dtype=torch.float64, device=self.device)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
     def close(self):
         if self.pg is not None:
             self.pg.destroy_process_group()
+
+
+def aggregate_gbs(bytes_per_step, world, steps, max_sec):
+    """Whole-job throughput: every rank streams bytes_per_step per step; the job
+    takes the slowest rank's time."""
+    return bytes_per_step * world * steps / max_sec / 1e9
 
 
 def time_graph(torch, graph, reps, stream):
@@ -497,7 +514,7 @@ def main():
     clocks = clk.summary()
     assert q.qmv_check(stream) == 0
 
-    value = sweep.weight_bytes * dist.world / (sec / args.steps) / 1e9
+    value = aggregate_gbs(sweep.weight_bytes, dist.world, args.steps, sec)
     ms_per_step = sec / args.steps * 1e3
     achieved = sweep.algo / sum(durs) / 1e9
     traffic = None

@@ -95,6 +95,28 @@ typedef enum {
 int qmv_f32(int fmt, const void *W_blocks, int64_t rows, int64_t cols,
             const float *x, float *y, qmv_stream_t stream);
 
+/* One matvec of a grouped launch (see qmv_multi). */
+typedef struct {
+    const void *W_blocks;   /* device, 16-byte aligned, rows x cols weights    */
+    int64_t rows;
+    int64_t cols;
+    const float *x;         /* device f32 [n_tok][cols], 16-byte aligned       */
+    float *y;               /* device f32 [n_tok][rows], 4-byte aligned        */
+} qmv_task;
+
+#define QMV_MAX_TASKS 4096
+
+/* Several independent matvecs of one format and token count in as few
+ * launches as possible: y_t = W_t x_t for every task t (same layouts as
+ * qmv_batched).  The tasks run concurrently and in no defined order, so no
+ * task may write memory another task of the call reads; the call as a whole
+ * is ordered in `stream` like any other.  Each task's rows are split into
+ * CTAs of roughly equal byte counts sized to the whole batch, so the CTAs of
+ * all tasks stream together and the launch-to-launch latency of a chain of
+ * small matvecs disappears.  `tasks` is a host array of n_tasks entries
+ * (1 <= n_tasks <= QMV_MAX_TASKS), read during the call only. */
+int qmv_multi(int fmt, int n_tok, const qmv_task *tasks, int n_tasks, qmv_stream_t stream);
+
 /* Multi-token variant for speculative verification (FlareLLM page,
  * §推理层面的深度优化: n-gram speculative decoding): every weight is read once
  * and applied to n_tok activation vectors.

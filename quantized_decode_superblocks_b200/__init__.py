@@ -25,9 +25,15 @@ STATUS_NAMES = {0: "QMV_OK", -1: "QMV_ERR_NULL", -2: "QMV_ERR_FMT", -3: "QMV_ERR
 DEVERR_EXPERT_ID = 1
 DEVERR_TIMEOUT = 2
 
-EXPORTED = ("qmv_f32", "qmv_batched", "moe_route", "moe_qmv", "moe_ffn", "qmv_dequant",
+EXPORTED = ("qmv_f32", "qmv_batched", "qmv_multi", "moe_route", "moe_qmv", "moe_ffn", "qmv_dequant",
             "qmv_check", "qmv_strerror", "qmv_block_bytes", "qmv_block_weights",
             "qmv_debug_fail_next_launches", "qmv_set_pdl", "qmv_get_pdl", "qmv_last_cuda_error")
+
+
+class QmvTask(ctypes.Structure):
+    """One matvec of a grouped launch (qmv_task in include/qmv.h)."""
+    _fields_ = [("W_blocks", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("x", ctypes.c_void_p), ("y", ctypes.c_void_p)]
 
 
 class QmvError(RuntimeError):
@@ -52,6 +58,7 @@ def lib() -> ctypes.CDLL:
         vp, i64, c_int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
         L.qmv_f32.argtypes = [c_int, vp, i64, i64, vp, vp, vp]
         L.qmv_batched.argtypes = [c_int, vp, i64, i64, vp, vp, c_int, vp]
+        L.qmv_multi.argtypes = [c_int, c_int, ctypes.POINTER(QmvTask), c_int, vp]
         L.moe_route.argtypes = [vp, vp, c_int, c_int, vp, vp, vp]
         L.moe_qmv.argtypes = [c_int, vp, i64, c_int, vp, c_int, i64, i64, vp, i64, vp, vp, vp]
         L.moe_ffn.argtypes = [c_int, vp, vp, i64, c_int, vp, i64, c_int, vp, vp, c_int, i64, i64,
@@ -136,6 +143,21 @@ def qmv_batched(fmt, W, rows, cols, x, y, n_tok, stream=None):
     """y[n_tok][rows] = W x[n_tok][cols]^T, 1 <= n_tok <= 8."""
     _check(lib().qmv_batched(fmt, _ptr(W), rows, cols, _ptr(x), _ptr(y), n_tok, _stream(stream)),
            "qmv_batched")
+
+
+def make_tasks(tasks):
+    """ctypes array of QmvTask from (W, rows, cols, x, y) tuples."""
+    arr = (QmvTask * len(tasks))()
+    for i, (W, rows, cols, x, y) in enumerate(tasks):
+        arr[i] = QmvTask(_ptr(W), rows, cols, _ptr(x), _ptr(y))
+    return arr
+
+
+def qmv_multi(fmt, n_tok, tasks, stream=None):
+    """Independent matvecs y_t = W_t x_t in grouped launches; `tasks` is a list of
+    (W, rows, cols, x, y) tuples or an array from make_tasks()."""
+    arr = tasks if isinstance(tasks, ctypes.Array) else make_tasks(tasks)
+    _check(lib().qmv_multi(fmt, n_tok, arr, len(arr), _stream(stream)), "qmv_multi")
 
 
 def moe_route(logits, bias, n_expert, top_k, ids_out, g_out, stream=None):

@@ -1,8 +1,10 @@
 // qmv_api.cu -- the C ABI of libqmv.so (declared in include/qmv.h): host-side
 // argument validation, launch planning and the launches themselves.  Nothing
 // here allocates device memory; every buffer is the caller's.
+#include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "../../include/qmv.h"
 #include "qmv_misc.cuh"
@@ -17,6 +19,8 @@ __device__ int g_dev_err;
 constexpr int STAGE_MAX = 36 * 1024;       // bytes of one pipeline stage
 constexpr int STAGES_BUDGET2 = 105 * 1024; // all stages of one CTA, two CTAs per SM (1-2 tokens)
 constexpr int STAGES_BUDGET1 = 192 * 1024; // one CTA per SM (3-8 tokens: more registers per thread)
+constexpr int MULTI_WAVES = 4;                   // grouped launch: CTA waves over the GPU
+constexpr int64_t MULTI_MIN_CTA_BYTES = 128 * 1024;
 #ifndef QMV_SMALL_CTA_BYTES
 #define QMV_SMALL_CTA_BYTES (96 * 1024)
 #endif
@@ -93,7 +97,7 @@ struct Plan {
 };
 
 int make_plan(int fmt, int64_t rows, int64_t cols, int n_tok, int G, int n_jobs, bool /*shared_x*/,
-              const DevInfo &di, Plan &pl)
+              const DevInfo &di, Plan &pl, int64_t rows_per_cta_override = 0)
 {
     const int bw = block_weights(fmt), bb = block_bytes(fmt);
     const int64_t rb = cols / bw * bb;
@@ -116,7 +120,8 @@ int make_plan(int fmt, int64_t rows, int64_t cols, int n_tok, int G, int n_jobs,
     const int target_ctas = ctas_per_sm * di.sm_count;
     const int64_t budget = n_tok <= 2 ? STAGES_BUDGET2 : STAGES_BUDGET1;
     const int64_t ctas_job0 = std::max<int64_t>(1, target_ctas / n_jobs);
-    const int64_t rows_cta0 = ceil_div(rows, ctas_job0);
+    const int64_t rows_cta0 = rows_per_cta_override > 0 ? std::min(rows, rows_per_cta_override)
+                                                         : ceil_div(rows, ctas_job0);
 
     // warps per row (K-segments): one token -> the fewest that keep a warp's x
     // in registers; several tokens -> segments of at most 2048 columns
@@ -266,6 +271,78 @@ int qmv_batched(int fmt, const void *W_blocks, int64_t rows, int64_t cols, const
     pl.p.y = y;
     pl.p.y_tok_stride = rows;
     return launch_plan(fmt, pl, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int qmv_multi(int fmt, int n_tok, const qmv_task *tasks, int n_tasks, qmv_stream_t stream)
+{
+    if (!tasks) return QMV_ERR_NULL;
+    if (!fmt_ok(fmt)) return QMV_ERR_FMT;
+    if (n_tasks < 1 || n_tasks > QMV_MAX_TASKS) return QMV_ERR_SHAPE;
+    if (n_tok < 1 || n_tok > QMV_MAX_NTOK) return QMV_ERR_NTOK;
+    int64_t total = 0;
+    for (int t = 0; t < n_tasks; ++t) {
+        const qmv_task &k = tasks[t];
+        if (!k.W_blocks || !k.x || !k.y) return QMV_ERR_NULL;
+        const int rc = check_matrix(fmt, k.rows, k.cols);
+        if (rc) return rc;
+        if (!aligned(k.W_blocks, 16) || !aligned(k.x, 16) || !aligned(k.y, 4)) return QMV_ERR_ALIGN;
+        total += k.rows * (k.cols / block_weights(fmt)) * block_bytes(fmt);
+    }
+    if (injected_failure()) return QMV_ERR_CUDA;
+    DevInfo di;
+    int rc = get_dev(di);
+    if (rc) return rc;
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+    // Every CTA streams about the same number of bytes, sized so the batch
+    // takes a few waves of two CTAs per SM: small tasks get few CTAs with many
+    // rows each, and all tasks' CTAs share the GPU at once.
+    const int64_t per_cta = std::max<int64_t>(MULTI_MIN_CTA_BYTES,
+                                              ceil_div(total, (int64_t)MULTI_WAVES * 2 * di.sm_count));
+    std::vector<Plan> plans((size_t)n_tasks);
+    for (int t = 0; t < n_tasks; ++t) {
+        const qmv_task &k = tasks[t];
+        const int64_t bytes = k.rows * (k.cols / block_weights(fmt)) * block_bytes(fmt);
+        const int64_t ctas = std::max<int64_t>(1, ceil_div(bytes, per_cta));
+        Plan &pl = plans[(size_t)t];
+        if ((rc = make_plan(fmt, k.rows, k.cols, n_tok, 1, 1, true, di, pl, ceil_div(k.rows, ctas)))) return rc;
+        pl.p.mode = MODE_SEPARATE;
+        pl.p.base0 = static_cast<const uint8_t *>(k.W_blocks);
+        pl.p.x = k.x;
+        pl.p.x_tok_stride = k.cols;
+        pl.p.y = k.y;
+        pl.p.y_tok_stride = k.rows;
+    }
+    // one launch per kernel instance (rows per warp, x in registers), at most
+    // MAX_MULTI tasks each
+    std::vector<char> done((size_t)n_tasks, 0);
+    static thread_local MultiParams mp;
+    for (int t0 = 0; t0 < n_tasks; ++t0) {
+        if (done[(size_t)t0]) continue;
+        const KernelChoice kc = plans[(size_t)t0].kc;
+        mp.n = 0;
+        size_t smem = 0;
+        int ctas = 0;
+        for (int t = t0; t < n_tasks && mp.n < MAX_MULTI; ++t) {
+            const Plan &pl = plans[(size_t)t];
+            if (done[(size_t)t] || pl.kc.R != kc.R || pl.kc.xreg != kc.xreg) continue;
+            done[(size_t)t] = 1;
+            mp.cta_begin[mp.n] = ctas;
+            mp.p[mp.n] = pl.p;
+            ctas += (int)pl.grid.x;
+            smem = std::max(smem, pl.smem);
+            ++mp.n;
+        }
+        mp.cta_begin[mp.n] = ctas;
+        cudaError_t e;
+        switch (fmt) {
+        case QMV_Q8_0: e = launch_multi<FMT_Q8_0>(mp, kc, ctas, smem, st); break;
+        case QMV_Q4_K: e = launch_multi<FMT_Q4_K>(mp, kc, ctas, smem, st); break;
+        default: e = launch_multi<FMT_Q6_K>(mp, kc, ctas, smem, st); break;
+        }
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return QMV_OK;
 }
 
 int qmv_f32(int fmt, const void *W_blocks, int64_t rows, int64_t cols, const float *x, float *y,

@@ -7,12 +7,12 @@
 
 namespace qmv {
 
-template <int FMT, int NTOK, int R, bool XREG>
-static cudaError_t launch_one(const Params &p, dim3 grid, size_t smem, cudaStream_t stream, bool pdl)
+// Launch `kern` with `arg`: raises the dynamic shared-memory limit once per
+// (kernel, device) and adds the programmatic-serialization attribute when asked.
+template <class Kern, class Arg>
+static cudaError_t launch_with(Kern kern, int *configured, const Arg &arg, dim3 grid, size_t smem,
+                               cudaStream_t stream, bool pdl)
 {
-    auto kern = qmv_pipeline_kernel<FMT, NTOK, R, XREG>;
-    // Raise the dynamic shared-memory limit once per (kernel, device).
-    static int configured[64] = {0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -32,51 +32,98 @@ static cudaError_t launch_one(const Params &p, dim3 grid, size_t smem, cudaStrea
     cfg.stream = stream;
     cfg.attrs = pdl ? attr : nullptr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kern, p);
+    return cudaLaunchKernelEx(&cfg, kern, arg);
 }
 
-template <int FMT, int NTOK>
-static cudaError_t launch_ntok(const Params &p, const KernelChoice &kc, dim3 grid, size_t smem,
-                               cudaStream_t stream)
+template <int FMT, int NTOK, int R, bool XREG>
+struct Instance {
+    static cudaError_t one(const Params &p, dim3 grid, size_t smem, cudaStream_t st, bool pdl)
+    {
+        static int configured[64] = {0};
+        return launch_with(qmv_pipeline_kernel<FMT, NTOK, R, XREG>, configured, p, grid, smem, st, pdl);
+    }
+    static cudaError_t multi(const MultiParams &mp, dim3 grid, size_t smem, cudaStream_t st, bool pdl)
+    {
+        static int configured[64] = {0};
+        return launch_with(qmv_multi_kernel<FMT, NTOK, R, XREG>, configured, mp, grid, smem, st, pdl);
+    }
+};
+
+// Calls Fn::template run<FMT, NTOK, R, XREG>() for the runtime choice.
+template <int FMT, int NTOK, class Fn>
+static cudaError_t pick_r(const KernelChoice &kc, Fn &&fn)
 {
     if (kc.xreg) {
         if constexpr (NTOK == 1) {
             switch (kc.R) {
-            case 1: return launch_one<FMT, 1, 1, true>(p, grid, smem, stream, kc.pdl);
-            case 2: return launch_one<FMT, 1, 2, true>(p, grid, smem, stream, kc.pdl);
-            case 4: return launch_one<FMT, 1, 4, true>(p, grid, smem, stream, kc.pdl);
-            case 8: return launch_one<FMT, 1, 8, true>(p, grid, smem, stream, kc.pdl);
+            case 1: return fn.template run<FMT, 1, 1, true>();
+            case 2: return fn.template run<FMT, 1, 2, true>();
+            case 4: return fn.template run<FMT, 1, 4, true>();
+            case 8: return fn.template run<FMT, 1, 8, true>();
             default: return cudaErrorInvalidValue;
             }
         }
         return cudaErrorInvalidValue;
     }
     switch (kc.R) {
-    case 1: return launch_one<FMT, NTOK, 1, false>(p, grid, smem, stream, kc.pdl);
-    case 2: return launch_one<FMT, NTOK, 2, false>(p, grid, smem, stream, kc.pdl);
-    case 4: return launch_one<FMT, NTOK, 4, false>(p, grid, smem, stream, kc.pdl);
+    case 1: return fn.template run<FMT, NTOK, 1, false>();
+    case 2: return fn.template run<FMT, NTOK, 2, false>();
+    case 4: return fn.template run<FMT, NTOK, 4, false>();
     case 8:
-        if constexpr (NTOK == 1) return launch_one<FMT, NTOK, 8, false>(p, grid, smem, stream, kc.pdl);
+        if constexpr (NTOK == 1) return fn.template run<FMT, NTOK, 8, false>();
         return cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
     }
 }
 
+template <int FMT, class Fn>
+static cudaError_t pick(const KernelChoice &kc, Fn &&fn)
+{
+    switch (kc.ntok) {
+    case 1: return pick_r<FMT, 1>(kc, fn);
+    case 2: return pick_r<FMT, 2>(kc, fn);
+    case 3: return pick_r<FMT, 3>(kc, fn);
+    case 4: return pick_r<FMT, 4>(kc, fn);
+    case 5: return pick_r<FMT, 5>(kc, fn);
+    case 6: return pick_r<FMT, 6>(kc, fn);
+    case 7: return pick_r<FMT, 7>(kc, fn);
+    case 8: return pick_r<FMT, 8>(kc, fn);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+struct OneLaunch {
+    const Params &p;
+    dim3 grid;
+    size_t smem;
+    cudaStream_t st;
+    bool pdl;
+    template <int FMT, int NTOK, int R, bool XREG>
+    cudaError_t run() const { return Instance<FMT, NTOK, R, XREG>::one(p, grid, smem, st, pdl); }
+};
+
+struct MultiLaunch {
+    const MultiParams &mp;
+    dim3 grid;
+    size_t smem;
+    cudaStream_t st;
+    bool pdl;
+    template <int FMT, int NTOK, int R, bool XREG>
+    cudaError_t run() const { return Instance<FMT, NTOK, R, XREG>::multi(mp, grid, smem, st, pdl); }
+};
+
 template <int FMT>
 cudaError_t launch_pipeline(const Params &p, const KernelChoice &kc, dim3 grid, size_t smem,
                             cudaStream_t stream)
 {
-    switch (kc.ntok) {
-    case 1: return launch_ntok<FMT, 1>(p, kc, grid, smem, stream);
-    case 2: return launch_ntok<FMT, 2>(p, kc, grid, smem, stream);
-    case 3: return launch_ntok<FMT, 3>(p, kc, grid, smem, stream);
-    case 4: return launch_ntok<FMT, 4>(p, kc, grid, smem, stream);
-    case 5: return launch_ntok<FMT, 5>(p, kc, grid, smem, stream);
-    case 6: return launch_ntok<FMT, 6>(p, kc, grid, smem, stream);
-    case 7: return launch_ntok<FMT, 7>(p, kc, grid, smem, stream);
-    case 8: return launch_ntok<FMT, 8>(p, kc, grid, smem, stream);
-    default: return cudaErrorInvalidValue;
-    }
+    return pick<FMT>(kc, OneLaunch{p, grid, smem, stream, kc.pdl});
+}
+
+template <int FMT>
+cudaError_t launch_multi(const MultiParams &mp, const KernelChoice &kc, int grid, size_t smem,
+                         cudaStream_t stream)
+{
+    return pick<FMT>(kc, MultiLaunch{mp, dim3((unsigned)grid), smem, stream, kc.pdl});
 }
 
 }  // namespace qmv

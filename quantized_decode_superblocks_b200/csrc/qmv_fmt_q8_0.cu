@@ -3,4 +3,5 @@
 
 namespace qmv {
 template cudaError_t launch_pipeline<FMT_Q8_0>(const Params &, const KernelChoice &, dim3, size_t, cudaStream_t);
+template cudaError_t launch_multi<FMT_Q8_0>(const MultiParams &, const KernelChoice &, int, size_t, cudaStream_t);
 }  // namespace qmv

@@ -173,8 +173,9 @@ __device__ __forceinline__ void fill_stage(const Params &p, const uint8_t *const
     }
 }
 
+// The whole pipeline for CTA `cta` of job `job` of one matvec launch.
 template <int FMT, int NTOK, int R, bool XREG>
-__global__ void __launch_bounds__(NTHREADS, (NTOK <= 2 ? 2 : 1)) qmv_pipeline_kernel(const __grid_constant__ Params p)
+__device__ __forceinline__ void qmv_pipeline_body(const Params &p, const int cta, const int job)
 {
     constexpr int NTP = Pow2Ceil<NTOK>::v;
     constexpr int V = R * NTP;
@@ -188,8 +189,7 @@ __global__ void __launch_bounds__(NTHREADS, (NTOK <= 2 ? 2 : 1)) qmv_pipeline_ke
     __shared__ const float *sX[MAX_GROUPS];
     __shared__ float sWgt[MAX_GROUPS];
 
-    const int job = blockIdx.y;
-    const int64_t r_begin = (int64_t)blockIdx.x * p.rows_per_cta;
+    const int64_t r_begin = (int64_t)cta * p.rows_per_cta;
     if (r_begin >= p.rows) return;                     // uniform for the whole CTA
     const int64_t r_end = min(p.rows, r_begin + (int64_t)p.rows_per_cta);
     const int T = p.tile_rows;
@@ -463,6 +463,30 @@ __global__ void __launch_bounds__(NTHREADS, (NTOK <= 2 ? 2 : 1)) qmv_pipeline_ke
     }
 }
 
+template <int FMT, int NTOK, int R, bool XREG>
+__global__ void __launch_bounds__(NTHREADS, (NTOK <= 2 ? 2 : 1)) qmv_pipeline_kernel(const __grid_constant__ Params p)
+{
+    qmv_pipeline_body<FMT, NTOK, R, XREG>(p, (int)blockIdx.x, (int)blockIdx.y);
+}
+
+// Several independent matvecs in one launch: task t owns CTAs
+// [cta_begin[t], cta_begin[t+1]).
+constexpr int MAX_MULTI = 64;
+struct MultiParams {
+    int32_t n;
+    int32_t cta_begin[MAX_MULTI + 1];
+    Params p[MAX_MULTI];
+};
+
+template <int FMT, int NTOK, int R, bool XREG>
+__global__ void __launch_bounds__(NTHREADS, (NTOK <= 2 ? 2 : 1)) qmv_multi_kernel(const __grid_constant__ MultiParams mp)
+{
+    const int b = (int)blockIdx.x;
+    int t = 0;
+    while (t + 1 < mp.n && b >= mp.cta_begin[t + 1]) ++t;
+    qmv_pipeline_body<FMT, NTOK, R, XREG>(mp.p[t], b - mp.cta_begin[t], 0);
+}
+
 // ------------------------------------------------------------ launchers --
 struct KernelChoice {
     int ntok;
@@ -475,5 +499,8 @@ struct KernelChoice {
 template <int FMT>
 cudaError_t launch_pipeline(const Params &p, const KernelChoice &kc, dim3 grid, size_t smem,
                             cudaStream_t stream);
+template <int FMT>
+cudaError_t launch_multi(const MultiParams &mp, const KernelChoice &kc, int grid, size_t smem,
+                         cudaStream_t stream);
 
 }  // namespace qmv

@@ -166,6 +166,46 @@ def test_results_are_deterministic():
         assert np.array_equal(y.view(np.uint32), ys[0].view(np.uint32))
 
 
+# ------------------------------------------------------- grouped launch --
+
+@pytest.mark.parametrize("fmt,n_tok", [(Q8_0, 1), (Q4_K, 1), (Q6_K, 1), (Q8_0, 4), (Q4_K, 8)])
+def test_qmv_multi_matches_each_task(fmt, n_tok):
+    bw = synth.BLOCK_WEIGHTS[fmt]
+    shapes = [(3072, 2048), (2048, 2048), (257, 4096), (1, bw), (5000, 1792 if fmt == Q8_0 else 2048),
+              (300, 8192), (17, 16384 if fmt != Q6_K else 8192), (1024, 1024 if fmt == Q8_0 else 2048)]
+    host, dev_args = [], []
+    for i, (rows, cols) in enumerate(shapes):
+        W = synth.gen_blocks(fmt, rows, cols, 60 + fmt, i)
+        x = synth.gen_x(n_tok, cols, 61, i)
+        y = torch.full((n_tok, rows), float("nan"), device="cuda")
+        host.append((W, rows, cols, x))
+        dev_args.append((dev(W), rows, cols, dev(x), y))
+    q.qmv_multi(fmt, n_tok, dev_args)
+    torch.cuda.synchronize()
+    for (W, rows, cols, x), (_, _, _, _, y) in zip(host, dev_args):
+        ref, bound = oracle.qmv(fmt, W, rows, cols, x)
+        within(y.cpu().numpy(), ref, bound)
+
+
+def test_qmv_multi_many_tasks_and_errors():
+    # more tasks than one launch takes, all from one shared weight matrix
+    fmt, rows, cols = Q4_K, 96, 512
+    W = synth.gen_blocks(fmt, rows, cols, 70, 0)
+    Wd = dev(W)
+    xs = synth.gen_x(130, cols, 70, 1)
+    xd = dev(xs)
+    y = torch.full((130, rows), float("nan"), device="cuda")
+    tasks = [(Wd, rows, cols, xd[i], y[i]) for i in range(130)]
+    q.qmv_multi(fmt, 1, tasks)
+    torch.cuda.synchronize()
+    ref, bound = oracle.qmv(fmt, W, rows, cols, xs)
+    within(y.cpu().numpy(), ref, bound)
+    with pytest.raises(q.QmvError):
+        q.qmv_multi(fmt, 1, [(Wd, rows, 100, xd[0], y[0])])
+    with pytest.raises(q.QmvError):
+        q.qmv_multi(fmt, 9, tasks[:2])
+
+
 # ---------------------------------------------------- full-size workloads --
 
 def test_cfg0_q8_0_1024x1024():
