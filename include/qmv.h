@@ -163,6 +163,29 @@ int moe_ffn(int fmt_gu, const void *gate_blocks, const void *up_blocks,
             const float *g, int n_sel, int64_t hidden, int64_t inter,
             const float *x, float *h_scratch, float *y, qmv_stream_t stream);
 
+/* moe_ffn without a caller-provided scratch buffer, for callers that cannot
+ * allocate device memory: code running while a stream is being captured into
+ * a CUDA graph (where cudaMalloc is not allowed), plugins and callbacks that
+ * are handed only their input and output buffers, and real-time paths that
+ * must not take an allocator's latency or locks.  (The pages have no
+ * counterpart; this is a usage variant of the same MoE step.)
+ * The SwiGLU activations go to a file-scope device array of
+ * QMV_STATIC_H_FLOATS floats (512 KiB) that every GPU which loads the library
+ * holds until the process exits; n_sel * inter above that is rejected with
+ * QMV_ERR_SHAPE.  Nothing is allocated by the call.  The first call on a
+ * device looks up the array's device address (a host call, no allocation):
+ * make that first call before capturing a stream.  All calls share the one
+ * array, which keeps the last call's contents (every call overwrites the part
+ * it uses before reading it), so calls that can overlap on the GPU -- on two
+ * streams of one device, say -- race and must be serialised by the caller.
+ * Arguments and results are those of moe_ffn. */
+#define QMV_STATIC_H_FLOATS (8 * 16384)
+int moe_ffn_static(int fmt_gu, const void *gate_blocks, const void *up_blocks,
+                   int64_t gu_stride_bytes, int fmt_down, const void *down_blocks,
+                   int64_t down_stride_bytes, int n_expert, const int32_t *expert_ids,
+                   const float *g, int n_sel, int64_t hidden, int64_t inter,
+                   const float *x, float *y, qmv_stream_t stream);
+
 /* Dequantize the whole matrix to f32: out[rows][cols].  The values are
  * bit-exact f32 evaluations of the block formulas above (every product in
  * them is exact in f32; Q4_K rounds once, in the subtraction). */

@@ -25,7 +25,8 @@ STATUS_NAMES = {0: "QMV_OK", -1: "QMV_ERR_NULL", -2: "QMV_ERR_FMT", -3: "QMV_ERR
 DEVERR_EXPERT_ID = 1
 DEVERR_TIMEOUT = 2
 
-EXPORTED = ("qmv_f32", "qmv_batched", "qmv_multi", "moe_route", "moe_qmv", "moe_ffn", "qmv_dequant",
+EXPORTED = ("qmv_f32", "qmv_batched", "qmv_multi", "moe_route", "moe_qmv", "moe_ffn", "moe_ffn_static",
+            "qmv_dequant",
             "qmv_check", "qmv_strerror", "qmv_block_bytes", "qmv_block_weights",
             "qmv_debug_fail_next_launches", "qmv_set_pdl", "qmv_get_pdl", "qmv_last_cuda_error")
 
@@ -63,6 +64,8 @@ def lib() -> ctypes.CDLL:
         L.moe_qmv.argtypes = [c_int, vp, i64, c_int, vp, c_int, i64, i64, vp, i64, vp, vp, vp]
         L.moe_ffn.argtypes = [c_int, vp, vp, i64, c_int, vp, i64, c_int, vp, vp, c_int, i64, i64,
                               vp, vp, vp, vp]
+        L.moe_ffn_static.argtypes = [c_int, vp, vp, i64, c_int, vp, i64, c_int, vp, vp, c_int, i64, i64,
+                                     vp, vp, vp]
         L.qmv_dequant.argtypes = [c_int, vp, i64, i64, vp, vp]
         L.qmv_check.argtypes = [vp, ctypes.POINTER(c_int)]
         L.qmv_strerror.argtypes = [c_int]
@@ -179,6 +182,14 @@ def moe_ffn(fmt_gu, gate_blocks, up_blocks, gu_stride_bytes, fmt_down, down_bloc
                          _ptr(down_blocks), down_stride_bytes, n_expert, _ptr(expert_ids), _ptr(g),
                          n_sel, hidden, inter, _ptr(x), _ptr(h_scratch), _ptr(y), _stream(stream)),
            "moe_ffn")
+
+
+def moe_ffn_static(fmt_gu, gate_blocks, up_blocks, gu_stride_bytes, fmt_down, down_blocks,
+                   down_stride_bytes, n_expert, expert_ids, g, n_sel, hidden, inter, x, y, stream=None):
+    """moe_ffn with the library's own fixed device scratch (see include/qmv.h)."""
+    _check(lib().moe_ffn_static(fmt_gu, _ptr(gate_blocks), _ptr(up_blocks), gu_stride_bytes, fmt_down,
+                                _ptr(down_blocks), down_stride_bytes, n_expert, _ptr(expert_ids), _ptr(g),
+                                n_sel, hidden, inter, _ptr(x), _ptr(y), _stream(stream)), "moe_ffn_static")
 
 
 def qmv_dequant(fmt, W, rows, cols, out, stream=None):

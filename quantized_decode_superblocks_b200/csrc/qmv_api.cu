@@ -16,6 +16,10 @@ using namespace qmv;
 // Sticky device error word (QMV_DEVERR_* bits), read and cleared by qmv_check.
 __device__ int g_dev_err;
 
+// Scratch of moe_ffn_static: the SwiGLU activations h[n_sel][inter].  Every
+// device that loads the library holds one copy until the process exits.
+static __device__ __align__(256) float g_static_h[QMV_STATIC_H_FLOATS];
+
 constexpr int STAGE_MAX = 36 * 1024;       // bytes of one pipeline stage
 constexpr int STAGES_BUDGET2 = 105 * 1024; // all stages of one CTA, two CTAs per SM (1-2 tokens)
 constexpr int STAGES_BUDGET1 = 192 * 1024; // one CTA per SM (3-8 tokens: more registers per thread)
@@ -30,6 +34,7 @@ struct DevInfo {
     int sm_count = 0;
     int smem_optin = 0;
     int *err = nullptr;
+    float *static_h = nullptr;   // device address of g_static_h, set up by moe_ffn_static
     bool ok = false;
 };
 
@@ -464,6 +469,35 @@ int moe_ffn(int fmt_gu, const void *gate_blocks, const void *up_blocks, int64_t 
     b.p.y = y;
     b.p.y_tok_stride = hidden;
     return launch_plan(fmt_down, b, st);
+}
+
+int moe_ffn_static(int fmt_gu, const void *gate_blocks, const void *up_blocks, int64_t gu_stride_bytes,
+                   int fmt_down, const void *down_blocks, int64_t down_stride_bytes, int n_expert,
+                   const int32_t *expert_ids, const float *g, int n_sel, int64_t hidden, int64_t inter,
+                   const float *x, float *y, qmv_stream_t stream)
+{
+    if (!gate_blocks || !up_blocks || !down_blocks || !expert_ids || !g || !x || !y) return QMV_ERR_NULL;
+    if (n_sel >= 1 && inter >= 1 && (int64_t)n_sel * inter > QMV_STATIC_H_FLOATS) return QMV_ERR_SHAPE;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        (void)cudaGetLastError();
+        return QMV_ERR_DEVICE;
+    }
+    float *h = nullptr;
+    {
+        // once per device, with that device current: the array's device address
+        // (its name in host code is only a host-side stand-in)
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_dev[dev].static_h) {
+            void *ptr = nullptr;
+            const cudaError_t e = cudaGetSymbolAddress(&ptr, g_static_h);
+            if (e != cudaSuccess) return cuda_fail(e);
+            g_dev[dev].static_h = static_cast<float *>(ptr);
+        }
+        h = g_dev[dev].static_h;
+    }
+    return moe_ffn(fmt_gu, gate_blocks, up_blocks, gu_stride_bytes, fmt_down, down_blocks, down_stride_bytes,
+                   n_expert, expert_ids, g, n_sel, hidden, inter, x, h, y, stream);
 }
 
 int qmv_dequant(int fmt, const void *W_blocks, int64_t rows, int64_t cols, float *out, qmv_stream_t stream)
