@@ -23,6 +23,7 @@ static __device__ __align__(256) float g_static_h[QMV_STATIC_H_FLOATS];
 constexpr int STAGE_MAX = 36 * 1024;       // bytes of one pipeline stage
 constexpr int STAGES_BUDGET2 = 105 * 1024; // all stages of one CTA, two CTAs per SM (1-2 tokens)
 constexpr int STAGES_BUDGET1 = 192 * 1024; // one CTA per SM (3-8 tokens: more registers per thread)
+constexpr int64_t X_SMEM_MAX = 64 * 1024;       // several tokens: largest x staged in shared memory
 constexpr int MULTI_WAVES = 4;                   // grouped launch: CTA waves over the GPU
 constexpr int64_t MULTI_MIN_CTA_BYTES = 128 * 1024;
 #ifndef QMV_SMALL_CTA_BYTES
@@ -164,9 +165,13 @@ int make_plan(int fmt, int64_t rows, int64_t cols, int n_tok, int G, int n_jobs,
     const int64_t last_cols = cols - (n_chunks - 1) * chunk_cols;
     const int64_t stage_bytes = (int64_t)G * T * chunk_bytes;
     const int64_t stage_pitch = ceil_div(stage_bytes + 16, 128) * 128;
-    int n_stage = (int)std::min<int64_t>(MAX_STAGES, std::max<int64_t>(2, budget / stage_pitch));
-    while (n_stage > 2 && 128 + SMEM_HDR + n_stage * stage_pitch > di.smem_optin) --n_stage;
-    const int64_t smem = 128 + SMEM_HDR + n_stage * stage_pitch;   // 128: base alignment slack
+    // several tokens of one group: stage x in shared memory when it fits
+    const int64_t x_bytes = (int64_t)n_tok * cols * 4;
+    const bool x_smem = n_tok > 1 && G == 1 && n_chunks == 1 && x_bytes <= X_SMEM_MAX;
+    const int64_t x_area = x_smem ? ceil_div(x_bytes, 128) * 128 : 0;
+    int n_stage = (int)std::min<int64_t>(MAX_STAGES, std::max<int64_t>(2, (budget - x_area) / stage_pitch));
+    while (n_stage > 2 && 128 + SMEM_HDR + n_stage * stage_pitch + x_area > di.smem_optin) --n_stage;
+    const int64_t smem = 128 + SMEM_HDR + n_stage * stage_pitch + x_area;   // 128: base alignment slack
     if (smem > di.smem_optin) return QMV_ERR_SHAPE;
 
     const int64_t rows_per_cta = std::max<int64_t>(1, rows_cta0);
@@ -192,6 +197,7 @@ int make_plan(int fmt, int64_t rows, int64_t cols, int n_tok, int G, int n_jobs,
     p.row_pitch = (int32_t)chunk_bytes;
     p.rows_per_cta = (int32_t)rows_per_cta;
     p.tma = tma ? 1 : 0;
+    p.x_smem = x_smem ? 1 : 0;
     p.err = di.err;
     pl.kc.ntok = n_tok;
     pl.kc.R = R;

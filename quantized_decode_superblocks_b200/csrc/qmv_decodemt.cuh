@@ -18,17 +18,23 @@
 
 namespace qmv {
 
-__device__ __forceinline__ float4 ldg4_mt(const float *p)
+// Staged x in shared memory: float4 group f of a token row lives at group
+// f ^ (((f >> 3) ^ (f >> 4)) & 7), so lanes reading the same offset of
+// consecutive slices fall in different banks.
+__device__ __forceinline__ uint32_t xs_swizzle(uint32_t f)
 {
-    return __ldg(reinterpret_cast<const float4 *>(p));
+    return f ^ (((f >> 3) ^ (f >> 4)) & 7u);
 }
 
 __device__ __forceinline__ float2 f2mul(float2 a, float2 b) { return __fmul2_rn(a, b); }
 
-// Q8_0: blk[k] = shared address of row k's block (2-byte aligned); xs = x of
-// token 0 at the block's first column; xts = floats between tokens.
-template <int NTOK, int R>
-__device__ __forceinline__ void q8_0_slice_mt(const uint32_t (&blk)[R], const float *xs, int64_t xts,
+// x accessors: xl(t, col) returns x[t][col .. col+3] as a float4 (col a
+// multiple of 4, relative to the current K-chunk).
+//
+// Q8_0: blk[k] = shared address of row k's block (2-byte aligned); col0 = the
+// block's first column.
+template <int NTOK, int R, class XL>
+__device__ __forceinline__ void q8_0_slice_mt(const uint32_t (&blk)[R], int col0, XL &&xl,
                                               float2 (&acc)[R][NTOK])
 {
     float2 d[R];
@@ -54,8 +60,8 @@ __device__ __forceinline__ void q8_0_slice_mt(const uint32_t (&blk)[R], const fl
         }
 #pragma unroll
         for (int t = 0; t < NTOK; ++t) {
-            const float4 a = ldg4_mt(xs + (int64_t)t * xts + 8 * st);
-            const float4 b = ldg4_mt(xs + (int64_t)t * xts + 8 * st + 4);
+            const float4 a = xl(t, col0 + 8 * st);
+            const float4 b = xl(t, col0 + 8 * st + 4);
             const float2 x02 = make_float2(a.x, a.z), x13 = make_float2(a.y, a.w);
             const float2 x46 = make_float2(b.x, b.z), x57 = make_float2(b.y, b.w);
 #pragma unroll
@@ -72,10 +78,10 @@ __device__ __forceinline__ void q8_0_slice_mt(const uint32_t (&blk)[R], const fl
 }
 
 // Q4_K: sb[k] = shared address of row k's superblock (16-byte aligned), c =
-// chunk; xs = x of token 0 at column 64c of the superblock.
-template <int NTOK, int R>
+// chunk; col0 = column 64c of the superblock.
+template <int NTOK, int R, class XL>
 __device__ __forceinline__ void q4_k_slice_mt(const uint32_t (&sb)[R], int c, const Q4kSel &sel,
-                                              const float *xs, int64_t xts, float2 (&acc)[R][NTOK])
+                                              int col0, XL &&xl, float2 (&acc)[R][NTOK])
 {
     float2 dscA[R], dmA[R], dscB[R], dmB[R];
 #pragma unroll
@@ -105,8 +111,8 @@ __device__ __forceinline__ void q4_k_slice_mt(const uint32_t (&sb)[R], int c, co
         }
 #pragma unroll
         for (int t = 0; t < NTOK; ++t) {
-            const float4 a = ldg4_mt(xs + (int64_t)t * xts + 4 * i);
-            const float4 b = ldg4_mt(xs + (int64_t)t * xts + 32 + 4 * i);
+            const float4 a = xl(t, col0 + 4 * i);
+            const float4 b = xl(t, col0 + 32 + 4 * i);
             const float2 xa02 = make_float2(a.x, a.z), xa13 = make_float2(a.y, a.w);
             const float2 xb02 = make_float2(b.x, b.z), xb13 = make_float2(b.y, b.w);
 #pragma unroll
@@ -123,10 +129,10 @@ __device__ __forceinline__ void q4_k_slice_mt(const uint32_t (&sb)[R], int c, co
 }
 
 // Q6_K: sb[k] = shared address of row k's superblock (2-byte aligned); half h,
-// l0 in {0, 16}; xs = x of token 0 at column 128h + l0 of the superblock.
-template <int NTOK, int R>
-__device__ __forceinline__ void q6_k_slice_mt(const uint32_t (&sb)[R], int h, int l0, const float *xs,
-                                              int64_t xts, float2 (&acc)[R][NTOK])
+// l0 in {0, 16}; col0 = column 128h + l0 of the superblock.
+template <int NTOK, int R, class XL>
+__device__ __forceinline__ void q6_k_slice_mt(const uint32_t (&sb)[R], int h, int l0, int col0, XL &&xl,
+                                              float2 (&acc)[R][NTOK])
 {
     float2 dsc[R][4];
     const uint32_t o = (uint32_t)(l0 >> 4);
@@ -169,7 +175,7 @@ __device__ __forceinline__ void q6_k_slice_mt(const uint32_t (&sb)[R], int h, in
         for (int n = 0; n < NTOK; ++n) {
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
-                const float4 a = ldg4_mt(xs + (int64_t)n * xts + 32 * t + 4 * i);
+                const float4 a = xl(n, col0 + 32 * t + 4 * i);
                 const float2 x02 = make_float2(a.x, a.z), x13 = make_float2(a.y, a.w);
 #pragma unroll
                 for (int k = 0; k < R; ++k) {

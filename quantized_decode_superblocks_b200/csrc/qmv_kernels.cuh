@@ -73,6 +73,7 @@ struct Params {
     int32_t rows_per_cta;
     int32_t mode;
     int32_t tma;             // 1: bulk async copies; 0: warp copies
+    int32_t x_smem;          // several tokens: x staged in shared memory after the stages
     // weights: group matrix = base + ids[idx] * expert_stride (or base)
     const uint8_t *base0;
     const uint8_t *base1;    // MODE_SWIGLU: up matrices (group 1)
@@ -279,6 +280,20 @@ __device__ __forceinline__ void qmv_pipeline_body(const Params &p, const int cta
         }
     }
 
+    // several tokens: stage every token's x once in shared memory (swizzled)
+    const uint32_t xsm = stage0 + (uint32_t)S * (uint32_t)p.stage_pitch;
+    const int nf = p.cols >> 2;                   // float4 groups per token row
+    if constexpr (NTOK > 1) {
+        if (p.x_smem) {
+            for (int idx = tid; idx < NTOK * nf; idx += NTHREADS) {
+                const int t = idx / nf, f = idx - t * nf;
+                sts_f4(xsm + 16u * (uint32_t)(t * nf + (int)xs_swizzle((uint32_t)f)),
+                       ldg4(sX[0] + (int64_t)t * p.x_tok_stride + 4 * f));
+            }
+            __syncthreads();
+        }
+    }
+
     float acc[V];
 #pragma unroll
     for (int v = 0; v < V; ++v) acc[v] = 0.f;
@@ -357,23 +372,31 @@ __device__ __forceinline__ void qmv_pipeline_body(const Params &p, const int cta
                     rowp[k] = st + (uint32_t)(g * T + (rl < tr ? rl : 0)) * (uint32_t)p.row_pitch;
                 }
                 const float *xg = sX[g] + col_base;
-                for (int s = ks * P + lane; s < s_end; s += 32) {
-                    uint32_t bp[R];
-                    if (FMT == FMT_Q8_0) {
+                auto xl_g = [&](int t, int col) { return ldg4(xg + (int64_t)t * p.x_tok_stride + col); };
+                auto xl_s = [&](int t, int col) {
+                    return lds_f4(xsm + 16u * (uint32_t)(t * nf + (int)xs_swizzle((uint32_t)col >> 2)));
+                };
+                auto slices = [&](auto &&xl) {
+                    for (int s = ks * P + lane; s < s_end; s += 32) {
+                        uint32_t bp[R];
+                        if (FMT == FMT_Q8_0) {
 #pragma unroll
-                        for (int k = 0; k < R; ++k) bp[k] = rowp[k] + 34u * (uint32_t)s;
-                        q8_0_slice_mt<NTOK, R>(bp, xg + 32 * s, p.x_tok_stride, accmt);
-                    } else if (FMT == FMT_Q4_K) {
+                            for (int k = 0; k < R; ++k) bp[k] = rowp[k] + 34u * (uint32_t)s;
+                            q8_0_slice_mt<NTOK, R>(bp, 32 * s, xl, accmt);
+                        } else if (FMT == FMT_Q4_K) {
 #pragma unroll
-                        for (int k = 0; k < R; ++k) bp[k] = rowp[k] + 144u * (uint32_t)(s >> 2);
-                        q4_k_slice_mt<NTOK, R>(bp, s & 3, sel, xg + 256 * (s >> 2) + 64 * (s & 3), p.x_tok_stride, accmt);
-                    } else {
+                            for (int k = 0; k < R; ++k) bp[k] = rowp[k] + 144u * (uint32_t)(s >> 2);
+                            q4_k_slice_mt<NTOK, R>(bp, s & 3, sel, 256 * (s >> 2) + 64 * (s & 3), xl, accmt);
+                        } else {
 #pragma unroll
-                        for (int k = 0; k < R; ++k) bp[k] = rowp[k] + 210u * (uint32_t)(s >> 2);
-                        const int h = (s >> 1) & 1, l0 = 16 * (s & 1);
-                        q6_k_slice_mt<NTOK, R>(bp, h, l0, xg + 256 * (s >> 2) + 128 * h + l0, p.x_tok_stride, accmt);
+                            for (int k = 0; k < R; ++k) bp[k] = rowp[k] + 210u * (uint32_t)(s >> 2);
+                            const int h = (s >> 1) & 1, l0 = 16 * (s & 1);
+                            q6_k_slice_mt<NTOK, R>(bp, h, l0, 256 * (s >> 2) + 128 * h + l0, xl, accmt);
+                        }
                     }
-                }
+                };
+                if (p.x_smem) slices(xl_s);
+                else slices(xl_g);
             }
         }
 
