@@ -250,7 +250,20 @@ class Sweep:
         self.y_host = torch.empty(y_off, dtype=torch.float32).pin_memory()
         self.weight_bytes = sum(synth.matrix_bytes(Q8_0, mm["rows"], mm["cols"]) for mm in self.mats)
         self.algo = sum(algo_bytes(Q8_0, mm["rows"], mm["cols"], n_tok) for mm in self.mats)
+        self.tasks = q.make_tasks([(mm["W"], mm["rows"], mm["cols"], self.x.data_ptr() + 4 * mm["x_off"],
+                                    self.y.data_ptr() + 4 * mm["y_off"]) for mm in self.mats])
+        self.mode = "launches"
         self.launches = len(self.mats)
+
+    def set_mode(self, mode):
+        """'launches': one library call per matvec, in order; 'chain': the
+        whole step as in-order chained calls (one token); 'grouped': the
+        matvecs as independent grouped launches."""
+        if mode == "chain" and self.n_tok != 1:
+            raise ValueError("the chained step is one-token")
+        self.mode = mode
+        self.launches = {"launches": len(self.mats), "chain": -(-len(self.mats) // 64),
+                         "grouped": None}[mode]
 
     def launch(self, i, stream=None):
         mm = self.mats[i]
@@ -262,8 +275,13 @@ class Sweep:
             self.q.qmv_batched(Q8_0, mm["W"], mm["rows"], mm["cols"], x, y, self.n_tok, stream)
 
     def step(self, stream=None):
-        for i in range(len(self.mats)):
-            self.launch(i, stream)
+        if self.mode == "chain":
+            self.q.qmv_chain(Q8_0, self.tasks, stream)
+        elif self.mode == "grouped":
+            self.q.qmv_multi(Q8_0, self.n_tok, self.tasks, stream)
+        else:
+            for i in range(len(self.mats)):
+                self.launch(i, stream)
 
 
 def per_launch_durations(torch, sweep, stream, reps=3):

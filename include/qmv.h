@@ -117,6 +117,24 @@ typedef struct {
  * (1 <= n_tasks <= QMV_MAX_TASKS), read during the call only. */
 int qmv_multi(int fmt, int n_tok, const qmv_task *tasks, int n_tasks, qmv_stream_t stream);
 
+/* One-token matvecs of one format executed IN ORDER, the way a decode step
+ * runs its projections layer after layer (BebeLM：纯Rust实现的端侧大模型推理引擎,
+ * §核心算子 and §性能表现: every layer's matvecs each decode step): task t+1
+ * starts only after every row of task t is written, so a task's x may be the
+ * y of any earlier task of the same call (tasks' n_tok is 1: x f32 [cols],
+ * y f32 [rows]).  The library runs up to 64 tasks in one persistent
+ * cooperative launch with a grid barrier between tasks, and keeps copying the
+ * next tasks' weights into shared memory while the GPU waits at a barrier;
+ * longer lists take several consecutive launches.  A task shape that the
+ * persistent kernel does not take turns the whole call into one launch per
+ * task, in order.  The grid barrier's state is one per device: do not run two
+ * qmv_chain calls on the same device at the same time (different streams);
+ * a barrier that waits about a second reports QMV_DEVERR_TIMEOUT through
+ * qmv_check, which also resets the barrier.  `tasks` is a host array of
+ * n_tasks entries (1 <= n_tasks <= QMV_MAX_TASKS), read during the call only.
+ * Errors as qmv_multi. */
+int qmv_chain(int fmt, const qmv_task *tasks, int n_tasks, qmv_stream_t stream);
+
 /* Multi-token variant for speculative verification (FlareLLM page,
  * §推理层面的深度优化: n-gram speculative decoding): every weight is read once
  * and applied to n_tok activation vectors.

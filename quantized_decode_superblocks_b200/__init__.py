@@ -25,7 +25,7 @@ STATUS_NAMES = {0: "QMV_OK", -1: "QMV_ERR_NULL", -2: "QMV_ERR_FMT", -3: "QMV_ERR
 DEVERR_EXPERT_ID = 1
 DEVERR_TIMEOUT = 2
 
-EXPORTED = ("qmv_f32", "qmv_batched", "qmv_multi", "moe_route", "moe_qmv", "moe_ffn", "moe_ffn_static",
+EXPORTED = ("qmv_f32", "qmv_batched", "qmv_multi", "qmv_chain", "moe_route", "moe_qmv", "moe_ffn", "moe_ffn_static",
             "qmv_dequant",
             "qmv_check", "qmv_strerror", "qmv_block_bytes", "qmv_block_weights",
             "qmv_debug_fail_next_launches", "qmv_set_pdl", "qmv_get_pdl", "qmv_last_cuda_error")
@@ -161,6 +161,13 @@ def qmv_multi(fmt, n_tok, tasks, stream=None):
     (W, rows, cols, x, y) tuples or an array from make_tasks()."""
     arr = tasks if isinstance(tasks, ctypes.Array) else make_tasks(tasks)
     _check(lib().qmv_multi(fmt, n_tok, arr, len(arr), _stream(stream)), "qmv_multi")
+
+
+def qmv_chain(fmt, tasks, stream=None):
+    """One-token matvecs executed in order (task t+1 may read task t's y);
+    `tasks` as for qmv_multi."""
+    arr = tasks if isinstance(tasks, ctypes.Array) else make_tasks(tasks)
+    _check(lib().qmv_chain(fmt, arr, len(arr), _stream(stream)), "qmv_chain")
 
 
 def moe_route(logits, bias, n_expert, top_k, ids_out, g_out, stream=None):

@@ -19,7 +19,7 @@ BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libqmv.so")
 
 SOURCES = ["qmv_api.cu", "qmv_fmt_q8_0.cu", "qmv_fmt_q4_k.cu", "qmv_fmt_q6_k.cu"]
-HEADERS = ["qmv_device.cuh", "qmv_decode1.cuh", "qmv_decodemt.cuh", "qmv_kernels.cuh", "qmv_dispatch.cuh", "qmv_misc.cuh"]
+HEADERS = ["qmv_device.cuh", "qmv_decode1.cuh", "qmv_decodemt.cuh", "qmv_kernels.cuh", "qmv_rw.cuh", "qmv_dispatch.cuh", "qmv_misc.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
                      "-I", os.path.join(ROOT, "include"), "--expt-relaxed-constexpr"]

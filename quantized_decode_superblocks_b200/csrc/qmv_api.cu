@@ -8,6 +8,7 @@
 
 #include "../../include/qmv.h"
 #include "qmv_misc.cuh"
+#include "qmv_rw.cuh"
 
 namespace {
 
@@ -15,6 +16,10 @@ using namespace qmv;
 
 // Sticky device error word (QMV_DEVERR_* bits), read and cleared by qmv_check.
 __device__ int g_dev_err;
+
+// Grid barrier of ordered chained launches: {arrivals, exits}, back to zero
+// at the end of every launch; qmv_check clears both after a device error.
+__device__ unsigned g_chain_sync[2];
 
 // Scratch of moe_ffn_static: the SwiGLU activations h[n_sel][inter].  Every
 // device that loads the library holds one copy until the process exits.
@@ -35,6 +40,7 @@ struct DevInfo {
     int sm_count = 0;
     int smem_optin = 0;
     int *err = nullptr;
+    unsigned *sync = nullptr;
     float *static_h = nullptr;   // device address of g_static_h, set up by moe_ffn_static
     bool ok = false;
 };
@@ -82,7 +88,8 @@ int get_dev(DevInfo &out)
         if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-            cudaGetSymbolAddress(reinterpret_cast<void **>(&d.err), g_dev_err) != cudaSuccess) {
+            cudaGetSymbolAddress(reinterpret_cast<void **>(&d.err), g_dev_err) != cudaSuccess ||
+            cudaGetSymbolAddress(reinterpret_cast<void **>(&d.sync), g_chain_sync) != cudaSuccess) {
             (void)cudaGetLastError();
             return QMV_ERR_DEVICE;
         }
@@ -220,6 +227,179 @@ int launch_plan(int fmt, const Plan &pl, cudaStream_t stream)
     return QMV_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Warp-private-ring kernel (one token, one matrix per task): tile = R rows x a
+// K-chunk of up to 2048 columns; per warp S stages.  R and S depend only on the
+// format (the bytes of a full K-chunk), so tasks of one format share them.
+constexpr int64_t RW_CTA_SMEM = 112 * 1024;      // per CTA, two CTAs per SM
+
+struct RwGeom {
+    int R = 0;
+    int S = 0;
+    int pitch = 0;
+    size_t smem = 0;
+};
+
+// x_floats: shared-memory x (tasks longer than one K-chunk), taken from the
+// stage budget.
+RwGeom rw_geom(int fmt, int64_t x_floats, int n_tasks)
+{
+    const int64_t cb = (RW_CK / block_weights(fmt)) * block_bytes(fmt);
+    const int64_t x_area = ceil_div(x_floats * 4, 128) * 128;
+    const int64_t hdr = rw_hdr_bytes(n_tasks);
+    const int64_t per_warp = (RW_CTA_SMEM - hdr - x_area) / NW;
+    auto pitch = [&](int R) { return ceil_div(R * cb + 16, 128) * 128; };
+    auto stages = [&](int R) { return std::min<int64_t>(RW_MAX_STAGES, per_warp / pitch(R)); };
+    RwGeom g;
+    for (int want_s : {3, 2}) {
+        for (int R : {4, 2, 1}) {
+            if (stages(R) >= want_s) {
+                g.R = R;
+                g.S = (int)stages(R);
+                g.pitch = (int)pitch(R);
+                g.smem = (size_t)(128 + hdr + x_area + (int64_t)NW * g.S * g.pitch);
+                return g;
+            }
+        }
+    }
+    return g;
+}
+
+// Whether a (rows x cols) matrix of fmt can take the warp-ring kernel: every
+// bulk copy (a row, a K-chunk of a row) must be a multiple of 16 bytes, and a
+// Q8_0 lane slice is a pair of blocks.
+bool rw_ok(int fmt, int64_t cols)
+{
+    const int bw = block_weights(fmt), bb = block_bytes(fmt);
+    if (fmt == QMV_Q8_0 && cols % 64 != 0) return false;
+    if (cols > RW_CK && cols > RW_X_SMEM_MAX) return false;     // x of a long row must fit in shared memory
+    const int64_t rb = cols / bw * bb;
+    const int64_t cb = (RW_CK / bw) * bb;
+    const int64_t last_cols = cols - (ceil_div(cols, RW_CK) - 1) * RW_CK;
+    const int64_t lb = last_cols / bw * bb;
+    return rb % 16 == 0 && cb % 16 == 0 && lb % 16 == 0;
+}
+
+// Split a task's row groups over its nw warps, starting at warp rot (see
+// rw_range in the kernel).
+void rw_split(RwTask &t, int64_t nw, int64_t rot = 0)
+{
+    t.rg_q = t.n_rg / nw;
+    t.rg_r = (int32_t)(t.n_rg % nw);
+    t.nw = (int32_t)nw;
+    t.rot = (int32_t)(rot % nw);
+}
+
+RwTask rw_task(int fmt, int R, const void *W, int64_t rows, int64_t cols, const float *x, float *y)
+{
+    const int bw = block_weights(fmt), bb = block_bytes(fmt);
+    RwTask t{};
+    t.W = static_cast<const uint8_t *>(W);
+    t.x = x;
+    t.y = y;
+    t.rows = rows;
+    t.row_bytes = cols / bw * bb;
+    t.n_rg = ceil_div(rows, R);
+    t.n_chunks = (int32_t)ceil_div(cols, RW_CK);
+    t.chunk_bytes = (int32_t)((RW_CK / bw) * bb);
+    t.last_cols = (int32_t)(cols - (int64_t)(t.n_chunks - 1) * RW_CK);
+    t.last_bytes = (int32_t)(t.last_cols / bw * bb);
+    if (t.n_chunks == 1) t.chunk_bytes = t.last_bytes;
+    return t;
+}
+
+template <int NT>
+cudaError_t rw_launch(int fmt, const RwParamsT<NT> &p, int R, dim3 grid, size_t smem, cudaStream_t st, bool pdl,
+                      bool coop)
+{
+    switch (fmt) {
+    case QMV_Q8_0: return launch_rw<FMT_Q8_0, NT>(p, R, grid, smem, st, pdl, coop);
+    case QMV_Q4_K: return launch_rw<FMT_Q4_K, NT>(p, R, grid, smem, st, pdl, coop);
+    default: return launch_rw<FMT_Q6_K, NT>(p, R, grid, smem, st, pdl, coop);
+    }
+}
+
+cudaError_t rw_occ(int fmt, int R, size_t smem, int *n)
+{
+    switch (fmt) {
+    case QMV_Q8_0: return rw_occupancy<FMT_Q8_0>(R, smem, n);
+    case QMV_Q4_K: return rw_occupancy<FMT_Q4_K>(R, smem, n);
+    default: return rw_occupancy<FMT_Q6_K>(R, smem, n);
+    }
+}
+
+// One matvec on the warp-ring kernel: enough CTAs that every warp has a row
+// group, at most two per SM.
+int rw_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x, float *y, const DevInfo &di,
+              cudaStream_t st)
+{
+    const int64_t x_floats = cols > RW_CK ? cols : 0;
+    const RwGeom g = rw_geom(fmt, x_floats, 1);
+    if (g.R == 0) return QMV_ERR_SHAPE;
+    RwParams1 p{};
+    p.n_tasks = 1;
+    p.chain = 0;
+    p.ordered = 0;
+    p.n_stage = g.S;
+    p.stage_pitch = g.pitch;
+    p.x_floats = (int32_t)x_floats;
+    p.sync = di.sync;
+    p.err = di.err;
+    p.t[0] = rw_task(fmt, g.R, W, rows, cols, x, y);
+    const int64_t ctas = std::max<int64_t>(1, std::min<int64_t>(2LL * di.sm_count, ceil_div(p.t[0].n_rg, NW)));
+    p.cta_begin[0] = 0;
+    p.cta_begin[1] = (int)ctas;
+    rw_split(p.t[0], ctas * NW);
+    const cudaError_t e = rw_launch(fmt, p, g.R, dim3((unsigned)ctas), g.smem, st, g_pdl.load() != 0, false);
+    return e == cudaSuccess ? QMV_OK : cuda_fail(e);
+}
+
+// Matvecs of one format on the warp-ring kernel, up to RW_MAX_TASKS per
+// launch.  Every CTA works on every task, in order, each task's row groups
+// spread over all warps (so small and large tasks alike use the whole GPU);
+// ordered: with a grid barrier between consecutive tasks (cooperative launch).
+int rw_group(int fmt, const qmv_task *tasks, int n_tasks, bool ordered, const DevInfo &di, cudaStream_t st)
+{
+    int64_t x_floats = 0;
+    for (int t = 0; t < n_tasks; ++t)
+        if (tasks[t].cols > RW_CK) x_floats = std::max<int64_t>(x_floats, tasks[t].cols);
+    const RwGeom g = rw_geom(fmt, x_floats, std::min(n_tasks, RW_MAX_TASKS));
+    if (g.R == 0) return QMV_ERR_SHAPE;
+    static thread_local RwParams p;
+    int ctas_per_sm = 2;
+    {
+        const cudaError_t e = rw_occ(fmt, g.R, g.smem, &ctas_per_sm);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if (ctas_per_sm < 1) return QMV_ERR_SHAPE;
+    }
+    const int64_t ctas = (int64_t)ctas_per_sm * di.sm_count;
+    for (int t0 = 0; t0 < n_tasks; t0 += RW_MAX_TASKS) {
+        const int n = std::min(RW_MAX_TASKS, n_tasks - t0);
+        p.n_tasks = n;
+        p.chain = 1;
+        p.ordered = ordered ? 1 : 0;
+        p.n_stage = g.S;
+        p.stage_pitch = g.pitch;
+        p.x_floats = (int32_t)x_floats;
+        p.sync = di.sync;
+        p.err = di.err;
+        // each task starts on the warp after the previous task's last row group
+        int64_t rot = 0;
+        for (int i = 0; i < n; ++i) {
+            const qmv_task &k = tasks[t0 + i];
+            p.t[i] = rw_task(fmt, g.R, k.W_blocks, k.rows, k.cols, k.x, k.y);
+            rw_split(p.t[i], ctas * NW, rot);
+            rot = (rot + p.t[i].n_rg) % (ctas * NW);
+        }
+        p.cta_begin[0] = 0;
+        p.cta_begin[1] = (int32_t)ctas;
+        const cudaError_t e = rw_launch(fmt, p, g.R, dim3((unsigned)ctas), g.smem, st,
+                                        !ordered && g_pdl.load() != 0, ordered);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return QMV_OK;
+}
+
 int check_matrix(int fmt, int64_t rows, int64_t cols)
 {
     if (!fmt_ok(fmt)) return QMV_ERR_FMT;
@@ -273,6 +453,8 @@ int qmv_batched(int fmt, const void *W_blocks, int64_t rows, int64_t cols, const
     if (injected_failure()) return QMV_ERR_CUDA;
     DevInfo di;
     if ((rc = get_dev(di))) return rc;
+    if (n_tok == 1 && rw_ok(fmt, cols))
+        return rw_single(fmt, W_blocks, rows, cols, x, y, di, reinterpret_cast<cudaStream_t>(stream));
     Plan pl;
     if ((rc = make_plan(fmt, rows, cols, n_tok, 1, 1, true, di, pl))) return rc;
     pl.p.mode = MODE_SEPARATE;
@@ -304,6 +486,11 @@ int qmv_multi(int fmt, int n_tok, const qmv_task *tasks, int n_tasks, qmv_stream
     int rc = get_dev(di);
     if (rc) return rc;
     const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (n_tok == 1) {
+        bool all = true;
+        for (int t = 0; t < n_tasks && all; ++t) all = rw_ok(fmt, tasks[t].cols);
+        if (all) return rw_group(fmt, tasks, n_tasks, false, di, st);
+    }
 
     // Every CTA streams about the same number of bytes, sized so the batch
     // takes a few waves of two CTAs per SM: small tasks get few CTAs with many
@@ -352,6 +539,34 @@ int qmv_multi(int fmt, int n_tok, const qmv_task *tasks, int n_tasks, qmv_stream
         default: e = launch_multi<FMT_Q6_K>(mp, kc, ctas, smem, st); break;
         }
         if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return QMV_OK;
+}
+
+int qmv_chain(int fmt, const qmv_task *tasks, int n_tasks, qmv_stream_t stream)
+{
+    if (!tasks) return QMV_ERR_NULL;
+    if (!fmt_ok(fmt)) return QMV_ERR_FMT;
+    if (n_tasks < 1 || n_tasks > QMV_MAX_TASKS) return QMV_ERR_SHAPE;
+    bool all = true;
+    for (int t = 0; t < n_tasks; ++t) {
+        const qmv_task &k = tasks[t];
+        if (!k.W_blocks || !k.x || !k.y) return QMV_ERR_NULL;
+        const int rc = check_matrix(fmt, k.rows, k.cols);
+        if (rc) return rc;
+        if (!aligned(k.W_blocks, 16) || !aligned(k.x, 16) || !aligned(k.y, 4)) return QMV_ERR_ALIGN;
+        all = all && rw_ok(fmt, k.cols);
+    }
+    if (injected_failure()) return QMV_ERR_CUDA;
+    DevInfo di;
+    int rc = get_dev(di);
+    if (rc) return rc;
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (all) return rw_group(fmt, tasks, n_tasks, true, di, st);
+    // a shape the chained kernel does not take: one launch per task, in order
+    for (int t = 0; t < n_tasks; ++t) {
+        const qmv_task &k = tasks[t];
+        if ((rc = qmv_batched(fmt, k.W_blocks, k.rows, k.cols, k.x, k.y, 1, stream))) return rc;
     }
     return QMV_OK;
 }
@@ -541,6 +756,10 @@ int qmv_check(qmv_stream_t stream, int *dev_err_out)
     int word = 0;
     if (cudaMemcpy(&word, di.err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
         cudaMemset(di.err, 0, sizeof(int)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+        (void)cudaGetLastError();
+        return QMV_ERR_CUDA;
+    }
+    if (word && (cudaMemset(di.sync, 0, 2 * sizeof(unsigned)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)) {
         (void)cudaGetLastError();
         return QMV_ERR_CUDA;
     }

@@ -3,7 +3,7 @@
 // parallel.
 #pragma once
 
-#include "qmv_kernels.cuh"
+#include "qmv_rw.cuh"
 
 namespace qmv {
 
@@ -11,7 +11,7 @@ namespace qmv {
 // (kernel, device) and adds the programmatic-serialization attribute when asked.
 template <class Kern, class Arg>
 static cudaError_t launch_with(Kern kern, int *configured, const Arg &arg, dim3 grid, size_t smem,
-                               cudaStream_t stream, bool pdl)
+                               cudaStream_t stream, bool pdl, bool cooperative = false)
 {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -22,16 +22,25 @@ static cudaError_t launch_with(Kern kern, int *configured, const Arg &arg, dim3 
         if (e != cudaSuccess) return e;
         configured[dev] = (int)smem;
     }
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    unsigned n_attr = 0;
+    if (pdl) {
+        attr[n_attr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n_attr].val.programmaticStreamSerializationAllowed = 1;
+        ++n_attr;
+    }
+    if (cooperative) {      // all CTAs co-resident, or the launch fails (grid barriers)
+        attr[n_attr].id = cudaLaunchAttributeCooperative;
+        attr[n_attr].val.cooperative = 1;
+        ++n_attr;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = dim3(NTHREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cfg.attrs = pdl ? attr : nullptr;
-    cfg.numAttrs = pdl ? 1 : 0;
+    cfg.attrs = n_attr ? attr : nullptr;
+    cfg.numAttrs = n_attr;
     return cudaLaunchKernelEx(&cfg, kern, arg);
 }
 
@@ -111,6 +120,56 @@ struct MultiLaunch {
     template <int FMT, int NTOK, int R, bool XREG>
     cudaError_t run() const { return Instance<FMT, NTOK, R, XREG>::multi(mp, grid, smem, st, pdl); }
 };
+
+template <int FMT, int R, int NT>
+struct RwInstance {
+    static int *configured()
+    {
+        static int c[64] = {0};
+        return c;
+    }
+    static cudaError_t go(const RwParamsT<NT> &p, dim3 grid, size_t smem, cudaStream_t st, bool pdl, bool coop)
+    {
+        return launch_with(qmv_rw_kernel<FMT, R, NT>, configured(), p, grid, smem, st, pdl, coop);
+    }
+    static cudaError_t occupancy(size_t smem, int *n)
+    {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+        if (configured()[dev] < (int)smem) {
+            e = cudaFuncSetAttribute(qmv_rw_kernel<FMT, R, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)smem);
+            if (e != cudaSuccess) return e;
+            configured()[dev] = (int)smem;
+        }
+        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(n, qmv_rw_kernel<FMT, R, NT>, NTHREADS, smem);
+    }
+};
+
+template <int FMT, int NT>
+cudaError_t launch_rw(const RwParamsT<NT> &p, int R, dim3 grid, size_t smem, cudaStream_t stream, bool pdl,
+                      bool cooperative)
+{
+    switch (R) {
+    case 1: return RwInstance<FMT, 1, NT>::go(p, grid, smem, stream, pdl, cooperative);
+    case 2: return RwInstance<FMT, 2, NT>::go(p, grid, smem, stream, pdl, cooperative);
+    case 4: return RwInstance<FMT, 4, NT>::go(p, grid, smem, stream, pdl, cooperative);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int FMT>
+cudaError_t rw_occupancy(int R, size_t smem, int *ctas_per_sm)
+{
+    switch (R) {
+    case 1: return RwInstance<FMT, 1, RW_MAX_TASKS>::occupancy(smem, ctas_per_sm);
+    case 2: return RwInstance<FMT, 2, RW_MAX_TASKS>::occupancy(smem, ctas_per_sm);
+    case 4: return RwInstance<FMT, 4, RW_MAX_TASKS>::occupancy(smem, ctas_per_sm);
+    default: return cudaErrorInvalidValue;
+    }
+}
 
 template <int FMT>
 cudaError_t launch_pipeline(const Params &p, const KernelChoice &kc, dim3 grid, size_t smem,

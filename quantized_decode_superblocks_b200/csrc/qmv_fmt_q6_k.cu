@@ -4,4 +4,7 @@
 namespace qmv {
 template cudaError_t launch_pipeline<FMT_Q6_K>(const Params &, const KernelChoice &, dim3, size_t, cudaStream_t);
 template cudaError_t launch_multi<FMT_Q6_K>(const MultiParams &, const KernelChoice &, int, size_t, cudaStream_t);
+template cudaError_t launch_rw<FMT_Q6_K, 1>(const RwParams1 &, int, dim3, size_t, cudaStream_t, bool, bool);
+template cudaError_t launch_rw<FMT_Q6_K, RW_MAX_TASKS>(const RwParams &, int, dim3, size_t, cudaStream_t, bool, bool);
+template cudaError_t rw_occupancy<FMT_Q6_K>(int, size_t, int *);
 }  // namespace qmv

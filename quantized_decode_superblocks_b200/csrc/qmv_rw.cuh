@@ -1,0 +1,584 @@
+// qmv_rw.cuh -- the one-token matvec with warp-private copy rings.
+//
+// A batch-1 decode matvec is bound by how fast the SM can decode weights once
+// the bytes stream at HBM speed (the decode costs a few instructions per
+// weight, and 148 SMs must decode ~10^13 weights/s).  This kernel therefore
+// spends as little as possible outside the decode itself:
+//   * every warp owns a contiguous run of row groups (R rows each) and runs its
+//     own ring of shared-memory stages: lane 0 moves a tile (R rows x one
+//     K-chunk of up to 2048 columns) with 1-D bulk async copies that complete
+//     on the stage's mbarrier, and refills the stage as soon as the warp has
+//     finished with it -- no cross-warp tickets or block barriers per tile;
+//   * the slice geometry is fixed at compile time: lane l decodes 64
+//     consecutive-in-layout weights of every row of the tile (a pair of Q8_0
+//     blocks, or a quarter of a Q4_K / Q6_K superblock) against x values that
+//     sit in its registers for the whole K-chunk;
+//   * one multi-row butterfly per row group reduces the lanes' partial sums.
+// Decode is memory-bandwidth bound on the pages' hardware (BebeLM：纯Rust实现的
+// 端侧大模型推理引擎, §性能表现); on this one the decode arithmetic is the
+// tighter limit, which is what the layout above optimises for.
+//
+// The same body serves three launch forms:
+//   * one matvec (one task, all CTAs);
+//   * several independent matvecs (each task owns a range of CTAs);
+//   * a chain: every CTA works on every task in order, with a grid-wide
+//     barrier between consecutive tasks, so task t+1 may read task t's output
+//     (the layer-after-layer order of a decode step).  Weights do not depend on
+//     earlier tasks, so each warp's ring keeps prefetching the next tasks'
+//     tiles while the CTA waits at the barrier.
+#pragma once
+
+#include "qmv_kernels.cuh"
+
+namespace qmv {
+
+constexpr int RW_CK = 2048;           // columns of one K-chunk: 64 per lane
+constexpr int RW_MAX_STAGES = 6;      // ring stages per warp
+constexpr int RW_MAX_TASKS = 64;
+constexpr int RW_CUR_OFF = 512;       // per-warp producer cursors (32 bytes each) after the mbarriers
+constexpr int RW_BAR_BYTES = 1024;    // mbarriers (NW x RW_MAX_STAGES x 8 bytes) + cursors, rounded up;
+                                      // the launch's task table follows (rw_hdr_bytes)
+constexpr int RW_X_SMEM_MAX = 12288;  // longest row (columns) whose x is staged in shared memory
+
+struct RwTask {
+    const uint8_t *W;         // rows x row_bytes of packed blocks
+    const float *x;           // [cols]
+    float *y;                 // [rows]
+    int64_t rows;
+    int64_t row_bytes;
+    int64_t n_rg;             // row groups: ceil(rows / R)
+    int64_t rg_q;             // warp w = (wg - rot) mod nw of the task's nw warps takes row
+    int32_t rg_r;             //   groups [w*rg_q + min(w, rg_r), +rg_q + (w < rg_r))
+    int32_t rot;              // first warp of the task: consecutive small tasks land on different warps
+    int32_t nw;               // warps the task is spread over
+    int32_t n_chunks;         // ceil(cols / RW_CK)
+    int32_t chunk_bytes;      // bytes of one full K-chunk of a row
+    int32_t last_bytes;       // bytes of the last K-chunk of a row
+    int32_t last_cols;        // columns of the last K-chunk
+    int32_t pad_[3];
+};
+static_assert(sizeof(RwTask) % 16 == 0, "task table is copied in 16-byte units");
+
+// Shared-memory header of a launch with n tasks: mbarriers, cursors, and a copy
+// of the task table (read at every task switch: shared memory, not the
+// constant bank, whose cache a 5 KB table with runtime indices keeps missing).
+__host__ __device__ constexpr int rw_hdr_bytes(int n_tasks)
+{
+    return RW_BAR_BYTES + ((n_tasks * (int)sizeof(RwTask) + 127) & ~127);
+}
+
+// Launch parameters for up to NT tasks (NT = 1 keeps a single matvec's
+// parameter block small: it is copied with every launch).
+template <int NT>
+struct RwParamsT {
+    int32_t n_tasks;
+    int32_t chain;            // 1: every CTA works on every task, in order
+    int32_t ordered;          // chained: grid barrier between consecutive tasks (cooperative launch)
+    int32_t n_stage;          // ring stages per warp
+    int32_t stage_pitch;      // bytes per stage (multiple of 128)
+    int32_t x_floats;         // shared-memory x of tasks longer than one K-chunk (0: none)
+    int32_t cta_begin[NT + 1];   // not chained: task t owns CTAs [cta_begin[t], cta_begin[t+1])
+    unsigned *sync;           // ordered: {arrivals, exits} of the grid barrier, zero between launches
+    int *err;
+    RwTask t[NT];
+};
+using RwParams1 = RwParamsT<1>;
+using RwParams = RwParamsT<RW_MAX_TASKS>;
+
+// Row groups [a, b) of a task that warp wg takes: contiguous, balanced, split
+// on the host (no divisions here).
+__device__ __forceinline__ void rw_range(const RwTask &tk, int wg, int64_t &a, int64_t &b)
+{
+    int w = wg - tk.rot;
+    if (w < 0) w += tk.nw;
+    a = (int64_t)w * tk.rg_q + min(w, tk.rg_r);
+    b = a + tk.rg_q + (w < tk.rg_r ? 1 : 0);
+}
+
+// The producer's position in a warp's tile sequence: task, row group, K-chunk
+// (with the task's K-chunk count cached).
+struct RwCursor {
+    int t;
+    int kc;
+    int nch;
+    int issued;         // tiles issued so far
+    int64_t rg;
+    int64_t rg_end;
+};
+static_assert(sizeof(RwCursor) == 32, "cursor slot");
+
+// Move c to the first tile of task t or, if the warp has none there, of the
+// next task where it has some (c.t == t_end: no tiles left).
+static __device__ __noinline__ void rw_seek(const RwTask *tasks, RwCursor &c, int t, int t_end, int wg)
+{
+    for (; t < t_end; ++t) {
+        int64_t a, b;
+        rw_range(tasks[t], wg, a, b);
+        if (a < b) {
+            c.t = t;
+            c.kc = 0;
+            c.nch = tasks[t].n_chunks;
+            c.rg = a;
+            c.rg_end = b;
+            return;
+        }
+    }
+    c.t = t_end;
+    c.kc = 0;
+    c.nch = 1;
+    c.rg = 0;
+    c.rg_end = 0;
+}
+
+__device__ __forceinline__ void rw_advance(const RwTask *tasks, RwCursor &c, int t_end, int wg)
+{
+    if (++c.kc < c.nch) return;
+    c.kc = 0;
+    if (++c.rg < c.rg_end) return;
+    rw_seek(tasks, c, c.t + 1, t_end, wg);
+}
+
+// Issue the copies of tile c into stage dst (called by one lane).
+template <int R>
+__device__ __forceinline__ void rw_issue(const RwTask *tasks, const RwCursor &c, uint32_t dst, uint32_t bar)
+{
+    const RwTask &tk = tasks[c.t];
+    const int64_t r0 = c.rg * R;
+    const int tr = (int)min((int64_t)R, tk.rows - r0);
+    const bool lastc = c.kc == c.nch - 1;
+    const uint32_t cb = (uint32_t)(lastc ? tk.last_bytes : tk.chunk_bytes);
+    mbar_arrive_expect_tx(bar, (uint32_t)tr * cb);
+    const uint8_t *src = tk.W + r0 * tk.row_bytes + (int64_t)c.kc * tk.chunk_bytes;
+    if (c.nch == 1) {
+        bulk_g2s(dst, src, (uint32_t)tr * cb, bar);      // the tile's rows are contiguous
+    } else {
+        for (int k = 0; k < tr; ++k) bulk_g2s(dst + (uint32_t)k * cb, src + k * tk.row_bytes, cb, bar);
+    }
+}
+
+// Two consecutive Q8_0 blocks (68 bytes at a 4-byte-aligned shared address):
+// block 0's quants straddle words 0..8 (two bytes in), block 1's are words
+// 9..16.  Groups gq = 0..15 of the x pairs are columns 4gq.. of the pair.
+// Block 0 is finished (scaled by its d) before block 1 starts, so only two
+// packed accumulators and nine words are live at a time.
+template <class XP>
+__device__ __forceinline__ float q8_0_dot_pair(uint32_t a, XP &&xp)
+{
+    float r;
+    {
+        uint32_t w[9];
+#pragma unroll
+        for (int i = 0; i < 9; ++i) w[i] = lds_u32(a + 4u * (uint32_t)i);
+        float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int gq = 0; gq < 8; ++gq) {           // bytes 2 + 4gq .. 5 + 4gq of the pair
+            float2 p02, p13, x02, x13;
+            bytes4_to_f2(__byte_perm(w[gq], w[gq + 1], 0x5432u) ^ 0x80808080u, 128.0f, p02, p13);
+            xp(gq, x02, x13);
+            s0 = f2fma(p02, x02, s0);
+            s1 = f2fma(p13, x13, s1);
+        }
+        r = half_bits_to_float(w[0]) * hsum2(s0, s1);
+    }
+    const float d1 = half_bits_to_float(lds_u32(a + 32u) >> 16);
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = lds_u32(a + 36u + 4u * (uint32_t)i);
+    float2 t0 = make_float2(0.f, 0.f), t1 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int gq = 0; gq < 8; ++gq) {               // aligned words 9 + gq
+        float2 p02, p13, x02, x13;
+        bytes4_to_f2(w[gq] ^ 0x80808080u, 128.0f, p02, p13);
+        xp(8 + gq, x02, x13);
+        t0 = f2fma(p02, x02, t0);
+        t1 = f2fma(p13, x13, t1);
+    }
+    return fmaf(d1, hsum2(t0, t1), r);
+}
+
+// Q4_K slice (chunk c of the superblock at shared address sb, 16-byte
+// aligned).  Each nibble becomes a float with one bitwise instruction: masked
+// in place under the exponent of 2^23 it reads 2^23 + q * 2^e, where e is the
+// nibble's bit offset (the upper three nibbles of a word are first shifted
+// down by 12 bits so that every field stays below bit 20); one packed
+// subtraction leaves q * 2^e exactly.  The x values in registers were scaled
+// by 2^-e to match (rw_scale_x_q4_k: exact powers of two), so each product is
+// q * x exactly as with unscaled operands.  xsa / xsb: the unscaled sums of the
+// slice's low / high 32 x (the min terms).
+//   word byte j: low nibble (bits 8j..8j+3)   -> column 4i + j      of the slice
+//                high nibble (bits 8j+4..8j+7) -> column 32 + 4i + j
+template <class XP>
+__device__ __forceinline__ float q4_k_dot_rw(uint32_t sb, int c, const Q4kSel &sel, XP &&xp, float xsa, float xsb)
+{
+    const uint32_t M = 0x4B000000u;
+    const float2 nm = make_float2(-8388608.0f, -8388608.0f);
+    float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+    float2 b0 = make_float2(0.f, 0.f), b1 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint4 q = lds_v4(sb + 16u + 32u * (uint32_t)c + 16u * (uint32_t)h);
+        const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t w = qw[i], w2 = qw[i] >> 12;
+            const float2 lo02 = f2add(make_float2(__uint_as_float((w & 0x0000000Fu) | M),
+                                                  __uint_as_float((w & 0x000F0000u) | M)), nm);
+            const float2 lo13 = f2add(make_float2(__uint_as_float((w & 0x00000F00u) | M),
+                                                  __uint_as_float((w2 & 0x0000F000u) | M)), nm);
+            const float2 hi02 = f2add(make_float2(__uint_as_float((w & 0x000000F0u) | M),
+                                                  __uint_as_float((w2 & 0x00000F00u) | M)), nm);
+            const float2 hi13 = f2add(make_float2(__uint_as_float((w & 0x0000F000u) | M),
+                                                  __uint_as_float((w2 & 0x000F0000u) | M)), nm);
+            float2 xl02, xl13, xh02, xh13;
+            xp(4 * h + i, xl02, xl13);
+            xp(8 + 4 * h + i, xh02, xh13);
+            a0 = f2fma(lo02, xl02, a0);
+            a1 = f2fma(lo13, xl13, a1);
+            b0 = f2fma(hi02, xh02, b0);
+            b1 = f2fma(hi13, xh13, b1);
+        }
+    }
+    const float sa = hsum2(a0, a1), sbv = hsum2(b0, b1);
+    const uint4 hdr = lds_v4(sb);
+    const uint32_t v = q4k_scales_mins(hdr.y, hdr.z, hdr.w, sel);   // bytes [sc0, sc1, m0, m1]
+    float2 sc0_m0, sc1_m1;
+    bytes4_to_f2(v, 0.0f, sc0_m0, sc1_m1);
+    const float d = half_bits_to_float(hdr.x);
+    const float dmin = half_bits_to_float(hdr.x >> 16);
+    float r = (d * sc0_m0.x) * sa;
+    r = fmaf(d * sc1_m1.x, sbv, r);
+    r = fmaf(-dmin * sc0_m0.y, xsa, r);
+    r = fmaf(-dmin * sc1_m1.y, xsb, r);
+    return r;
+}
+
+// The matching x scaling (see q4_k_dot_rw): groups 0..7 (low nibbles) by
+// (2^0, 2^-16) / (2^-8, 2^-12), groups 8..15 (high) by (2^-4, 2^-8) / (2^-12, 2^-16).
+__device__ __forceinline__ void rw_scale_x_q4_k(float2 (&xr)[16][2])
+{
+#pragma unroll
+    for (int gq = 0; gq < 16; ++gq) {
+        const bool lo = gq < 8;
+        xr[gq][0] = __fmul2_rn(xr[gq][0], lo ? make_float2(1.0f, 0x1p-16f) : make_float2(0x1p-4f, 0x1p-8f));
+        xr[gq][1] = __fmul2_rn(xr[gq][1], lo ? make_float2(0x1p-8f, 0x1p-12f) : make_float2(0x1p-12f, 0x1p-16f));
+    }
+}
+
+// Column (within the K-chunk) of x group gq of lane l's 64-weight slice.
+template <int FMT>
+__device__ __forceinline__ int rw_group_col(int l, int gq)
+{
+    if (FMT == FMT_Q8_0) return 64 * l + 4 * gq;
+    return slice1_group_col<FMT>(l, gq);
+}
+
+// Shared address of lane l's slice within one row of a stage.
+template <int FMT>
+__device__ __forceinline__ uint32_t rw_slice_addr(uint32_t rowp, int l)
+{
+    if (FMT == FMT_Q8_0) return rowp + 68u * (uint32_t)l;
+    if (FMT == FMT_Q4_K) return rowp + 144u * (uint32_t)(l >> 2);
+    return rowp + 210u * (uint32_t)(l >> 2);
+}
+
+// Lane l's x slice of K-chunk kc in registers (zeros where the chunk is short),
+// with the Q4_K half sums.  Chained launches read x through L2 only: it may
+// have been written by another SM earlier in the same launch.
+template <int FMT>
+__device__ __forceinline__ void rw_load_x(const float *x, int kc, int ncols, bool coherent, int lane,
+                                          float2 (&xr)[16][2], float &xsa, float &xsb)
+{
+    const bool have = 64 * (lane + 1) <= ncols;
+    float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
+    const float *xc = x + (int64_t)kc * RW_CK;
+#pragma unroll
+    for (int gq = 0; gq < 16; ++gq) {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (have) {
+            const float4 *src = reinterpret_cast<const float4 *>(xc + rw_group_col<FMT>(lane, gq));
+            v = coherent ? __ldcg(src) : __ldg(src);
+        }
+        xr[gq][0] = make_float2(v.x, v.z);
+        xr[gq][1] = make_float2(v.y, v.w);
+        if (gq < 8) sa = f2add(sa, f2add(xr[gq][0], xr[gq][1]));
+        else sb = f2add(sb, f2add(xr[gq][0], xr[gq][1]));
+    }
+    xsa = sa.x + sa.y;
+    xsb = sb.x + sb.y;
+    if (FMT == FMT_Q4_K) rw_scale_x_q4_k(xr);
+}
+
+// x of a task longer than one K-chunk sits in shared memory for the whole task
+// (all warps read every K-chunk of it).  float4 f of the row is stored at
+// f ^ ((f >> 4) & 7): the eight lanes of a quarter-warp that read the same
+// group of their 64-column slices hit eight different bank groups.
+__device__ __forceinline__ uint32_t rw_xswz(uint32_t f) { return f ^ ((f >> 4) & 7u); }
+
+__device__ __forceinline__ void rw_stage_x(uint32_t xs, const float *x, int cols, bool coherent)
+{
+    for (int f = (int)threadIdx.x; f < (cols >> 2); f += NTHREADS) {
+        const float4 *src = reinterpret_cast<const float4 *>(x) + f;
+        sts_f4(xs + 16u * rw_xswz((uint32_t)f), coherent ? __ldcg(src) : __ldg(src));
+    }
+}
+
+template <int FMT>
+__device__ __forceinline__ void rw_load_x_smem(uint32_t xs, int kc, int ncols, int lane, float2 (&xr)[16][2],
+                                               float &xsa, float &xsb)
+{
+    const bool have = 64 * (lane + 1) <= ncols;
+    float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int gq = 0; gq < 16; ++gq) {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (have) v = lds_f4(xs + 16u * rw_xswz((uint32_t)((kc * RW_CK + rw_group_col<FMT>(lane, gq)) >> 2)));
+        xr[gq][0] = make_float2(v.x, v.z);
+        xr[gq][1] = make_float2(v.y, v.w);
+        if (gq < 8) sa = f2add(sa, f2add(xr[gq][0], xr[gq][1]));
+        else sb = f2add(sb, f2add(xr[gq][0], xr[gq][1]));
+    }
+    xsa = sa.x + sa.y;
+    xsb = sb.x + sb.y;
+    if (FMT == FMT_Q4_K) rw_scale_x_q4_k(xr);
+}
+
+// Grid-wide barrier of an ordered chained launch (all CTAs co-resident:
+// cooperative launch).  sync[0] counts arrivals and only grows within a
+// launch: barrier k is passed once it reaches (k + 1) * n_ctas.  One thread
+// per CTA fences the CTA's writes, adds its arrival, polls with relaxed loads
+// and fences once more on the way out; the last CTA to leave the kernel
+// (sync[1]) puts both words back to zero for the next launch.  A wait gives
+// up after about a second and returns false (the caller records the error;
+// the kernel still finishes).
+__device__ __forceinline__ bool rw_grid_barrier(unsigned *sync, unsigned target)
+{
+    bool ok = true;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" :: "l"(sync) : "memory");
+        uint64_t t0 = 0;
+        for (uint32_t i = 0;; ++i) {
+            unsigned c;
+            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(sync) : "memory");
+            if ((int)(c - target) >= 0) break;
+            if ((i & 63u) == 0u) {
+                const uint64_t now = global_timer_ns();
+                if (i == 0u) t0 = now;
+                else if (now - t0 > 1000000000ull) {
+                    ok = false;
+                    break;
+                }
+            }
+        }
+        __threadfence();
+    }
+    __syncthreads();
+    return ok;
+}
+
+__device__ __forceinline__ void rw_grid_exit(unsigned *sync, unsigned n_ctas)
+{
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const unsigned old = atomicAdd(sync + 1, 1u);
+        if (old == n_ctas - 1u) {       // every CTA has passed its last barrier
+            atomicExch(sync, 0u);
+            atomicExch(sync + 1, 0u);
+        }
+    }
+}
+
+template <int FMT, int R, int NT>
+__global__ void __launch_bounds__(NTHREADS, 2) qmv_rw_kernel(const __grid_constant__ RwParamsT<NT> p)
+{
+    static_assert(R == 1 || R == 2 || R == 4 || R == 8, "R");
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int warp = (int)threadIdx.x >> 5, lane = (int)threadIdx.x & 31;
+    const uint32_t sraw = smem_addr(smem);
+    const uint32_t sbase = (sraw + 127u) & ~127u;          // the launch adds 128 spare bytes
+    const int S = p.n_stage;
+    const uint32_t full0 = sbase + 8u * (uint32_t)(warp * RW_MAX_STAGES);
+    RwTask *const tasks = reinterpret_cast<RwTask *>(smem + (sbase - sraw) + RW_BAR_BYTES);
+    const uint32_t xs = sbase + (uint32_t)rw_hdr_bytes(p.n_tasks);
+    const uint32_t x_area = (uint32_t)(((p.x_floats * 4) + 127) & ~127);
+    const uint32_t stage0 = xs + x_area + (uint32_t)(warp * S) * (uint32_t)p.stage_pitch;
+
+    int t_begin, t_end, wg;
+    if (p.chain) {
+        t_begin = 0;
+        t_end = p.n_tasks;
+        wg = (int)blockIdx.x * NW + warp;
+    } else {
+        int t = 0;
+        while (t + 1 < p.n_tasks && (int)blockIdx.x >= p.cta_begin[t + 1]) ++t;
+        t_begin = t;
+        t_end = t + 1;
+        wg = ((int)blockIdx.x - p.cta_begin[t]) * NW + warp;
+    }
+
+    {
+        const uint4 *src = reinterpret_cast<const uint4 *>(&p.t[0]);
+        uint4 *dst = reinterpret_cast<uint4 *>(tasks);
+        for (int i = (int)threadIdx.x; i < p.n_tasks * (int)(sizeof(RwTask) / 16); i += NTHREADS) dst[i] = src[i];
+    }
+    if (lane == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(full0 + 8u * (uint32_t)s, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    pdl_launch_dependents();
+
+    // The producer cursor lives in shared memory and only lane 0 touches it
+    // (keeps the consumer's registers for x and the decode).
+    RwCursor *const cur = reinterpret_cast<RwCursor *>(smem + (sbase - sraw) + RW_CUR_OFF) + warp;
+    // prologue: the first S tiles (weights only: no dependence on earlier kernels)
+    if (lane == 0) {
+        RwCursor f;
+        rw_seek(tasks, f, t_begin, t_end, wg);
+        f.issued = 0;
+        for (int s = 0; s < S && f.t < t_end; ++s) {
+            rw_issue<R>(tasks, f, stage0 + (uint32_t)s * (uint32_t)p.stage_pitch, full0 + 8u * (uint32_t)s);
+            rw_advance(tasks, f, t_end, wg);
+            ++f.issued;
+        }
+        *cur = f;
+    }
+    int consumed = 0;
+
+    pdl_wait();                                    // x is the previous kernel's output
+    const Q4kSel sel = q4k_sel(lane & 3);
+    const bool coherent = p.ordered != 0;
+    bool dead = false;
+    int slot = 0;
+    uint32_t phase = 0;
+    const uint32_t pitch = (uint32_t)p.stage_pitch;
+
+    float2 xr[16][2];
+    float xsa = 0.f, xsb = 0.f;
+    for (int t = t_begin; t < t_end; ++t) {
+        if (p.ordered && t > t_begin) {
+            if (!rw_grid_barrier(p.sync, (unsigned)(t - t_begin) * gridDim.x) && threadIdx.x == 0)
+                atomicOr(p.err, DEVERR_TIMEOUT);
+        }
+        const RwTask &tk = tasks[t];
+        const int nch = tk.n_chunks;
+        if (nch > 1) {
+            // every warp of the CTA takes part (the task's x for all K-chunks)
+            rw_stage_x(xs, tk.x, (nch - 1) * RW_CK + tk.last_cols, coherent);
+            __syncthreads();
+        }
+        int64_t a, b;
+        rw_range(tk, wg, a, b);
+        if (a >= b || dead) {
+            if (nch > 1) __syncthreads();         // matches the one after the task below
+            continue;
+        }
+        // the task's fields, once
+        const float *tx = tk.x;
+        float *ty = tk.y;
+        const int64_t rows = tk.rows;
+        const int last_cols = tk.last_cols;
+        const uint32_t last_bytes = (uint32_t)tk.last_bytes;
+        const uint32_t chunk_bytes = (uint32_t)tk.chunk_bytes;
+        // one tile: wait for the stage, decode R rows of it, hand the stage back
+        // to the producer (refilled with the tile S ahead)
+        auto tile = [&](float (&acc)[R], int ncols, uint32_t cb) -> bool {
+            const uint32_t full = full0 + 8u * (uint32_t)slot;
+            // every lane times its own wait: agree on the outcome so the warp stays converged
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(full, phase))) {
+                if (lane == 0) atomicOr(p.err, DEVERR_TIMEOUT);
+                return false;
+            }
+            ++consumed;
+            const uint32_t st = stage0 + (uint32_t)slot * pitch;
+            if (64 * (lane + 1) <= ncols) {
+                auto xp = [&](int gq, float2 &x02, float2 &x13) {
+                    x02 = xr[gq][0];
+                    x13 = xr[gq][1];
+                };
+                uint32_t sa = rw_slice_addr<FMT>(st, lane);
+#pragma unroll
+                for (int k = 0; k < R; ++k, sa += cb) {
+                    if (FMT == FMT_Q8_0) acc[k] += q8_0_dot_pair(sa, xp);
+                    else if (FMT == FMT_Q4_K) acc[k] += q4_k_dot_rw(sa, lane & 3, sel, xp, xsa, xsb);
+                    else acc[k] += q6_k_dot1(sa, (lane >> 1) & 1, 16 * (lane & 1), xp);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) {
+                RwCursor f = *cur;
+                if (f.t < t_end) {
+                    fence_proxy_async_smem();
+                    rw_issue<R>(tasks, f, st, full);
+                    rw_advance(tasks, f, t_end, wg);
+                    ++f.issued;
+                    *cur = f;
+                }
+            }
+            if (++slot == S) {
+                slot = 0;
+                phase ^= 1u;
+            }
+            return true;
+        };
+        auto finish = [&](float (&acc)[R], int64_t rg) {
+            warp_transpose_reduce<R>(acc, lane);
+            constexpr int SH = 5 - Log2<R>::v;
+            const int64_t row = rg * R + (lane >> SH);
+            if ((lane & ((1 << SH) - 1)) == 0 && row < rows) ty[row] = acc[0];
+        };
+        if (nch == 1) {
+            // x stays in registers for the whole task
+            rw_load_x<FMT>(tx, 0, last_cols, coherent, lane, xr, xsa, xsb);
+            for (int64_t rg = a; rg < b; ++rg) {
+                float acc[R];
+#pragma unroll
+                for (int k = 0; k < R; ++k) acc[k] = 0.f;
+                if (!tile(acc, last_cols, last_bytes)) {
+                    dead = true;
+                    break;
+                }
+                finish(acc, rg);
+            }
+        } else {
+            for (int64_t rg = a; rg < b && !dead; ++rg) {
+                float acc[R];
+#pragma unroll
+                for (int k = 0; k < R; ++k) acc[k] = 0.f;
+                for (int kc = 0; kc < nch; ++kc) {
+                    const bool lastc = kc == nch - 1;
+                    const int ncols = lastc ? last_cols : RW_CK;
+                    rw_load_x_smem<FMT>(xs, kc, ncols, lane, xr, xsa, xsb);
+                    if (!tile(acc, ncols, lastc ? last_bytes : chunk_bytes)) {
+                        dead = true;
+                        break;
+                    }
+                }
+                if (!dead) finish(acc, rg);
+            }
+            __syncthreads();                      // x stays until every warp is done with it
+        }
+    }
+    if (p.ordered) rw_grid_exit(p.sync, gridDim.x);
+    // after a timeout: let the copies still in flight land before the CTA exits
+    if (dead) {
+        int pending = __shfl_sync(0xFFFFFFFFu, lane == 0 ? cur->issued : 0, 0) - consumed;
+        for (; pending > 0; --pending) {
+            (void)mbar_wait_bounded(full0 + 8u * (uint32_t)slot, phase);
+            if (++slot == S) {
+                slot = 0;
+                phase ^= 1u;
+            }
+        }
+    }
+}
+
+// Defined per format in qmv_fmt_*.cu.
+template <int FMT, int NT>
+cudaError_t launch_rw(const RwParamsT<NT> &p, int R, dim3 grid, size_t smem, cudaStream_t stream, bool pdl,
+                      bool cooperative);
+template <int FMT>
+cudaError_t rw_occupancy(int R, size_t smem, int *ctas_per_sm);
+
+}  // namespace qmv

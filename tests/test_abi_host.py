@@ -105,6 +105,23 @@ def test_multi_argument_validation(L):
     q.lib().qmv_debug_fail_next_launches(0)
 
 
+def test_chain_argument_validation(L):
+    T = q.make_tasks([(A, 4, 256, A, A), (A, 8, 512, A, A)])
+    assert L.qmv_chain(1, None, 2, None) == NULL
+    assert L.qmv_chain(1, T, 0, None) == SHAPE
+    assert L.qmv_chain(1, T, 4097, None) == SHAPE
+    assert L.qmv_chain(5, T, 2, None) == FMT
+    bad = q.make_tasks([(A, 4, 256, A, A), (A, 8, 500, A, A)])
+    assert L.qmv_chain(1, bad, 2, None) == SHAPE
+    bad = q.make_tasks([(A, 4, 256, A, A), (A + 8, 8, 512, A, A)])
+    assert L.qmv_chain(1, bad, 2, None) == ALIGN
+    bad = q.make_tasks([(A, 4, 256, A, A), (A, 8, 512, A, None)])
+    assert L.qmv_chain(1, bad, 2, None) == NULL
+    q.lib().qmv_debug_fail_next_launches(1)
+    assert L.qmv_chain(1, T, 2, None) == CUDA
+    q.lib().qmv_debug_fail_next_launches(0)
+
+
 def test_injected_launch_failure_is_reported(L):
     q.lib().qmv_debug_fail_next_launches(2)
     assert qb(L) == CUDA

@@ -206,6 +206,74 @@ def test_qmv_multi_many_tasks_and_errors():
         q.qmv_multi(fmt, 9, tasks[:2])
 
 
+# ------------------------------------------------------- chained launch --
+
+def _chain_case(fmt, dims, seed):
+    """Tasks t = 0..len(dims)-2 with W_t of shape dims[t+1] x dims[t]; task t
+    reads task t-1's output as x (task 0 reads a fresh x).  Outputs start as NaN,
+    so a task that ran before its input was complete would be caught."""
+    Ws, dev_args = [], []
+    x0 = synth.gen_x(1, dims[0], seed, 99)[0]
+    bufs = [dev(x0)] + [torch.full((d,), float("nan"), device="cuda") for d in dims[1:]]
+    for t in range(len(dims) - 1):
+        cols, rows = dims[t], dims[t + 1]
+        W = synth.gen_blocks(fmt, rows, cols, seed, t)
+        Wd = dev(W)
+        Ws.append((W, Wd))
+        dev_args.append((Wd, rows, cols, bufs[t], bufs[t + 1]))
+    q.qmv_chain(fmt, dev_args)
+    torch.cuda.synchronize()
+    outs = [b.cpu().numpy() for b in bufs]
+    worst = 0.0
+    for t in range(len(dims) - 1):
+        # each step against the oracle on the input the GPU actually had
+        ref, bound = oracle.qmv(fmt, Ws[t][0], dims[t + 1], dims[t], outs[t][None, :])
+        worst = max(worst, within(outs[t + 1][None, :], ref, bound))
+    return worst
+
+
+@pytest.mark.parametrize("fmt", [Q8_0, Q4_K, Q6_K])
+def test_qmv_chain_dependent_tasks(fmt):
+    # x of every task is the previous task's y: the grid barrier must order them
+    dims = [2048, 3072, 2048, 16384, 2048, 8192, 2048] if fmt != Q6_K else [2048, 4096, 2048, 6144, 2048]
+    _chain_case(fmt, dims, 80 + fmt)
+
+
+def test_qmv_chain_crosses_launch_split():
+    # 70 tasks (more than one persistent launch holds) on 512 x 512 Q4_K
+    # matrices; task t reads task t-1's output unless t % 3 == 0 (then a fresh
+    # x), so activations stay finite and task 64 depends on task 63 across the
+    # launch boundary
+    fmt, n, T = Q4_K, 512, 70
+    x0 = synth.gen_x(1, n, 93, 0)[0]
+    x0d = dev(x0)
+    ys = torch.full((T, n), float("nan"), device="cuda")
+    Ws, args = [], []
+    for t in range(T):
+        W = synth.gen_blocks(fmt, n, n, 93, 1 + t)
+        Wd = dev(W)
+        Ws.append(W)
+        args.append((Wd, n, n, x0d if t % 3 == 0 else ys[t - 1], ys[t]))
+    q.qmv_chain(fmt, args)
+    torch.cuda.synchronize()
+    yh = ys.cpu().numpy()
+    for t in range(T):
+        xin = x0 if t % 3 == 0 else yh[t - 1]
+        ref, bound = oracle.qmv(fmt, Ws[t], n, n, xin[None, :])
+        within(yh[t][None, :], ref, bound)
+
+
+def test_qmv_chain_fallback_shape_keeps_order():
+    # 96 columns is not a whole number of Q8_0 block pairs: one launch per task
+    dims = [1024, 96, 2048, 1024]
+    _chain_case(Q8_0, dims, 91)
+
+
+def test_qmv_chain_repeated_calls_reuse_the_barrier():
+    for rep in range(3):
+        _chain_case(Q8_0, [1024, 2048, 512, 1024], 92 + rep)
+
+
 # ---------------------------------------------------- full-size workloads --
 
 def test_cfg0_q8_0_1024x1024():
