@@ -4,13 +4,19 @@
 Headline step: the full decode-step matvec sweep of a 16-layer dense stack
 (hidden 2048, intermediate 8192, 32 query / 8 KV heads of head_dim 64), all
 weights Q8_0, one token: per layer the fused QKV 3072x2048, O 2048x2048, fused
-gate/up 16384x2048 and down 2048x8192 matvecs -- 64 launches, 1.034 GB of
-weights per step (larger than the 126 MB L2, so no flush is needed).  The step
-is captured once as a CUDA graph of the library's C-ABI calls and replayed.
+gate/up 16384x2048 and down 2048x8192 matvecs -- 64 matvecs, 1.034 GB of
+weights per step (larger than the 126 MB L2, so no flush is needed) -- run in
+decode order (each matvec starts after the previous one is complete, as its
+input would be the previous output in a model): by default as one qmv_chain
+call (a persistent launch with a grid barrier between matvecs), or with
+--mode launches as 64 separate calls.  The step is captured once as a CUDA
+graph of the library's C-ABI calls and replayed.
 Metric: weight bytes streamed per second (GB/s), with the fraction of the
 measured HBM peak.  The other workloads (Q8_0 1024^2, Q4_K fused QKV, Q6_K
 vocab projection at 1 and 4 tokens, the MoE FFN step, the sweep at 2/4/8
-tokens) are measured in the same run and reported under "per_config".
+tokens, and the sweep as independent grouped launches -- an upper bound for
+matvecs that need no ordering) are measured in the same run and reported
+under "per_config".
 
   python bench.py [--gpus N --steps K --warmup W]      # our CUDA path
   python bench.py --impl reference ...                   # the oracle on host cores
@@ -460,6 +466,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--n-tok", type=int, default=1)
+    ap.add_argument("--mode", choices=["auto", "chain", "launches"], default="auto",
+                    help="how the step runs, in decode order either way: 'chain' = qmv_chain "
+                         "(persistent, grid barrier between matvecs; one token), 'launches' = one "
+                         "library call per matvec; auto = chain for one token, else launches")
     ap.add_argument("--headline-only", action="store_true",
                     help="skip the per-config measurements and the CPU baseline")
     ap.add_argument("--profile-case", choices=["q8_0", "q4_k", "q6_k", "q8_0_down", "q8_0_o"])
@@ -481,7 +491,9 @@ def main():
     props = torch.cuda.get_device_properties(torch.cuda.current_device())
     cache = {}
 
+    mode = args.mode if args.mode != "auto" else ("chain" if args.n_tok == 1 else "launches")
     sweep = Sweep(torch, q, args.n_tok, cache)
+    sweep.set_mode(mode)
     graph = capture(torch, lambda: sweep.step(), stream)
     assert q.qmv_check(stream) == 0
 
@@ -499,7 +511,8 @@ def main():
         dist.barrier(torch)
         sec = dist.max(torch, sec)
         # the dominant kernel: every launch of the step, event-timed on its stream
-        durs = per_launch_durations(torch, sweep, stream)
+        durs = per_launch_durations(torch, sweep, stream) if mode == "launches" else [
+            time_graph(torch, graph, 20, stream) / 20]
         # end to end: pinned x -> device, the step's library calls, y -> pinned host
         e2e_reps = max(3, min(200, args.steps // 5))
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -521,14 +534,21 @@ def main():
                     torch, q, stream, Q6_K, 128000, 2048, nt, 2, reps=20)
             per_config["cfg3_moe_ffn_step"] = measure_moe(torch, q, stream)
             for nt in (1, 2, 4, 8):
-                if nt == args.n_tok:
-                    continue
                 sw = Sweep(torch, q, nt, cache)
-                gr = capture(torch, lambda: sw.step(), stream)
-                s2 = time_graph(torch, gr, max(3, args.steps // 10), stream) / max(3, args.steps // 10)
-                per_config[f"cfg4_sweep_ntok{nt}"] = {"us": s2 * 1e6, "weight_gbs": sw.weight_bytes / s2 / 1e9,
-                                                      "launches": sw.launches}
-                del gr, sw
+                for md in (("launches", "chain", "grouped") if nt == 1 else ("launches", "grouped")):
+                    if nt == args.n_tok and md == mode:
+                        continue
+                    sw.set_mode(md)
+                    gr = capture(torch, lambda: sw.step(), stream)
+                    reps = max(3, args.steps // 10)
+                    s2 = time_graph(torch, gr, reps, stream) / reps
+                    key = f"cfg4_sweep_ntok{nt}" + ("" if md == "launches" else f"_{md}")
+                    per_config[key] = {"us": s2 * 1e6, "weight_gbs": sw.weight_bytes / s2 / 1e9,
+                                       "launches": sw.launches, "mode": md,
+                                       "order": "independent (grouped, no ordering)" if md == "grouped"
+                                       else "decode order"}
+                    del gr
+                del sw
     clocks = clk.summary()
     assert q.qmv_check(stream) == 0
 
@@ -542,9 +562,9 @@ def main():
             t = json.load(f)
         if t.get("source_hash") == source_hash() and t.get("n_tok") == args.n_tok:
             traffic = t.get("step_traffic_bytes_per_launch")
-    cfg4_key = f"cfg4_sweep_ntok{args.n_tok}"
+    cfg4_key = f"cfg4_sweep_ntok{args.n_tok}" + ("" if mode == "launches" else f"_{mode}")
     per_config[cfg4_key] = {"us": ms_per_step * 1e3, "weight_gbs": sweep.weight_bytes / (sec / args.steps) / 1e9,
-                            "launches": sweep.launches}
+                            "launches": sweep.launches, "mode": mode, "order": "decode order"}
     for v in per_config.values():
         if "weight_gbs" in v:
             v["frac_of_hbm_peak"] = round(v["weight_gbs"] / hbm_peak, 4)
@@ -565,13 +585,16 @@ def main():
                    "weight_bytes_per_step": sweep.weight_bytes, "launches_per_step": sweep.launches,
                    "l2": "inputs larger than L2 (1.03 GB of weights per step, L2 126 MB)",
                    "timing": "CUDA graph of the step's C-ABI calls, replayed; CUDA events on the launch stream",
+                   "mode": mode,
+                   "order": "decode order: every matvec starts after the previous one has finished",
                    "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"},
         "frac_of_hbm_peak": round(value / dist.world / hbm_peak, 4),
         "us_per_step": round(ms_per_step * 1e3, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6.65 TB/s",
-                     "kernel": "qmv_pipeline_kernel (Q8_0, every launch of the step)",
+                     "kernel": ("qmv_rw_kernel, chained (Q8_0, the whole step in one launch)" if mode == "chain"
+                                else "the step's matvec launches (Q8_0)"),
                      "algorithmic_bytes_per_step": sweep.algo,
                      "mean_launch_us": round(sum(durs) / len(durs) * 1e6, 3)},
         "e2e": {"value": round(sweep.weight_bytes * dist.world / e2e_sec / 1e9, 1), "unit": "GB/s",

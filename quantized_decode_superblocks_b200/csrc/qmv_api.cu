@@ -231,7 +231,9 @@ int launch_plan(int fmt, const Plan &pl, cudaStream_t stream)
 // Warp-private-ring kernel (one token, one matrix per task): tile = R rows x a
 // K-chunk of up to 2048 columns; per warp S stages.  R and S depend only on the
 // format (the bytes of a full K-chunk), so tasks of one format share them.
-constexpr int64_t RW_CTA_SMEM = 112 * 1024;      // per CTA, two CTAs per SM
+// Dynamic shared memory of one CTA, two per SM: (228 KB - 2 x 1 KB reserved) / 2
+// = 113 KB, less the 128 bytes of alignment slack each launch adds.
+constexpr int64_t RW_CTA_SMEM = 113 * 1024 - 128;
 
 struct RwGeom {
     int R = 0;

@@ -196,74 +196,6 @@ __device__ __forceinline__ float q8_0_dot_pair(uint32_t a, XP &&xp)
     return fmaf(d1, hsum2(t0, t1), r);
 }
 
-// Q4_K slice (chunk c of the superblock at shared address sb, 16-byte
-// aligned).  Each nibble becomes a float with one bitwise instruction: masked
-// in place under the exponent of 2^23 it reads 2^23 + q * 2^e, where e is the
-// nibble's bit offset (the upper three nibbles of a word are first shifted
-// down by 12 bits so that every field stays below bit 20); one packed
-// subtraction leaves q * 2^e exactly.  The x values in registers were scaled
-// by 2^-e to match (rw_scale_x_q4_k: exact powers of two), so each product is
-// q * x exactly as with unscaled operands.  xsa / xsb: the unscaled sums of the
-// slice's low / high 32 x (the min terms).
-//   word byte j: low nibble (bits 8j..8j+3)   -> column 4i + j      of the slice
-//                high nibble (bits 8j+4..8j+7) -> column 32 + 4i + j
-template <class XP>
-__device__ __forceinline__ float q4_k_dot_rw(uint32_t sb, int c, const Q4kSel &sel, XP &&xp, float xsa, float xsb)
-{
-    const uint32_t M = 0x4B000000u;
-    const float2 nm = make_float2(-8388608.0f, -8388608.0f);
-    float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
-    float2 b0 = make_float2(0.f, 0.f), b1 = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const uint4 q = lds_v4(sb + 16u + 32u * (uint32_t)c + 16u * (uint32_t)h);
-        const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t w = qw[i], w2 = qw[i] >> 12;
-            const float2 lo02 = f2add(make_float2(__uint_as_float((w & 0x0000000Fu) | M),
-                                                  __uint_as_float((w & 0x000F0000u) | M)), nm);
-            const float2 lo13 = f2add(make_float2(__uint_as_float((w & 0x00000F00u) | M),
-                                                  __uint_as_float((w2 & 0x0000F000u) | M)), nm);
-            const float2 hi02 = f2add(make_float2(__uint_as_float((w & 0x000000F0u) | M),
-                                                  __uint_as_float((w2 & 0x00000F00u) | M)), nm);
-            const float2 hi13 = f2add(make_float2(__uint_as_float((w & 0x0000F000u) | M),
-                                                  __uint_as_float((w2 & 0x000F0000u) | M)), nm);
-            float2 xl02, xl13, xh02, xh13;
-            xp(4 * h + i, xl02, xl13);
-            xp(8 + 4 * h + i, xh02, xh13);
-            a0 = f2fma(lo02, xl02, a0);
-            a1 = f2fma(lo13, xl13, a1);
-            b0 = f2fma(hi02, xh02, b0);
-            b1 = f2fma(hi13, xh13, b1);
-        }
-    }
-    const float sa = hsum2(a0, a1), sbv = hsum2(b0, b1);
-    const uint4 hdr = lds_v4(sb);
-    const uint32_t v = q4k_scales_mins(hdr.y, hdr.z, hdr.w, sel);   // bytes [sc0, sc1, m0, m1]
-    float2 sc0_m0, sc1_m1;
-    bytes4_to_f2(v, 0.0f, sc0_m0, sc1_m1);
-    const float d = half_bits_to_float(hdr.x);
-    const float dmin = half_bits_to_float(hdr.x >> 16);
-    float r = (d * sc0_m0.x) * sa;
-    r = fmaf(d * sc1_m1.x, sbv, r);
-    r = fmaf(-dmin * sc0_m0.y, xsa, r);
-    r = fmaf(-dmin * sc1_m1.y, xsb, r);
-    return r;
-}
-
-// The matching x scaling (see q4_k_dot_rw): groups 0..7 (low nibbles) by
-// (2^0, 2^-16) / (2^-8, 2^-12), groups 8..15 (high) by (2^-4, 2^-8) / (2^-12, 2^-16).
-__device__ __forceinline__ void rw_scale_x_q4_k(float2 (&xr)[16][2])
-{
-#pragma unroll
-    for (int gq = 0; gq < 16; ++gq) {
-        const bool lo = gq < 8;
-        xr[gq][0] = __fmul2_rn(xr[gq][0], lo ? make_float2(1.0f, 0x1p-16f) : make_float2(0x1p-4f, 0x1p-8f));
-        xr[gq][1] = __fmul2_rn(xr[gq][1], lo ? make_float2(0x1p-8f, 0x1p-12f) : make_float2(0x1p-12f, 0x1p-16f));
-    }
-}
-
 // Column (within the K-chunk) of x group gq of lane l's 64-weight slice.
 template <int FMT>
 __device__ __forceinline__ int rw_group_col(int l, int gq)
@@ -305,7 +237,6 @@ __device__ __forceinline__ void rw_load_x(const float *x, int kc, int ncols, boo
     }
     xsa = sa.x + sa.y;
     xsb = sb.x + sb.y;
-    if (FMT == FMT_Q4_K) rw_scale_x_q4_k(xr);
 }
 
 // x of a task longer than one K-chunk sits in shared memory for the whole task
@@ -339,7 +270,6 @@ __device__ __forceinline__ void rw_load_x_smem(uint32_t xs, int kc, int ncols, i
     }
     xsa = sa.x + sa.y;
     xsb = sb.x + sb.y;
-    if (FMT == FMT_Q4_K) rw_scale_x_q4_k(xr);
 }
 
 // Grid-wide barrier of an ordered chained launch (all CTAs co-resident:
@@ -355,23 +285,20 @@ __device__ __forceinline__ bool rw_grid_barrier(unsigned *sync, unsigned target)
     bool ok = true;
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence();
+        asm volatile("fence.acq_rel.gpu;" ::: "memory");
         asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" :: "l"(sync) : "memory");
-        uint64_t t0 = 0;
-        for (uint32_t i = 0;; ++i) {
+        // bounded by the SM cycle counter (cheap to read): about a second at 2 GHz
+        const long long c0 = clock64();
+        for (;;) {
             unsigned c;
             asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(sync) : "memory");
             if ((int)(c - target) >= 0) break;
-            if ((i & 63u) == 0u) {
-                const uint64_t now = global_timer_ns();
-                if (i == 0u) t0 = now;
-                else if (now - t0 > 1000000000ull) {
-                    ok = false;
-                    break;
-                }
+            if (clock64() - c0 > 2000000000LL) {
+                ok = false;
+                break;
             }
         }
-        __threadfence();
+        asm volatile("fence.acq_rel.gpu;" ::: "memory");
     }
     __syncthreads();
     return ok;
@@ -501,7 +428,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) qmv_rw_kernel(const __grid_consta
 #pragma unroll
                 for (int k = 0; k < R; ++k, sa += cb) {
                     if (FMT == FMT_Q8_0) acc[k] += q8_0_dot_pair(sa, xp);
-                    else if (FMT == FMT_Q4_K) acc[k] += q4_k_dot_rw(sa, lane & 3, sel, xp, xsa, xsb);
+                    else if (FMT == FMT_Q4_K) acc[k] += q4_k_dot1<false>(sa, lane & 3, sel, xp, xsa, xsb);
                     else acc[k] += q6_k_dot1(sa, (lane >> 1) & 1, 16 * (lane & 1), xp);
                 }
             }
