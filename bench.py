@@ -6,11 +6,13 @@ Headline step: the full decode-step matvec sweep of a 16-layer dense stack
 weights Q8_0, one token: per layer the fused QKV 3072x2048, O 2048x2048, fused
 gate/up 16384x2048 and down 2048x8192 matvecs -- 64 matvecs, 1.034 GB of
 weights per step (larger than the 126 MB L2, so no flush is needed) -- run in
-decode order (each matvec starts after the previous one is complete, as its
-input would be the previous output in a model): by default as one qmv_chain
-call (a persistent launch with a grid barrier between matvecs), or with
---mode launches as 64 separate calls.  The step is captured once as a CUDA
-graph of the library's C-ABI calls and replayed.
+decode order (each matvec reads its x only after the previous one is complete,
+as its input would be the previous output in a model): 64 library calls with
+programmatic dependent launch (each launch may copy its weights while the
+previous one finishes; --no-pdl turns it off), or with --mode chain one
+qmv_chain call (a persistent launch with a grid barrier between matvecs).  The
+step is captured once as a CUDA graph of the library's C-ABI calls and
+replayed.
 Metric: weight bytes streamed per second (GB/s), with the fraction of the
 measured HBM peak.  The other workloads (Q8_0 1024^2, Q4_K fused QKV, Q6_K
 vocab projection at 1 and 4 tokens, the MoE FFN step, the sweep at 2/4/8
@@ -290,22 +292,19 @@ class Sweep:
                 self.launch(i, stream)
 
 
-def per_launch_durations(torch, sweep, stream, reps=3):
-    """CUDA-event duration of every launch of the step, on its stream."""
-    n = sweep.launches
-    tot = [0.0] * n
-    for _ in range(reps):
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
-        torch.cuda.synchronize()
-        with torch.cuda.stream(stream):
-            for i in range(n):
-                evs[i][0].record(stream)
-                sweep.launch(i, stream)
-                evs[i][1].record(stream)
-        torch.cuda.synchronize()
-        for i in range(n):
-            tot[i] += evs[i][0].elapsed_time(evs[i][1]) / 1e3
-    return [t / reps for t in tot]
+def per_kind_durations(torch, sweep, stream, reps=20):
+    """Average duration of each projection type's launch as it runs in the
+    step: a CUDA graph of that type's 16 launches (in layer order, same launch
+    attributes), replayed and timed with CUDA events on the launch stream."""
+    out = {}
+    layers = sweep_layers()
+    for kind in dict.fromkeys(name for (_, _, name, _, _) in layers):
+        idx = [i for i, (_, _, name, _, _) in enumerate(layers) if name == kind]
+        g = capture(torch, lambda: [sweep.launch(i, stream) for i in idx], stream)
+        time_graph(torch, g, 3, stream)
+        out[kind] = (time_graph(torch, g, reps, stream) / (reps * len(idx)), len(idx))
+        del g
+    return out
 
 
 # --------------------------------------------------------- per-config runs --
@@ -466,10 +465,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--n-tok", type=int, default=1)
-    ap.add_argument("--mode", choices=["auto", "chain", "launches"], default="auto",
-                    help="how the step runs, in decode order either way: 'chain' = qmv_chain "
-                         "(persistent, grid barrier between matvecs; one token), 'launches' = one "
-                         "library call per matvec; auto = chain for one token, else launches")
+    ap.add_argument("--mode", choices=["launches", "chain"], default="launches",
+                    help="how the step runs, in decode order either way: 'launches' = one library "
+                         "call per matvec (default), 'chain' = qmv_chain (one persistent launch with a "
+                         "grid barrier between matvecs; one token)")
+    ap.add_argument("--no-pdl", action="store_true",
+                    help="launch without programmatic dependent launch (qmv_set_pdl(0))")
     ap.add_argument("--headline-only", action="store_true",
                     help="skip the per-config measurements and the CPU baseline")
     ap.add_argument("--profile-case", choices=["q8_0", "q4_k", "q6_k", "q8_0_down", "q8_0_o"])
@@ -491,7 +492,8 @@ def main():
     props = torch.cuda.get_device_properties(torch.cuda.current_device())
     cache = {}
 
-    mode = args.mode if args.mode != "auto" else ("chain" if args.n_tok == 1 else "launches")
+    mode = args.mode
+    q.qmv_set_pdl(0 if args.no_pdl else 1)
     sweep = Sweep(torch, q, args.n_tok, cache)
     sweep.set_mode(mode)
     graph = capture(torch, lambda: sweep.step(), stream)
@@ -511,8 +513,8 @@ def main():
         dist.barrier(torch)
         sec = dist.max(torch, sec)
         # the dominant kernel: every launch of the step, event-timed on its stream
-        durs = per_launch_durations(torch, sweep, stream) if mode == "launches" else [
-            time_graph(torch, graph, 20, stream) / 20]
+        durs = per_kind_durations(torch, sweep, stream) if mode == "launches" else {
+            "chain": (time_graph(torch, graph, 20, stream) / 20, 1)}
         # end to end: pinned x -> device, the step's library calls, y -> pinned host
         e2e_reps = max(3, min(200, args.steps // 5))
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -554,14 +556,31 @@ def main():
 
     value = aggregate_gbs(sweep.weight_bytes, dist.world, args.steps, sec)
     ms_per_step = sec / args.steps * 1e3
-    achieved = sweep.algo / sum(durs) / 1e9
+    # the dominant kernel: the projection type with the largest share of the
+    # step's kernel time; achieved = its algorithmic bytes per launch / its
+    # average event-timed duration
+    shapes = {name: (rows, cols) for (_, _, name, rows, cols) in sweep_layers()}
+    total_kernel_sec = sum(sec1 * n for sec1, n in durs.values())
+    dom_name = max(durs, key=lambda k: durs[k][0] * durs[k][1])
+    dom_launch_sec, dom_n = durs[dom_name]
+    dom_share = dom_launch_sec * dom_n / total_kernel_sec
+    shares = {k: round(v[0] * v[1] / total_kernel_sec, 4) for k, v in durs.items()}
+    if mode == "launches":
+        rows, cols = shapes[dom_name]
+        dom_bytes = algo_bytes(Q8_0, rows, cols, args.n_tok)
+        dom_kernel = f"Q8_0 {dom_name} matvec {rows}x{cols} (warp-ring kernel), {dom_n} launches per step"
+    else:
+        dom_bytes = sweep.algo
+        dom_kernel = "qmv_rw_kernel, chained: the whole step in one launch"
+    achieved = dom_bytes / dom_launch_sec / 1e9
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if os.path.exists(tpath):
         with open(tpath) as f:
             t = json.load(f)
-        if t.get("source_hash") == source_hash() and t.get("n_tok") == args.n_tok:
-            traffic = t.get("step_traffic_bytes_per_launch")
+        if (t.get("source_hash") == source_hash() and t.get("n_tok") == args.n_tok
+                and t.get("kernel") == dom_name):
+            traffic = t.get("traffic_bytes_per_launch")
     cfg4_key = f"cfg4_sweep_ntok{args.n_tok}" + ("" if mode == "launches" else f"_{mode}")
     per_config[cfg4_key] = {"us": ms_per_step * 1e3, "weight_gbs": sweep.weight_bytes / (sec / args.steps) / 1e9,
                             "launches": sweep.launches, "mode": mode, "order": "decode order"}
@@ -586,17 +605,21 @@ def main():
                    "l2": "inputs larger than L2 (1.03 GB of weights per step, L2 126 MB)",
                    "timing": "CUDA graph of the step's C-ABI calls, replayed; CUDA events on the launch stream",
                    "mode": mode,
-                   "order": "decode order: every matvec starts after the previous one has finished",
+                   "pdl": not args.no_pdl,
+                   "order": "decode order: every matvec reads its x after the previous one has finished",
                    "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"},
         "frac_of_hbm_peak": round(value / dist.world / hbm_peak, 4),
         "us_per_step": round(ms_per_step * 1e3, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6.65 TB/s",
-                     "kernel": ("qmv_rw_kernel, chained (Q8_0, the whole step in one launch)" if mode == "chain"
-                                else "the step's matvec launches (Q8_0)"),
-                     "algorithmic_bytes_per_step": sweep.algo,
-                     "mean_launch_us": round(sum(durs) / len(durs) * 1e6, 3)},
+                     "kernel": dom_kernel,
+                     "algorithmic_bytes_per_launch": dom_bytes,
+                     "launch_us": round(dom_launch_sec * 1e6, 3),
+                     "share_of_step_kernel_time": round(dom_share, 4),
+                     "kernel_time_shares": shares,
+                     "step_kernel_gbs": round(sweep.algo / total_kernel_sec / 1e9, 1),
+                     "timing": "each projection type's 16 launches as a replayed CUDA graph, CUDA events"},
         "e2e": {"value": round(sweep.weight_bytes * dist.world / e2e_sec / 1e9, 1), "unit": "GB/s",
                 "h2d_bytes_per_step": int(sweep.x_host.numel() * 4),
                 "d2h_bytes_per_step": int(sweep.y_host.numel() * 4)},

@@ -282,6 +282,17 @@ bool rw_ok(int fmt, int64_t cols)
     return rb % 16 == 0 && cb % 16 == 0 && lb % 16 == 0;
 }
 
+// Whether a single one-token matvec should take the warp-ring kernel rather
+// than the general one (measured on B200): Q8_0 and Q6_K yes, except for
+// tall matrices with rows longer than one K-chunk (there the general kernel's
+// register-resident K-segments stay ahead); Q4_K no (its general-kernel decode
+// keeps more rows in flight per warp).
+bool rw_preferred(int fmt, int64_t rows, int64_t cols)
+{
+    if (!rw_ok(fmt, cols) || fmt == QMV_Q4_K) return false;
+    return cols <= RW_CK || rows <= 4096;
+}
+
 // Split a task's row groups over its nw warps, starting at warp rot (see
 // rw_range in the kernel).
 void rw_split(RwTask &t, int64_t nw, int64_t rot = 0)
@@ -356,11 +367,12 @@ int rw_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x
     return e == cudaSuccess ? QMV_OK : cuda_fail(e);
 }
 
-// Matvecs of one format on the warp-ring kernel, up to RW_MAX_TASKS per
-// launch.  Every CTA works on every task, in order, each task's row groups
-// spread over all warps (so small and large tasks alike use the whole GPU);
-// ordered: with a grid barrier between consecutive tasks (cooperative launch).
-int rw_group(int fmt, const qmv_task *tasks, int n_tasks, bool ordered, const DevInfo &di, cudaStream_t st)
+// In-order one-token matvecs of one format on the warp-ring kernel, up to
+// RW_MAX_TASKS per launch.  Every CTA works on every task, in order, each
+// task's row groups spread over all warps (so small and large tasks alike use
+// the whole GPU), with a grid barrier between consecutive tasks (cooperative
+// launch).
+int rw_chain(int fmt, const qmv_task *tasks, int n_tasks, const DevInfo &di, cudaStream_t st)
 {
     int64_t x_floats = 0;
     for (int t = 0; t < n_tasks; ++t)
@@ -379,7 +391,7 @@ int rw_group(int fmt, const qmv_task *tasks, int n_tasks, bool ordered, const De
         const int n = std::min(RW_MAX_TASKS, n_tasks - t0);
         p.n_tasks = n;
         p.chain = 1;
-        p.ordered = ordered ? 1 : 0;
+        p.ordered = 1;
         p.n_stage = g.S;
         p.stage_pitch = g.pitch;
         p.x_floats = (int32_t)x_floats;
@@ -395,8 +407,7 @@ int rw_group(int fmt, const qmv_task *tasks, int n_tasks, bool ordered, const De
         }
         p.cta_begin[0] = 0;
         p.cta_begin[1] = (int32_t)ctas;
-        const cudaError_t e = rw_launch(fmt, p, g.R, dim3((unsigned)ctas), g.smem, st,
-                                        !ordered && g_pdl.load() != 0, ordered);
+        const cudaError_t e = rw_launch(fmt, p, g.R, dim3((unsigned)ctas), g.smem, st, false, true);
         if (e != cudaSuccess) return cuda_fail(e);
     }
     return QMV_OK;
@@ -455,7 +466,7 @@ int qmv_batched(int fmt, const void *W_blocks, int64_t rows, int64_t cols, const
     if (injected_failure()) return QMV_ERR_CUDA;
     DevInfo di;
     if ((rc = get_dev(di))) return rc;
-    if (n_tok == 1 && rw_ok(fmt, cols))
+    if (n_tok == 1 && rw_preferred(fmt, rows, cols))
         return rw_single(fmt, W_blocks, rows, cols, x, y, di, reinterpret_cast<cudaStream_t>(stream));
     Plan pl;
     if ((rc = make_plan(fmt, rows, cols, n_tok, 1, 1, true, di, pl))) return rc;
@@ -488,12 +499,6 @@ int qmv_multi(int fmt, int n_tok, const qmv_task *tasks, int n_tasks, qmv_stream
     int rc = get_dev(di);
     if (rc) return rc;
     const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (n_tok == 1) {
-        bool all = true;
-        for (int t = 0; t < n_tasks && all; ++t) all = rw_ok(fmt, tasks[t].cols);
-        if (all) return rw_group(fmt, tasks, n_tasks, false, di, st);
-    }
-
     // Every CTA streams about the same number of bytes, sized so the batch
     // takes a few waves of two CTAs per SM: small tasks get few CTAs with many
     // rows each, and all tasks' CTAs share the GPU at once.
@@ -564,7 +569,7 @@ int qmv_chain(int fmt, const qmv_task *tasks, int n_tasks, qmv_stream_t stream)
     int rc = get_dev(di);
     if (rc) return rc;
     const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (all) return rw_group(fmt, tasks, n_tasks, true, di, st);
+    if (all) return rw_chain(fmt, tasks, n_tasks, di, st);
     // a shape the chained kernel does not take: one launch per task, in order
     for (int t = 0; t < n_tasks; ++t) {
         const qmv_task &k = tasks[t];
