@@ -250,7 +250,10 @@ RwGeom rw_geom(int fmt, int64_t x_floats, int n_tasks)
     const int64_t x_area = ceil_div(x_floats * 4, 128) * 128;
     const int64_t hdr = rw_hdr_bytes(n_tasks);
     const int64_t per_warp = (RW_CTA_SMEM - hdr - x_area) / NW;
-    auto pitch = [&](int R) { return ceil_div(R * cb + 16, 128) * 128; };
+    // Q6_K's decode reads up to 4 bytes past a slice (2-byte-aligned words):
+    // its stages carry 16 spare bytes
+    const int64_t pad = fmt == QMV_Q6_K ? 16 : 0;
+    auto pitch = [&](int R) { return ceil_div(R * cb + pad, 128) * 128; };
     auto stages = [&](int R) { return std::min<int64_t>(RW_MAX_STAGES, per_warp / pitch(R)); };
     RwGeom g;
     for (int want_s : {3, 2}) {
@@ -346,7 +349,7 @@ cudaError_t rw_occ(int fmt, int R, size_t smem, int *n)
 int rw_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x, float *y, const DevInfo &di,
               cudaStream_t st)
 {
-    const int64_t x_floats = cols > RW_CK ? cols : 0;
+    const int64_t x_floats = cols;
     const RwGeom g = rw_geom(fmt, x_floats, 1);
     if (g.R == 0) return QMV_ERR_SHAPE;
     RwParams1 p{};
@@ -375,8 +378,7 @@ int rw_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x
 int rw_chain(int fmt, const qmv_task *tasks, int n_tasks, const DevInfo &di, cudaStream_t st)
 {
     int64_t x_floats = 0;
-    for (int t = 0; t < n_tasks; ++t)
-        if (tasks[t].cols > RW_CK) x_floats = std::max<int64_t>(x_floats, tasks[t].cols);
+    for (int t = 0; t < n_tasks; ++t) x_floats = std::max<int64_t>(x_floats, tasks[t].cols);
     const RwGeom g = rw_geom(fmt, x_floats, std::min(n_tasks, RW_MAX_TASKS));
     if (g.R == 0) return QMV_ERR_SHAPE;
     static thread_local RwParams p;

@@ -76,7 +76,7 @@ struct RwParamsT {
     int32_t ordered;          // chained: grid barrier between consecutive tasks (cooperative launch)
     int32_t n_stage;          // ring stages per warp
     int32_t stage_pitch;      // bytes per stage (multiple of 128)
-    int32_t x_floats;         // shared-memory x of tasks longer than one K-chunk (0: none)
+    int32_t x_floats;         // shared-memory x: the longest task row (floats)
     int32_t cta_begin[NT + 1];   // not chained: task t owns CTAs [cta_begin[t], cta_begin[t+1])
     unsigned *sync;           // ordered: {arrivals, exits} of the grid barrier, zero between launches
     int *err;
@@ -213,36 +213,13 @@ __device__ __forceinline__ uint32_t rw_slice_addr(uint32_t rowp, int l)
     return rowp + 210u * (uint32_t)(l >> 2);
 }
 
-// Lane l's x slice of K-chunk kc in registers (zeros where the chunk is short),
-// with the Q4_K half sums.  Chained launches read x through L2 only: it may
-// have been written by another SM earlier in the same launch.
-template <int FMT>
-__device__ __forceinline__ void rw_load_x(const float *x, int kc, int ncols, bool coherent, int lane,
-                                          float2 (&xr)[16][2], float &xsa, float &xsb)
-{
-    const bool have = 64 * (lane + 1) <= ncols;
-    float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
-    const float *xc = x + (int64_t)kc * RW_CK;
-#pragma unroll
-    for (int gq = 0; gq < 16; ++gq) {
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (have) {
-            const float4 *src = reinterpret_cast<const float4 *>(xc + rw_group_col<FMT>(lane, gq));
-            v = coherent ? __ldcg(src) : __ldg(src);
-        }
-        xr[gq][0] = make_float2(v.x, v.z);
-        xr[gq][1] = make_float2(v.y, v.w);
-        if (gq < 8) sa = f2add(sa, f2add(xr[gq][0], xr[gq][1]));
-        else sb = f2add(sb, f2add(xr[gq][0], xr[gq][1]));
-    }
-    xsa = sa.x + sa.y;
-    xsb = sb.x + sb.y;
-}
-
-// x of a task longer than one K-chunk sits in shared memory for the whole task
-// (all warps read every K-chunk of it).  float4 f of the row is stored at
-// f ^ ((f >> 4) & 7): the eight lanes of a quarter-warp that read the same
-// group of their 64-column slices hit eight different bank groups.
+// A task's x sits in shared memory for the whole task; a lane loads its 64
+// values of a K-chunk into registers from there (once per task for rows of
+// one K-chunk, once per tile for longer rows).  float4 f of the row is stored
+// at f ^ ((f >> 4) & 7): the eight lanes of a quarter-warp that read the same
+// group of their 64-column slices hit eight different bank groups.  Chained
+// launches read x through L2 only: it may have been written by another SM
+// earlier in the same launch.
 __device__ __forceinline__ uint32_t rw_xswz(uint32_t f) { return f ^ ((f >> 4) & 7u); }
 
 __device__ __forceinline__ void rw_stage_x(uint32_t xs, const float *x, int cols, bool coherent)
@@ -390,19 +367,19 @@ __global__ void __launch_bounds__(NTHREADS, 2) qmv_rw_kernel(const __grid_consta
         }
         const RwTask &tk = tasks[t];
         const int nch = tk.n_chunks;
-        if (nch > 1) {
-            // every warp of the CTA takes part (the task's x for all K-chunks)
-            rw_stage_x(xs, tk.x, (nch - 1) * RW_CK + tk.last_cols, coherent);
-            __syncthreads();
-        }
+        // The CTA copies the task's x into shared memory once (every thread a
+        // few float4s) and every warp takes its slices from there: one 8 KB
+        // read per CTA from L2 instead of one per warp, which matters because
+        // those L2 reads queue behind the weight copies in flight.
+        rw_stage_x(xs, tk.x, (nch - 1) * RW_CK + tk.last_cols, coherent);
+        __syncthreads();
         int64_t a, b;
         rw_range(tk, wg, a, b);
         if (a >= b || dead) {
-            if (nch > 1) __syncthreads();         // matches the one after the task below
+            __syncthreads();                      // matches the one after the task below
             continue;
         }
         // the task's fields, once
-        const float *tx = tk.x;
         float *ty = tk.y;
         const int64_t rows = tk.rows;
         const int last_cols = tk.last_cols;
@@ -457,7 +434,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) qmv_rw_kernel(const __grid_consta
         };
         if (nch == 1) {
             // x stays in registers for the whole task
-            rw_load_x<FMT>(tx, 0, last_cols, coherent, lane, xr, xsa, xsb);
+            rw_load_x_smem<FMT>(xs, 0, last_cols, lane, xr, xsa, xsb);
             for (int64_t rg = a; rg < b; ++rg) {
                 float acc[R];
 #pragma unroll
@@ -484,8 +461,8 @@ __global__ void __launch_bounds__(NTHREADS, 2) qmv_rw_kernel(const __grid_consta
                 }
                 if (!dead) finish(acc, rg);
             }
-            __syncthreads();                      // x stays until every warp is done with it
         }
+        __syncthreads();                          // x stays until every warp is done with it
     }
     if (p.ordered) rw_grid_exit(p.sync, gridDim.x);
     // after a timeout: let the copies still in flight land before the CTA exits
