@@ -29,6 +29,7 @@ constexpr int STAGE_MAX = 36 * 1024;       // bytes of one pipeline stage
 constexpr int STAGES_BUDGET2 = 105 * 1024; // all stages of one CTA, two CTAs per SM (1-2 tokens)
 constexpr int STAGES_BUDGET1 = 192 * 1024; // one CTA per SM (3-8 tokens: more registers per thread)
 constexpr int64_t X_SMEM_MAX = 64 * 1024;       // several tokens: largest x staged in shared memory
+constexpr int64_t X1_SMEM_MAX = 32 * 1024;      // one token: largest x (all groups) staged in shared memory
 constexpr int MULTI_WAVES = 4;                   // grouped launch: CTA waves over the GPU
 constexpr int64_t MULTI_MIN_CTA_BYTES = 128 * 1024;
 #ifndef QMV_SMALL_CTA_BYTES
@@ -172,9 +173,12 @@ int make_plan(int fmt, int64_t rows, int64_t cols, int n_tok, int G, int n_jobs,
     const int64_t last_cols = cols - (n_chunks - 1) * chunk_cols;
     const int64_t stage_bytes = (int64_t)G * T * chunk_bytes;
     const int64_t stage_pitch = ceil_div(stage_bytes + 16, 128) * 128;
-    // several tokens of one group: stage x in shared memory when it fits
-    const int64_t x_bytes = (int64_t)n_tok * cols * 4;
-    const bool x_smem = n_tok > 1 && G == 1 && n_chunks == 1 && x_bytes <= X_SMEM_MAX;
+    // x staged in shared memory when it fits: several tokens of one group, or
+    // one token's x of every group (x then goes to registers from there)
+    const bool xreg = n_tok == 1 && n_chunks == 1 && ceil_div(n1, wpr) <= xcap;
+    const int64_t x_bytes = (int64_t)(n_tok > 1 ? n_tok : G) * cols * 4;
+    const bool x_smem = n_chunks == 1 && x_bytes <= (n_tok > 1 ? X_SMEM_MAX : X1_SMEM_MAX) &&
+                        (n_tok > 1 ? G == 1 : xreg);
     const int64_t x_area = x_smem ? ceil_div(x_bytes, 128) * 128 : 0;
     int n_stage = (int)std::min<int64_t>(MAX_STAGES, std::max<int64_t>(2, (budget - x_area) / stage_pitch));
     while (n_stage > 2 && 128 + SMEM_HDR + n_stage * stage_pitch + x_area > di.smem_optin) --n_stage;
@@ -208,7 +212,7 @@ int make_plan(int fmt, int64_t rows, int64_t cols, int n_tok, int G, int n_jobs,
     p.err = di.err;
     pl.kc.ntok = n_tok;
     pl.kc.R = R;
-    pl.kc.xreg = n_tok == 1 && n_chunks == 1 && ceil_div(n1, wpr) <= xcap;
+    pl.kc.xreg = xreg;
     pl.kc.pdl = g_pdl.load() != 0;
     pl.grid = dim3((unsigned)ctas_per_job, (unsigned)n_jobs);
     pl.smem = (size_t)smem;
@@ -286,14 +290,16 @@ bool rw_ok(int fmt, int64_t cols)
 }
 
 // Whether a single one-token matvec should take the warp-ring kernel rather
-// than the general one (measured on B200): Q8_0 and Q6_K yes, except for
-// tall matrices with rows longer than one K-chunk (there the general kernel's
-// register-resident K-segments stay ahead); Q4_K no (its general-kernel decode
-// keeps more rows in flight per warp).
+// than the general one (measured on B200).  Rows of one K-chunk: yes, except
+// very tall Q4_K matrices (beyond ~32K rows the general kernel's Q4_K decode,
+// with more rows in flight per warp, streams faster).  Longer rows: only for
+// Q8_0 / Q6_K matrices of at most 4096 rows (taller ones run faster on the
+// general kernel's register-resident K-segments).
 bool rw_preferred(int fmt, int64_t rows, int64_t cols)
 {
-    if (!rw_ok(fmt, cols) || fmt == QMV_Q4_K) return false;
-    return cols <= RW_CK || rows <= 4096;
+    if (!rw_ok(fmt, cols)) return false;
+    if (cols <= RW_CK) return fmt != QMV_Q4_K || rows <= 32768;
+    return fmt != QMV_Q4_K && rows <= 4096;
 }
 
 // Split a task's row groups over its nw warps, starting at warp rot (see

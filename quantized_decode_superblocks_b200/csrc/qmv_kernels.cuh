@@ -73,7 +73,8 @@ struct Params {
     int32_t rows_per_cta;
     int32_t mode;
     int32_t tma;             // 1: bulk async copies; 0: warp copies
-    int32_t x_smem;          // several tokens: x staged in shared memory after the stages
+    int32_t x_smem;          // x staged in shared memory after the stages: every token of one
+                             // group, or (one token, x in registers) every group's x
     // weights: group matrix = base + ids[idx] * expert_stride (or base)
     const uint8_t *base0;
     const uint8_t *base1;    // MODE_SWIGLU: up matrices (group 1)
@@ -255,6 +256,21 @@ __device__ __forceinline__ void qmv_pipeline_body(const Params &p, const int cta
 
     pdl_wait();                                   // x is the previous kernel's output
 
+    // x staged once per CTA in shared memory (swizzled): every token of one
+    // group, or (one token) every group's x -- one L2 read per CTA instead of
+    // one per warp, which queues behind the weight copies in flight
+    const uint32_t xsm = stage0 + (uint32_t)S * (uint32_t)p.stage_pitch;
+    const int nf = p.cols >> 2;                   // float4 groups per row of x
+    if (p.x_smem) {
+        const int nrow = NTOK > 1 ? NTOK : p.G;
+        for (int idx = tid; idx < nrow * nf; idx += NTHREADS) {
+            const int t = idx / nf, f = idx - t * nf;
+            const float *src = NTOK > 1 ? sX[0] + (int64_t)t * p.x_tok_stride : sX[t];
+            sts_f4(xsm + 16u * (uint32_t)(t * nf + (int)xs_swizzle((uint32_t)f)), ldg4(src + 4 * f));
+        }
+        __syncthreads();
+    }
+
     // one token: this warp's x slices in registers for the whole kernel
     float2 xr[XREG ? SPL1 : 1][XREG ? NG1 : 1][2];
     float xsa[XREG ? SPL1 : 1], xsb[XREG ? SPL1 : 1];
@@ -269,7 +285,11 @@ __device__ __forceinline__ void qmv_pipeline_body(const Params &p, const int cta
             float2 sa = make_float2(0.f, 0.f), sbv = make_float2(0.f, 0.f);
 #pragma unroll
             for (int gq = 0; gq < NG1; ++gq) {
-                const float4 v = have ? ldg4(sX[g] + slice1_group_col<FMT>(s, gq)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                const int col = slice1_group_col<FMT>(s, gq);
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (have)
+                    v = p.x_smem ? lds_f4(xsm + 16u * (uint32_t)(g * nf + (int)xs_swizzle((uint32_t)col >> 2)))
+                                 : ldg4(sX[g] + col);
                 xr[q][gq][0] = make_float2(v.x, v.z);
                 xr[q][gq][1] = make_float2(v.y, v.w);
                 if (gq < NG1 / 2) sa = f2add(sa, f2add(xr[q][gq][0], xr[q][gq][1]));
@@ -277,20 +297,6 @@ __device__ __forceinline__ void qmv_pipeline_body(const Params &p, const int cta
             }
             xsa[q] = sa.x + sa.y;
             xsb[q] = sbv.x + sbv.y;
-        }
-    }
-
-    // several tokens: stage every token's x once in shared memory (swizzled)
-    const uint32_t xsm = stage0 + (uint32_t)S * (uint32_t)p.stage_pitch;
-    const int nf = p.cols >> 2;                   // float4 groups per token row
-    if constexpr (NTOK > 1) {
-        if (p.x_smem) {
-            for (int idx = tid; idx < NTOK * nf; idx += NTHREADS) {
-                const int t = idx / nf, f = idx - t * nf;
-                sts_f4(xsm + 16u * (uint32_t)(t * nf + (int)xs_swizzle((uint32_t)f)),
-                       ldg4(sX[0] + (int64_t)t * p.x_tok_stride + 4 * f));
-            }
-            __syncthreads();
         }
     }
 
