@@ -316,17 +316,21 @@ def rotating_pool(torch, fmt, rows, cols, seed, min_total):
     return [base] + [base.clone() for _ in range(copies - 1)]
 
 
-def measure_matvec(torch, q, stream, fmt, rows, cols, n_tok, seed, reps=200):
-    """µs per matvec over a pool of weight copies larger than L2 (replayed graph)."""
+def measure_matvec(torch, q, stream, fmt, rows, cols, n_tok, seed, reps=200, argmax=False):
+    """µs per matvec over a pool of weight copies larger than L2 (replayed graph);
+    argmax: the projection followed by the greedy argmax (qmv_argmax)."""
     pool = rotating_pool(torch, fmt, rows, cols, seed, 2 * L2_BYTES)
     x = torch.from_numpy(synth.gen_x(n_tok, cols, seed, 1)).cuda()
     y = torch.empty((n_tok, rows), device="cuda")
+    idx = torch.empty(n_tok, dtype=torch.int32, device="cuda")
     per_graph = min(len(pool) * max(1, 64 // len(pool)), 256)
 
     def body():
         for i in range(per_graph):
             W = pool[i % len(pool)]
-            if n_tok == 1:
+            if argmax:
+                q.qmv_argmax(fmt, W, rows, cols, x, y, n_tok, idx)
+            elif n_tok == 1:
                 q.qmv_f32(fmt, W, rows, cols, x, y)
             else:
                 q.qmv_batched(fmt, W, rows, cols, x, y, n_tok)
@@ -534,6 +538,8 @@ def main():
             for nt in (1, 4):
                 per_config[f"cfg2_q6_k_vocab_128000x2048_ntok{nt}"] = measure_matvec(
                     torch, q, stream, Q6_K, 128000, 2048, nt, 2, reps=20)
+            per_config["cfg2_q6_k_vocab_128000x2048_ntok1_greedy_argmax"] = measure_matvec(
+                torch, q, stream, Q6_K, 128000, 2048, 1, 2, reps=20, argmax=True)
             per_config["cfg3_moe_ffn_step"] = measure_moe(torch, q, stream)
             for nt in (1, 2, 4, 8):
                 sw = Sweep(torch, q, nt, cache)

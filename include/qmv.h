@@ -43,9 +43,11 @@
  *   - The arithmetic is f32: dequantized weights are exact f32 values, dot
  *     products accumulate in f32 (order unspecified, deterministic for a
  *     given shape).  There is no CPU fallback and no other backend.
- *   - Thread safety: calls may be made from several host threads; the only
- *     global state is a per-device properties cache and the sticky device
- *     error word read by qmv_check().
+ *   - Thread safety: calls may be made from several host threads.  Global
+ *     state: a per-device properties cache, the programmatic-dependent-launch
+ *     switch (qmv_set_pdl), and per device the sticky error word read by
+ *     qmv_check(), the two grid-barrier words of qmv_chain and the scratch
+ *     array of moe_ffn_static.
  */
 #ifndef QMV_H
 #define QMV_H
@@ -203,6 +205,17 @@ int moe_ffn_static(int fmt_gu, const void *gate_blocks, const void *up_blocks,
                    int64_t down_stride_bytes, int n_expert, const int32_t *expert_ids,
                    const float *g, int n_sel, int64_t hidden, int64_t inter,
                    const float *x, float *y, qmv_stream_t stream);
+
+/* Greedy next-token choice on the device (FlareLLM page, §推理层面的深度优化:
+ * greedy decoding of the vocabulary projection): y = W x as qmv_batched (the
+ * logits are kept in the caller's y, f32 [n_tok][rows]), then
+ * idx_out[t] = the row of the largest y[t][row] -- IEEE > on f32, ties to
+ * the lower row, NaN values skipped, -1 if every value of the token is NaN.
+ * idx_out: device int32 [n_tok], 4-byte aligned.  rows <= INT32_MAX.
+ * Deterministic (no atomics); two launches on `stream`.  Errors as
+ * qmv_batched. */
+int qmv_argmax(int fmt, const void *W_blocks, int64_t rows, int64_t cols,
+               const float *x, float *y, int n_tok, int32_t *idx_out, qmv_stream_t stream);
 
 /* Dequantize the whole matrix to f32: out[rows][cols].  The values are
  * bit-exact f32 evaluations of the block formulas above (every product in

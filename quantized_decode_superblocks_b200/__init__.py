@@ -25,7 +25,7 @@ STATUS_NAMES = {0: "QMV_OK", -1: "QMV_ERR_NULL", -2: "QMV_ERR_FMT", -3: "QMV_ERR
 DEVERR_EXPERT_ID = 1
 DEVERR_TIMEOUT = 2
 
-EXPORTED = ("qmv_f32", "qmv_batched", "qmv_multi", "qmv_chain", "moe_route", "moe_qmv", "moe_ffn", "moe_ffn_static",
+EXPORTED = ("qmv_f32", "qmv_batched", "qmv_multi", "qmv_chain", "qmv_argmax", "moe_route", "moe_qmv", "moe_ffn", "moe_ffn_static",
             "qmv_dequant",
             "qmv_check", "qmv_strerror", "qmv_block_bytes", "qmv_block_weights",
             "qmv_debug_fail_next_launches", "qmv_set_pdl", "qmv_get_pdl", "qmv_last_cuda_error")
@@ -60,6 +60,8 @@ def lib() -> ctypes.CDLL:
         L.qmv_f32.argtypes = [c_int, vp, i64, i64, vp, vp, vp]
         L.qmv_batched.argtypes = [c_int, vp, i64, i64, vp, vp, c_int, vp]
         L.qmv_multi.argtypes = [c_int, c_int, ctypes.POINTER(QmvTask), c_int, vp]
+        L.qmv_chain.argtypes = [c_int, ctypes.POINTER(QmvTask), c_int, vp]
+        L.qmv_argmax.argtypes = [c_int, vp, i64, i64, vp, vp, c_int, vp, vp]
         L.moe_route.argtypes = [vp, vp, c_int, c_int, vp, vp, vp]
         L.moe_qmv.argtypes = [c_int, vp, i64, c_int, vp, c_int, i64, i64, vp, i64, vp, vp, vp]
         L.moe_ffn.argtypes = [c_int, vp, vp, i64, c_int, vp, i64, c_int, vp, vp, c_int, i64, i64,
@@ -168,6 +170,13 @@ def qmv_chain(fmt, tasks, stream=None):
     `tasks` as for qmv_multi."""
     arr = tasks if isinstance(tasks, ctypes.Array) else make_tasks(tasks)
     _check(lib().qmv_chain(fmt, arr, len(arr), _stream(stream)), "qmv_chain")
+
+
+def qmv_argmax(fmt, W, rows, cols, x, y, n_tok, idx_out, stream=None):
+    """y = W x (kept in y) and idx_out[t] = argmax over rows of y[t] (ties to the
+    lower row, NaN skipped, -1 if all NaN)."""
+    _check(lib().qmv_argmax(fmt, _ptr(W), rows, cols, _ptr(x), _ptr(y), n_tok, _ptr(idx_out),
+                            _stream(stream)), "qmv_argmax")
 
 
 def moe_route(logits, bias, n_expert, top_k, ids_out, g_out, stream=None):

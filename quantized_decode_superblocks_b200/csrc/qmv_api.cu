@@ -2,6 +2,7 @@
 // argument validation, launch planning and the launches themselves.  Nothing
 // here allocates device memory; every buffer is the caller's.
 #include <algorithm>
+#include <climits>
 #include <atomic>
 #include <mutex>
 #include <vector>
@@ -734,6 +735,22 @@ int moe_ffn_static(int fmt_gu, const void *gate_blocks, const void *up_blocks, i
     }
     return moe_ffn(fmt_gu, gate_blocks, up_blocks, gu_stride_bytes, fmt_down, down_blocks, down_stride_bytes,
                    n_expert, expert_ids, g, n_sel, hidden, inter, x, h, y, stream);
+}
+
+int qmv_argmax(int fmt, const void *W_blocks, int64_t rows, int64_t cols, const float *x, float *y, int n_tok,
+               int32_t *idx_out, qmv_stream_t stream)
+{
+    if (!W_blocks || !x || !y || !idx_out) return QMV_ERR_NULL;
+    int rc = check_matrix(fmt, rows, cols);
+    if (rc) return rc;
+    if (rows > INT32_MAX) return QMV_ERR_SHAPE;
+    if (n_tok < 1 || n_tok > QMV_MAX_NTOK) return QMV_ERR_NTOK;
+    if (!aligned(W_blocks, 16) || !aligned(x, 16) || !aligned(y, 4) || !aligned(idx_out, 4)) return QMV_ERR_ALIGN;
+    if ((rc = qmv_batched(fmt, W_blocks, rows, cols, x, y, n_tok, stream))) return rc;
+    argmax_rows_kernel<<<n_tok, 1024, 0, reinterpret_cast<cudaStream_t>(stream)>>>(y, rows, rows, idx_out);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e);
+    return QMV_OK;
 }
 
 int qmv_dequant(int fmt, const void *W_blocks, int64_t rows, int64_t cols, float *out, qmv_stream_t stream)

@@ -6,6 +6,61 @@
 
 namespace qmv {
 
+// ------------------------------------------------------- greedy argmax --
+// FlareLLM page, §推理层面的深度优化 (greedy decoding picks the next token from
+// the logits on the device): idx[t] = the row of the largest y[t][row] (IEEE >
+// on f32), ties to the lower row, NaN skipped; -1 when every value is NaN.
+// One CTA of 1024 threads per token: each thread scans rows tid, tid + 1024,
+// ... in float4 groups, then a warp and a block reduction.  Reads y once
+// (512 KB per token for a 128000-row vocabulary, from L2 right after the
+// matvec that wrote it); deterministic, no atomics, no scratch.
+__device__ __forceinline__ void argmax_merge(float &bv, int &bi, float ov, int oi)
+{
+    if (oi < 0) return;
+    if (bi < 0 || ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+    }
+}
+
+__global__ void __launch_bounds__(1024) argmax_rows_kernel(const float *y, int64_t rows, int64_t y_tok_stride,
+                                                           int32_t *idx)
+{
+    __shared__ float s_v[32];
+    __shared__ int s_i[32];
+    const float *yt = y + (int64_t)blockIdx.x * y_tok_stride;
+    float bv = 0.f;
+    int bi = -1;
+    const bool vec = (reinterpret_cast<uintptr_t>(yt) & 15u) == 0;
+    const int64_t n4 = vec ? rows / 4 : 0;
+    for (int64_t i = threadIdx.x; i < n4; i += blockDim.x) {
+        const float4 v = __ldcg(reinterpret_cast<const float4 *>(yt) + i);
+        const float e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            if (e[k] == e[k]) argmax_merge(bv, bi, e[k], (int)(4 * i + k));
+    }
+    for (int64_t r = 4 * n4 + threadIdx.x; r < rows; r += blockDim.x) {
+        const float e = __ldcg(yt + r);
+        if (e == e) argmax_merge(bv, bi, e, (int)r);
+    }
+    for (int o = 16; o >= 1; o >>= 1)
+        argmax_merge(bv, bi, __shfl_xor_sync(0xFFFFFFFFu, bv, o), __shfl_xor_sync(0xFFFFFFFFu, bi, o));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) {
+        s_v[warp] = bv;
+        s_i[warp] = bi;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        bv = lane < (int)(blockDim.x >> 5) ? s_v[lane] : 0.f;
+        bi = lane < (int)(blockDim.x >> 5) ? s_i[lane] : -1;
+        for (int o = 16; o >= 1; o >>= 1)
+            argmax_merge(bv, bi, __shfl_xor_sync(0xFFFFFFFFu, bv, o), __shfl_xor_sync(0xFFFFFFFFu, bi, o));
+        if (lane == 0) idx[blockIdx.x] = bi;
+    }
+}
+
 // -------------------------------------------------------------- router --
 // BebeLM page, §核心算子 (MoE前馈网络): sigmoid scores, the per-expert bias
 // added for the choice only, top_k by biased score (ties to the lower index),

@@ -122,6 +122,18 @@ def test_chain_argument_validation(L):
     q.lib().qmv_debug_fail_next_launches(0)
 
 
+def test_argmax_argument_validation(L):
+    assert L.qmv_argmax(0, A, 4, 64, A, A, 1, None, None) == NULL
+    assert L.qmv_argmax(0, None, 4, 64, A, A, 1, A, None) == NULL
+    assert L.qmv_argmax(7, A, 4, 64, A, A, 1, A, None) == FMT
+    assert L.qmv_argmax(0, A, 4, 60, A, A, 1, A, None) == SHAPE
+    assert L.qmv_argmax(0, A, 0, 64, A, A, 1, A, None) == SHAPE
+    assert L.qmv_argmax(0, A, 4, 64, A, A, 0, A, None) == NTOK
+    assert L.qmv_argmax(0, A, 4, 64, A, A, 9, A, None) == NTOK
+    assert L.qmv_argmax(0, A + 8, 4, 64, A, A, 1, A, None) == ALIGN
+    assert L.qmv_argmax(0, A, 4, 64, A, A, 1, A + 2, None) == ALIGN
+
+
 def test_injected_launch_failure_is_reported(L):
     q.lib().qmv_debug_fail_next_launches(2)
     assert qb(L) == CUDA

@@ -274,6 +274,68 @@ def test_qmv_chain_repeated_calls_reuse_the_barrier():
         _chain_case(Q8_0, [1024, 2048, 512, 1024], 92 + rep)
 
 
+# ------------------------------------------------------------ greedy argmax --
+
+def _argmax_check(fmt, W, rows, cols, x, seed_note=""):
+    n_tok = x.shape[0]
+    yd = torch.full((n_tok, rows), float("nan"), device="cuda")
+    idx = torch.full((n_tok,), -7, dtype=torch.int32, device="cuda")
+    q.qmv_argmax(fmt, dev(W), rows, cols, dev(x), yd, n_tok, idx)
+    torch.cuda.synchronize()
+    y, i = yd.cpu().numpy(), idx.cpu().numpy()
+    ref, bound = oracle.qmv(fmt, W, rows, cols, x)
+    within(y, ref, bound)
+    for t in range(n_tok):
+        # exact: the first maximum of the GPU's own logits (numpy's tie rule)
+        assert i[t] == int(np.argmax(y[t])), (t, i[t], int(np.argmax(y[t])))
+        # against the oracle: equal where the top two are further apart than
+        # the error allowed on either; else the pick must be a near-maximum
+        r = ref[t]
+        lim = REL * bound[t] + ABS
+        order = np.argsort(r, kind="stable")
+        top = int(np.argmax(r))
+        clear = rows == 1 or r[top] - r[order[-2]] > lim[top] + lim[order[-2]]
+        if clear:
+            assert i[t] == top
+        else:
+            assert r[i[t]] >= r[top] - 2 * lim.max()
+    return i
+
+
+@pytest.mark.parametrize("fmt,rows,cols,n_tok", [(Q6_K, 128000, 2048, 1), (Q6_K, 128000, 2048, 4),
+                                                 (Q8_0, 5000, 1024, 1), (Q4_K, 777, 512, 8)])
+def test_argmax_matches_logits_and_oracle(fmt, rows, cols, n_tok):
+    W = synth.gen_blocks(fmt, rows, cols, 40 + n_tok, fmt)
+    x = synth.gen_x(n_tok, cols, 41, n_tok)
+    _argmax_check(fmt, W, rows, cols, x)
+
+
+def test_argmax_ties_go_to_the_lower_row_and_nan_is_skipped():
+    # rows of zero blocks (d = 0: logit 0) and three copies of one row with a
+    # positive logit at rows 5, 9 and 14: bit-identical maxima, row 5 wins
+    fmt, cols, rows = Q8_0, 256, 16
+    one = synth.gen_blocks(fmt, 1, cols, 50, 0)
+    x = synth.gen_x(1, cols, 53, 0)
+    if oracle.qmv(fmt, one, 1, cols, x)[0][0, 0] < 0:
+        x = -x
+    W = np.zeros((rows, one.size), np.uint8)
+    for r in (5, 9, 14):
+        W[r] = one
+    i = _argmax_check(fmt, W.reshape(-1), rows, cols, x)
+    assert i[0] == 5
+    # every row the same: row 0
+    i = _argmax_check(fmt, np.tile(one, rows), rows, cols, x)
+    assert i[0] == 0
+    # a NaN activation makes every logit NaN: no row is chosen
+    xn = x.copy()
+    xn[0, 3] = np.nan
+    yd = torch.empty((1, rows), device="cuda")
+    idx = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q.qmv_argmax(fmt, dev(W), rows, cols, dev(xn), yd, 1, idx)
+    torch.cuda.synchronize()
+    assert np.isnan(yd.cpu().numpy()).all() and int(idx.cpu()[0]) == -1
+
+
 # ---------------------------------------------------- full-size workloads --
 
 def test_cfg0_q8_0_1024x1024():
