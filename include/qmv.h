@@ -46,8 +46,8 @@
  *   - Thread safety: calls may be made from several host threads.  Global
  *     state: a per-device properties cache, the programmatic-dependent-launch
  *     switch (qmv_set_pdl), and per device the sticky error word read by
- *     qmv_check(), the two grid-barrier words of qmv_chain and the scratch
- *     array of moe_ffn_static.
+ *     qmv_check(), the two grid-barrier words of qmv_chain, qmv_argmax's
+ *     per-token keys and the scratch array of moe_ffn_static.
  */
 #ifndef QMV_H
 #define QMV_H
@@ -212,8 +212,11 @@ int moe_ffn_static(int fmt_gu, const void *gate_blocks, const void *up_blocks,
  * idx_out[t] = the row of the largest y[t][row] -- IEEE > on f32, ties to
  * the lower row, NaN values skipped, -1 if every value of the token is NaN.
  * idx_out: device int32 [n_tok], 4-byte aligned.  rows <= INT32_MAX.
- * Deterministic (no atomics); two launches on `stream`.  Errors as
- * qmv_batched. */
+ * Two launches on `stream`; the choice is deterministic (the CTAs combine
+ * their candidates with an order-independent 64-bit atomic max).  The
+ * reduction keeps one key and one counter per token in device memory of the
+ * library, back to zero after every call: do not run two qmv_argmax calls on
+ * the same device at the same time.  Errors as qmv_batched. */
 int qmv_argmax(int fmt, const void *W_blocks, int64_t rows, int64_t cols,
                const float *x, float *y, int n_tok, int32_t *idx_out, qmv_stream_t stream);
 

@@ -22,6 +22,11 @@ __device__ int g_dev_err;
 // at the end of every launch; qmv_check clears both after a device error.
 __device__ unsigned g_chain_sync[2];
 
+// Greedy argmax: one 64-bit key and one arrival counter per token, back to
+// zero at the end of every call; qmv_check clears them after a device error.
+__device__ unsigned long long g_amax_key[QMV_MAX_NTOK];
+__device__ unsigned g_amax_done[QMV_MAX_NTOK];
+
 // Scratch of moe_ffn_static: the SwiGLU activations h[n_sel][inter].  Every
 // device that loads the library holds one copy until the process exits.
 static __device__ __align__(256) float g_static_h[QMV_STATIC_H_FLOATS];
@@ -43,6 +48,8 @@ struct DevInfo {
     int smem_optin = 0;
     int *err = nullptr;
     unsigned *sync = nullptr;
+    unsigned long long *amax_key = nullptr;
+    unsigned *amax_done = nullptr;
     float *static_h = nullptr;   // device address of g_static_h, set up by moe_ffn_static
     bool ok = false;
 };
@@ -91,7 +98,9 @@ int get_dev(DevInfo &out)
             cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaGetSymbolAddress(reinterpret_cast<void **>(&d.err), g_dev_err) != cudaSuccess ||
-            cudaGetSymbolAddress(reinterpret_cast<void **>(&d.sync), g_chain_sync) != cudaSuccess) {
+            cudaGetSymbolAddress(reinterpret_cast<void **>(&d.sync), g_chain_sync) != cudaSuccess ||
+            cudaGetSymbolAddress(reinterpret_cast<void **>(&d.amax_key), g_amax_key) != cudaSuccess ||
+            cudaGetSymbolAddress(reinterpret_cast<void **>(&d.amax_done), g_amax_done) != cudaSuccess) {
             (void)cudaGetLastError();
             return QMV_ERR_DEVICE;
         }
@@ -746,8 +755,12 @@ int qmv_argmax(int fmt, const void *W_blocks, int64_t rows, int64_t cols, const 
     if (rows > INT32_MAX) return QMV_ERR_SHAPE;
     if (n_tok < 1 || n_tok > QMV_MAX_NTOK) return QMV_ERR_NTOK;
     if (!aligned(W_blocks, 16) || !aligned(x, 16) || !aligned(y, 4) || !aligned(idx_out, 4)) return QMV_ERR_ALIGN;
+    DevInfo di;
+    if ((rc = get_dev(di))) return rc;
     if ((rc = qmv_batched(fmt, W_blocks, rows, cols, x, y, n_tok, stream))) return rc;
-    argmax_rows_kernel<<<n_tok, 1024, 0, reinterpret_cast<cudaStream_t>(stream)>>>(y, rows, rows, idx_out);
+    const dim3 grid((unsigned)ceil_div(rows, ARGMAX_ROWS_PER_CTA), (unsigned)n_tok);
+    argmax_rows_kernel<<<grid, ARGMAX_THREADS, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        y, rows, rows, idx_out, di.amax_key, di.amax_done);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e);
     return QMV_OK;
@@ -791,7 +804,10 @@ int qmv_check(qmv_stream_t stream, int *dev_err_out)
         (void)cudaGetLastError();
         return QMV_ERR_CUDA;
     }
-    if (word && (cudaMemset(di.sync, 0, 2 * sizeof(unsigned)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)) {
+    if (word && (cudaMemset(di.sync, 0, 2 * sizeof(unsigned)) != cudaSuccess ||
+                 cudaMemset(di.amax_key, 0, QMV_MAX_NTOK * sizeof(unsigned long long)) != cudaSuccess ||
+                 cudaMemset(di.amax_done, 0, QMV_MAX_NTOK * sizeof(unsigned)) != cudaSuccess ||
+                 cudaDeviceSynchronize() != cudaSuccess)) {
         (void)cudaGetLastError();
         return QMV_ERR_CUDA;
     }

@@ -10,10 +10,14 @@ namespace qmv {
 // FlareLLM page, §推理层面的深度优化 (greedy decoding picks the next token from
 // the logits on the device): idx[t] = the row of the largest y[t][row] (IEEE >
 // on f32), ties to the lower row, NaN skipped; -1 when every value is NaN.
-// One CTA of 1024 threads per token: each thread scans rows tid, tid + 1024,
-// ... in float4 groups, then a warp and a block reduction.  Reads y once
-// (512 KB per token for a 128000-row vocabulary, from L2 right after the
-// matvec that wrote it); deterministic, no atomics, no scratch.
+// A grid of CTAs per token scans the rows (float4 loads from L2, where the
+// projection just wrote them); each CTA folds its best (value, row) into one
+// 64-bit key per token with atomicMax -- the value's bits mapped to an
+// order-preserving unsigned in the high word, the complement of the row in the
+// low word, so a larger key is a larger value or, for equal values, a lower
+// row: the result does not depend on the order of the atomics.  The last CTA
+// of the token (an arrival counter) writes idx and puts the key and the
+// counter back to zero for the next call.
 __device__ __forceinline__ void argmax_merge(float &bv, int &bi, float ov, int oi)
 {
     if (oi < 0) return;
@@ -23,24 +27,38 @@ __device__ __forceinline__ void argmax_merge(float &bv, int &bi, float ov, int o
     }
 }
 
-__global__ void __launch_bounds__(1024) argmax_rows_kernel(const float *y, int64_t rows, int64_t y_tok_stride,
-                                                           int32_t *idx)
+__device__ __forceinline__ unsigned long long argmax_key(float v, int row)
 {
-    __shared__ float s_v[32];
-    __shared__ int s_i[32];
-    const float *yt = y + (int64_t)blockIdx.x * y_tok_stride;
+    const uint32_t u = v == 0.f ? 0u : __float_as_uint(v);            // -0 and +0 compare equal
+    const uint32_t hi = (u & 0x80000000u) ? ~u : (u | 0x80000000u);   // order-preserving for non-NaN
+    return ((unsigned long long)hi << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)row);
+}
+
+constexpr int ARGMAX_THREADS = 256;
+constexpr int ARGMAX_ROWS_PER_CTA = 2048;
+
+__global__ void __launch_bounds__(ARGMAX_THREADS) argmax_rows_kernel(const float *y, int64_t rows,
+                                                                     int64_t y_tok_stride, int32_t *idx,
+                                                                     unsigned long long *keys, unsigned *done)
+{
+    __shared__ float s_v[ARGMAX_THREADS / 32];
+    __shared__ int s_i[ARGMAX_THREADS / 32];
+    const int t = (int)blockIdx.y;
+    const float *yt = y + (int64_t)t * y_tok_stride;
+    const int64_t r0 = (int64_t)blockIdx.x * ARGMAX_ROWS_PER_CTA;
+    const int64_t r1 = min(rows, r0 + ARGMAX_ROWS_PER_CTA);
     float bv = 0.f;
     int bi = -1;
-    const bool vec = (reinterpret_cast<uintptr_t>(yt) & 15u) == 0;
-    const int64_t n4 = vec ? rows / 4 : 0;
-    for (int64_t i = threadIdx.x; i < n4; i += blockDim.x) {
-        const float4 v = __ldcg(reinterpret_cast<const float4 *>(yt) + i);
+    const bool vec = ((reinterpret_cast<uintptr_t>(yt + r0) & 15u) == 0);
+    const int64_t n4 = vec ? (r1 - r0) / 4 : 0;
+    for (int64_t i = threadIdx.x; i < n4; i += ARGMAX_THREADS) {
+        const float4 v = __ldcg(reinterpret_cast<const float4 *>(yt + r0) + i);
         const float e[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-            if (e[k] == e[k]) argmax_merge(bv, bi, e[k], (int)(4 * i + k));
+            if (e[k] == e[k]) argmax_merge(bv, bi, e[k], (int)(r0 + 4 * i + k));
     }
-    for (int64_t r = 4 * n4 + threadIdx.x; r < rows; r += blockDim.x) {
+    for (int64_t r = r0 + 4 * n4 + threadIdx.x; r < r1; r += ARGMAX_THREADS) {
         const float e = __ldcg(yt + r);
         if (e == e) argmax_merge(bv, bi, e, (int)r);
     }
@@ -53,11 +71,20 @@ __global__ void __launch_bounds__(1024) argmax_rows_kernel(const float *y, int64
     }
     __syncthreads();
     if (warp == 0) {
-        bv = lane < (int)(blockDim.x >> 5) ? s_v[lane] : 0.f;
-        bi = lane < (int)(blockDim.x >> 5) ? s_i[lane] : -1;
+        bv = lane < ARGMAX_THREADS / 32 ? s_v[lane] : 0.f;
+        bi = lane < ARGMAX_THREADS / 32 ? s_i[lane] : -1;
         for (int o = 16; o >= 1; o >>= 1)
             argmax_merge(bv, bi, __shfl_xor_sync(0xFFFFFFFFu, bv, o), __shfl_xor_sync(0xFFFFFFFFu, bi, o));
-        if (lane == 0) idx[blockIdx.x] = bi;
+        if (lane == 0) {
+            if (bi >= 0) atomicMax(keys + t, argmax_key(bv, bi));
+            __threadfence();
+            if (atomicAdd(done + t, 1u) == gridDim.x - 1u) {      // the token's last CTA
+                __threadfence();
+                const unsigned long long k = atomicExch(keys + t, 0ull);
+                atomicExch(done + t, 0u);
+                idx[t] = k ? (int32_t)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFull)) : -1;
+            }
+        }
     }
 }
 
