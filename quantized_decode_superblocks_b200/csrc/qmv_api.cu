@@ -258,18 +258,31 @@ struct RwGeom {
 
 // x_floats: shared-memory x (tasks longer than one K-chunk), taken from the
 // stage budget.
-RwGeom rw_geom(int fmt, int64_t x_floats, int n_tasks)
+RwGeom rw_geom(int fmt, int64_t x_floats, int n_tasks, int n_tok = 1)
 {
     const int64_t cb = (RW_CK / block_weights(fmt)) * block_bytes(fmt);
-    const int64_t x_area = ceil_div(x_floats * 4, 128) * 128;
+    const int64_t x_area = n_tok * ceil_div(x_floats * 4, 128) * 128;
     const int64_t hdr = rw_hdr_bytes(n_tasks);
     const int64_t per_warp = (RW_CTA_SMEM - hdr - x_area) / NW;
-    // Q6_K's decode reads up to 4 bytes past a slice (2-byte-aligned words):
-    // its stages carry 16 spare bytes
-    const int64_t pad = fmt == QMV_Q6_K ? 16 : 0;
+    // the Q6_K decode and the several-token units read up to 4 bytes past a
+    // slice (2-byte-aligned words): their stages carry 16 spare bytes
+    const int64_t pad = (fmt == QMV_Q6_K || n_tok > 1) ? 16 : 0;
     auto pitch = [&](int R) { return ceil_div(R * cb + pad, 128) * 128; };
     auto stages = [&](int R) { return std::min<int64_t>(RW_MAX_STAGES, per_warp / pitch(R)); };
     RwGeom g;
+    if (n_tok > 1) {
+        // several tokens: two rows per warp share every x load; two stages
+        for (int R : {2, 1}) {
+            if (stages(R) >= 2 && R * pow2ceil(n_tok) <= 32) {
+                g.R = R;
+                g.S = (int)stages(R);
+                g.pitch = (int)pitch(R);
+                g.smem = (size_t)(128 + hdr + x_area + (int64_t)NW * g.S * g.pitch);
+                return g;
+            }
+        }
+        return g;
+    }
     for (int want_s : {3, 2}) {
         for (int R : {4, 2, 1}) {
             if (stages(R) >= want_s) {
@@ -310,6 +323,19 @@ bool rw_preferred(int fmt, int64_t rows, int64_t cols)
     if (!rw_ok(fmt, cols)) return false;
     if (cols <= RW_CK) return fmt != QMV_Q4_K || rows <= 32768;
     return fmt != QMV_Q4_K && rows <= 4096;
+}
+
+// Several tokens on the warp-ring kernel (measured on B200): two tokens for
+// every format, up to four for Q6_K; beyond that the general kernel's
+// weight-stationary loop with more rows per warp is faster.  Every token's x
+// must fit in shared memory beside two stages per warp (n_tok x cols <= 16384
+// floats).
+bool rw_mt_preferred(int fmt, int64_t rows, int64_t cols, int n_tok)
+{
+    (void)rows;
+    if (n_tok > (fmt == QMV_Q6_K ? 4 : 2)) return false;
+    if (!rw_ok(fmt, cols) || (int64_t)n_tok * cols > 16384) return false;
+    return rw_geom(fmt, cols, 1, n_tok).R > 0;
 }
 
 // Split a task's row groups over its nw warps, starting at warp rot (see
@@ -362,11 +388,11 @@ cudaError_t rw_occ(int fmt, int R, size_t smem, int *n)
 
 // One matvec on the warp-ring kernel: enough CTAs that every warp has a row
 // group, at most two per SM.
-int rw_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x, float *y, const DevInfo &di,
-              cudaStream_t st)
+int rw_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x, float *y, int n_tok,
+              const DevInfo &di, cudaStream_t st)
 {
     const int64_t x_floats = cols;
-    const RwGeom g = rw_geom(fmt, x_floats, 1);
+    const RwGeom g = rw_geom(fmt, x_floats, 1, n_tok);
     if (g.R == 0) return QMV_ERR_SHAPE;
     RwParams1 p{};
     p.n_tasks = 1;
@@ -382,7 +408,17 @@ int rw_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x
     p.cta_begin[0] = 0;
     p.cta_begin[1] = (int)ctas;
     rw_split(p.t[0], ctas * NW);
-    const cudaError_t e = rw_launch(fmt, p, g.R, dim3((unsigned)ctas), g.smem, st, g_pdl.load() != 0, false);
+    const bool pdl = g_pdl.load() != 0;
+    cudaError_t e;
+    if (n_tok == 1) {
+        e = rw_launch(fmt, p, g.R, dim3((unsigned)ctas), g.smem, st, pdl, false);
+    } else {
+        switch (fmt) {
+        case QMV_Q8_0: e = launch_rw_mt<FMT_Q8_0>(p, n_tok, g.R, dim3((unsigned)ctas), g.smem, st, pdl); break;
+        case QMV_Q4_K: e = launch_rw_mt<FMT_Q4_K>(p, n_tok, g.R, dim3((unsigned)ctas), g.smem, st, pdl); break;
+        default: e = launch_rw_mt<FMT_Q6_K>(p, n_tok, g.R, dim3((unsigned)ctas), g.smem, st, pdl); break;
+        }
+    }
     return e == cudaSuccess ? QMV_OK : cuda_fail(e);
 }
 
@@ -484,8 +520,8 @@ int qmv_batched(int fmt, const void *W_blocks, int64_t rows, int64_t cols, const
     if (injected_failure()) return QMV_ERR_CUDA;
     DevInfo di;
     if ((rc = get_dev(di))) return rc;
-    if (n_tok == 1 && rw_preferred(fmt, rows, cols))
-        return rw_single(fmt, W_blocks, rows, cols, x, y, di, reinterpret_cast<cudaStream_t>(stream));
+    if (n_tok == 1 ? rw_preferred(fmt, rows, cols) : rw_mt_preferred(fmt, rows, cols, n_tok))
+        return rw_single(fmt, W_blocks, rows, cols, x, y, n_tok, di, reinterpret_cast<cudaStream_t>(stream));
     Plan pl;
     if ((rc = make_plan(fmt, rows, cols, n_tok, 1, 1, true, di, pl))) return rc;
     pl.p.mode = MODE_SEPARATE;

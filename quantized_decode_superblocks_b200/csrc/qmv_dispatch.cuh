@@ -121,7 +121,7 @@ struct MultiLaunch {
     cudaError_t run() const { return Instance<FMT, NTOK, R, XREG>::multi(mp, grid, smem, st, pdl); }
 };
 
-template <int FMT, int R, int NT>
+template <int FMT, int R, int NT, int NTOK = 1>
 struct RwInstance {
     static int *configured()
     {
@@ -130,7 +130,7 @@ struct RwInstance {
     }
     static cudaError_t go(const RwParamsT<NT> &p, dim3 grid, size_t smem, cudaStream_t st, bool pdl, bool coop)
     {
-        return launch_with(qmv_rw_kernel<FMT, R, NT>, configured(), p, grid, smem, st, pdl, coop);
+        return launch_with(qmv_rw_kernel<FMT, R, NT, NTOK>, configured(), p, grid, smem, st, pdl, coop);
     }
     static cudaError_t occupancy(size_t smem, int *n)
     {
@@ -139,12 +139,12 @@ struct RwInstance {
         if (e != cudaSuccess) return e;
         if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
         if (configured()[dev] < (int)smem) {
-            e = cudaFuncSetAttribute(qmv_rw_kernel<FMT, R, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            e = cudaFuncSetAttribute(qmv_rw_kernel<FMT, R, NT, NTOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)smem);
             if (e != cudaSuccess) return e;
             configured()[dev] = (int)smem;
         }
-        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(n, qmv_rw_kernel<FMT, R, NT>, NTHREADS, smem);
+        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(n, qmv_rw_kernel<FMT, R, NT, NTOK>, NTHREADS, smem);
     }
 };
 
@@ -157,6 +157,27 @@ cudaError_t launch_rw(const RwParamsT<NT> &p, int R, dim3 grid, size_t smem, cud
     case 2: return RwInstance<FMT, 2, NT>::go(p, grid, smem, stream, pdl, cooperative);
     case 4: return RwInstance<FMT, 4, NT>::go(p, grid, smem, stream, pdl, cooperative);
     default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int FMT, int NTOK>
+static cudaError_t launch_rw_mt_r(const RwParams1 &p, int R, dim3 grid, size_t smem, cudaStream_t stream, bool pdl)
+{
+    switch (R) {
+    case 1: return RwInstance<FMT, 1, 1, NTOK>::go(p, grid, smem, stream, pdl, false);
+    case 2: return RwInstance<FMT, 2, 1, NTOK>::go(p, grid, smem, stream, pdl, false);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int FMT>
+cudaError_t launch_rw_mt(const RwParams1 &p, int n_tok, int R, dim3 grid, size_t smem, cudaStream_t stream, bool pdl)
+{
+    switch (n_tok) {
+    case 2: return launch_rw_mt_r<FMT, 2>(p, R, grid, smem, stream, pdl);
+    case 3: return launch_rw_mt_r<FMT, 3>(p, R, grid, smem, stream, pdl);
+    case 4: return launch_rw_mt_r<FMT, 4>(p, R, grid, smem, stream, pdl);
+    default: return cudaErrorInvalidValue;      // 5..8 tokens take the general kernel
     }
 }
 

@@ -76,7 +76,7 @@ struct RwParamsT {
     int32_t ordered;          // chained: grid barrier between consecutive tasks (cooperative launch)
     int32_t n_stage;          // ring stages per warp
     int32_t stage_pitch;      // bytes per stage (multiple of 128)
-    int32_t x_floats;         // shared-memory x: the longest task row (floats)
+    int32_t x_floats;         // shared-memory x: the longest task row (floats), one such row per token
     int32_t cta_begin[NT + 1];   // not chained: task t owns CTAs [cta_begin[t], cta_begin[t+1])
     unsigned *sync;           // ordered: {arrivals, exits} of the grid barrier, zero between launches
     int *err;
@@ -293,10 +293,35 @@ __device__ __forceinline__ void rw_grid_exit(unsigned *sync, unsigned n_ctas)
     }
 }
 
-template <int FMT, int R, int NT>
+// Accumulators of one row group: one token -> a float per row (factored
+// decode); several tokens -> a packed pair per (row, token) (weight-stationary
+// decode units of qmv_decodemt.cuh).
+template <int R, int NTOK> struct RwAcc {
+    float2 v[R][NTOK];
+    __device__ __forceinline__ void zero()
+    {
+#pragma unroll
+        for (int k = 0; k < R; ++k)
+#pragma unroll
+            for (int t = 0; t < NTOK; ++t) v[k][t] = make_float2(0.f, 0.f);
+    }
+};
+template <int R> struct RwAcc<R, 1> {
+    float v[R];
+    __device__ __forceinline__ void zero()
+    {
+#pragma unroll
+        for (int k = 0; k < R; ++k) v[k] = 0.f;
+    }
+};
+
+template <int FMT, int R, int NT, int NTOK>
 __global__ void __launch_bounds__(NTHREADS, 2) qmv_rw_kernel(const __grid_constant__ RwParamsT<NT> p)
 {
     static_assert(R == 1 || R == 2 || R == 4 || R == 8, "R");
+    static_assert(NTOK >= 1 && NTOK <= 8 && (NTOK == 1 || NT == 1), "several tokens: single launches only");
+    constexpr int NTP = Pow2Ceil<NTOK>::v;
+    static_assert(R * NTP <= 32, "R * n_tok too large for one warp reduction");
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = (int)threadIdx.x >> 5, lane = (int)threadIdx.x & 31;
     const uint32_t sraw = smem_addr(smem);
@@ -305,7 +330,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) qmv_rw_kernel(const __grid_consta
     const uint32_t full0 = sbase + 8u * (uint32_t)(warp * RW_MAX_STAGES);
     RwTask *const tasks = reinterpret_cast<RwTask *>(smem + (sbase - sraw) + RW_BAR_BYTES);
     const uint32_t xs = sbase + (uint32_t)rw_hdr_bytes(p.n_tasks);
-    const uint32_t x_area = (uint32_t)(((p.x_floats * 4) + 127) & ~127);
+    const uint32_t x_area = (uint32_t)NTOK * (uint32_t)(((p.x_floats * 4) + 127) & ~127);   // one row per token
     const uint32_t stage0 = xs + x_area + (uint32_t)(warp * S) * (uint32_t)p.stage_pitch;
 
     int t_begin, t_end, wg;
@@ -371,7 +396,10 @@ __global__ void __launch_bounds__(NTHREADS, 2) qmv_rw_kernel(const __grid_consta
         // few float4s) and every warp takes its slices from there: one 8 KB
         // read per CTA from L2 instead of one per warp, which matters because
         // those L2 reads queue behind the weight copies in flight.
-        rw_stage_x(xs, tk.x, (nch - 1) * RW_CK + tk.last_cols, coherent);
+        const int cols_t = (nch - 1) * RW_CK + tk.last_cols;
+        const uint32_t xrow = (uint32_t)((cols_t * 4 + 127) & ~127);   // bytes per token row of staged x
+#pragma unroll 1
+        for (int n = 0; n < NTOK; ++n) rw_stage_x(xs + (uint32_t)n * xrow, tk.x + (int64_t)n * cols_t, cols_t, coherent);
         __syncthreads();
         int64_t a, b;
         rw_range(tk, wg, a, b);
@@ -387,7 +415,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) qmv_rw_kernel(const __grid_consta
         const uint32_t chunk_bytes = (uint32_t)tk.chunk_bytes;
         // one tile: wait for the stage, decode R rows of it, hand the stage back
         // to the producer (refilled with the tile S ahead)
-        auto tile = [&](float (&acc)[R], int ncols, uint32_t cb) -> bool {
+        auto tile = [&](RwAcc<R, NTOK> &acc, int ncols, uint32_t cb, int kc) -> bool {
             const uint32_t full = full0 + 8u * (uint32_t)slot;
             // every lane times its own wait: agree on the outcome so the warp stays converged
             if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(full, phase))) {
@@ -397,16 +425,43 @@ __global__ void __launch_bounds__(NTHREADS, 2) qmv_rw_kernel(const __grid_consta
             ++consumed;
             const uint32_t st = stage0 + (uint32_t)slot * pitch;
             if (64 * (lane + 1) <= ncols) {
-                auto xp = [&](int gq, float2 &x02, float2 &x13) {
-                    x02 = xr[gq][0];
-                    x13 = xr[gq][1];
-                };
-                uint32_t sa = rw_slice_addr<FMT>(st, lane);
+                if constexpr (NTOK == 1) {
+                    auto xp = [&](int gq, float2 &x02, float2 &x13) {
+                        x02 = xr[gq][0];
+                        x13 = xr[gq][1];
+                    };
+                    uint32_t sa = rw_slice_addr<FMT>(st, lane);
 #pragma unroll
-                for (int k = 0; k < R; ++k, sa += cb) {
-                    if (FMT == FMT_Q8_0) acc[k] += q8_0_dot_pair(sa, xp);
-                    else if (FMT == FMT_Q4_K) acc[k] += q4_k_dot1<false>(sa, lane & 3, sel, xp, xsa, xsb);
-                    else acc[k] += q6_k_dot1(sa, (lane >> 1) & 1, 16 * (lane & 1), xp);
+                    for (int k = 0; k < R; ++k, sa += cb) {
+                        if (FMT == FMT_Q8_0) acc.v[k] += q8_0_dot_pair(sa, xp);
+                        else if (FMT == FMT_Q4_K) acc.v[k] += q4_k_dot1<false>(sa, lane & 3, sel, xp, xsa, xsb);
+                        else acc.v[k] += q6_k_dot1(sa, (lane >> 1) & 1, 16 * (lane & 1), xp);
+                    }
+                } else {
+                    // several tokens: weights decoded once per step, each token's
+                    // x (staged, swizzled) spent on all R rows
+                    auto xl = [&](int n, int col) {
+                        return lds_f4(xs + (uint32_t)n * xrow + 16u * rw_xswz((uint32_t)col >> 2));
+                    };
+                    const int cbase = kc * RW_CK;
+                    uint32_t bp[R];
+                    if (FMT == FMT_Q8_0) {
+#pragma unroll
+                        for (int b = 0; b < 2; ++b) {
+#pragma unroll
+                            for (int k = 0; k < R; ++k) bp[k] = st + (uint32_t)k * cb + 68u * (uint32_t)lane + 34u * (uint32_t)b;
+                            q8_0_slice_mt<NTOK, R>(bp, cbase + 64 * lane + 32 * b, xl, acc.v);
+                        }
+                    } else if (FMT == FMT_Q4_K) {
+#pragma unroll
+                        for (int k = 0; k < R; ++k) bp[k] = st + (uint32_t)k * cb + 144u * (uint32_t)(lane >> 2);
+                        q4_k_slice_mt<NTOK, R>(bp, lane & 3, sel, cbase + 64 * lane, xl, acc.v);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < R; ++k) bp[k] = st + (uint32_t)k * cb + 210u * (uint32_t)(lane >> 2);
+                        const int h = (lane >> 1) & 1, l0 = 16 * (lane & 1);
+                        q6_k_slice_mt<NTOK, R>(bp, h, l0, cbase + 256 * (lane >> 2) + 128 * h + l0, xl, acc.v);
+                    }
                 }
             }
             __syncwarp();
@@ -426,20 +481,29 @@ __global__ void __launch_bounds__(NTHREADS, 2) qmv_rw_kernel(const __grid_consta
             }
             return true;
         };
-        auto finish = [&](float (&acc)[R], int64_t rg) {
-            warp_transpose_reduce<R>(acc, lane);
-            constexpr int SH = 5 - Log2<R>::v;
-            const int64_t row = rg * R + (lane >> SH);
-            if ((lane & ((1 << SH) - 1)) == 0 && row < rows) ty[row] = acc[0];
+        auto finish = [&](RwAcc<R, NTOK> &acc, int64_t rg) {
+            constexpr int V = R * NTP;
+            float vals[V];
+#pragma unroll
+            for (int k = 0; k < R; ++k)
+#pragma unroll
+                for (int n = 0; n < NTP; ++n) {
+                    if constexpr (NTOK == 1) vals[k] = acc.v[k];
+                    else vals[k * NTP + n] = n < NTOK ? acc.v[k][n < NTOK ? n : 0].x + acc.v[k][n < NTOK ? n : 0].y : 0.f;
+                }
+            warp_transpose_reduce<V>(vals, lane);
+            constexpr int SH = 5 - Log2<V>::v;
+            const int idx = lane >> SH, k = idx / NTP, n = idx % NTP;
+            const int64_t row = rg * R + k;
+            if ((lane & ((1 << SH) - 1)) == 0 && n < NTOK && row < rows) ty[(int64_t)n * rows + row] = vals[0];
         };
         if (nch == 1) {
-            // x stays in registers for the whole task
-            rw_load_x_smem<FMT>(xs, 0, last_cols, lane, xr, xsa, xsb);
+            // one token: x stays in registers for the whole task
+            if constexpr (NTOK == 1) rw_load_x_smem<FMT>(xs, 0, last_cols, lane, xr, xsa, xsb);
             for (int64_t rg = a; rg < b; ++rg) {
-                float acc[R];
-#pragma unroll
-                for (int k = 0; k < R; ++k) acc[k] = 0.f;
-                if (!tile(acc, last_cols, last_bytes)) {
+                RwAcc<R, NTOK> acc;
+                acc.zero();
+                if (!tile(acc, last_cols, last_bytes, 0)) {
                     dead = true;
                     break;
                 }
@@ -447,14 +511,13 @@ __global__ void __launch_bounds__(NTHREADS, 2) qmv_rw_kernel(const __grid_consta
             }
         } else {
             for (int64_t rg = a; rg < b && !dead; ++rg) {
-                float acc[R];
-#pragma unroll
-                for (int k = 0; k < R; ++k) acc[k] = 0.f;
+                RwAcc<R, NTOK> acc;
+                acc.zero();
                 for (int kc = 0; kc < nch; ++kc) {
                     const bool lastc = kc == nch - 1;
                     const int ncols = lastc ? last_cols : RW_CK;
-                    rw_load_x_smem<FMT>(xs, kc, ncols, lane, xr, xsa, xsb);
-                    if (!tile(acc, ncols, lastc ? last_bytes : chunk_bytes)) {
+                    if constexpr (NTOK == 1) rw_load_x_smem<FMT>(xs, kc, ncols, lane, xr, xsa, xsb);
+                    if (!tile(acc, ncols, lastc ? last_bytes : chunk_bytes, kc)) {
                         dead = true;
                         break;
                     }
@@ -482,6 +545,9 @@ __global__ void __launch_bounds__(NTHREADS, 2) qmv_rw_kernel(const __grid_consta
 template <int FMT, int NT>
 cudaError_t launch_rw(const RwParamsT<NT> &p, int R, dim3 grid, size_t smem, cudaStream_t stream, bool pdl,
                       bool cooperative);
+// Several tokens (2..4), single launches.
+template <int FMT>
+cudaError_t launch_rw_mt(const RwParams1 &p, int n_tok, int R, dim3 grid, size_t smem, cudaStream_t stream, bool pdl);
 template <int FMT>
 cudaError_t rw_occupancy(int R, size_t smem, int *ctas_per_sm);
 
