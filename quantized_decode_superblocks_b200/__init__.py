@@ -28,7 +28,8 @@ DEVERR_TIMEOUT = 2
 EXPORTED = ("qmv_f32", "qmv_batched", "qmv_multi", "qmv_chain", "qmv_argmax", "moe_route", "moe_qmv", "moe_ffn", "moe_ffn_static",
             "qmv_dequant",
             "qmv_check", "qmv_strerror", "qmv_block_bytes", "qmv_block_weights",
-            "qmv_debug_fail_next_launches", "qmv_set_pdl", "qmv_get_pdl", "qmv_last_cuda_error")
+            "qmv_debug_fail_next_launches", "qmv_debug_short_copies", "qmv_set_pdl", "qmv_get_pdl",
+            "qmv_last_cuda_error")
 
 
 class QmvTask(ctypes.Structure):
@@ -77,14 +78,16 @@ def lib() -> ctypes.CDLL:
         L.qmv_block_weights.argtypes = [c_int]
         L.qmv_debug_fail_next_launches.argtypes = [c_int]
         L.qmv_debug_fail_next_launches.restype = None
+        L.qmv_debug_short_copies.argtypes = [c_int]
+        L.qmv_debug_short_copies.restype = None
         L.qmv_set_pdl.argtypes = [c_int]
         L.qmv_set_pdl.restype = None
         L.qmv_get_pdl.argtypes = []
         L.qmv_last_cuda_error.argtypes = []
         L.qmv_last_cuda_error.restype = ctypes.c_char_p
         for name in EXPORTED:
-            if name not in ("qmv_strerror", "qmv_block_bytes", "qmv_debug_fail_next_launches", "qmv_set_pdl",
-                            "qmv_last_cuda_error"):
+            if name not in ("qmv_strerror", "qmv_block_bytes", "qmv_debug_fail_next_launches",
+                            "qmv_debug_short_copies", "qmv_set_pdl", "qmv_last_cuda_error"):
                 getattr(L, name).restype = c_int
         _lib = L
     return _lib

@@ -58,6 +58,7 @@ std::mutex g_mu;
 DevInfo g_dev[64];
 std::atomic<int> g_fail_launches{0};
 std::atomic<int> g_pdl{0};
+std::atomic<unsigned> g_debug_extra_tx{0};
 thread_local cudaError_t t_last_cuda = cudaSuccess;
 
 int cuda_fail(cudaError_t e)
@@ -403,6 +404,7 @@ int rw_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x
     p.x_floats = (int32_t)x_floats;
     p.sync = di.sync;
     p.err = di.err;
+    p.debug_extra_tx = g_debug_extra_tx.load();
     p.t[0] = rw_task(fmt, g.R, W, rows, cols, x, y);
     const int64_t ctas = std::max<int64_t>(1, std::min<int64_t>(2LL * di.sm_count, ceil_div(p.t[0].n_rg, NW)));
     p.cta_begin[0] = 0;
@@ -451,6 +453,7 @@ int rw_chain(int fmt, const qmv_task *tasks, int n_tasks, const DevInfo &di, cud
         p.x_floats = (int32_t)x_floats;
         p.sync = di.sync;
         p.err = di.err;
+        p.debug_extra_tx = g_debug_extra_tx.load();
         // each task starts on the warp after the previous task's last row group
         int64_t rot = 0;
         for (int i = 0; i < n; ++i) {
@@ -485,6 +488,8 @@ int qmv_block_weights(int fmt) { return block_weights(fmt); }
 void qmv_debug_fail_next_launches(int count) { g_fail_launches.store(count > 0 ? count : 0); }
 
 void qmv_set_pdl(int enable) { g_pdl.store(enable ? 1 : 0); }
+
+void qmv_debug_short_copies(int bytes) { g_debug_extra_tx.store(bytes > 0 ? (unsigned)bytes : 0u); }
 
 int qmv_get_pdl(void) { return g_pdl.load(); }
 

@@ -80,6 +80,7 @@ struct RwParamsT {
     int32_t cta_begin[NT + 1];   // not chained: task t owns CTAs [cta_begin[t], cta_begin[t+1])
     unsigned *sync;           // ordered: {arrivals, exits} of the grid barrier, zero between launches
     int *err;
+    uint32_t debug_extra_tx;  // test hook: bytes expected per tile beyond those copied (0 in use)
     RwTask t[NT];
 };
 using RwParams1 = RwParamsT<1>;
@@ -140,14 +141,15 @@ __device__ __forceinline__ void rw_advance(const RwTask *tasks, RwCursor &c, int
 
 // Issue the copies of tile c into stage dst (called by one lane).
 template <int R>
-__device__ __forceinline__ void rw_issue(const RwTask *tasks, const RwCursor &c, uint32_t dst, uint32_t bar)
+__device__ __forceinline__ void rw_issue(const RwTask *tasks, const RwCursor &c, uint32_t dst, uint32_t bar,
+                                         uint32_t extra_tx)
 {
     const RwTask &tk = tasks[c.t];
     const int64_t r0 = c.rg * R;
     const int tr = (int)min((int64_t)R, tk.rows - r0);
     const bool lastc = c.kc == c.nch - 1;
     const uint32_t cb = (uint32_t)(lastc ? tk.last_bytes : tk.chunk_bytes);
-    mbar_arrive_expect_tx(bar, (uint32_t)tr * cb);
+    mbar_arrive_expect_tx(bar, (uint32_t)tr * cb + extra_tx);
     const uint8_t *src = tk.W + r0 * tk.row_bytes + (int64_t)c.kc * tk.chunk_bytes;
     if (c.nch == 1) {
         bulk_g2s(dst, src, (uint32_t)tr * cb, bar);      // the tile's rows are contiguous
@@ -367,7 +369,8 @@ __global__ void __launch_bounds__(NTHREADS, 2) qmv_rw_kernel(const __grid_consta
         rw_seek(tasks, f, t_begin, t_end, wg);
         f.issued = 0;
         for (int s = 0; s < S && f.t < t_end; ++s) {
-            rw_issue<R>(tasks, f, stage0 + (uint32_t)s * (uint32_t)p.stage_pitch, full0 + 8u * (uint32_t)s);
+            rw_issue<R>(tasks, f, stage0 + (uint32_t)s * (uint32_t)p.stage_pitch, full0 + 8u * (uint32_t)s,
+                        p.debug_extra_tx);
             rw_advance(tasks, f, t_end, wg);
             ++f.issued;
         }
@@ -469,7 +472,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) qmv_rw_kernel(const __grid_consta
                 RwCursor f = *cur;
                 if (f.t < t_end) {
                     fence_proxy_async_smem();
-                    rw_issue<R>(tasks, f, st, full);
+                    rw_issue<R>(tasks, f, st, full, p.debug_extra_tx);
                     rw_advance(tasks, f, t_end, wg);
                     ++f.issued;
                     *cur = f;

@@ -479,6 +479,26 @@ def test_moe_bad_expert_id_is_dropped_and_reported():
     assert np.array_equal(yh[1], np.zeros(rows, np.float32))
 
 
+def test_stage_wait_timeout_is_reported_and_the_gpu_stays_usable():
+    # the test hook makes every tile of the warp-ring kernel expect 16 bytes
+    # more than are copied: each stage wait runs out (about a second), the
+    # kernel records the timeout and finishes, and the context stays usable
+    fmt, rows, cols = Q8_0, 512, 2048
+    W = synth.gen_blocks(fmt, rows, cols, 45, 0)
+    x = synth.gen_x(1, cols, 45, 1)
+    y = torch.empty((1, rows), device="cuda")
+    q.lib().qmv_debug_short_copies(16)
+    try:
+        q.qmv_f32(fmt, dev(W), rows, cols, dev(x), y)
+        err = q.qmv_check()
+    finally:
+        q.lib().qmv_debug_short_copies(0)
+    assert err & q.DEVERR_TIMEOUT
+    assert q.qmv_check() == 0                      # cleared by the read
+    ref, bound = oracle.qmv(fmt, W, rows, cols, x)
+    within(run_qmv(fmt, W, rows, cols, x), ref, bound)
+
+
 def _check_moe_ffn(n_expert, hidden, inter, seed, ids, g32):
     gate, up, down, gus, ds, x = _moe_weights(n_expert, hidden, inter, seed)
     n_sel = len(ids)
