@@ -565,3 +565,45 @@ def test_moe_ffn_cfg3_routed_on_device():
 def test_moe_ffn_other_expert_counts(ids):
     g = np.random.default_rng(len(ids)).uniform(0.1, 1.0, len(ids)).astype(np.float32)
     _check_moe_ffn(8, 512, 768, 50 + len(ids), ids, g)
+
+
+@pytest.mark.parametrize("fmt,hidden,inter", [(Q4_K, 2048, 1792), (Q8_0, 1024, 512), (Q8_0, 4096, 1024)])
+def test_moe_ffn_formats_and_a_bad_expert_id(fmt, hidden, inter):
+    # Q8_0 experts, rows of more than one K-chunk (hidden 4096), and an expert id
+    # out of range: that expert contributes nothing (h row zero) and is reported
+    n_expert, ids, g32 = 6, [4, 1, 9, 3], np.array([0.4, 0.3, 0.2, 0.1], np.float32)
+    gus, ds = synth.matrix_bytes(fmt, inter, hidden), synth.matrix_bytes(fmt, hidden, inter)
+    gate = synth.gen_blocks(fmt, inter * n_expert, hidden, 61, 1)
+    up = synth.gen_blocks(fmt, inter * n_expert, hidden, 61, 2)
+    down = synth.gen_blocks(fmt, hidden * n_expert, inter, 61, 3)
+    x = synth.gen_x(1, hidden, 61, 4)[0]
+    h = torch.full((4, inter), float("nan"), device="cuda")
+    y = torch.full((hidden,), float("nan"), device="cuda")
+    q.moe_ffn(fmt, dev(gate), dev(up), gus, fmt, dev(down), ds, n_expert, dev(np.array(ids, np.int32)),
+              dev(g32), 4, hidden, inter, dev(x), h, y)
+    err = q.qmv_check()
+    assert err & q.DEVERR_EXPERT_ID
+    hh, yy = h.cpu().numpy(), y.cpu().numpy()
+    assert np.array_equal(hh[2], np.zeros(inter, np.float32))
+    good = [0, 1, 3]
+    ref = oracle.moe_ffn(fmt, gate, up, gus, fmt, down, ds, n_expert, np.array([ids[k] for k in good]),
+                         g32[good].astype(np.float64), hidden, inter, x)
+    # h of the valid experts: the composite rule (i) of _check_moe_ffn
+    for j, k in enumerate(good):
+        e = ids[k]
+        _, bu = oracle.qmv(fmt, gate[e * gus:(e + 1) * gus], inter, hidden, x)
+        _, bv = oracle.qmv(fmt, up[e * gus:(e + 1) * gus], inter, hidden, x)
+        du, dv = REL * bu[0] + ABS, REL * bv[0] + ABS
+        u, v = ref["u"][j], ref["v"][j]
+        su = u / (1 + np.exp(-u))
+        dh = 1.1 * du * np.abs(v) + np.abs(su) * dv + 1.1 * du * dv + 1e-6 * np.abs(ref["h"][j])
+        assert (np.abs(hh[k] - ref["h"][j]) <= dh + ABS).all(), k
+    # y from the GPU's own h: the weighted down sum over the valid experts
+    yref = np.zeros(hidden)
+    bnd = np.zeros(hidden)
+    for k in good:
+        r, b = oracle.qmv(fmt, down[ids[k] * ds:(ids[k] + 1) * ds], hidden, inter, hh[k][None, :])
+        yref += float(g32[k]) * r[0]
+        bnd += abs(float(g32[k])) * b[0]
+    within(yy[None, :], yref[None, :], bnd[None, :])
+    assert np.isfinite(ref["y"]).all()
