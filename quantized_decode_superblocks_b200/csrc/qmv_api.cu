@@ -249,6 +249,7 @@ int launch_plan(int fmt, const Plan &pl, cudaStream_t stream)
 // Dynamic shared memory of one CTA, two per SM: (228 KB - 2 x 1 KB reserved) / 2
 // = 113 KB, less the 128 bytes of alignment slack each launch adds.
 constexpr int64_t RW_CTA_SMEM = 113 * 1024 - 128;
+constexpr int64_t RW_CTA_SMEM_ONE = 227 * 1024 - 128;    // one CTA per SM (3-4 tokens)
 
 struct RwGeom {
     int R = 0;
@@ -264,7 +265,8 @@ RwGeom rw_geom(int fmt, int64_t x_floats, int n_tasks, int n_tok = 1)
     const int64_t cb = (RW_CK / block_weights(fmt)) * block_bytes(fmt);
     const int64_t x_area = n_tok * ceil_div(x_floats * 4, 128) * 128;
     const int64_t hdr = rw_hdr_bytes(n_tasks);
-    const int64_t per_warp = (RW_CTA_SMEM - hdr - x_area) / NW;
+    const int64_t budget = n_tok > 2 ? RW_CTA_SMEM_ONE : RW_CTA_SMEM;   // 3+ tokens: one CTA per SM
+    const int64_t per_warp = (budget - hdr - x_area) / NW;
     // the Q6_K decode and the several-token units read up to 4 bytes past a
     // slice (2-byte-aligned words): their stages carry 16 spare bytes
     const int64_t pad = (fmt == QMV_Q6_K || n_tok > 1) ? 16 : 0;
@@ -326,16 +328,15 @@ bool rw_preferred(int fmt, int64_t rows, int64_t cols)
     return fmt != QMV_Q4_K && rows <= 4096;
 }
 
-// Several tokens on the warp-ring kernel (measured on B200): two tokens for
-// every format, up to four for Q6_K; beyond that the general kernel's
-// weight-stationary loop with more rows per warp is faster.  Every token's x
-// must fit in shared memory beside two stages per warp (n_tok x cols <= 16384
-// floats).
+// Several tokens on the warp-ring kernel (measured on B200): up to four
+// tokens (three and four with one CTA per SM); beyond that the general
+// kernel's weight-stationary loop is faster.  Every token's x must fit in
+// shared memory beside two stages per warp (n_tok x cols <= 32768 floats).
 bool rw_mt_preferred(int fmt, int64_t rows, int64_t cols, int n_tok)
 {
     (void)rows;
-    if (n_tok > (fmt == QMV_Q6_K ? 4 : 2)) return false;
-    if (!rw_ok(fmt, cols) || (int64_t)n_tok * cols > 16384) return false;
+    if (n_tok > 4) return false;
+    if (!rw_ok(fmt, cols) || (int64_t)n_tok * cols > 32768) return false;
     return rw_geom(fmt, cols, 1, n_tok).R > 0;
 }
 
@@ -406,7 +407,8 @@ int rw_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x
     p.err = di.err;
     p.debug_extra_tx = g_debug_extra_tx.load();
     p.t[0] = rw_task(fmt, g.R, W, rows, cols, x, y);
-    const int64_t ctas = std::max<int64_t>(1, std::min<int64_t>(2LL * di.sm_count, ceil_div(p.t[0].n_rg, NW)));
+    const int64_t per_sm = n_tok > 2 ? 1 : 2;
+    const int64_t ctas = std::max<int64_t>(1, std::min<int64_t>(per_sm * di.sm_count, ceil_div(p.t[0].n_rg, NW)));
     p.cta_begin[0] = 0;
     p.cta_begin[1] = (int)ctas;
     rw_split(p.t[0], ctas * NW);

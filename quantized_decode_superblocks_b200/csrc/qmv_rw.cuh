@@ -317,8 +317,10 @@ template <int R> struct RwAcc<R, 1> {
     }
 };
 
+// Three or more tokens: one CTA per SM, with the SM's whole shared memory
+// (every token's x) and registers (the accumulators) -- no spills.
 template <int FMT, int R, int NT, int NTOK>
-__global__ void __launch_bounds__(NTHREADS, 2) qmv_rw_kernel(const __grid_constant__ RwParamsT<NT> p)
+__global__ void __launch_bounds__(NTHREADS, (NTOK > 2 ? 1 : 2)) qmv_rw_kernel(const __grid_constant__ RwParamsT<NT> p)
 {
     static_assert(R == 1 || R == 2 || R == 4 || R == 8, "R");
     static_assert(NTOK >= 1 && NTOK <= 8 && (NTOK == 1 || NT == 1), "several tokens: single launches only");
@@ -548,7 +550,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) qmv_rw_kernel(const __grid_consta
 template <int FMT, int NT>
 cudaError_t launch_rw(const RwParamsT<NT> &p, int R, dim3 grid, size_t smem, cudaStream_t stream, bool pdl,
                       bool cooperative);
-// Several tokens (2..4), single launches.
+// Several tokens (2..4), single launches (3 and 4: one CTA per SM).
 template <int FMT>
 cudaError_t launch_rw_mt(const RwParams1 &p, int n_tok, int R, dim3 grid, size_t smem, cudaStream_t stream, bool pdl);
 template <int FMT>
