@@ -10,6 +10,7 @@
 #include "../../include/qmv.h"
 #include "qmv_misc.cuh"
 #include "qmv_rw.cuh"
+#include "qmv_tc.cuh"
 
 namespace {
 
@@ -426,6 +427,74 @@ int rw_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x
     return e == cudaSuccess ? QMV_OK : cuda_fail(e);
 }
 
+// Several tokens of a Q8_0 matrix on the tensor-core kernel: one CTA of
+// TC_WARPS warps per SM, x in shared memory when it fits next to rings of at
+// least two stages, else read through L2.
+struct TcGeom {
+    bool ok = false;
+    bool x_smem = false;
+    int S = 0;
+    int ksplit = 1;
+    size_t smem = 0;
+};
+
+TcGeom tc_geom(int64_t cols, int n_tok, const DevInfo &di)
+{
+    TcGeom g;
+    const int tile = TC_ROWS * (TC_KCOLS / 32) * 34;
+    const int64_t kc_n = cols / TC_KCOLS;
+    g.ksplit = kc_n % 8 == 0 ? 8 : kc_n % 4 == 0 ? 4 : kc_n % 2 == 0 ? 2 : 1;
+    const int64_t budget = (int64_t)std::min(di.smem_optin, 227 * 1024) - 128 - TC_BAR_BYTES - tc_part_bytes(TC_WARPS);
+    int64_t xb = ((int64_t)n_tok * (cols + 4) * 4 + 127) & ~(int64_t)127;
+    int64_t S = (budget - xb) / ((int64_t)TC_WARPS * tile);
+    g.x_smem = S >= 2;
+    if (!g.x_smem) {
+        xb = 0;
+        S = budget / ((int64_t)TC_WARPS * tile);
+    }
+    S = std::min<int64_t>(S, TC_MAX_STAGES);
+    if (S < 2) return g;
+    g.S = (int)S;
+    g.smem = (size_t)(128 + TC_BAR_BYTES + xb + tc_part_bytes(TC_WARPS) + (int64_t)TC_WARPS * S * tile);
+    g.ok = true;
+    return g;
+}
+
+// Q8_0 with 4..8 tokens whose rows are whole 256-column K-chunks.
+bool tc_preferred(int fmt, int64_t rows, int64_t cols, int n_tok)
+{
+    return fmt == QMV_Q8_0 && n_tok >= 4 && n_tok <= 8 && cols % TC_KCOLS == 0 && cols <= (int64_t)1 << 24 &&
+           rows <= (int64_t)INT_MAX;
+}
+
+int tc_single(const void *W, int64_t rows, int64_t cols, const float *x, float *y, int n_tok, const DevInfo &di,
+              cudaStream_t st)
+{
+    const TcGeom g = tc_geom(cols, n_tok, di);
+    if (!g.ok) return QMV_ERR_SHAPE;
+    TcParams p{};
+    p.W = static_cast<const uint8_t *>(W);
+    p.x = x;
+    p.y = y;
+    p.rows = rows;
+    p.row_bytes = cols / 32 * 34;
+    p.cols = (int32_t)cols;
+    p.n_tok = n_tok;
+    p.kc_n = (int32_t)(cols / TC_KCOLS);
+    p.chunk_bytes = TC_KCOLS / 32 * 34;
+    p.ksplit = g.ksplit;
+    const int64_t n_rt = ceil_div(rows, (int64_t)TC_ROWS);
+    p.n_rt = (int32_t)n_rt;
+    const int64_t ctas = std::max<int64_t>(1, std::min<int64_t>(n_rt, di.sm_count));
+    p.rt_q = (int32_t)(n_rt / ctas);
+    p.rt_r = (int32_t)(n_rt % ctas);
+    p.n_stage = g.S;
+    p.x_pitch = (int32_t)(cols + 4);
+    p.err = di.err;
+    const cudaError_t e = launch_tc<FMT_Q8_0>(p, g.x_smem, dim3((unsigned)ctas), g.smem, st, g_pdl.load() != 0);
+    return e == cudaSuccess ? QMV_OK : cuda_fail(e);
+}
+
 // In-order one-token matvecs of one format on the warp-ring kernel, up to
 // RW_MAX_TASKS per launch.  Every CTA works on every task, in order, each
 // task's row groups spread over all warps (so small and large tasks alike use
@@ -527,6 +596,8 @@ int qmv_batched(int fmt, const void *W_blocks, int64_t rows, int64_t cols, const
     if (injected_failure()) return QMV_ERR_CUDA;
     DevInfo di;
     if ((rc = get_dev(di))) return rc;
+    if (tc_preferred(fmt, rows, cols, n_tok) && tc_geom(cols, n_tok, di).ok)
+        return tc_single(W_blocks, rows, cols, x, y, n_tok, di, reinterpret_cast<cudaStream_t>(stream));
     if (n_tok == 1 ? rw_preferred(fmt, rows, cols) : rw_mt_preferred(fmt, rows, cols, n_tok))
         return rw_single(fmt, W_blocks, rows, cols, x, y, n_tok, di, reinterpret_cast<cudaStream_t>(stream));
     Plan pl;

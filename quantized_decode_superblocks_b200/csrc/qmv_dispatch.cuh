@@ -4,6 +4,7 @@
 #pragma once
 
 #include "qmv_rw.cuh"
+#include "qmv_tc.cuh"
 
 namespace qmv {
 
@@ -11,7 +12,7 @@ namespace qmv {
 // (kernel, device) and adds the programmatic-serialization attribute when asked.
 template <class Kern, class Arg>
 static cudaError_t launch_with(Kern kern, int *configured, const Arg &arg, dim3 grid, size_t smem,
-                               cudaStream_t stream, bool pdl, bool cooperative = false)
+                               cudaStream_t stream, bool pdl, bool cooperative = false, int threads = NTHREADS)
 {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -36,7 +37,7 @@ static cudaError_t launch_with(Kern kern, int *configured, const Arg &arg, dim3 
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
-    cfg.blockDim = dim3(NTHREADS);
+    cfg.blockDim = dim3((unsigned)threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cfg.attrs = n_attr ? attr : nullptr;
@@ -204,6 +205,16 @@ cudaError_t launch_multi(const MultiParams &mp, const KernelChoice &kc, int grid
                          cudaStream_t stream)
 {
     return pick<FMT>(kc, MultiLaunch{mp, dim3((unsigned)grid), smem, stream, kc.pdl});
+}
+
+// The tensor-core several-token kernel (Q8_0): x in shared memory or through L2.
+template <int FMT>
+cudaError_t launch_tc(const TcParams &p, bool x_smem, dim3 grid, size_t smem, cudaStream_t st, bool pdl)
+{
+    static int configured_s[64] = {0}, configured_g[64] = {0};
+    if (x_smem)
+        return launch_with(qmv_tc_kernel<FMT, TC_WARPS, true>, configured_s, p, grid, smem, st, pdl, false, TC_WARPS * 32);
+    return launch_with(qmv_tc_kernel<FMT, TC_WARPS, false>, configured_g, p, grid, smem, st, pdl, false, TC_WARPS * 32);
 }
 
 }  // namespace qmv
