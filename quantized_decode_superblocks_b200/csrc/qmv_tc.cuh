@@ -1,26 +1,28 @@
-// qmv_tc.cuh -- several-token (3..8) Q8_0 matvec on the tensor cores.
+// qmv_tc.cuh -- several-token (4..8) Q8_0 matvec on the tensor cores.
 //
 // With n_tok tokens every weight feeds n_tok products; on the CUDA cores that
 // is n_tok FMAs plus n_tok x reads per weight, which made the 8-token decode
-// step six times slower than the 1-token one.  Here the weights of a tile of
-// 16 rows are decoded exactly (Q8_0 quants are small integers, exact in
-// TF32) straight into the A fragments of mma.m16n8k8 (TF32 in, f32
-// accumulate) and the tokens form the N = 8 columns.  x is split as
-// hi = tf32(x), lo = x - hi: two MMAs per k-step keep the products within
-// about 2^-21 of f32 (TF32 alone would lose 11 bits of x).  Each 32-column
-// block's sum is scaled by its f32 d in registers (GGUF Q8_0 layout: one fp16
-// d and 32 int8 quants per block; dequantized weight d * q), so only
-// integers go through the tensor cores.
+// step several times slower than the 1-token one.  Here the weights of a
+// tile of 16 rows are decoded exactly (Q8_0 quants are integers in
+// [-128, 127], exact in bf16) straight into the A fragments of
+// mma.m16n8k16 (bf16 in, f32 accumulate), and the tokens form the N = 8
+// columns.  x is split into two bf16 halves, hi (the float's upper 16 bits)
+// and lo (the remainder, rounded): two MMAs per k-step keep every product
+// within 2^-16 of f32, against a tolerance of 1e-4 of sum |w x|.  Each
+// 32-column block's sum is scaled by its f32 d in registers (GGUF Q8_0
+// layout: one fp16 d and 32 int8 quants per block; the dequantized weight is
+// d * q), so only integers and the split x go through the tensor cores.
 //
-// Data flow: one CTA per SM (16 warps); the CTA's x rows sit in shared
-// memory (token-major, row pitch cols + 4 floats so a warp's 16-byte loads
-// hit all banks once) or, when they do not fit next to the rings, are read
-// through L2.  A unit is one tile (16 rows x 256 columns = 4352 bytes),
-// copied by `cp.async.bulk` (one copy per row) into a warp-private ring of
-// stages on an mbarrier, as in the warp-ring kernel.  The CTA's row tiles go
-// to groups of `ksplit` warps; the warps of a group split the K-chunks of a
-// tile, add their partial sums in a fixed order through shared memory
-// (named barrier per group) and write y.
+// Data flow: one CTA per SM (16 warps).  The CTA's x rows sit in shared
+// memory already split (token-major; 32 bytes per 8 columns, 16 of hi pairs
+// and 16 of lo pairs; row pitch cols * 4 + 16 bytes, so a warp's 16-byte
+// loads hit all banks once) or, when they do not fit next to the rings, are
+// read through L2 and split per tile.  A unit is one tile (16 rows x 256
+// columns = 4352 bytes), copied by `cp.async.bulk` (one copy per row) into a
+// warp-private ring of stages on an mbarrier, as in the warp-ring kernel.
+// The CTA's row tiles go to groups of `ksplit` warps; the warps of a group
+// split the K-chunks of a tile, add their partial sums in a fixed order
+// through shared memory (a named barrier per group) and write y.
 #pragma once
 
 #include "qmv_kernels.cuh"
@@ -48,33 +50,11 @@ struct TcParams {
     int32_t n_rt;          // row tiles in the matrix
     int32_t rt_q, rt_r;    // CTA c owns rt_q + (c < rt_r) consecutive row tiles
     int32_t n_stage;       // ring stages per warp
-    int32_t x_pitch;       // floats per token row of shared x (cols + 4)
+    int32_t x_pitch;       // 4-byte words per token row of shared x (cols + 4)
     int *err;
 };
 
 __host__ __device__ constexpr uint32_t tc_round128(uint32_t b) { return (b + 127u) & ~127u; }
-
-// Round-to-nearest TF32 of v, as a 32-bit pattern with the low 13 bits clear.
-__device__ __forceinline__ uint32_t tf32_rna(float v)
-{
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(v));
-    return r;
-}
-
-// d[0..3] += A (16x8, TF32) * B (8x8, TF32), f32 accumulation.  Fragments as
-// the PTX ISA defines them for m16n8k8 (g = lane / 4, t = lane % 4):
-// a0 (g, t), a1 (g + 8, t), a2 (g, t + 4), a3 (g + 8, t + 4);
-// b0 (k = t, n = g), b1 (k = t + 4, n = g);
-// d0 (g, 2t), d1 (g, 2t + 1), d2 (g + 8, 2t), d3 (g + 8, 2t + 1).
-__device__ __forceinline__ void mma_tf32(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1)
-{
-    asm("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
-                 "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 
 // Bytes 8t .. 8t + 7 of block b's quants in one row of a stage (row at
 // shared address rp, 16-byte aligned; block b at rp + 34 b, its quants two
@@ -91,30 +71,6 @@ __device__ __forceinline__ void tc_q8_words(uint32_t rp, int t, uint32_t &u0, ui
         const uint32_t w0 = lds_u32(a), w1 = lds_u32(a + 4u), w2 = lds_u32(a + 8u);
         u0 = __byte_perm(w0, w1, 0x5432u);
         u1 = __byte_perm(w1, w2, 0x5432u);
-    }
-}
-
-// x[token g][32b + 8t .. + 7] of block b as TF32 hi / lo halves (B fragments),
-// from shared memory (XS; xrow a shared address) or through L2 (xg).
-template <bool XS>
-__device__ __forceinline__ void tc_x_frag(uint32_t xrow, const float *xg, int b, int t, bool have_x,
-                                          uint32_t (&bh)[8], uint32_t (&bl)[8])
-{
-    float4 xa = make_float4(0.f, 0.f, 0.f, 0.f), xb = xa;
-    if (have_x) {
-        if (XS) {
-            xa = lds_f4(xrow + 4u * (uint32_t)(32 * b + 8 * t));
-            xb = lds_f4(xrow + 4u * (uint32_t)(32 * b + 8 * t + 4));
-        } else {
-            xa = __ldg(reinterpret_cast<const float4 *>(xg + 32 * b + 8 * t));
-            xb = __ldg(reinterpret_cast<const float4 *>(xg + 32 * b + 8 * t + 4));
-        }
-    }
-    const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        bh[i] = tf32_rna(xv[i]);
-        bl[i] = __float_as_uint(xv[i] - __uint_as_float(bh[i]));
     }
 }
 
@@ -140,36 +96,100 @@ __device__ __forceinline__ void tc_q8_frag(uint32_t ra, uint32_t rb, int t, floa
     }
 }
 
-// One 16 x 256 Q8_0 tile against the 8 token columns: acc (rows g, g + 8;
-// tokens 2t, 2t + 1) += sum over the 8 blocks of d_row * (q . x).
-// Column map: the k-step s of block b gives thread t the columns
-// 32b + 8t + 2s (logical k = t) and 32b + 8t + 2s + 1 (k = t + 4), on both
-// the A and the B side, so a thread's A bytes and x values are 8 consecutive
-// columns.  Two blocks at a time, each with separate hi and lo accumulators:
-// four independent MMA chains of four, so a warp does not wait out the MMA
-// latency at every step.
-template <int B0, bool XS>
-__device__ __forceinline__ void tc_q8_pair(uint32_t ra, uint32_t rb, uint32_t xrow, const float *xg, bool have_x, int t,
-                                           float (&acc)[4])
+// d[0..3] += A (16x16, bf16) * B (16x8, bf16), f32 accumulation.  Fragments
+// (PTX ISA, m16n8k16; each register holds two bf16, the lower column / row
+// in the low half): a0 (g; 2t, 2t+1), a1 (g + 8; 2t, 2t+1), a2 (g; 2t+8,
+// 2t+9), a3 (g + 8; 2t+8, 2t+9); b0 (k = 2t, 2t+1; n = g), b1 (k = 2t+8,
+// 2t+9; n = g); d as for m16n8k8.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1)
 {
-    uint32_t h0[8], l0[8], h1[8], l1[8];
-    tc_x_frag<XS>(xrow, xg, B0, t, have_x, h0, l0);
-    tc_x_frag<XS>(xrow, xg, B0 + 1, t, have_x, h1, l1);
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// bf16x2 {lo, hi} rounded to nearest from two floats.
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Columns c .. c + 7 of one x row as bf16 pairs: hi = the upper 16 bits of
+// each float (exact truncation), lo = bf16 of the remainder x - hi (exact in
+// f32), so |x - hi - lo| <= 2^-16 |x| and every product q (hi + lo) is
+// within 2^-16 of q x.  Pair i holds columns c + 2i, c + 2i + 1.
+__device__ __forceinline__ void tc_split_x8(float4 xa, float4 xb, uint4 &bh, uint4 &bl)
+{
+    const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t u0 = __float_as_uint(xv[2 * i]), u1 = __float_as_uint(xv[2 * i + 1]);
+        h[i] = __byte_perm(u0, u1, 0x7632u);
+        const float2 r = f2fma(make_float2(__uint_as_float(u0 & 0xFFFF0000u), __uint_as_float(u1 & 0xFFFF0000u)),
+                               make_float2(-1.0f, -1.0f), make_float2(xv[2 * i], xv[2 * i + 1]));
+        l[i] = bf16x2_rn(r.x, r.y);
+    }
+    bh = make_uint4(h[0], h[1], h[2], h[3]);
+    bl = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// B fragments of block b for thread t: x[token g][32b + 8t .. + 7] as hi /
+// lo bf16 pairs.  XS: already split in shared memory (xrow: the token's row
+// there, 32 bytes per 8 columns: 16 of hi pairs, 16 of lo pairs); else
+// read through L2 (xg) and split here.
+template <bool XS>
+__device__ __forceinline__ void tc_x_frag(uint32_t xrow, const float *xg, int b, int t, bool have_x, uint4 &bh,
+                                          uint4 &bl)
+{
+    bh = make_uint4(0u, 0u, 0u, 0u);
+    bl = bh;
+    if (!have_x) return;
+    if (XS) {
+        const uint32_t a = xrow + 32u * (uint32_t)(4 * b + t);
+        bh = lds_v4(a);
+        bl = lds_v4(a + 16u);
+    } else {
+        const float4 xa = __ldg(reinterpret_cast<const float4 *>(xg + 32 * b + 8 * t));
+        const float4 xb = __ldg(reinterpret_cast<const float4 *>(xg + 32 * b + 8 * t + 4));
+        tc_split_x8(xa, xb, bh, bl);
+    }
+}
+
+// Two blocks on bf16 MMAs: the quants (|q| <= 128, exact in bf16) packed in
+// column pairs; k-step s (0, 1) of block b gives thread t the columns
+// 32b + 8t + 4s, +1 (k = 2t, 2t+1) and +2, +3 (k = 2t+8, 2t+9).
+template <int B0, bool XS>
+__device__ __forceinline__ void tc_q8_pair_bf16(uint32_t ra, uint32_t rb, uint32_t xrow, const float *xg, bool have_x,
+                                                int t, float (&acc)[4])
+{
+    uint4 x0h, x0l, x1h, x1l;
+    tc_x_frag<XS>(xrow, xg, B0, t, have_x, x0h, x0l);
+    tc_x_frag<XS>(xrow, xg, B0 + 1, t, have_x, x1h, x1l);
+    const uint32_t h0[4] = {x0h.x, x0h.y, x0h.z, x0h.w}, l0[4] = {x0l.x, x0l.y, x0l.z, x0l.w};
+    const uint32_t h1[4] = {x1h.x, x1h.y, x1h.z, x1h.w}, l1[4] = {x1l.x, x1l.y, x1l.z, x1l.w};
     float q0[16], q1[16];
     tc_q8_frag<B0>(ra, rb, t, q0);
     tc_q8_frag<B0 + 1>(ra, rb, t, q1);
+    uint32_t p0[8], p1[8];       // [row half h][pair i]: columns 2i, 2i + 1
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        p0[i] = bf16x2_rn(q0[2 * i], q0[2 * i + 1]);
+        p1[i] = bf16x2_rn(q1[2 * i], q1[2 * i + 1]);
+    }
     float c0h[4] = {0.f, 0.f, 0.f, 0.f}, c0l[4] = {0.f, 0.f, 0.f, 0.f};
     float c1h[4] = {0.f, 0.f, 0.f, 0.f}, c1l[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
-        const uint32_t a0 = __float_as_uint(q0[2 * s]), a2 = __float_as_uint(q0[2 * s + 1]);
-        const uint32_t a1 = __float_as_uint(q0[8 + 2 * s]), a3 = __float_as_uint(q0[8 + 2 * s + 1]);
-        const uint32_t e0 = __float_as_uint(q1[2 * s]), e2 = __float_as_uint(q1[2 * s + 1]);
-        const uint32_t e1 = __float_as_uint(q1[8 + 2 * s]), e3 = __float_as_uint(q1[8 + 2 * s + 1]);
-        mma_tf32(c0h, a0, a1, a2, a3, h0[2 * s], h0[2 * s + 1]);
-        mma_tf32(c1h, e0, e1, e2, e3, h1[2 * s], h1[2 * s + 1]);
-        mma_tf32(c0l, a0, a1, a2, a3, l0[2 * s], l0[2 * s + 1]);
-        mma_tf32(c1l, e0, e1, e2, e3, l1[2 * s], l1[2 * s + 1]);
+    for (int s = 0; s < 2; ++s) {
+        // a0: row g pair 2s; a2: row g pair 2s + 1; a1 / a3: row g + 8
+        mma_bf16(c0h, p0[2 * s], p0[4 + 2 * s], p0[2 * s + 1], p0[4 + 2 * s + 1], h0[2 * s], h0[2 * s + 1]);
+        mma_bf16(c1h, p1[2 * s], p1[4 + 2 * s], p1[2 * s + 1], p1[4 + 2 * s + 1], h1[2 * s], h1[2 * s + 1]);
+        mma_bf16(c0l, p0[2 * s], p0[4 + 2 * s], p0[2 * s + 1], p0[4 + 2 * s + 1], l0[2 * s], l0[2 * s + 1]);
+        mma_bf16(c1l, p1[2 * s], p1[4 + 2 * s], p1[2 * s + 1], p1[4 + 2 * s + 1], l1[2 * s], l1[2 * s + 1]);
     }
     const float da0 = half_bits_to_float(lds_u16(ra + 34u * B0)), db0 = half_bits_to_float(lds_u16(rb + 34u * B0));
     const float da1 = half_bits_to_float(lds_u16(ra + 34u * (B0 + 1))), db1 = half_bits_to_float(lds_u16(rb + 34u * (B0 + 1)));
@@ -183,16 +203,18 @@ __device__ __forceinline__ void tc_q8_pair(uint32_t ra, uint32_t rb, uint32_t xr
     acc[3] = fmaf(db1, c1h[3] + c1l[3], acc[3]);
 }
 
+// One 16 x 256 Q8_0 tile against the 8 token columns: acc (rows g, g + 8;
+// tokens 2t, 2t + 1) += sum over the 8 blocks of d_row * (q . x).
 template <bool XS>
 __device__ __forceinline__ void tc_q8_tile(uint32_t st, int chunk_bytes, uint32_t xrow, const float *xg, bool have_x,
                                            int g, int t, float (&acc)[4])
 {
     const uint32_t ra = st + (uint32_t)(g * chunk_bytes);
     const uint32_t rb = ra + 8u * (uint32_t)chunk_bytes;
-    tc_q8_pair<0, XS>(ra, rb, xrow, xg, have_x, t, acc);
-    tc_q8_pair<2, XS>(ra, rb, xrow, xg, have_x, t, acc);
-    tc_q8_pair<4, XS>(ra, rb, xrow, xg, have_x, t, acc);
-    tc_q8_pair<6, XS>(ra, rb, xrow, xg, have_x, t, acc);
+    tc_q8_pair_bf16<0, XS>(ra, rb, xrow, xg, have_x, t, acc);
+    tc_q8_pair_bf16<2, XS>(ra, rb, xrow, xg, have_x, t, acc);
+    tc_q8_pair_bf16<4, XS>(ra, rb, xrow, xg, have_x, t, acc);
+    tc_q8_pair_bf16<6, XS>(ra, rb, xrow, xg, have_x, t, acc);
 }
 
 template <int FMT, int NWARP, bool XS>
@@ -251,12 +273,16 @@ __global__ void __launch_bounds__(NWARP * 32, 1) qmv_tc_kernel(const TcParams p)
     for (; issued < S && issued < n_units; ++issued) issue(issued);   // weights: no dependence on earlier kernels
 
     pdl_wait();                                         // x is the previous kernel's output
-    if (XS) {
-        const int c4 = p.cols >> 2;
-        for (int i = (int)threadIdx.x; i < p.n_tok * c4; i += TC_NT) {
-            const int tok = i / c4, f = i - tok * c4;
-            const float4 v = __ldg(reinterpret_cast<const float4 *>(p.x + (int64_t)tok * p.cols) + f);
-            sts_f4(xs + 4u * (uint32_t)(tok * p.x_pitch + 4 * f), v);
+    if (XS) {           // split once per CTA: 32 bytes per 8 columns, hi pairs then lo pairs
+        const int c8 = p.cols >> 3;
+        for (int i = (int)threadIdx.x; i < p.n_tok * c8; i += TC_NT) {
+            const int tok = i / c8, j = i - tok * c8;
+            const float4 *src = reinterpret_cast<const float4 *>(p.x + (int64_t)tok * p.cols) + 2 * j;
+            uint4 h, l;
+            tc_split_x8(__ldg(src), __ldg(src + 1), h, l);
+            const uint32_t a = xs + 4u * (uint32_t)(tok * p.x_pitch) + 32u * (uint32_t)j;
+            sts_v4(a, h);
+            sts_v4(a + 16u, l);
         }
     }
     __syncthreads();
