@@ -460,10 +460,10 @@ TcGeom tc_geom(int64_t cols, int n_tok, const DevInfo &di)
     return g;
 }
 
-// Q8_0 with 4..8 tokens whose rows are whole 256-column K-chunks.
+// Q8_0 with 3..8 tokens whose rows are whole 256-column K-chunks.
 bool tc_preferred(int fmt, int64_t rows, int64_t cols, int n_tok)
 {
-    return fmt == QMV_Q8_0 && n_tok >= 4 && n_tok <= 8 && cols % TC_KCOLS == 0 && cols <= (int64_t)1 << 24 &&
+    return fmt == QMV_Q8_0 && n_tok >= 3 && n_tok <= 8 && cols % TC_KCOLS == 0 && cols <= (int64_t)1 << 24 &&
            rows <= (int64_t)INT_MAX;
 }
 

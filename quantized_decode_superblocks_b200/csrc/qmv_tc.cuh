@@ -1,4 +1,4 @@
-// qmv_tc.cuh -- several-token (4..8) Q8_0 matvec on the tensor cores.
+// qmv_tc.cuh -- several-token (3..8) Q8_0 matvec on the tensor cores.
 //
 // With n_tok tokens every weight feeds n_tok products; on the CUDA cores that
 // is n_tok FMAs plus n_tok x reads per weight, which made the 8-token decode
