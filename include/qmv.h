@@ -258,8 +258,8 @@ int qmv_get_pdl(void);
  * this library fail with QMV_ERR_CUDA without reaching the GPU. */
 void qmv_debug_fail_next_launches(int count);
 
-/* Test hook for the device-side failure path: while bytes > 0, the one-token
- * and several-token warp-ring launches (qmv_f32 / qmv_batched on the shapes
+/* Test hook for the device-side failure path: while bytes > 0, the
+ * warp-ring and tensor-core launches (qmv_f32 / qmv_batched on the shapes
  * that take them, qmv_chain) expect `bytes` more per copied tile than they
  * copy, so every stage wait runs into its bound (about a second), records
  * QMV_DEVERR_TIMEOUT for qmv_check, and the kernel still finishes; results

@@ -491,6 +491,7 @@ int tc_single(const void *W, int64_t rows, int64_t cols, const float *x, float *
     p.n_stage = g.S;
     p.x_pitch = (int32_t)(cols + 4);
     p.err = di.err;
+    p.debug_extra_tx = g_debug_extra_tx.load();
     const cudaError_t e = launch_tc<FMT_Q8_0>(p, g.x_smem, dim3((unsigned)ctas), g.smem, st, g_pdl.load() != 0);
     return e == cudaSuccess ? QMV_OK : cuda_fail(e);
 }

@@ -52,6 +52,7 @@ struct TcParams {
     int32_t n_stage;       // ring stages per warp
     int32_t x_pitch;       // 4-byte words per token row of shared x (cols + 4)
     int *err;
+    uint32_t debug_extra_tx;   // test hook: bytes expected per tile beyond those copied (0 in use)
 };
 
 __host__ __device__ constexpr uint32_t tc_round128(uint32_t b) { return (b + 127u) & ~127u; }
@@ -263,7 +264,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1) qmv_tc_kernel(const TcParams p)
         const int valid = (int)min((int64_t)TC_ROWS, p.rows - r0);
         const int sl = j % S;
         const uint32_t bar = bar0 + 8u * (uint32_t)sl;
-        if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(valid * p.chunk_bytes));
+        if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(valid * p.chunk_bytes) + p.debug_extra_tx);
         __syncwarp();
         if (lane < valid)
             bulk_g2s(stage0 + (uint32_t)sl * tile_bytes + (uint32_t)(lane * p.chunk_bytes),

@@ -514,17 +514,22 @@ def test_moe_bad_expert_id_is_dropped_and_reported():
     assert np.array_equal(yh[1], np.zeros(rows, np.float32))
 
 
-def test_stage_wait_timeout_is_reported_and_the_gpu_stays_usable():
-    # the test hook makes every tile of the warp-ring kernel expect 16 bytes
-    # more than are copied: each stage wait runs out (about a second), the
-    # kernel records the timeout and finishes, and the context stays usable
+@pytest.mark.parametrize("n_tok", [1, 8])
+def test_stage_wait_timeout_is_reported_and_the_gpu_stays_usable(n_tok):
+    # the test hook makes every tile expect 16 bytes more than are copied
+    # (one token: the warp-ring kernel; eight: the tensor-core kernel): each
+    # stage wait runs out (about a second), the kernel records the timeout
+    # and finishes, and the context stays usable
     fmt, rows, cols = Q8_0, 512, 2048
     W = synth.gen_blocks(fmt, rows, cols, 45, 0)
-    x = synth.gen_x(1, cols, 45, 1)
-    y = torch.empty((1, rows), device="cuda")
+    x = synth.gen_x(n_tok, cols, 45, 1)
+    y = torch.empty((n_tok, rows), device="cuda")
     q.lib().qmv_debug_short_copies(16)
     try:
-        q.qmv_f32(fmt, dev(W), rows, cols, dev(x), y)
+        if n_tok == 1:
+            q.qmv_f32(fmt, dev(W), rows, cols, dev(x), y)
+        else:
+            q.qmv_batched(fmt, dev(W), rows, cols, dev(x), y, n_tok)
         err = q.qmv_check()
     finally:
         q.lib().qmv_debug_short_copies(0)
