@@ -427,7 +427,7 @@ int rw_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x
     return e == cudaSuccess ? QMV_OK : cuda_fail(e);
 }
 
-// Several tokens of a Q8_0 matrix on the tensor-core kernel: one CTA of
+// Several tokens of a Q8_0 or Q4_K matrix on the tensor-core kernel: one CTA of
 // TC_WARPS warps per SM, x in shared memory when it fits next to rings of at
 // least two stages, else read through L2.
 struct TcGeom {
@@ -438,13 +438,17 @@ struct TcGeom {
     size_t smem = 0;
 };
 
-TcGeom tc_geom(int64_t cols, int n_tok, const DevInfo &di)
+int tc_chunk_bytes(int fmt) { return fmt == QMV_Q8_0 ? TC_KCOLS / 32 * 34 : TC_KCOLS / 256 * 144; }
+
+TcGeom tc_geom(int fmt, int64_t cols, int n_tok, const DevInfo &di)
 {
     TcGeom g;
-    const int tile = TC_ROWS * (TC_KCOLS / 32) * 34;
+    const int tile = TC_ROWS * tc_chunk_bytes(fmt);
     const int64_t kc_n = cols / TC_KCOLS;
     g.ksplit = kc_n % 8 == 0 ? 8 : kc_n % 4 == 0 ? 4 : kc_n % 2 == 0 ? 2 : 1;
-    const int64_t budget = (int64_t)std::min(di.smem_optin, 227 * 1024) - 128 - TC_BAR_BYTES - tc_part_bytes(TC_WARPS);
+    const int64_t sx = fmt == QMV_Q4_K ? ((cols + 127) & ~(int64_t)127) : 0;   // sum-x table
+    const int64_t budget =
+        (int64_t)std::min(di.smem_optin, 227 * 1024) - 128 - TC_BAR_BYTES - tc_part_bytes(TC_WARPS) - sx;
     int64_t xb = ((int64_t)n_tok * (cols + 4) * 4 + 127) & ~(int64_t)127;
     int64_t S = (budget - xb) / ((int64_t)TC_WARPS * tile);
     g.x_smem = S >= 2;
@@ -455,33 +459,33 @@ TcGeom tc_geom(int64_t cols, int n_tok, const DevInfo &di)
     S = std::min<int64_t>(S, TC_MAX_STAGES);
     if (S < 2) return g;
     g.S = (int)S;
-    g.smem = (size_t)(128 + TC_BAR_BYTES + xb + tc_part_bytes(TC_WARPS) + (int64_t)TC_WARPS * S * tile);
+    g.smem = (size_t)(128 + TC_BAR_BYTES + xb + tc_part_bytes(TC_WARPS) + sx + (int64_t)TC_WARPS * S * tile);
     g.ok = true;
     return g;
 }
 
-// Q8_0 with 3..8 tokens whose rows are whole 256-column K-chunks.
+// Q8_0 / Q4_K with 3..8 tokens whose rows are whole 256-column K-chunks.
 bool tc_preferred(int fmt, int64_t rows, int64_t cols, int n_tok)
 {
-    return fmt == QMV_Q8_0 && n_tok >= 3 && n_tok <= 8 && cols % TC_KCOLS == 0 && cols <= (int64_t)1 << 24 &&
-           rows <= (int64_t)INT_MAX;
+    return (fmt == QMV_Q8_0 || fmt == QMV_Q4_K) && n_tok >= 3 && n_tok <= 8 && cols % TC_KCOLS == 0 &&
+           cols <= (int64_t)1 << 24 && rows <= (int64_t)INT_MAX;
 }
 
-int tc_single(const void *W, int64_t rows, int64_t cols, const float *x, float *y, int n_tok, const DevInfo &di,
-              cudaStream_t st)
+int tc_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x, float *y, int n_tok,
+              const DevInfo &di, cudaStream_t st)
 {
-    const TcGeom g = tc_geom(cols, n_tok, di);
+    const TcGeom g = tc_geom(fmt, cols, n_tok, di);
     if (!g.ok) return QMV_ERR_SHAPE;
     TcParams p{};
     p.W = static_cast<const uint8_t *>(W);
     p.x = x;
     p.y = y;
     p.rows = rows;
-    p.row_bytes = cols / 32 * 34;
+    p.row_bytes = cols / TC_KCOLS * tc_chunk_bytes(fmt);
     p.cols = (int32_t)cols;
     p.n_tok = n_tok;
     p.kc_n = (int32_t)(cols / TC_KCOLS);
-    p.chunk_bytes = TC_KCOLS / 32 * 34;
+    p.chunk_bytes = tc_chunk_bytes(fmt);
     p.ksplit = g.ksplit;
     const int64_t n_rt = ceil_div(rows, (int64_t)TC_ROWS);
     p.n_rt = (int32_t)n_rt;
@@ -492,7 +496,9 @@ int tc_single(const void *W, int64_t rows, int64_t cols, const float *x, float *
     p.x_pitch = (int32_t)(cols + 4);
     p.err = di.err;
     p.debug_extra_tx = g_debug_extra_tx.load();
-    const cudaError_t e = launch_tc<FMT_Q8_0>(p, g.x_smem, dim3((unsigned)ctas), g.smem, st, g_pdl.load() != 0);
+    const bool pdl = g_pdl.load() != 0;
+    const cudaError_t e = fmt == QMV_Q8_0 ? launch_tc<FMT_Q8_0>(p, g.x_smem, dim3((unsigned)ctas), g.smem, st, pdl)
+                                          : launch_tc<FMT_Q4_K>(p, g.x_smem, dim3((unsigned)ctas), g.smem, st, pdl);
     return e == cudaSuccess ? QMV_OK : cuda_fail(e);
 }
 
@@ -597,8 +603,8 @@ int qmv_batched(int fmt, const void *W_blocks, int64_t rows, int64_t cols, const
     if (injected_failure()) return QMV_ERR_CUDA;
     DevInfo di;
     if ((rc = get_dev(di))) return rc;
-    if (tc_preferred(fmt, rows, cols, n_tok) && tc_geom(cols, n_tok, di).ok)
-        return tc_single(W_blocks, rows, cols, x, y, n_tok, di, reinterpret_cast<cudaStream_t>(stream));
+    if (tc_preferred(fmt, rows, cols, n_tok) && tc_geom(fmt, cols, n_tok, di).ok)
+        return tc_single(fmt, W_blocks, rows, cols, x, y, n_tok, di, reinterpret_cast<cudaStream_t>(stream));
     if (n_tok == 1 ? rw_preferred(fmt, rows, cols) : rw_mt_preferred(fmt, rows, cols, n_tok))
         return rw_single(fmt, W_blocks, rows, cols, x, y, n_tok, di, reinterpret_cast<cudaStream_t>(stream));
     Plan pl;

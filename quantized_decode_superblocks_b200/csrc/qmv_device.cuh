@@ -60,6 +60,13 @@ __device__ __forceinline__ float4 lds_f4(uint32_t a)
     return v;
 }
 
+__device__ __forceinline__ float2 lds_f2(uint32_t a)
+{
+    float2 v;
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
+    return v;
+}
+
 __device__ __forceinline__ void sts_f4(uint32_t a, float4 v)
 {
     asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};"

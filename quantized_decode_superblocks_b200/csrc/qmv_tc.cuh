@@ -1,17 +1,19 @@
-// qmv_tc.cuh -- several-token (3..8) Q8_0 matvec on the tensor cores.
+// qmv_tc.cuh -- several-token (3..8) Q8_0 and Q4_K matvec on the tensor cores.
 //
 // With n_tok tokens every weight feeds n_tok products; on the CUDA cores that
 // is n_tok FMAs plus n_tok x reads per weight, which made the 8-token decode
 // step several times slower than the 1-token one.  Here the weights of a
 // tile of 16 rows are decoded exactly (Q8_0 quants are integers in
-// [-128, 127], exact in bf16) straight into the A fragments of
-// mma.m16n8k16 (bf16 in, f32 accumulate), and the tokens form the N = 8
-// columns.  x is split into two bf16 halves, hi (the float's upper 16 bits)
-// and lo (the remainder, rounded): two MMAs per k-step keep every product
-// within 2^-16 of f32, against a tolerance of 1e-4 of sum |w x|.  Each
-// 32-column block's sum is scaled by its f32 d in registers (GGUF Q8_0
-// layout: one fp16 d and 32 int8 quants per block; the dequantized weight is
-// d * q), so only integers and the split x go through the tensor cores.
+// [-128, 127], Q4_K quants nibbles: both exact in bf16) straight into the A
+// fragments of mma.m16n8k16 (bf16 in, f32 accumulate), and the tokens form
+// the N = 8 columns.  x is split into two bf16 halves, hi (the float's upper
+// 16 bits) and lo (the remainder, rounded): two MMAs per k-step keep every
+// product within 2^-16 of f32, against a tolerance of 1e-4 of sum |w x|.
+// The scales are applied in f32 in registers after each 32-column block's
+// MMAs (GGUF layouts: Q8_0 w = d q with one fp16 d per 32 quants; Q4_K
+// w = d sc q - dmin m per 32-column sub-block, the min term taken as
+// dmin m * sum x), so only integers and the split x go through the tensor
+// cores.
 //
 // Data flow: one CTA per SM (16 warps).  The CTA's x rows sit in shared
 // memory already split (token-major; 32 bytes per 8 columns, 16 of hi pairs
@@ -218,13 +220,95 @@ __device__ __forceinline__ void tc_q8_tile(uint32_t st, int chunk_bytes, uint32_
     tc_q8_pair_bf16<6, XS>(ra, rb, xrow, xg, have_x, t, acc);
 }
 
+// ------------------------------------------------------------------ Q4_K --
+// Four quants (nibbles 0..15, one per byte of nb) of columns c .. c + 3 as
+// two exact bf16 pairs: each byte under the exponent of 128 (bf16 0x43qq =
+// 128 + q), then one exact bf16x2 FMA q' * 1 - 128.
+__device__ __forceinline__ void tc_nib_pairs(uint32_t nb, uint32_t &p01, uint32_t &p23)
+{
+    const uint32_t v01 = __byte_perm(nb, 0x43434343u, 0x5140u);
+    const uint32_t v23 = __byte_perm(nb, 0x43434343u, 0x7362u);
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(p01) : "r"(v01), "r"(0x3F803F80u), "r"(0xC300C300u));
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(p23) : "r"(v23), "r"(0x3F803F80u), "r"(0xC300C300u));
+}
+
+// Sub-blocks 2C (low nibbles of qs[32C .. 32C + 31]) and 2C + 1 (their high
+// nibbles) of one Q4_K superblock per row (GGUF layout: d, dmin, 12 bytes of
+// packed 6-bit scales / mins, 128 bytes of quants; w = d sc q - dmin m):
+// sum_i w_i x_i = d sc (q . x) - dmin m (sum x), with q . x from the tensor
+// cores and sum x per 32 columns and token from the table at sxc.  Thread t
+// takes columns 8t .. 8t + 7 of each sub-block, as for Q8_0.
+template <int C, bool XS>
+__device__ __forceinline__ void tc_q4k_pair(uint32_t ra, uint32_t rb, const uint4 &ha, const uint4 &hb, float da,
+                                            float dma, float db, float dmb, uint32_t xrow, const float *xg,
+                                            bool have_x, int t, uint32_t sxc, float (&acc)[4])
+{
+    uint4 x0h, x0l, x1h, x1l;
+    tc_x_frag<XS>(xrow, xg, 2 * C, t, have_x, x0h, x0l);
+    tc_x_frag<XS>(xrow, xg, 2 * C + 1, t, have_x, x1h, x1l);
+    const uint32_t h0[4] = {x0h.x, x0h.y, x0h.z, x0h.w}, l0[4] = {x0l.x, x0l.y, x0l.z, x0l.w};
+    const uint32_t h1[4] = {x1h.x, x1h.y, x1h.z, x1h.w}, l1[4] = {x1l.x, x1l.y, x1l.z, x1l.w};
+    const uint32_t off = 16u + 32u * C + 8u * (uint32_t)t;
+    const uint32_t wa0 = lds_u32(ra + off), wa1 = lds_u32(ra + off + 4u);
+    const uint32_t wb0 = lds_u32(rb + off), wb1 = lds_u32(rb + off + 4u);
+    uint32_t p0[8], p1[8];       // [row half][pair]: columns 2i, 2i + 1 (low nibbles: p0, high: p1)
+    tc_nib_pairs(wa0 & 0x0F0F0F0Fu, p0[0], p0[1]);
+    tc_nib_pairs(wa1 & 0x0F0F0F0Fu, p0[2], p0[3]);
+    tc_nib_pairs(wb0 & 0x0F0F0F0Fu, p0[4], p0[5]);
+    tc_nib_pairs(wb1 & 0x0F0F0F0Fu, p0[6], p0[7]);
+    tc_nib_pairs((wa0 >> 4) & 0x0F0F0F0Fu, p1[0], p1[1]);
+    tc_nib_pairs((wa1 >> 4) & 0x0F0F0F0Fu, p1[2], p1[3]);
+    tc_nib_pairs((wb0 >> 4) & 0x0F0F0F0Fu, p1[4], p1[5]);
+    tc_nib_pairs((wb1 >> 4) & 0x0F0F0F0Fu, p1[6], p1[7]);
+    float c0h[4] = {0.f, 0.f, 0.f, 0.f}, c0l[4] = {0.f, 0.f, 0.f, 0.f};
+    float c1h[4] = {0.f, 0.f, 0.f, 0.f}, c1l[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+        mma_bf16(c0h, p0[2 * s], p0[4 + 2 * s], p0[2 * s + 1], p0[4 + 2 * s + 1], h0[2 * s], h0[2 * s + 1]);
+        mma_bf16(c1h, p1[2 * s], p1[4 + 2 * s], p1[2 * s + 1], p1[4 + 2 * s + 1], h1[2 * s], h1[2 * s + 1]);
+        mma_bf16(c0l, p0[2 * s], p0[4 + 2 * s], p0[2 * s + 1], p0[4 + 2 * s + 1], l0[2 * s], l0[2 * s + 1]);
+        mma_bf16(c1l, p1[2 * s], p1[4 + 2 * s], p1[2 * s + 1], p1[4 + 2 * s + 1], l1[2 * s], l1[2 * s + 1]);
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int j = 2 * C + h;
+        uint32_t sca, ma, scb, mb;
+        q4k_scale_min(ha.y, ha.z, ha.w, j, sca, ma);
+        q4k_scale_min(hb.y, hb.z, hb.w, j, scb, mb);
+        const float2 sx = lds_f2(sxc + 4u * (uint32_t)(8 * j + 2 * t));   // sum x of this sub-block, tokens 2t, 2t + 1
+        const float *ch = h ? c1h : c0h, *cl = h ? c1l : c0l;
+        const float aa = da * (float)sca, ba = dma * (float)ma, ab = db * (float)scb, bb = dmb * (float)mb;
+        acc[0] = fmaf(aa, ch[0] + cl[0], fmaf(-ba, sx.x, acc[0]));
+        acc[1] = fmaf(aa, ch[1] + cl[1], fmaf(-ba, sx.y, acc[1]));
+        acc[2] = fmaf(ab, ch[2] + cl[2], fmaf(-bb, sx.x, acc[2]));
+        acc[3] = fmaf(ab, ch[3] + cl[3], fmaf(-bb, sx.y, acc[3]));
+    }
+}
+
+// One 16-row tile of one Q4_K superblock (256 columns) against the 8 token
+// columns; sxc: the sum-x table of this K-chunk ([32-column block][8 tokens]).
+template <bool XS>
+__device__ __forceinline__ void tc_q4k_tile(uint32_t st, int chunk_bytes, uint32_t xrow, const float *xg, bool have_x,
+                                            int g, int t, uint32_t sxc, float (&acc)[4])
+{
+    const uint32_t ra = st + (uint32_t)(g * chunk_bytes);
+    const uint32_t rb = ra + 8u * (uint32_t)chunk_bytes;
+    const uint4 ha = lds_v4(ra), hb = lds_v4(rb);
+    const float da = half_bits_to_float(ha.x), dma = half_bits_to_float(ha.x >> 16);
+    const float db = half_bits_to_float(hb.x), dmb = half_bits_to_float(hb.x >> 16);
+    tc_q4k_pair<0, XS>(ra, rb, ha, hb, da, dma, db, dmb, xrow, xg, have_x, t, sxc, acc);
+    tc_q4k_pair<1, XS>(ra, rb, ha, hb, da, dma, db, dmb, xrow, xg, have_x, t, sxc, acc);
+    tc_q4k_pair<2, XS>(ra, rb, ha, hb, da, dma, db, dmb, xrow, xg, have_x, t, sxc, acc);
+    tc_q4k_pair<3, XS>(ra, rb, ha, hb, da, dma, db, dmb, xrow, xg, have_x, t, sxc, acc);
+}
+
 template <int FMT, int NWARP, bool XS>
 __global__ void __launch_bounds__(NWARP * 32, 1) qmv_tc_kernel(const TcParams p)
 {
     constexpr int TC_NW = NWARP;
     constexpr int TC_NT = NWARP * 32;
     constexpr int TC_PART_BYTES = tc_part_bytes(NWARP);
-    static_assert(FMT == FMT_Q8_0, "tensor-core path: Q8_0");
+    static_assert(FMT == FMT_Q8_0 || FMT == FMT_Q4_K, "tensor-core path: Q8_0, Q4_K");
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = (int)threadIdx.x >> 5, lane = (int)threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -236,7 +320,9 @@ __global__ void __launch_bounds__(NWARP * 32, 1) qmv_tc_kernel(const TcParams p)
     const uint32_t x_bytes = XS ? tc_round128((uint32_t)(p.n_tok * p.x_pitch * 4)) : 0u;
     const uint32_t part = xs + x_bytes;
     const uint32_t tile_bytes = (uint32_t)(TC_ROWS * p.chunk_bytes);
-    const uint32_t stage0 = part + (uint32_t)TC_PART_BYTES + (uint32_t)(warp * S) * tile_bytes;
+    const uint32_t sx = part + (uint32_t)TC_PART_BYTES;       // Q4_K: sum x per 32 columns, [block][8 tokens]
+    const uint32_t sx_bytes = FMT == FMT_Q4_K ? tc_round128((uint32_t)p.cols) : 0u;
+    const uint32_t stage0 = sx + sx_bytes + (uint32_t)(warp * S) * tile_bytes;
 
     // this CTA's row tiles, this warp's group and K-chunks
     const int c = (int)blockIdx.x;
@@ -286,6 +372,21 @@ __global__ void __launch_bounds__(NWARP * 32, 1) qmv_tc_kernel(const TcParams p)
             sts_v4(a + 16u, l);
         }
     }
+    if (FMT == FMT_Q4_K) {   // sum x of every 32-column block and token (zero for the missing tokens)
+        for (int i = (int)threadIdx.x; i < (p.cols >> 5) * 8; i += TC_NT) {
+            const int blk = i >> 3, tok = i & 7;
+            float sum = 0.f;
+            if (tok < p.n_tok) {
+                const float4 *src = reinterpret_cast<const float4 *>(p.x + (int64_t)tok * p.cols + 32 * blk);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const float4 v = __ldg(src + k);
+                    sum += (v.x + v.y) + (v.z + v.w);
+                }
+            }
+            sts_f32(sx + 4u * (uint32_t)i, sum);
+        }
+    }
     __syncthreads();
 
     const bool have_x = g < p.n_tok;
@@ -307,8 +408,13 @@ __global__ void __launch_bounds__(NWARP * 32, 1) qmv_tc_kernel(const TcParams p)
                     if (lane == 0) atomicOr(p.err, DEVERR_TIMEOUT);
                 } else {
                     const int kc = kg * kpw + k;
-                    tc_q8_tile<XS>(stage0 + (uint32_t)sl * tile_bytes, p.chunk_bytes,
-                                   xrow0 + 4u * (uint32_t)(kc * TC_KCOLS), xg0 + kc * TC_KCOLS, have_x, g, t, acc);
+                    if (FMT == FMT_Q8_0)
+                        tc_q8_tile<XS>(stage0 + (uint32_t)sl * tile_bytes, p.chunk_bytes,
+                                       xrow0 + 4u * (uint32_t)(kc * TC_KCOLS), xg0 + kc * TC_KCOLS, have_x, g, t, acc);
+                    else
+                        tc_q4k_tile<XS>(stage0 + (uint32_t)sl * tile_bytes, p.chunk_bytes,
+                                        xrow0 + 4u * (uint32_t)(kc * TC_KCOLS), xg0 + kc * TC_KCOLS, have_x, g, t,
+                                        sx + 4u * (uint32_t)(kc * (TC_KCOLS / 32) * 8), acc);
                     consumed = j + 1;
                     __syncwarp();
                     if (issued < n_units) { issue(issued); ++issued; }

@@ -124,38 +124,41 @@ def test_qmv_long_rows_k_chunked(fmt, rows, cols, n_tok):
     within(y, ref, bound)
 
 
-# Q8_0 with 4..8 tokens and rows of whole 256-column K-chunks takes the
-# tensor-core kernel: partial row tiles, more tiles than CTAs, every K-split
-# (1, 2, 4, 8 warps per tile), x in shared memory and through L2, and x over
-# a wide range of magnitudes (the hi / lo TF32 split of x).
+# Q8_0 and Q4_K with 3..8 tokens and rows of whole 256-column K-chunks take
+# the tensor-core kernel: partial row tiles, more tiles than CTAs, every
+# K-split (1, 2, 4, 8 warps per tile), x in shared memory and through L2, and
+# x over a wide range of magnitudes (the hi / lo bf16 split of x).
+@pytest.mark.parametrize("fmt", [Q8_0, Q4_K])
 @pytest.mark.parametrize("rows,cols", [(5, 256), (16, 768), (33, 512), (2371, 1024), (300, 2048),
                                        (16 * 148 * 2 + 7, 2048), (40, 8192)])
-@pytest.mark.parametrize("n_tok", [4, 6, 7, 8])
-def test_q8_0_tensor_core_tiles(rows, cols, n_tok):
-    W = synth.gen_blocks(Q8_0, rows, cols, seed=11, tensor_id=rows)
+@pytest.mark.parametrize("n_tok", [3, 4, 6, 7, 8])
+def test_tensor_core_tiles(fmt, rows, cols, n_tok):
+    W = synth.gen_blocks(fmt, rows, cols, seed=11, tensor_id=rows)
     x = synth.gen_x(n_tok, cols, seed=11, tensor_id=cols + n_tok)
-    y = run_qmv(Q8_0, W, rows, cols, x)
-    ref, bound = oracle.qmv(Q8_0, W, rows, cols, x, nthreads=8)
+    y = run_qmv(fmt, W, rows, cols, x)
+    ref, bound = oracle.qmv(fmt, W, rows, cols, x, nthreads=8)
     within(y, ref, bound)
 
 
+@pytest.mark.parametrize("fmt", [Q8_0, Q4_K])
 @pytest.mark.parametrize("scale", [1e-30, 1e-6, 1e6, 1e30])
-def test_q8_0_tensor_core_x_magnitudes(scale):
+def test_tensor_core_x_magnitudes(fmt, scale):
     rows, cols, n_tok = 64, 1024, 8
-    W = synth.gen_blocks(Q8_0, rows, cols, seed=12, tensor_id=0)
+    W = synth.gen_blocks(fmt, rows, cols, seed=12, tensor_id=0)
     x = (synth.gen_x(n_tok, cols, seed=12, tensor_id=1) * np.float32(scale)).astype(np.float32)
-    y = run_qmv(Q8_0, W, rows, cols, x)
-    ref, bound = oracle.qmv(Q8_0, W, rows, cols, x)
+    y = run_qmv(fmt, W, rows, cols, x)
+    ref, bound = oracle.qmv(fmt, W, rows, cols, x)
     within(y, ref, bound, abs_=ABS * min(1.0, scale))
 
 
-def test_q8_0_tensor_core_repeatable():
+@pytest.mark.parametrize("fmt", [Q8_0, Q4_K])
+def test_tensor_core_repeatable(fmt):
     # the K-split partial sums are added in a fixed order: identical bits every call
     rows, cols, n_tok = 3072, 2048, 8
-    W = synth.gen_blocks(Q8_0, rows, cols, seed=13, tensor_id=0)
+    W = synth.gen_blocks(fmt, rows, cols, seed=13, tensor_id=0)
     x = synth.gen_x(n_tok, cols, seed=13, tensor_id=1)
-    a = run_qmv(Q8_0, W, rows, cols, x)
-    b = run_qmv(Q8_0, W, rows, cols, x)
+    a = run_qmv(fmt, W, rows, cols, x)
+    b = run_qmv(fmt, W, rows, cols, x)
     assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
 
 
