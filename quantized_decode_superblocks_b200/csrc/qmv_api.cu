@@ -438,12 +438,15 @@ struct TcGeom {
     size_t smem = 0;
 };
 
-int tc_chunk_bytes(int fmt) { return fmt == QMV_Q8_0 ? TC_KCOLS / 32 * 34 : TC_KCOLS / 256 * 144; }
+// Bytes of one row's 256-column K-chunk, and of its slot in a stage (Q6_K:
+// the 16-byte-aligned 224 bytes around a 210-byte superblock).
+int tc_chunk_bytes(int fmt) { return fmt == QMV_Q8_0 ? TC_KCOLS / 32 * 34 : fmt == QMV_Q4_K ? 144 : 210; }
+int tc_slot_bytes(int fmt) { return fmt == QMV_Q6_K ? 224 : tc_chunk_bytes(fmt); }
 
 TcGeom tc_geom(int fmt, int64_t cols, int n_tok, const DevInfo &di)
 {
     TcGeom g;
-    const int tile = TC_ROWS * tc_chunk_bytes(fmt);
+    const int tile = TC_ROWS * tc_slot_bytes(fmt);
     const int64_t kc_n = cols / TC_KCOLS;
     g.ksplit = kc_n % 8 == 0 ? 8 : kc_n % 4 == 0 ? 4 : kc_n % 2 == 0 ? 2 : 1;
     const int64_t sx = fmt == QMV_Q4_K ? ((cols + 127) & ~(int64_t)127) : 0;   // sum-x table
@@ -457,18 +460,20 @@ TcGeom tc_geom(int fmt, int64_t cols, int n_tok, const DevInfo &di)
         S = budget / ((int64_t)TC_WARPS * tile);
     }
     S = std::min<int64_t>(S, TC_MAX_STAGES);
-    if (S < 2) return g;
+    if (S < 2 || (fmt == QMV_Q6_K && !g.x_smem)) return g;
     g.S = (int)S;
     g.smem = (size_t)(128 + TC_BAR_BYTES + xb + tc_part_bytes(TC_WARPS) + sx + (int64_t)TC_WARPS * S * tile);
     g.ok = true;
     return g;
 }
 
-// Q8_0 / Q4_K with 3..8 tokens whose rows are whole 256-column K-chunks.
+// Q8_0 / Q4_K with 3..8 tokens whose rows are whole 256-column K-chunks;
+// Q6_K when rows are whole 2048-column runs (a multiple of 16 bytes, so a
+// superblock's offset in its 16-byte-aligned slot is the same in every row).
 bool tc_preferred(int fmt, int64_t rows, int64_t cols, int n_tok)
 {
-    return (fmt == QMV_Q8_0 || fmt == QMV_Q4_K) && n_tok >= 3 && n_tok <= 8 && cols % TC_KCOLS == 0 &&
-           cols <= (int64_t)1 << 24 && rows <= (int64_t)INT_MAX;
+    const bool shape = fmt == QMV_Q6_K ? cols % 2048 == 0 : (fmt == QMV_Q8_0 || fmt == QMV_Q4_K) && cols % TC_KCOLS == 0;
+    return shape && n_tok >= 3 && n_tok <= 8 && cols <= (int64_t)1 << 24 && rows <= (int64_t)INT_MAX;
 }
 
 int tc_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x, float *y, int n_tok,
@@ -481,11 +486,12 @@ int tc_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x
     p.x = x;
     p.y = y;
     p.rows = rows;
-    p.row_bytes = cols / TC_KCOLS * tc_chunk_bytes(fmt);
+    p.row_bytes = cols / TC_KCOLS * tc_chunk_bytes(fmt);   // Q6_K: a multiple of 16 (cols % 2048 == 0)
     p.cols = (int32_t)cols;
     p.n_tok = n_tok;
     p.kc_n = (int32_t)(cols / TC_KCOLS);
     p.chunk_bytes = tc_chunk_bytes(fmt);
+    p.slot_bytes = tc_slot_bytes(fmt);
     p.ksplit = g.ksplit;
     const int64_t n_rt = ceil_div(rows, (int64_t)TC_ROWS);
     p.n_rt = (int32_t)n_rt;
@@ -497,8 +503,9 @@ int tc_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x
     p.err = di.err;
     p.debug_extra_tx = g_debug_extra_tx.load();
     const bool pdl = g_pdl.load() != 0;
-    const cudaError_t e = fmt == QMV_Q8_0 ? launch_tc<FMT_Q8_0>(p, g.x_smem, dim3((unsigned)ctas), g.smem, st, pdl)
-                                          : launch_tc<FMT_Q4_K>(p, g.x_smem, dim3((unsigned)ctas), g.smem, st, pdl);
+    const cudaError_t e = fmt == QMV_Q8_0   ? launch_tc<FMT_Q8_0>(p, g.x_smem, dim3((unsigned)ctas), g.smem, st, pdl)
+                          : fmt == QMV_Q4_K ? launch_tc<FMT_Q4_K>(p, g.x_smem, dim3((unsigned)ctas), g.smem, st, pdl)
+                                            : launch_tc<FMT_Q6_K>(p, g.x_smem, dim3((unsigned)ctas), g.smem, st, pdl);
     return e == cudaSuccess ? QMV_OK : cuda_fail(e);
 }
 

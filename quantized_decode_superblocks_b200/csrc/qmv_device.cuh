@@ -60,6 +60,13 @@ __device__ __forceinline__ float4 lds_f4(uint32_t a)
     return v;
 }
 
+__device__ __forceinline__ uint2 lds_v2(uint32_t a)
+{
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
+
 __device__ __forceinline__ float2 lds_f2(uint32_t a)
 {
     float2 v;

@@ -212,9 +212,16 @@ template <int FMT>
 cudaError_t launch_tc(const TcParams &p, bool x_smem, dim3 grid, size_t smem, cudaStream_t st, bool pdl)
 {
     static int configured_s[64] = {0}, configured_g[64] = {0};
-    if (x_smem)
+    if constexpr (FMT == FMT_Q6_K) {       // x always in shared memory
+        if (!x_smem) return cudaErrorInvalidValue;
         return launch_with(qmv_tc_kernel<FMT, TC_WARPS, true>, configured_s, p, grid, smem, st, pdl, false, TC_WARPS * 32);
-    return launch_with(qmv_tc_kernel<FMT, TC_WARPS, false>, configured_g, p, grid, smem, st, pdl, false, TC_WARPS * 32);
+    } else {
+        if (x_smem)
+            return launch_with(qmv_tc_kernel<FMT, TC_WARPS, true>, configured_s, p, grid, smem, st, pdl, false,
+                               TC_WARPS * 32);
+        return launch_with(qmv_tc_kernel<FMT, TC_WARPS, false>, configured_g, p, grid, smem, st, pdl, false,
+                           TC_WARPS * 32);
+    }
 }
 
 }  // namespace qmv

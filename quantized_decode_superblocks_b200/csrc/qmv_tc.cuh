@@ -47,7 +47,8 @@ struct TcParams {
     int32_t cols;
     int32_t n_tok;         // 1..8 (missing tokens are zero columns of B)
     int32_t kc_n;          // K-chunks per row
-    int32_t chunk_bytes;   // bytes of one row's K-chunk
+    int32_t chunk_bytes;   // bytes of one row's K-chunk (its stride along the row)
+    int32_t slot_bytes;    // bytes of one row's slot in a stage (Q6_K: a 16-byte-aligned superset of the chunk)
     int32_t ksplit;        // warps per row-tile group (divides TC_NW and kc_n)
     int32_t n_rt;          // row tiles in the matrix
     int32_t rt_q, rt_r;    // CTA c owns rt_q + (c < rt_r) consecutive row tiles
@@ -302,13 +303,84 @@ __device__ __forceinline__ void tc_q4k_tile(uint32_t st, int chunk_bytes, uint32
     tc_q4k_pair<3, XS>(ra, rb, ha, hb, da, dma, db, dmb, xrow, xg, have_x, t, sxc, acc);
 }
 
+// ------------------------------------------------------------------ Q6_K --
+// Four bytes at a 2-byte-aligned shared address.
+__device__ __forceinline__ uint32_t tc_lds_u32_a2(uint32_t a)
+{
+    const uint32_t a4 = a & ~3u;
+    return __byte_perm(lds_u32(a4), lds_u32(a4 + 4u), (a & 2u) ? 0x5432u : 0x3210u);
+}
+
+__device__ __forceinline__ int tc_lds_s8(uint32_t a)
+{
+    int v;
+    asm volatile("ld.shared.s8 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+
+// Four 6-bit quants u (one per byte, 0..63) as two exact bf16 pairs of
+// q = u - 32: each byte under the exponent of 128, then an exact bf16x2 FMA
+// subtracts 160.
+__device__ __forceinline__ void tc_q6_pairs(uint32_t u, uint32_t &p01, uint32_t &p23)
+{
+    const uint32_t v01 = __byte_perm(u, 0x43434343u, 0x5140u);
+    const uint32_t v23 = __byte_perm(u, 0x43434343u, 0x7362u);
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(p01) : "r"(v01), "r"(0x3F803F80u), "r"(0xC320C320u));
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(p23) : "r"(v23), "r"(0x3F803F80u), "r"(0xC320C320u));
+}
+
+// One 16-row tile of one Q6_K superblock (GGUF layout: ql[128], qh[64],
+// int8 scales[16], fp16 d; weight i of the superblock: half h = i / 128,
+// quarter t = (i / 32) % 4, l = i % 32; low 4 bits from ql[64h + 32(t & 1) +
+// l] (high nibble when t >= 2), high 2 bits from qh[32h + l] >> 2t;
+// w = d * scales[i / 16] * (q - 32)).  One k-step per 16-column scale group:
+// thread t takes its columns 4t .. 4t + 3 (k = 2t, 2t + 1 and 2t + 8,
+// 2t + 9).  The superblock starts `sofs` bytes into each row's slot.
+__device__ __forceinline__ void tc_q6k_tile(uint32_t st, int slot_bytes, int sofs, uint32_t xrow, bool have_x, int g,
+                                            int t, float (&acc)[4])
+{
+    const uint32_t ra = st + (uint32_t)(g * slot_bytes + sofs);
+    const uint32_t rb = ra + 8u * (uint32_t)slot_bytes;
+    const float da = half_bits_to_float(lds_u16(ra + 208u)), db = half_bits_to_float(lds_u16(rb + 208u));
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const int h = j >> 3, q4 = (j >> 1) & 3;
+        const uint32_t lo_off = (uint32_t)(64 * h + 32 * (q4 & 1) + 16 * (j & 1) + 4 * t);
+        const uint32_t hi_off = (uint32_t)(128 + 32 * h + 16 * (j & 1) + 4 * t);
+        const int nsh = q4 >= 2 ? 4 : 0;
+        const uint32_t ua = ((tc_lds_u32_a2(ra + lo_off) >> nsh) & 0x0F0F0F0Fu) |
+                            (((tc_lds_u32_a2(ra + hi_off) >> (2 * q4)) & 0x03030303u) << 4);
+        const uint32_t ub = ((tc_lds_u32_a2(rb + lo_off) >> nsh) & 0x0F0F0F0Fu) |
+                            (((tc_lds_u32_a2(rb + hi_off) >> (2 * q4)) & 0x03030303u) << 4);
+        uint32_t a01, a23, b01, b23;
+        tc_q6_pairs(ua, a01, a23);
+        tc_q6_pairs(ub, b01, b23);
+        // x: columns 16j + 4t .. + 3 = pairs 2(t & 1), 2(t & 1) + 1 of 8-column group 2j + t / 2
+        uint32_t xh0 = 0u, xh1 = 0u, xl0 = 0u, xl1 = 0u;
+        if (have_x) {
+            const uint32_t xa = xrow + 32u * (uint32_t)(2 * j + (t >> 1)) + 8u * (uint32_t)(t & 1);
+            const uint2 vh = lds_v2(xa), vl = lds_v2(xa + 16u);
+            xh0 = vh.x; xh1 = vh.y; xl0 = vl.x; xl1 = vl.y;
+        }
+        float ch[4] = {0.f, 0.f, 0.f, 0.f}, cl[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_bf16(ch, a01, b01, a23, b23, xh0, xh1);
+        mma_bf16(cl, a01, b01, a23, b23, xl0, xl1);
+        const float sa = da * (float)tc_lds_s8(ra + 192u + (uint32_t)j);
+        const float sb = db * (float)tc_lds_s8(rb + 192u + (uint32_t)j);
+        acc[0] = fmaf(sa, ch[0] + cl[0], acc[0]);
+        acc[1] = fmaf(sa, ch[1] + cl[1], acc[1]);
+        acc[2] = fmaf(sb, ch[2] + cl[2], acc[2]);
+        acc[3] = fmaf(sb, ch[3] + cl[3], acc[3]);
+    }
+}
+
 template <int FMT, int NWARP, bool XS>
 __global__ void __launch_bounds__(NWARP * 32, 1) qmv_tc_kernel(const TcParams p)
 {
     constexpr int TC_NW = NWARP;
     constexpr int TC_NT = NWARP * 32;
     constexpr int TC_PART_BYTES = tc_part_bytes(NWARP);
-    static_assert(FMT == FMT_Q8_0 || FMT == FMT_Q4_K, "tensor-core path: Q8_0, Q4_K");
+    static_assert(FMT == FMT_Q8_0 || FMT == FMT_Q4_K || (FMT == FMT_Q6_K && XS), "tensor-core path: Q8_0, Q4_K, Q6_K");
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = (int)threadIdx.x >> 5, lane = (int)threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -319,7 +391,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1) qmv_tc_kernel(const TcParams p)
     const uint32_t xs = sbase + (uint32_t)TC_BAR_BYTES;
     const uint32_t x_bytes = XS ? tc_round128((uint32_t)(p.n_tok * p.x_pitch * 4)) : 0u;
     const uint32_t part = xs + x_bytes;
-    const uint32_t tile_bytes = (uint32_t)(TC_ROWS * p.chunk_bytes);
+    const uint32_t tile_bytes = (uint32_t)(TC_ROWS * p.slot_bytes);
     const uint32_t sx = part + (uint32_t)TC_PART_BYTES;       // Q4_K: sum x per 32 columns, [block][8 tokens]
     const uint32_t sx_bytes = FMT == FMT_Q4_K ? tc_round128((uint32_t)p.cols) : 0u;
     const uint32_t stage0 = sx + sx_bytes + (uint32_t)(warp * S) * tile_bytes;
@@ -350,11 +422,20 @@ __global__ void __launch_bounds__(NWARP * 32, 1) qmv_tc_kernel(const TcParams p)
         const int valid = (int)min((int64_t)TC_ROWS, p.rows - r0);
         const int sl = j % S;
         const uint32_t bar = bar0 + 8u * (uint32_t)sl;
-        if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(valid * p.chunk_bytes) + p.debug_extra_tx);
+        // Q6_K chunks (210 bytes) start on 2-byte boundaries: copy the 16-byte-aligned
+        // slot around each, cut at the end of the matrix (which is 16-byte aligned)
+        int64_t off = (r0 + lane) * p.row_bytes + (int64_t)kc * p.chunk_bytes;
+        uint32_t size = (uint32_t)p.chunk_bytes;
+        if (FMT == FMT_Q6_K) {
+            off &= ~(int64_t)15;
+            size = (uint32_t)min((int64_t)p.slot_bytes, p.rows * p.row_bytes - off);
+        }
+        if (lane >= valid) size = 0u;
+        const uint32_t total = __reduce_add_sync(0xffffffffu, size);
+        if (lane == 0) mbar_arrive_expect_tx(bar, total + p.debug_extra_tx);
         __syncwarp();
         if (lane < valid)
-            bulk_g2s(stage0 + (uint32_t)sl * tile_bytes + (uint32_t)(lane * p.chunk_bytes),
-                     p.W + (r0 + lane) * p.row_bytes + (int64_t)kc * p.chunk_bytes, (uint32_t)p.chunk_bytes, bar);
+            bulk_g2s(stage0 + (uint32_t)sl * tile_bytes + (uint32_t)(lane * p.slot_bytes), p.W + off, size, bar);
     };
     int issued = 0;
     for (; issued < S && issued < n_units; ++issued) issue(issued);   // weights: no dependence on earlier kernels
@@ -411,6 +492,9 @@ __global__ void __launch_bounds__(NWARP * 32, 1) qmv_tc_kernel(const TcParams p)
                     if (FMT == FMT_Q8_0)
                         tc_q8_tile<XS>(stage0 + (uint32_t)sl * tile_bytes, p.chunk_bytes,
                                        xrow0 + 4u * (uint32_t)(kc * TC_KCOLS), xg0 + kc * TC_KCOLS, have_x, g, t, acc);
+                    else if (FMT == FMT_Q6_K)
+                        tc_q6k_tile(stage0 + (uint32_t)sl * tile_bytes, p.slot_bytes, (2 * kc) & 15,
+                                    xrow0 + 4u * (uint32_t)(kc * TC_KCOLS), have_x, g, t, acc);
                     else
                         tc_q4k_tile<XS>(stage0 + (uint32_t)sl * tile_bytes, p.chunk_bytes,
                                         xrow0 + 4u * (uint32_t)(kc * TC_KCOLS), xg0 + kc * TC_KCOLS, have_x, g, t,

@@ -140,10 +140,23 @@ def test_tensor_core_tiles(fmt, rows, cols, n_tok):
     within(y, ref, bound)
 
 
-@pytest.mark.parametrize("fmt", [Q8_0, Q4_K])
+# Q6_K takes it when rows are whole 2048-column runs: superblocks at every
+# 2-byte offset within their 16-byte-aligned slots, the last row's copy cut at
+# the end of the matrix
+@pytest.mark.parametrize("rows,cols", [(5, 2048), (16 * 148 * 2 + 7, 2048), (300, 4096), (16, 6144)])
+@pytest.mark.parametrize("n_tok", [3, 4, 8])
+def test_tensor_core_q6_k_tiles(rows, cols, n_tok):
+    W = synth.gen_blocks(Q6_K, rows, cols, seed=14, tensor_id=rows)
+    x = synth.gen_x(n_tok, cols, seed=14, tensor_id=cols + n_tok)
+    y = run_qmv(Q6_K, W, rows, cols, x)
+    ref, bound = oracle.qmv(Q6_K, W, rows, cols, x, nthreads=8)
+    within(y, ref, bound)
+
+
+@pytest.mark.parametrize("fmt", [Q8_0, Q4_K, Q6_K])
 @pytest.mark.parametrize("scale", [1e-30, 1e-6, 1e6, 1e30])
 def test_tensor_core_x_magnitudes(fmt, scale):
-    rows, cols, n_tok = 64, 1024, 8
+    rows, cols, n_tok = 64, 2048, 8
     W = synth.gen_blocks(fmt, rows, cols, seed=12, tensor_id=0)
     x = (synth.gen_x(n_tok, cols, seed=12, tensor_id=1) * np.float32(scale)).astype(np.float32)
     y = run_qmv(fmt, W, rows, cols, x)
@@ -151,7 +164,7 @@ def test_tensor_core_x_magnitudes(fmt, scale):
     within(y, ref, bound, abs_=ABS * min(1.0, scale))
 
 
-@pytest.mark.parametrize("fmt", [Q8_0, Q4_K])
+@pytest.mark.parametrize("fmt", [Q8_0, Q4_K, Q6_K])
 def test_tensor_core_repeatable(fmt):
     # the K-split partial sums are added in a fixed order: identical bits every call
     rows, cols, n_tok = 3072, 2048, 8
