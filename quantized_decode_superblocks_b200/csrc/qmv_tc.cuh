@@ -1,10 +1,11 @@
-// qmv_tc.cuh -- several-token (3..8) Q8_0 and Q4_K matvec on the tensor cores.
+// qmv_tc.cuh -- several-token (3..8) Q8_0, Q4_K and Q6_K matvec on the tensor cores.
 //
 // With n_tok tokens every weight feeds n_tok products; on the CUDA cores that
 // is n_tok FMAs plus n_tok x reads per weight, which made the 8-token decode
 // step several times slower than the 1-token one.  Here the weights of a
 // tile of 16 rows are decoded exactly (Q8_0 quants are integers in
-// [-128, 127], Q4_K quants nibbles: both exact in bf16) straight into the A
+// [-128, 127], Q4_K quants nibbles, Q6_K quants q - 32 in [-32, 31]: all
+// exact in bf16) straight into the A
 // fragments of mma.m16n8k16 (bf16 in, f32 accumulate), and the tokens form
 // the N = 8 columns.  x is split into two bf16 halves, hi (the float's upper
 // 16 bits) and lo (the remainder, rounded): two MMAs per k-step keep every
@@ -12,15 +13,16 @@
 // The scales are applied in f32 in registers after each 32-column block's
 // MMAs (GGUF layouts: Q8_0 w = d q with one fp16 d per 32 quants; Q4_K
 // w = d sc q - dmin m per 32-column sub-block, the min term taken as
-// dmin m * sum x), so only integers and the split x go through the tensor
-// cores.
+// dmin m * sum x; Q6_K w = d scale (q - 32) per 16 columns), so only
+// integers and the split x go through the tensor cores.
 //
 // Data flow: one CTA per SM (16 warps).  The CTA's x rows sit in shared
 // memory already split (token-major; 32 bytes per 8 columns, 16 of hi pairs
 // and 16 of lo pairs; row pitch cols * 4 + 16 bytes, so a warp's 16-byte
 // loads hit all banks once) or, when they do not fit next to the rings, are
-// read through L2 and split per tile.  A unit is one tile (16 rows x 256
-// columns = 4352 bytes), copied by `cp.async.bulk` (one copy per row) into a
+// read through L2 and split per tile.  A unit is one tile of 16 rows x 256
+// columns (4352 bytes of Q8_0, 2304 of Q4_K, 16 slots of 224 bytes around
+// the Q6_K superblocks), copied by `cp.async.bulk` (one copy per row) into a
 // warp-private ring of stages on an mbarrier, as in the warp-ring kernel.
 // The CTA's row tiles go to groups of `ksplit` warps; the warps of a group
 // split the K-chunks of a tile, add their partial sums in a fixed order
