@@ -439,9 +439,11 @@ struct TcGeom {
 };
 
 // Bytes of one row's 256-column K-chunk, and of its slot in a stage (Q6_K:
-// the 16-byte-aligned 224 bytes around a 210-byte superblock).
+// the 16-byte-aligned 224 bytes around a 210-byte superblock, in a 240-byte
+// slot whose 60-word pitch keeps the rows a quad group reads in different
+// banks).
 int tc_chunk_bytes(int fmt) { return fmt == QMV_Q8_0 ? TC_KCOLS / 32 * 34 : fmt == QMV_Q4_K ? 144 : 210; }
-int tc_slot_bytes(int fmt) { return fmt == QMV_Q6_K ? 224 : tc_chunk_bytes(fmt); }
+int tc_slot_bytes(int fmt) { return fmt == QMV_Q6_K ? 240 : tc_chunk_bytes(fmt); }
 
 TcGeom tc_geom(int fmt, int64_t cols, int n_tok, const DevInfo &di)
 {

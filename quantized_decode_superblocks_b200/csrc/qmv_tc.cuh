@@ -21,8 +21,10 @@
 // and 16 of lo pairs; row pitch cols * 4 + 16 bytes, so a warp's 16-byte
 // loads hit all banks once) or, when they do not fit next to the rings, are
 // read through L2 and split per tile.  A unit is one tile of 16 rows x 256
-// columns (4352 bytes of Q8_0, 2304 of Q4_K, 16 slots of 224 bytes around
-// the Q6_K superblocks), copied by `cp.async.bulk` (one copy per row) into a
+// columns (4352 bytes of Q8_0, 2304 of Q4_K, 224 bytes around each row's
+// Q6_K superblock in a 240-byte slot: the 60-word pitch puts the eight rows a
+// quad group reads in different banks), copied by `cp.async.bulk` (one copy
+// per row) into a
 // warp-private ring of stages on an mbarrier, as in the warp-ring kernel.
 // The CTA's row tiles go to groups of `ksplit` warps; the warps of a group
 // split the K-chunks of a tile, add their partial sums in a fixed order
@@ -37,6 +39,7 @@ constexpr int TC_KCOLS = 256;          // columns per K-chunk (a multiple of 16 
 constexpr int TC_ROWS = 16;            // rows per tile (MMA M)
 constexpr int TC_MAX_STAGES = 6;
 constexpr int TC_WARPS = 16;           // warps per CTA (one CTA per SM)
+constexpr int TC_Q6K_COPY = 224;       // Q6_K: bytes copied per row (16-byte-aligned cover of a 210-byte superblock)
 constexpr int TC_BAR_BYTES = 1024;
 __host__ __device__ constexpr int tc_part_bytes(int nw) { return 2 * nw * 512; }   // double-buffered partial tiles (16 x 8 floats per warp)
 
@@ -430,7 +433,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1) qmv_tc_kernel(const TcParams p)
         uint32_t size = (uint32_t)p.chunk_bytes;
         if (FMT == FMT_Q6_K) {
             off &= ~(int64_t)15;
-            size = (uint32_t)min((int64_t)p.slot_bytes, p.rows * p.row_bytes - off);
+            size = (uint32_t)min((int64_t)TC_Q6K_COPY, p.rows * p.row_bytes - off);
         }
         if (lane >= valid) size = 0u;
         const uint32_t total = __reduce_add_sync(0xffffffffu, size);
