@@ -316,31 +316,72 @@ def rotating_pool(torch, fmt, rows, cols, seed, min_total):
     return [base] + [base.clone() for _ in range(copies - 1)]
 
 
+POOL_L2_MULTIPLE = 4      # rotating weight pools hold at least this many L2s of data
+
+
+def single_launch_us(torch, q, stream, fn, n, reps=30):
+    """Median device time of ONE call fn(i) with programmatic dependent launch
+    off: each call is bracketed by its own CUDA events on the launch stream,
+    behind a ~20 µs sleep kernel so the host has queued both events and the
+    call before the GPU reaches them (the events then time the GPU's work for
+    that call alone, launch gap included).  fn(i) uses weight copy i % n."""
+    pdl = q.qmv_get_pdl()
+    q.qmv_set_pdl(0)
+    out = []
+    try:
+        with torch.cuda.stream(stream):
+            for i in range(reps + 3):
+                ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                torch.cuda._sleep(40000)
+                ev0.record(stream)
+                fn(i % n)
+                ev1.record(stream)
+                ev1.synchronize()
+                if i >= 3:
+                    out.append(ev0.elapsed_time(ev1) * 1e3)
+    finally:
+        q.qmv_set_pdl(pdl)
+    return statistics.median(out)
+
+
 def measure_matvec(torch, q, stream, fmt, rows, cols, n_tok, seed, reps=200, argmax=False):
-    """µs per matvec over a pool of weight copies larger than L2 (replayed graph);
-    argmax: the projection followed by the greedy argmax (qmv_argmax)."""
-    pool = rotating_pool(torch, fmt, rows, cols, seed, 2 * L2_BYTES)
+    """µs per matvec over a pool of weight copies of at least 4x L2: (a) a
+    replayed graph of back-to-back launches with programmatic dependent launch
+    (each launch's prologue and first weight copies overlap the previous
+    launch: throughput of a stream of such matvecs), and (b) one launch alone,
+    PDL off, event-timed (its latency).  argmax: the projection followed by
+    the greedy argmax (qmv_argmax)."""
+    pool = rotating_pool(torch, fmt, rows, cols, seed, POOL_L2_MULTIPLE * L2_BYTES)
     x = torch.from_numpy(synth.gen_x(n_tok, cols, seed, 1)).cuda()
     y = torch.empty((n_tok, rows), device="cuda")
     idx = torch.empty(n_tok, dtype=torch.int32, device="cuda")
-    per_graph = min(len(pool) * max(1, 64 // len(pool)), 256)
+    per_graph = len(pool) if len(pool) >= 64 else len(pool) * (64 // len(pool))
+
+    def one(i):
+        W = pool[i % len(pool)]
+        if argmax:
+            q.qmv_argmax(fmt, W, rows, cols, x, y, n_tok, idx)
+        elif n_tok == 1:
+            q.qmv_f32(fmt, W, rows, cols, x, y)
+        else:
+            q.qmv_batched(fmt, W, rows, cols, x, y, n_tok)
 
     def body():
         for i in range(per_graph):
-            W = pool[i % len(pool)]
-            if argmax:
-                q.qmv_argmax(fmt, W, rows, cols, x, y, n_tok, idx)
-            elif n_tok == 1:
-                q.qmv_f32(fmt, W, rows, cols, x, y)
-            else:
-                q.qmv_batched(fmt, W, rows, cols, x, y, n_tok)
+            one(i)
     g = capture(torch, body, stream)
     time_graph(torch, g, 3, stream)
     n_rep = max(2, reps // per_graph)
     sec = time_graph(torch, g, n_rep, stream) / (n_rep * per_graph)
+    del g
     wb = synth.matrix_bytes(fmt, rows, cols)
+    us1 = single_launch_us(torch, q, stream, one, len(pool))
     return {"fmt": synth.FORMAT_NAMES[fmt], "rows": rows, "cols": cols, "n_tok": n_tok,
-            "us": sec * 1e6, "weight_gbs": wb / sec / 1e9, "copies": len(pool)}
+            "us": sec * 1e6, "weight_gbs": wb / sec / 1e9, "copies": len(pool),
+            "pool_bytes": wb * len(pool),
+            "timing": "graph of back-to-back launches, programmatic dependent launch on (pipelined)",
+            "us_single_launch": round(us1, 3), "weight_gbs_single_launch": round(wb / us1 / 1e3, 1),
+            "single_launch_timing": "one launch, PDL off, CUDA events around it"}
 
 
 def measure_moe(torch, q, stream, reps=200):
@@ -351,7 +392,10 @@ def measure_moe(torch, q, stream, reps=200):
     host = [synth.gen_blocks(Q4_K, inter * E, hidden, seed, 1), synth.gen_blocks(Q4_K, inter * E, hidden, seed, 2),
             synth.gen_blocks(Q4_K, hidden * E, inter, seed, 3)]
     base = [torch.from_numpy(h).cuda() for h in host]
-    n_copies = 6      # each step touches 24.8 MB; six copies keep reuse distance > L2
+    touched = 4 * (2 * gus + ds)
+    # each step touches 24.8 MB of the selected experts: enough copies that the
+    # steps of one graph replay cycle through at least 4x L2 of weights
+    n_copies = -(-POOL_L2_MULTIPLE * L2_BYTES // touched)
     sets = [base] + [[t.clone() for t in base] for _ in range(n_copies - 1)]
     logits, bias = synth.gen_router(E, seed, 5)
     lg, bs = torch.from_numpy(logits).cuda(), torch.from_numpy(bias).cuda()
@@ -360,30 +404,77 @@ def measure_moe(torch, q, stream, reps=200):
     g = torch.empty(4, device="cuda")
     h = torch.empty((4, inter), device="cuda")
     y = torch.empty(hidden, device="cuda")
-    per_graph = 4 * n_copies
+    per_graph = 2 * n_copies
+
+    def one(i):
+        G, U, D = sets[i % n_copies]
+        q.moe_route(lg, bs, E, 4, ids, g)
+        q.moe_ffn(Q4_K, G, U, gus, Q4_K, D, ds, E, ids, g, 4, hidden, inter, x, h, y)
 
     def body():
         for i in range(per_graph):
-            G, U, D = sets[i % n_copies]
-            q.moe_route(lg, bs, E, 4, ids, g)
-            q.moe_ffn(Q4_K, G, U, gus, Q4_K, D, ds, E, ids, g, 4, hidden, inter, x, h, y)
+            one(i)
     gr = capture(torch, body, stream)
     time_graph(torch, gr, 3, stream)
     n_rep = max(2, reps // per_graph)
     sec = time_graph(torch, gr, n_rep, stream) / (n_rep * per_graph)
-    touched = 4 * (2 * gus + ds)
+    del gr
+    us1 = single_launch_us(torch, q, stream, one, n_copies)
     return {"workload": "MoE FFN step: route top-4 of 32 + Q4_K gate/up 1792x2048 + down 2048x1792",
             "us": sec * 1e6, "weight_gbs": touched / sec / 1e9, "launches_per_step": 3,
-            "weight_bytes_touched": touched}
+            "weight_bytes_touched": touched, "copies": n_copies,
+            "timing": "graph of back-to-back steps, programmatic dependent launch on (pipelined)",
+            "us_single_launch": round(us1, 3), "weight_gbs_single_launch": round(touched / us1 / 1e3, 1),
+            "single_launch_timing": "one step alone, PDL off, CUDA events around it"}
 
 
 # ----------------------------------------------------------- reference arm --
 
-def oracle_rate(seconds, cache):
-    """The oracle on the host cores over a bounded sample of the sweep: GB/s of
-    weight bytes, the threads it used, and the sample description."""
+def cpu_info():
+    """CPU model, physical cores and logical CPUs of this host (lscpu)."""
+    info = {"model": None, "physical_cores": None, "logical_cpus": os.cpu_count()}
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        kv = {}
+        for line in out.splitlines():
+            if ":" in line:
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+        info["model"] = kv.get("Model name")
+        cps, sockets = kv.get("Core(s) per socket"), kv.get("Socket(s)")
+        if cps and sockets and cps.isdigit() and sockets.isdigit():
+            info["physical_cores"] = int(cps) * int(sockets)
+    except (OSError, subprocess.SubprocessError):
+        pass
+    return info
+
+
+def oracle_baseline(seconds_single, seconds_all, cache):
+    """The oracle timed on this host's cores over a bounded sample of the sweep
+    (layer 0's four Q8_0 matvecs): single-threaded and with OpenMP over rows on
+    every logical CPU, each the median GB/s of 5 timed passes."""
     import oracle
-    threads = os.cpu_count() or 1
+    info = cpu_info()
+    out = {}
+    for label, threads, secs in (("single_thread", 1, seconds_single),
+                                 ("all_cores", os.cpu_count() or 1, seconds_all)):
+        rate, used, sample = oracle_rate(secs, cache, threads)
+        out[label] = {"value": round(rate, 3), "cores": used, "sample": sample}
+    return {"value": out["all_cores"]["value"], "unit": "GB/s", "cores": out["all_cores"]["cores"],
+            "kind": "oracle", "sample": out["all_cores"]["sample"],
+            "single_thread": {"value": out["single_thread"]["value"], "unit": "GB/s", "cores": 1,
+                              "sample": out["single_thread"]["sample"]},
+            "cpu_model": info["model"], "physical_cores": info["physical_cores"],
+            "logical_cpus": info["logical_cpus"],
+            "method": "oracle (plain C, f64 accumulation, OpenMP over rows), median of 5 timed passes"}
+
+
+def oracle_rate(seconds, cache, threads=None):
+    """The oracle on the host cores over a bounded sample of the sweep: GB/s of
+    weight bytes (median of 5 passes, each about seconds / 5), the threads it
+    used, and the sample description."""
+    import oracle
+    threads = threads or os.cpu_count() or 1
     mats = [(l, m, name, rows, cols) for (l, m, name, rows, cols) in sweep_layers() if l == 0]
     data = []
     for (l, m, name, rows, cols) in mats:
@@ -391,16 +482,22 @@ def oracle_rate(seconds, cache):
         if key not in cache:
             cache[key] = synth.gen_blocks(Q8_0, rows, cols, synth.CFG4_SEED, 16 * l + m)
         data.append((cache[key], rows, cols, synth.gen_x(1, cols, synth.CFG4_SEED, 5000 + m)))
-    done_bytes, t0, passes = 0, time.perf_counter(), 0
-    while True:
-        for W, rows, cols, x in data:
-            oracle.qmv(Q8_0, W, rows, cols, x, nthreads=threads)
-            done_bytes += W.nbytes
-        passes += 1
-        if time.perf_counter() - t0 >= seconds:
-            break
-    dt = time.perf_counter() - t0
-    return done_bytes / dt / 1e9, threads, f"{passes} passes over layer 0's four Q8_0 matvecs ({dt:.1f} s)"
+    rates, total_t, total_passes = [], 0.0, 0
+    for _ in range(5):
+        done_bytes, t0, passes = 0, time.perf_counter(), 0
+        while True:
+            for W, rows, cols, x in data:
+                oracle.qmv(Q8_0, W, rows, cols, x, nthreads=threads)
+                done_bytes += W.nbytes
+            passes += 1
+            if time.perf_counter() - t0 >= seconds / 5:
+                break
+        dt = time.perf_counter() - t0
+        rates.append(done_bytes / dt / 1e9)
+        total_t += dt
+        total_passes += passes
+    return (statistics.median(rates), threads,
+            f"{total_passes} passes over layer 0's four Q8_0 matvecs ({total_t:.1f} s, {threads} threads)")
 
 
 def run_reference(args):
@@ -439,14 +536,50 @@ def run_reference(args):
 
 # ------------------------------------------------------------ profile case --
 
-def run_profile_case(args):
-    """A few launches of one large matvec (weights larger than L2, < 1 GB on the
-    device) -- the small case that ncu captures."""
+PROFILE_CASES = {
+    # name: (fmt, rows, cols) -- one matvec, a few launches, < 1 GB on the device
+    "q8_0": (Q8_0, 65536, 2048), "q4_k": (Q4_K, 131072, 2048), "q6_k": (Q6_K, 96000, 2048),
+    "q8_0_down": (Q8_0, 16384, 8192), "q8_0_o": (Q8_0, 2048, 2048),
+    "gate_up": (Q8_0, 16384, 2048), "down": (Q8_0, 2048, 8192), "qkv": (Q8_0, 3072, 2048),
+    "cfg0": (Q8_0, 1024, 1024), "cfg1": (Q4_K, 3072, 2048), "cfg2": (Q6_K, 128000, 2048),
+}
+
+
+def run_profile_moe(args):
+    """A few MoE FFN steps of the 32-expert workload (router, gate/up with the
+    SwiGLU epilogue, weighted down), 198 MB of experts on the device."""
     import torch
     import quantized_decode_superblocks_b200 as q
-    fmt = {"q8_0": Q8_0, "q4_k": Q4_K, "q6_k": Q6_K, "q8_0_down": Q8_0, "q8_0_o": Q8_0}[args.profile_case]
-    rows, cols = {"q8_0": (65536, 2048), "q4_k": (131072, 2048), "q6_k": (96000, 2048),
-                  "q8_0_down": (16384, 8192), "q8_0_o": (2048, 2048)}[args.profile_case]
+    torch.cuda.set_device(0)
+    w = synth.workload_cfg3()
+    E, hidden, inter, seed = w["n_expert"], w["hidden"], w["inter"], w["seed"]
+    gus, ds = synth.matrix_bytes(Q4_K, inter, hidden), synth.matrix_bytes(Q4_K, hidden, inter)
+    G = torch.from_numpy(synth.gen_blocks(Q4_K, inter * E, hidden, seed, 1)).cuda()
+    U = torch.from_numpy(synth.gen_blocks(Q4_K, inter * E, hidden, seed, 2)).cuda()
+    D = torch.from_numpy(synth.gen_blocks(Q4_K, hidden * E, inter, seed, 3)).cuda()
+    logits, bias = synth.gen_router(E, seed, 5)
+    lg, bs = torch.from_numpy(logits).cuda(), torch.from_numpy(bias).cuda()
+    x = torch.from_numpy(synth.gen_x(1, hidden, seed, 4)[0]).cuda()
+    ids = torch.empty(4, dtype=torch.int32, device="cuda")
+    g = torch.empty(4, device="cuda")
+    h = torch.empty((4, inter), device="cuda")
+    y = torch.empty(hidden, device="cuda")
+    for _ in range(max(1, args.steps)):
+        q.moe_route(lg, bs, E, 4, ids, g)
+        q.moe_ffn(Q4_K, G, U, gus, Q4_K, D, ds, E, ids, g, 4, hidden, inter, x, h, y)
+    torch.cuda.synchronize()
+    assert q.qmv_check() == 0
+    print(json.dumps({"profile_case": "moe", "weight_bytes_touched": 4 * (2 * gus + ds)}))
+    return 0
+
+
+def run_profile_case(args):
+    """A few launches of one matvec -- the small case that ncu captures."""
+    if args.profile_case == "moe":
+        return run_profile_moe(args)
+    import torch
+    import quantized_decode_superblocks_b200 as q
+    fmt, rows, cols = PROFILE_CASES[args.profile_case]
     torch.cuda.set_device(0)
     W = torch.from_numpy(synth.gen_blocks(fmt, rows, cols, 77, 0)).cuda()
     x = torch.from_numpy(synth.gen_x(args.n_tok, cols, 77, 1)).cuda()
@@ -477,7 +610,7 @@ def main():
                     help="launch without programmatic dependent launch (qmv_set_pdl(0))")
     ap.add_argument("--headline-only", action="store_true",
                     help="skip the per-config measurements and the CPU baseline")
-    ap.add_argument("--profile-case", choices=["q8_0", "q4_k", "q6_k", "q8_0_down", "q8_0_o"])
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES) + ["moe"])
     args = ap.parse_args()
     if args.warmup < 3 and not args.profile_case:
         raise SystemExit("--warmup must be at least 3")
@@ -598,8 +731,7 @@ def main():
 
     cpu = None
     if dist.rank == 0 and args.gpus == 1 and not args.headline_only:
-        rate, threads, sample = oracle_rate(10.0, cache)
-        cpu = {"value": round(rate, 3), "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample}
+        cpu = oracle_baseline(8.0, 8.0, cache)
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": args.gpus,

@@ -89,6 +89,11 @@ typedef enum {
 #define QMV_DEVERR_EXPERT_ID 1      /* an expert id was outside [0, n_expert); that
                                        expert's contribution was dropped        */
 #define QMV_DEVERR_TIMEOUT 2        /* a pipeline wait gave up (bounded wait)   */
+#define QMV_DEVERR_DRAIN 4          /* after a timeout, a CTA also gave up waiting for
+                                       its own copies in flight and exited: they may
+                                       still land in shared memory reused by later
+                                       kernels, so later results on this device are
+                                       suspect (recreate the context to be sure)   */
 
 /* y[rows] = W x.  x: f32 [cols]; y: f32 [rows].
  * One launch covers a whole fused projection: pass the row-concatenation of
@@ -253,6 +258,16 @@ int qmv_block_weights(int fmt);
  * (true for inference weights loaded once).  qmv_get_pdl returns the setting. */
 void qmv_set_pdl(int enable);
 int qmv_get_pdl(void);
+
+/* Test hook: which kernel served the calling host thread's most recent
+ * matvec call (qmv_f32, qmv_batched, qmv_multi, qmv_chain, moe_qmv, moe_ffn,
+ * qmv_argmax), so tests can show that each kernel path is exercised.
+ * QMV_KERNEL_NONE before the first such call on the thread. */
+#define QMV_KERNEL_NONE 0
+#define QMV_KERNEL_WARP_RING 1      /* one to four tokens, per-warp copy rings   */
+#define QMV_KERNEL_GENERAL 2        /* general pipeline (groups, grouped launches) */
+#define QMV_KERNEL_TENSOR_CORE 3    /* three to eight tokens, mma.sync          */
+int qmv_debug_last_kernel(void);
 
 /* Test hook for host-side failure handling: the next `count` launches made by
  * this library fail with QMV_ERR_CUDA without reaching the GPU. */

@@ -24,12 +24,14 @@ STATUS_NAMES = {0: "QMV_OK", -1: "QMV_ERR_NULL", -2: "QMV_ERR_FMT", -3: "QMV_ERR
                 -8: "QMV_ERR_DEVICE"}
 DEVERR_EXPERT_ID = 1
 DEVERR_TIMEOUT = 2
+DEVERR_DRAIN = 4
+KERNEL_WARP_RING, KERNEL_GENERAL, KERNEL_TENSOR_CORE = 1, 2, 3
 
 EXPORTED = ("qmv_f32", "qmv_batched", "qmv_multi", "qmv_chain", "qmv_argmax", "moe_route", "moe_qmv", "moe_ffn", "moe_ffn_static",
             "qmv_dequant",
             "qmv_check", "qmv_strerror", "qmv_block_bytes", "qmv_block_weights",
             "qmv_debug_fail_next_launches", "qmv_debug_short_copies", "qmv_set_pdl", "qmv_get_pdl",
-            "qmv_last_cuda_error")
+            "qmv_last_cuda_error", "qmv_debug_last_kernel")
 
 
 class QmvTask(ctypes.Structure):
@@ -83,6 +85,7 @@ def lib() -> ctypes.CDLL:
         L.qmv_set_pdl.argtypes = [c_int]
         L.qmv_set_pdl.restype = None
         L.qmv_get_pdl.argtypes = []
+        L.qmv_debug_last_kernel.argtypes = []
         L.qmv_last_cuda_error.argtypes = []
         L.qmv_last_cuda_error.restype = ctypes.c_char_p
         for name in EXPORTED:
@@ -132,6 +135,11 @@ def qmv_set_pdl(enable: bool) -> None:
 
 def qmv_get_pdl() -> bool:
     return bool(lib().qmv_get_pdl())
+
+
+def qmv_debug_last_kernel() -> int:
+    """Which kernel served this thread's most recent matvec call (KERNEL_*)."""
+    return lib().qmv_debug_last_kernel()
 
 
 def qmv_block_bytes(fmt: int) -> int:

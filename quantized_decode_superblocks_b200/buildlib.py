@@ -19,7 +19,6 @@ BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libqmv.so")
 
 SOURCES = ["qmv_api.cu", "qmv_fmt_q8_0.cu", "qmv_fmt_q4_k.cu", "qmv_fmt_q6_k.cu"]
-HEADERS = ["qmv_device.cuh", "qmv_decode1.cuh", "qmv_decodemt.cuh", "qmv_kernels.cuh", "qmv_rw.cuh", "qmv_dispatch.cuh", "qmv_misc.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
                      "-I", os.path.join(ROOT, "include"), "--expt-relaxed-constexpr"]
@@ -32,8 +31,13 @@ def nvcc() -> str:
     return path
 
 
+def headers():
+    """Every header under csrc/ (all of them are included by some source)."""
+    return sorted(f for f in os.listdir(CSRC) if f.endswith((".cuh", ".h")))
+
+
 def _inputs():
-    files = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
+    files = [os.path.join(CSRC, f) for f in SOURCES + headers()]
     files.append(os.path.join(ROOT, "include", "qmv.h"))
     files.append(os.path.abspath(__file__))
     return files

@@ -61,6 +61,9 @@ std::atomic<int> g_fail_launches{0};
 std::atomic<int> g_pdl{0};
 std::atomic<unsigned> g_debug_extra_tx{0};
 thread_local cudaError_t t_last_cuda = cudaSuccess;
+// The kernel that served this host thread's most recent matvec call
+// (QMV_KERNEL_*; test hook qmv_debug_last_kernel).
+thread_local int t_last_kernel = QMV_KERNEL_NONE;
 
 int cuda_fail(cudaError_t e)
 {
@@ -233,6 +236,7 @@ int make_plan(int fmt, int64_t rows, int64_t cols, int n_tok, int G, int n_jobs,
 
 int launch_plan(int fmt, const Plan &pl, cudaStream_t stream)
 {
+    t_last_kernel = QMV_KERNEL_GENERAL;
     cudaError_t e;
     switch (fmt) {
     case QMV_Q8_0: e = launch_pipeline<FMT_Q8_0>(pl.p, pl.kc, pl.grid, pl.smem, stream); break;
@@ -414,6 +418,7 @@ int rw_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x
     p.cta_begin[1] = (int)ctas;
     rw_split(p.t[0], ctas * NW);
     const bool pdl = g_pdl.load() != 0;
+    t_last_kernel = QMV_KERNEL_WARP_RING;
     cudaError_t e;
     if (n_tok == 1) {
         e = rw_launch(fmt, p, g.R, dim3((unsigned)ctas), g.smem, st, pdl, false);
@@ -505,6 +510,7 @@ int tc_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x
     p.err = di.err;
     p.debug_extra_tx = g_debug_extra_tx.load();
     const bool pdl = g_pdl.load() != 0;
+    t_last_kernel = QMV_KERNEL_TENSOR_CORE;
     const cudaError_t e = fmt == QMV_Q8_0   ? launch_tc<FMT_Q8_0>(p, g.x_smem, dim3((unsigned)ctas), g.smem, st, pdl)
                           : fmt == QMV_Q4_K ? launch_tc<FMT_Q4_K>(p, g.x_smem, dim3((unsigned)ctas), g.smem, st, pdl)
                                             : launch_tc<FMT_Q6_K>(p, g.x_smem, dim3((unsigned)ctas), g.smem, st, pdl);
@@ -530,6 +536,7 @@ int rw_chain(int fmt, const qmv_task *tasks, int n_tasks, const DevInfo &di, cud
         if (ctas_per_sm < 1) return QMV_ERR_SHAPE;
     }
     const int64_t ctas = (int64_t)ctas_per_sm * di.sm_count;
+    t_last_kernel = QMV_KERNEL_WARP_RING;
     for (int t0 = 0; t0 < n_tasks; t0 += RW_MAX_TASKS) {
         const int n = std::min(RW_MAX_TASKS, n_tasks - t0);
         p.n_tasks = n;
@@ -579,6 +586,8 @@ void qmv_set_pdl(int enable) { g_pdl.store(enable ? 1 : 0); }
 void qmv_debug_short_copies(int bytes) { g_debug_extra_tx.store(bytes > 0 ? (unsigned)bytes : 0u); }
 
 int qmv_get_pdl(void) { return g_pdl.load(); }
+
+int qmv_debug_last_kernel(void) { return t_last_kernel; }
 
 const char *qmv_last_cuda_error(void)
 {
@@ -670,6 +679,7 @@ int qmv_multi(int fmt, int n_tok, const qmv_task *tasks, int n_tasks, qmv_stream
     // MAX_MULTI tasks each
     std::vector<char> done((size_t)n_tasks, 0);
     static thread_local MultiParams mp;
+    t_last_kernel = QMV_KERNEL_GENERAL;
     for (int t0 = 0; t0 < n_tasks; ++t0) {
         if (done[(size_t)t0]) continue;
         const KernelChoice kc = plans[(size_t)t0].kc;

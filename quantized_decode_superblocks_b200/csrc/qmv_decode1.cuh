@@ -9,10 +9,7 @@
 //     quantized GEMMs, e.g. Kim et al. 2022, "Who Says Elephants Can't Run:
 //     Bringing Large Scale MoE Models into Cloud Scale Production"): a byte u
 //     placed under the exponent of 2^23 gives the float 2^23 + u, and one
-//     subtraction leaves u exactly.  With QMV_CVT_HALF the byte is placed
-//     under the fp16 exponent of 1024 instead and a mixed-precision
-//     f16 + f32 -> f32 add removes the offset.  Either way every value is an
-//     exact small integer.
+//     subtraction leaves u exactly, an exact small integer.
 //   * Packed f32x2 FMAs (sm_100) with several independent accumulators.
 //   * The factored form per scale group: sum_i w_i x_i =
 //     scale * sum_i q_i x_i (- min * sum_i x_i), so scales are applied once per
@@ -29,27 +26,9 @@ namespace qmv {
 __device__ __forceinline__ float2 f2add(float2 a, float2 b) { return __fadd2_rn(a, b); }
 __device__ __forceinline__ float2 f2fma(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
-#ifdef QMV_CVT_HALF
-// fp16 bit pattern (low 16 bits of h) converted to f32 and added to c, one
-// rounding (exact for the small integers used here).
-__device__ __forceinline__ float h16_add(uint32_t h, float c)
-{
-    float r;
-    asm("add.rn.f32.f16 %0, %1, %2;" : "=f"(r) : "h"((unsigned short)(h & 0xFFFFu)), "f"(c));
-    return r;
-}
-#endif
-
 // Four unsigned bytes of w -> (b0 - bias, b2 - bias), (b1 - bias, b3 - bias) as exact f32.
 __device__ __forceinline__ void bytes4_to_f2(uint32_t w, float bias, float2 &p02, float2 &p13)
 {
-#ifdef QMV_CVT_HALF
-    const float nb = -(1024.0f + bias);
-    const uint32_t h02 = __byte_perm(w, 0x64646464u, 0x4240u);   // [b0, 0x64, b2, 0x64]
-    const uint32_t h13 = __byte_perm(w, 0x64646464u, 0x4341u);   // [b1, 0x64, b3, 0x64]
-    p02 = make_float2(h16_add(h02, nb), h16_add(h02 >> 16, nb));
-    p13 = make_float2(h16_add(h13, nb), h16_add(h13 >> 16, nb));
-#else
     const float nb = -(8388608.0f + bias);
     const float2 a = make_float2(__uint_as_float(__byte_perm(w, 0x4B000000u, 0x7650u)),
                                  __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7652u)));
@@ -57,33 +36,14 @@ __device__ __forceinline__ void bytes4_to_f2(uint32_t w, float bias, float2 &p02
                                  __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7653u)));
     p02 = f2add(a, make_float2(nb, nb));
     p13 = f2add(b, make_float2(nb, nb));
-#endif
 }
 
-// Eight nibbles of w: the low nibbles (lo02, lo13) exactly, the high nibbles
-// multiplied by NIB_HI_SCALE (hi02, hi13).
-#ifdef QMV_CVT_HALF
-constexpr float NIB_HI_SCALE = 16.0f;
-#else
-constexpr float NIB_HI_SCALE = 1.0f;
-#endif
-
+// Eight nibbles of w as exact f32: the low nibbles (lo02, lo13) and the high
+// nibbles (hi02, hi13), each pair in the order of bytes4_to_f2.
 __device__ __forceinline__ void nibbles8_to_f2(uint32_t w, float2 &lo02, float2 &lo13, float2 &hi02, float2 &hi13)
 {
-#ifdef QMV_CVT_HALF
-    const uint32_t w8 = w >> 8;
-    const uint32_t l02 = (w & 0x000F000Fu) | 0x64006400u;
-    const uint32_t l13 = (w8 & 0x000F000Fu) | 0x64006400u;
-    const uint32_t h02 = (w & 0x00F000F0u) | 0x64006400u;     // 1024 + 16 q
-    const uint32_t h13 = (w8 & 0x00F000F0u) | 0x64006400u;
-    lo02 = make_float2(h16_add(l02, -1024.0f), h16_add(l02 >> 16, -1024.0f));
-    lo13 = make_float2(h16_add(l13, -1024.0f), h16_add(l13 >> 16, -1024.0f));
-    hi02 = make_float2(h16_add(h02, -1024.0f), h16_add(h02 >> 16, -1024.0f));
-    hi13 = make_float2(h16_add(h13, -1024.0f), h16_add(h13 >> 16, -1024.0f));
-#else
     bytes4_to_f2(w & 0x0F0F0F0Fu, 0.0f, lo02, lo13);
     bytes4_to_f2((w >> 4) & 0x0F0F0F0Fu, 0.0f, hi02, hi13);
-#endif
 }
 
 __device__ __forceinline__ float hsum2(float2 a, float2 b) { return (a.x + a.y) + (b.x + b.y); }
@@ -191,9 +151,9 @@ __device__ __forceinline__ float q4_k_dot1(uint32_t sb, int c, const Q4kSel &sel
     bytes4_to_f2(v, 0.0f, sc0_m0, sc1_m1);
     const float d = half_bits_to_float(hdr.x);
     const float dmin = half_bits_to_float(hdr.x >> 16);
-    // d*sc0*sa + d*sc1*sb - dmin*m0*xsa - dmin*m1*xsb (sb carries NIB_HI_SCALE)
+    // d*sc0*sa + d*sc1*sb - dmin*m0*xsa - dmin*m1*xsb
     float r = (d * sc0_m0.x) * sa;
-    r = fmaf(d * (sc1_m1.x * (1.0f / NIB_HI_SCALE)), sbv, r);
+    r = fmaf(d * sc1_m1.x, sbv, r);
     r = fmaf(-dmin * sc0_m0.y, xsa, r);
     r = fmaf(-dmin * sc1_m1.y, xsb, r);
     return r;

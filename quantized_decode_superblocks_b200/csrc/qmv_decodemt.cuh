@@ -91,7 +91,7 @@ __device__ __forceinline__ void q4_k_slice_mt(const uint32_t (&sb)[R], int c, co
         float2 sc0_m0, sc1_m1;
         bytes4_to_f2(v, 0.0f, sc0_m0, sc1_m1);
         const float d = half_bits_to_float(hdr.x), dmin = half_bits_to_float(hdr.x >> 16);
-        const float a = d * sc0_m0.x, b = d * (sc1_m1.x * (1.0f / NIB_HI_SCALE));
+        const float a = d * sc0_m0.x, b = d * sc1_m1.x;
         const float ma = -(dmin * sc0_m0.y), mb = -(dmin * sc1_m1.y);
         dscA[k] = make_float2(a, a); dmA[k] = make_float2(ma, ma);
         dscB[k] = make_float2(b, b); dmB[k] = make_float2(mb, mb);

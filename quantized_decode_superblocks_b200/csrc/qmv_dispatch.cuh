@@ -3,26 +3,45 @@
 // parallel.
 #pragma once
 
+#include <atomic>
+#include <mutex>
+
 #include "qmv_rw.cuh"
 #include "qmv_tc.cuh"
 
 namespace qmv {
 
-// Launch `kern` with `arg`: raises the dynamic shared-memory limit once per
-// (kernel, device) and adds the programmatic-serialization attribute when asked.
-template <class Kern, class Arg>
-static cudaError_t launch_with(Kern kern, int *configured, const Arg &arg, dim3 grid, size_t smem,
-                               cudaStream_t stream, bool pdl, bool cooperative = false, int threads = NTHREADS)
+// Per (kernel, device): the dynamic shared-memory limit set so far.
+using SmemCfg = std::atomic<int>[64];
+
+// Raises kern's dynamic shared-memory limit on the current device to at least
+// smem.  Host threads may race here: the fast path is one atomic load, and the
+// raise itself runs under a lock so the limit only ever grows.
+template <class Kern>
+static cudaError_t ensure_smem(Kern kern, SmemCfg &configured, size_t smem)
 {
+    static std::mutex mu;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (configured[dev] < (int)smem) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        configured[dev] = (int)smem;
-    }
+    if (configured[dev].load(std::memory_order_acquire) >= (int)smem) return cudaSuccess;
+    std::lock_guard<std::mutex> lk(mu);
+    if (configured[dev].load(std::memory_order_relaxed) >= (int)smem) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured[dev].store((int)smem, std::memory_order_release);
+    return cudaSuccess;
+}
+
+// Launch `kern` with `arg`: raises the dynamic shared-memory limit once per
+// (kernel, device) and adds the programmatic-serialization attribute when asked.
+template <class Kern, class Arg>
+static cudaError_t launch_with(Kern kern, SmemCfg &configured, const Arg &arg, dim3 grid, size_t smem,
+                               cudaStream_t stream, bool pdl, bool cooperative = false, int threads = NTHREADS)
+{
+    cudaError_t e = ensure_smem(kern, configured, smem);
+    if (e != cudaSuccess) return e;
     cudaLaunchAttribute attr[2];
     unsigned n_attr = 0;
     if (pdl) {
@@ -49,12 +68,12 @@ template <int FMT, int NTOK, int R, bool XREG>
 struct Instance {
     static cudaError_t one(const Params &p, dim3 grid, size_t smem, cudaStream_t st, bool pdl)
     {
-        static int configured[64] = {0};
+        static SmemCfg configured;
         return launch_with(qmv_pipeline_kernel<FMT, NTOK, R, XREG>, configured, p, grid, smem, st, pdl);
     }
     static cudaError_t multi(const MultiParams &mp, dim3 grid, size_t smem, cudaStream_t st, bool pdl)
     {
-        static int configured[64] = {0};
+        static SmemCfg configured;
         return launch_with(qmv_multi_kernel<FMT, NTOK, R, XREG>, configured, mp, grid, smem, st, pdl);
     }
 };
@@ -124,9 +143,9 @@ struct MultiLaunch {
 
 template <int FMT, int R, int NT, int NTOK = 1>
 struct RwInstance {
-    static int *configured()
+    static SmemCfg &configured()
     {
-        static int c[64] = {0};
+        static SmemCfg c;
         return c;
     }
     static cudaError_t go(const RwParamsT<NT> &p, dim3 grid, size_t smem, cudaStream_t st, bool pdl, bool coop)
@@ -135,16 +154,8 @@ struct RwInstance {
     }
     static cudaError_t occupancy(size_t smem, int *n)
     {
-        int dev = 0;
-        cudaError_t e = cudaGetDevice(&dev);
+        const cudaError_t e = ensure_smem(qmv_rw_kernel<FMT, R, NT, NTOK>, configured(), smem);
         if (e != cudaSuccess) return e;
-        if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-        if (configured()[dev] < (int)smem) {
-            e = cudaFuncSetAttribute(qmv_rw_kernel<FMT, R, NT, NTOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)smem);
-            if (e != cudaSuccess) return e;
-            configured()[dev] = (int)smem;
-        }
         return cudaOccupancyMaxActiveBlocksPerMultiprocessor(n, qmv_rw_kernel<FMT, R, NT, NTOK>, NTHREADS, smem);
     }
 };
@@ -211,7 +222,7 @@ cudaError_t launch_multi(const MultiParams &mp, const KernelChoice &kc, int grid
 template <int FMT>
 cudaError_t launch_tc(const TcParams &p, bool x_smem, dim3 grid, size_t smem, cudaStream_t st, bool pdl)
 {
-    static int configured_s[64] = {0}, configured_g[64] = {0};
+    static SmemCfg configured_s, configured_g;
     if constexpr (FMT == FMT_Q6_K) {       // x always in shared memory
         if (!x_smem) return cudaErrorInvalidValue;
         return launch_with(qmv_tc_kernel<FMT, TC_WARPS, true>, configured_s, p, grid, smem, st, pdl, false, TC_WARPS * 32);

@@ -48,7 +48,7 @@ constexpr int SMEM_RES = 128;                // partial-sum exchange: 2 x 256 fl
 constexpr int SMEM_HDR = 128 + 2 * 256 * 4;
 
 enum { MODE_SEPARATE = 0, MODE_WEIGHTED = 1, MODE_SWIGLU = 2 };
-enum { DEVERR_EXPERT_ID = 1, DEVERR_TIMEOUT = 2 };
+enum { DEVERR_EXPERT_ID = 1, DEVERR_TIMEOUT = 2, DEVERR_DRAIN = 4 };
 
 struct Params {
     // geometry

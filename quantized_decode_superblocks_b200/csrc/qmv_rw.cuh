@@ -533,11 +533,16 @@ __global__ void __launch_bounds__(NTHREADS, (NTOK > 2 ? 1 : 2)) qmv_rw_kernel(co
         __syncthreads();                          // x stays until every warp is done with it
     }
     if (p.ordered) rw_grid_exit(p.sync, gridDim.x);
-    // after a timeout: let the copies still in flight land before the CTA exits
+    // after a timeout: let the copies still in flight land before the CTA
+    // exits; if that wait runs out too, DEVERR_DRAIN marks the device's later
+    // results as suspect (copies may land in shared memory after the exit)
     if (dead) {
         int pending = __shfl_sync(0xFFFFFFFFu, lane == 0 ? cur->issued : 0, 0) - consumed;
         for (; pending > 0; --pending) {
-            (void)mbar_wait_bounded(full0 + 8u * (uint32_t)slot, phase);
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(full0 + 8u * (uint32_t)slot, phase))) {
+                if (lane == 0) atomicOr(p.err, DEVERR_DRAIN);
+                break;
+            }
             if (++slot == S) {
                 slot = 0;
                 phase ^= 1u;

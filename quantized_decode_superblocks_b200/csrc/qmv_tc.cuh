@@ -539,10 +539,16 @@ __global__ void __launch_bounds__(NWARP * 32, 1) qmv_tc_kernel(const TcParams p)
             }
         }
     }
-    // a warp that gave up waits (again bounded) for the copies it still has in flight
+    // a warp that gave up waits (again bounded) for the copies it still has in
+    // flight; if that wait runs out too, copies may still land in this CTA's
+    // shared memory after it exits: DEVERR_DRAIN marks the device's later
+    // results as suspect
     for (int j = consumed; j < issued; ++j) {
         const int sl = j % S;
-        (void)mbar_wait_bounded(bar0 + 8u * (uint32_t)sl, (uint32_t)((j / S) & 1));
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar0 + 8u * (uint32_t)sl, (uint32_t)((j / S) & 1)))) {
+            if (lane == 0) atomicOr(p.err, DEVERR_DRAIN);
+            break;
+        }
     }
 }
 

@@ -138,3 +138,61 @@ def decode2(fmt: int, blk) -> np.ndarray:
     f = fields_q6_k(blk)
     return np.array([f["d"] * f["scales"][i // 16] * (f["q"][i] - 32) for i in range(256)],
                     dtype=np.float64).astype(np.float32)
+
+
+# ------------------------------------------------------ vectorised encoders
+# The same placements as the encoders above, for many blocks at once (the
+# full-value-range GPU tests pack whole matrices).  Pinned against the
+# one-block encoders by a CPU test.
+
+def pack_q8_0_many(d_bits, q) -> np.ndarray:
+    d_bits = np.asarray(d_bits, dtype=np.uint16)
+    q = np.asarray(q, dtype=np.int64)
+    n = d_bits.shape[0]
+    assert q.shape == (n, 32) and q.min() >= -128 and q.max() <= 127
+    out = np.zeros((n, 34), dtype=np.uint8)
+    out[:, 0] = d_bits & 0xFF
+    out[:, 1] = d_bits >> 8
+    out[:, 2:] = (q & 0xFF).astype(np.uint8)
+    return out.reshape(-1)
+
+
+def pack_q4_k_many(d_bits, dmin_bits, sc, m, q) -> np.ndarray:
+    d_bits = np.asarray(d_bits, dtype=np.uint16)
+    dmin_bits = np.asarray(dmin_bits, dtype=np.uint16)
+    sc, m, q = (np.asarray(a, dtype=np.int64) for a in (sc, m, q))
+    n = d_bits.shape[0]
+    assert sc.shape == (n, 8) and m.shape == (n, 8) and q.shape == (n, 256)
+    assert sc.min() >= 0 and sc.max() < 64 and m.min() >= 0 and m.max() < 64
+    assert q.min() >= 0 and q.max() < 16
+    out = np.zeros((n, 144), dtype=np.int64)
+    out[:, 0], out[:, 1] = d_bits & 0xFF, d_bits >> 8
+    out[:, 2], out[:, 3] = dmin_bits & 0xFF, dmin_bits >> 8
+    s = np.zeros((n, 12), dtype=np.int64)
+    s[:, 0:4] |= sc[:, 0:4]
+    s[:, 4:8] |= m[:, 0:4]
+    s[:, 8:12] |= (sc[:, 4:8] & 15) | ((m[:, 4:8] & 15) << 4)
+    s[:, 0:4] |= (sc[:, 4:8] >> 4) << 6
+    s[:, 4:8] |= (m[:, 4:8] >> 4) << 6
+    out[:, 4:16] = s
+    qq = q.reshape(n, 4, 2, 32)                  # [chunk c][low / high nibble][l]
+    out[:, 16:] = (qq[:, :, 0, :] | (qq[:, :, 1, :] << 4)).reshape(n, 128)
+    return out.astype(np.uint8).reshape(-1)
+
+
+def pack_q6_k_many(d_bits, scales, q) -> np.ndarray:
+    d_bits = np.asarray(d_bits, dtype=np.uint16)
+    scales, q = np.asarray(scales, dtype=np.int64), np.asarray(q, dtype=np.int64)
+    n = d_bits.shape[0]
+    assert scales.shape == (n, 16) and q.shape == (n, 256)
+    assert scales.min() >= -128 and scales.max() <= 127 and q.min() >= 0 and q.max() < 64
+    out = np.zeros((n, 210), dtype=np.int64)
+    qq = q.reshape(n, 2, 4, 32)                  # [half h][t][l]
+    for h in range(2):
+        for t in range(4):
+            k0 = 64 * h + 32 * (t & 1)
+            out[:, k0:k0 + 32] |= (qq[:, h, t, :] & 15) << (0 if t < 2 else 4)
+            out[:, 128 + 32 * h:160 + 32 * h] |= (qq[:, h, t, :] >> 4) << (2 * t)
+    out[:, 192:208] = scales & 0xFF
+    out[:, 208], out[:, 209] = d_bits & 0xFF, d_bits >> 8
+    return out.astype(np.uint8).reshape(-1)
