@@ -267,6 +267,7 @@ int qmv_get_pdl(void);
 #define QMV_KERNEL_WARP_RING 1      /* one to four tokens, per-warp copy rings   */
 #define QMV_KERNEL_GENERAL 2        /* general pipeline (groups, grouped launches) */
 #define QMV_KERNEL_TENSOR_CORE 3    /* three to eight tokens, mma.sync          */
+#define QMV_KERNEL_STREAM 4         /* one token, producer warp + whole-row stages */
 int qmv_debug_last_kernel(void);
 
 /* Test hook for host-side failure handling: the next `count` launches made by
@@ -274,11 +275,13 @@ int qmv_debug_last_kernel(void);
 void qmv_debug_fail_next_launches(int count);
 
 /* Test hook for the device-side failure path: while bytes > 0, the
- * warp-ring and tensor-core launches (qmv_f32 / qmv_batched on the shapes
- * that take them, qmv_chain) expect `bytes` more per copied tile than they
- * copy, so every stage wait runs into its bound (about a second), records
- * QMV_DEVERR_TIMEOUT for qmv_check, and the kernel still finishes; results
- * are then undefined.  0 (the default) turns it off.  Not for production. */
+ * streaming, warp-ring and tensor-core launches (qmv_f32 / qmv_batched on the
+ * shapes that take them, qmv_chain) expect `bytes` more per copied tile than
+ * they copy, so every stage wait runs into its bound (about a second), records
+ * QMV_DEVERR_TIMEOUT (and, where a kernel then also gives up waiting for its
+ * own copies, QMV_DEVERR_DRAIN) for qmv_check, and the kernel still finishes;
+ * results are then undefined.  0 (the default) turns it off.  Not for
+ * production. */
 void qmv_debug_short_copies(int bytes);
 
 #ifdef __cplusplus

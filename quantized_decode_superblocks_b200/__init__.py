@@ -25,7 +25,7 @@ STATUS_NAMES = {0: "QMV_OK", -1: "QMV_ERR_NULL", -2: "QMV_ERR_FMT", -3: "QMV_ERR
 DEVERR_EXPERT_ID = 1
 DEVERR_TIMEOUT = 2
 DEVERR_DRAIN = 4
-KERNEL_WARP_RING, KERNEL_GENERAL, KERNEL_TENSOR_CORE = 1, 2, 3
+KERNEL_WARP_RING, KERNEL_GENERAL, KERNEL_TENSOR_CORE, KERNEL_STREAM = 1, 2, 3, 4
 
 EXPORTED = ("qmv_f32", "qmv_batched", "qmv_multi", "qmv_chain", "qmv_argmax", "moe_route", "moe_qmv", "moe_ffn", "moe_ffn_static",
             "qmv_dequant",

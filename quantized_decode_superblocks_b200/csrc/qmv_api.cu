@@ -10,6 +10,7 @@
 #include "../../include/qmv.h"
 #include "qmv_misc.cuh"
 #include "qmv_rw.cuh"
+#include "qmv_sk.cuh"
 #include "qmv_tc.cuh"
 
 namespace {
@@ -432,6 +433,90 @@ int rw_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x
     return e == cudaSuccess ? QMV_OK : cuda_fail(e);
 }
 
+// ---------------------------------------------------------------------------
+// One-token streaming kernel (qmv_sk.cuh): one CTA of 12 consumer warps and a
+// producer warp per SM, stages of T whole rows in up to ~210 KB of shared
+// memory.
+constexpr int64_t SK_CTA_SMEM = 210 * 1024;
+
+struct SkGeom {
+    bool ok = false;
+    int R = 0, T = 0, S = 0, ksegs = 1, gran = 1, x_in_ring = 0;
+    int64_t pitch = 0, x_off = 0;
+    size_t smem = 0;
+};
+
+SkGeom sk_geom(int fmt, int64_t rows, int64_t cols)
+{
+    SkGeom g;
+    const int bw = block_weights(fmt), bb = block_bytes(fmt);
+    if (cols > (int64_t)SK_SEG * SK_MAX_KSEGS || (fmt == QMV_Q8_0 && cols % 64 != 0)) return g;
+    const int64_t rb = cols / bw * bb;
+    if ((rows * rb) % 16 != 0) return g;          // every copy a multiple of 16 bytes
+    const int nseg = (int)ceil_div(cols, SK_SEG);
+    g.ksegs = pow2ceil(nseg);
+    while ((g.gran * rb) % 16 != 0) g.gran *= 2;
+    const int64_t x_bytes = ceil_div(cols * 4, 128) * 128;
+    const int64_t budget = SK_CTA_SMEM - SK_HDR - SK_PART;
+    // rows per consumer warp: two (more independent work per warp), four for
+    // Q4_K (short rows), one if a stage would not fit three times
+    const int r_pref = fmt == QMV_Q4_K ? 4 : 2;
+    for (int R = r_pref; R >= 1; R >>= 1) {
+        const int T = (SK_NC / g.ksegs) * R;
+        if (T % g.gran != 0) continue;
+        const int64_t pitch = ceil_div(T * rb + 16, 128) * 128;
+        const bool in_ring = x_bytes <= pitch;
+        const int64_t S = std::min<int64_t>(SK_MAX_STAGES, (budget - (in_ring ? 0 : x_bytes)) / pitch);
+        if (S < (R > 1 ? 3 : 2)) continue;
+        g.R = R;
+        g.T = T;
+        g.S = (int)S;
+        g.pitch = pitch;
+        g.x_in_ring = in_ring ? 1 : 0;
+        g.x_off = in_ring ? 0 : S * pitch;
+        g.smem = (size_t)(128 + SK_HDR + SK_PART + S * pitch + (in_ring ? 0 : x_bytes));
+        g.ok = true;
+        return g;
+    }
+    return g;
+}
+
+int sk_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x, float *y, const SkGeom &g,
+              const DevInfo &di, cudaStream_t st)
+{
+    const int bw = block_weights(fmt), bb = block_bytes(fmt);
+    SkParams p{};
+    p.W = static_cast<const uint8_t *>(W);
+    p.x = x;
+    p.y = y;
+    p.rows = rows;
+    p.row_bytes = cols / bw * bb;
+    const int64_t units = ceil_div(rows, (int64_t)g.gran);
+    const int64_t ctas = std::max<int64_t>(1, std::min<int64_t>(di.sm_count, units));
+    p.units_q = units / ctas;
+    p.units_r = (int32_t)(units % ctas);
+    p.gran = g.gran;
+    p.cols = (int32_t)cols;
+    p.ksegs = g.ksegs;
+    p.seg_bytes = (int32_t)(SK_SEG / bw * bb);
+    p.tile_rows = g.T;
+    p.n_stage = g.S;
+    p.stage_pitch = (int32_t)g.pitch;
+    p.x_in_ring = g.x_in_ring;
+    p.x_off = (int32_t)g.x_off;
+    p.err = di.err;
+    p.debug_extra_tx = g_debug_extra_tx.load();
+    const bool pdl = g_pdl.load() != 0;
+    t_last_kernel = QMV_KERNEL_STREAM;
+    cudaError_t e;
+    switch (fmt) {
+    case QMV_Q8_0: e = launch_sk<FMT_Q8_0>(p, g.R, dim3((unsigned)ctas), g.smem, st, pdl); break;
+    case QMV_Q4_K: e = launch_sk<FMT_Q4_K>(p, g.R, dim3((unsigned)ctas), g.smem, st, pdl); break;
+    default: e = launch_sk<FMT_Q6_K>(p, g.R, dim3((unsigned)ctas), g.smem, st, pdl); break;
+    }
+    return e == cudaSuccess ? QMV_OK : cuda_fail(e);
+}
+
 // Several tokens of a Q8_0 or Q4_K matrix on the tensor-core kernel: one CTA of
 // TC_WARPS warps per SM, x in shared memory when it fits next to rings of at
 // least two stages, else read through L2.
@@ -623,6 +708,10 @@ int qmv_batched(int fmt, const void *W_blocks, int64_t rows, int64_t cols, const
     if ((rc = get_dev(di))) return rc;
     if (tc_preferred(fmt, rows, cols, n_tok) && tc_geom(fmt, cols, n_tok, di).ok)
         return tc_single(fmt, W_blocks, rows, cols, x, y, n_tok, di, reinterpret_cast<cudaStream_t>(stream));
+    if (n_tok == 1) {
+        const SkGeom g = sk_geom(fmt, rows, cols);
+        if (g.ok) return sk_single(fmt, W_blocks, rows, cols, x, y, g, di, reinterpret_cast<cudaStream_t>(stream));
+    }
     if (n_tok == 1 ? rw_preferred(fmt, rows, cols) : rw_mt_preferred(fmt, rows, cols, n_tok))
         return rw_single(fmt, W_blocks, rows, cols, x, y, n_tok, di, reinterpret_cast<cudaStream_t>(stream));
     Plan pl;

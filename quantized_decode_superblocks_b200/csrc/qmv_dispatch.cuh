@@ -7,6 +7,7 @@
 #include <mutex>
 
 #include "qmv_rw.cuh"
+#include "qmv_sk.cuh"
 #include "qmv_tc.cuh"
 
 namespace qmv {
@@ -216,6 +217,19 @@ cudaError_t launch_multi(const MultiParams &mp, const KernelChoice &kc, int grid
                          cudaStream_t stream)
 {
     return pick<FMT>(kc, MultiLaunch{mp, dim3((unsigned)grid), smem, stream, kc.pdl});
+}
+
+// The one-token streaming kernel, R rows per consumer warp.
+template <int FMT>
+cudaError_t launch_sk(const SkParams &p, int R, dim3 grid, size_t smem, cudaStream_t st, bool pdl)
+{
+    static SmemCfg c1, c2, c4;
+    switch (R) {
+    case 1: return launch_with(qmv_sk_kernel<FMT, 1>, c1, p, grid, smem, st, pdl, false, SK_THREADS);
+    case 2: return launch_with(qmv_sk_kernel<FMT, 2>, c2, p, grid, smem, st, pdl, false, SK_THREADS);
+    case 4: return launch_with(qmv_sk_kernel<FMT, 4>, c4, p, grid, smem, st, pdl, false, SK_THREADS);
+    default: return cudaErrorInvalidValue;
+    }
 }
 
 // The tensor-core several-token kernel (Q8_0): x in shared memory or through L2.

@@ -24,7 +24,7 @@ torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
 Q8_0, Q4_K, Q6_K = synth.Q8_0, synth.Q4_K, synth.Q6_K
-WR, GEN, TC = q.KERNEL_WARP_RING, q.KERNEL_GENERAL, q.KERNEL_TENSOR_CORE
+WR, GEN, TC, SK = q.KERNEL_WARP_RING, q.KERNEL_GENERAL, q.KERNEL_TENSOR_CORE, q.KERNEL_STREAM
 REL, ABS = 1e-4, 1e-6
 
 
@@ -105,9 +105,11 @@ def test_dequant_full_range_bit_exact(fmt, rows, cols):
 
 # (fmt, rows, cols, n_tok, kernel that must serve the call)
 PATHS = [
-    (Q8_0, 300, 2048, 1, WR), (Q4_K, 300, 2048, 1, WR), (Q6_K, 300, 2048, 1, WR),     # warp-ring, one K-chunk
-    (Q8_0, 70, 8192, 1, WR), (Q6_K, 40, 4096, 1, WR),                                  # warp-ring, K-chunked rows
-    (Q4_K, 50, 8192, 1, GEN), (Q8_0, 37, 96, 1, GEN),                                  # general, one token
+    (Q8_0, 300, 2048, 1, SK), (Q4_K, 300, 2048, 1, SK), (Q6_K, 300, 2048, 1, SK),     # streaming, one K-segment
+    (Q8_0, 70, 8192, 1, SK), (Q6_K, 40, 4096, 1, SK), (Q4_K, 50, 8192, 1, SK),        # streaming, K-split rows
+    (Q6_K, 24, 1792, 1, SK),                                                           # rows not 16-byte multiples
+    (Q8_0, 33, 12288, 1, WR), (Q6_K, 9, 10240, 1, WR),                                 # warp-ring, K-chunked rows
+    (Q4_K, 5, 12288, 1, GEN), (Q8_0, 37, 96, 1, GEN),                                  # general, one token
     (Q8_0, 300, 2048, 2, WR), (Q4_K, 300, 2048, 2, WR), (Q6_K, 300, 2048, 2, WR),     # warp-ring, two tokens
     (Q8_0, 300, 2048, 3, TC), (Q4_K, 300, 2048, 3, TC), (Q6_K, 300, 2048, 3, TC),     # tensor cores
     (Q8_0, 300, 2048, 8, TC), (Q4_K, 300, 2048, 8, TC), (Q6_K, 300, 2048, 8, TC),

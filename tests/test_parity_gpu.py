@@ -530,12 +530,12 @@ def test_moe_bad_expert_id_is_dropped_and_reported():
     assert np.array_equal(yh[1], np.zeros(rows, np.float32))
 
 
-@pytest.mark.parametrize("n_tok", [1, 8])
-def test_stage_wait_timeout_is_reported_and_the_gpu_stays_usable(n_tok):
+@pytest.mark.parametrize("n_tok,kernel", [(1, q.KERNEL_STREAM), (2, q.KERNEL_WARP_RING), (8, q.KERNEL_TENSOR_CORE)])
+def test_stage_wait_timeout_is_reported_and_the_gpu_stays_usable(n_tok, kernel):
     # the test hook makes every tile expect 16 bytes more than are copied
-    # (one token: the warp-ring kernel; eight: the tensor-core kernel): each
-    # stage wait runs out (about a second), the kernel records the timeout
-    # and finishes, and the context stays usable
+    # (one token: the streaming kernel; two: the warp-ring kernel; eight: the
+    # tensor-core kernel): each stage wait runs out (about a second), the
+    # kernel records the timeout and finishes, and the context stays usable
     fmt, rows, cols = Q8_0, 512, 2048
     W = synth.gen_blocks(fmt, rows, cols, 45, 0)
     x = synth.gen_x(n_tok, cols, 45, 1)
@@ -546,6 +546,7 @@ def test_stage_wait_timeout_is_reported_and_the_gpu_stays_usable(n_tok):
             q.qmv_f32(fmt, dev(W), rows, cols, dev(x), y)
         else:
             q.qmv_batched(fmt, dev(W), rows, cols, dev(x), y, n_tok)
+        assert q.qmv_debug_last_kernel() == kernel
         err = q.qmv_check()
     finally:
         q.lib().qmv_debug_short_copies(0)
