@@ -292,19 +292,25 @@ class Sweep:
                 self.launch(i, stream)
 
 
-def per_kind_durations(torch, sweep, stream, reps=20):
+KERNEL_NAMES = {1: "warp-ring kernel", 2: "general pipeline kernel", 3: "tensor-core kernel",
+                4: "streaming kernel"}
+
+
+def per_kind_durations(torch, q, sweep, stream, reps=20):
     """Average duration of each projection type's launch as it runs in the
     step: a CUDA graph of that type's 16 launches (in layer order, same launch
-    attributes), replayed and timed with CUDA events on the launch stream."""
-    out = {}
+    attributes), replayed and timed with CUDA events on the launch stream.
+    Also returns which library kernel serves each type."""
+    out, kernels = {}, {}
     layers = sweep_layers()
     for kind in dict.fromkeys(name for (_, _, name, _, _) in layers):
         idx = [i for i, (_, _, name, _, _) in enumerate(layers) if name == kind]
         g = capture(torch, lambda: [sweep.launch(i, stream) for i in idx], stream)
+        kernels[kind] = KERNEL_NAMES.get(q.qmv_debug_last_kernel(), "?")
         time_graph(torch, g, 3, stream)
         out[kind] = (time_graph(torch, g, reps, stream) / (reps * len(idx)), len(idx))
         del g
-    return out
+    return out, kernels
 
 
 # --------------------------------------------------------- per-config runs --
@@ -650,8 +656,10 @@ def main():
         dist.barrier(torch)
         sec = dist.max(torch, sec)
         # the dominant kernel: every launch of the step, event-timed on its stream
-        durs = per_kind_durations(torch, sweep, stream) if mode == "launches" else {
-            "chain": (time_graph(torch, graph, 20, stream) / 20, 1)}
+        if mode == "launches":
+            durs, kinds = per_kind_durations(torch, q, sweep, stream)
+        else:
+            durs, kinds = {"chain": (time_graph(torch, graph, 20, stream) / 20, 1)}, {}
         # end to end: pinned x -> device, the step's library calls, y -> pinned host
         e2e_reps = max(3, min(200, args.steps // 5))
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -707,7 +715,7 @@ def main():
     if mode == "launches":
         rows, cols = shapes[dom_name]
         dom_bytes = algo_bytes(Q8_0, rows, cols, args.n_tok)
-        dom_kernel = f"Q8_0 {dom_name} matvec {rows}x{cols} (warp-ring kernel), {dom_n} launches per step"
+        dom_kernel = f"Q8_0 {dom_name} matvec {rows}x{cols} ({kinds[dom_name]}), {dom_n} launches per step"
     else:
         dom_bytes = sweep.algo
         dom_kernel = "qmv_rw_kernel, chained: the whole step in one launch"

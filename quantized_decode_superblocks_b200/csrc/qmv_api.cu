@@ -441,37 +441,54 @@ constexpr int64_t SK_CTA_SMEM = 210 * 1024;
 
 struct SkGeom {
     bool ok = false;
-    int R = 0, T = 0, S = 0, ksegs = 1, gran = 1, x_in_ring = 0;
-    int64_t pitch = 0, x_off = 0;
+    int R = 0, T = 0, S = 0, ksegs = 1, x_in_ring = 0;
+    int64_t pitch = 0, rs_bytes = 0, x_off = 0;
     size_t smem = 0;
 };
 
-SkGeom sk_geom(int fmt, int64_t rows, int64_t cols)
+// K-segments per row: the smallest divisor of the twelve consumer warps that
+// covers nseg segments (0 if none does).
+int sk_ksegs(int64_t nseg)
+{
+    if (nseg < 1) return 0;
+    for (int d : {1, 2, 3, 4, 6, 12})
+        if (d >= nseg) return d;
+    return 0;
+}
+
+// Geometry of a streaming-kernel launch.  mode SK_PLAIN: rows x cols; SK_SWIGLU:
+// n_sel experts of inter rows x cols (gate and up); SK_GATHER: rows of n_sel
+// expert segments of cols columns each.
+SkGeom sk_geom(int fmt, int mode, int64_t rows, int64_t cols, int n_sel = 1, int64_t inter = 0)
 {
     SkGeom g;
     const int bw = block_weights(fmt), bb = block_bytes(fmt);
-    if (cols > (int64_t)SK_SEG * SK_MAX_KSEGS || (fmt == QMV_Q8_0 && cols % 64 != 0)) return g;
+    if (fmt == QMV_Q8_0 && cols % 64 != 0) return g;     // a Q8_0 lane slice is a 4-byte-aligned block pair
     const int64_t rb = cols / bw * bb;
-    if ((rows * rb) % 16 != 0) return g;          // every copy a multiple of 16 bytes
-    const int nseg = (int)ceil_div(cols, SK_SEG);
-    g.ksegs = pow2ceil(nseg);
-    while ((g.gran * rb) % 16 != 0) g.gran *= 2;
-    const int64_t x_bytes = ceil_div(cols * 4, 128) * 128;
+    // GATHER: one K-segment per routed expert, each expert row at most one segment long
+    const int64_t nseg = mode == SK_GATHER ? (cols <= SK_SEG ? n_sel : 0) : ceil_div(cols, SK_SEG);
+    g.ksegs = sk_ksegs(nseg);
+    if (g.ksegs == 0 || (mode == SK_GATHER && g.ksegs < n_sel)) return g;
+    if (mode != SK_SWIGLU && (rows * rb) % 16 != 0) return g;   // the last copy ends on a 16-byte boundary
+    // x staged in shared memory (GATHER: one 2048-column row per expert)
+    const int64_t x_bytes = mode == SK_GATHER ? (int64_t)g.ksegs * SK_SEG * 4 : ceil_div(cols * 4, 128) * 128;
+    if (x_bytes > SK_X_MAX_BYTES) return g;
     const int64_t budget = SK_CTA_SMEM - SK_HDR - SK_PART;
-    // rows per consumer warp: two (more independent work per warp), four for
-    // Q4_K (short rows), one if a stage would not fit three times
-    const int r_pref = fmt == QMV_Q4_K ? 4 : 2;
+    const int r_pref = mode == SK_PLAIN && fmt == QMV_Q4_K ? 4 : 2;
     for (int R = r_pref; R >= 1; R >>= 1) {
-        const int T = (SK_NC / g.ksegs) * R;
-        if (T % g.gran != 0) continue;
-        const int64_t pitch = ceil_div(T * rb + 16, 128) * 128;
+        if ((R * rb) % 16 != 0) continue;                 // every row slot's copies 16-byte aligned
+        if (mode == SK_SWIGLU && inter % R != 0) continue; // a row slot never straddles two experts
+        const int nrs = SK_NC / g.ksegs;
+        const int64_t rs_bytes = (mode == SK_SWIGLU ? 2 : mode == SK_GATHER ? g.ksegs : 1) * R * rb;
+        const int64_t pitch = ceil_div(nrs * rs_bytes + 16, 128) * 128;
         const bool in_ring = x_bytes <= pitch;
         const int64_t S = std::min<int64_t>(SK_MAX_STAGES, (budget - (in_ring ? 0 : x_bytes)) / pitch);
         if (S < (R > 1 ? 3 : 2)) continue;
         g.R = R;
-        g.T = T;
+        g.T = nrs * R;
         g.S = (int)S;
         g.pitch = pitch;
+        g.rs_bytes = rs_bytes;
         g.x_in_ring = in_ring ? 1 : 0;
         g.x_off = in_ring ? 0 : S * pitch;
         g.smem = (size_t)(128 + SK_HDR + SK_PART + S * pitch + (in_ring ? 0 : x_bytes));
@@ -481,27 +498,22 @@ SkGeom sk_geom(int fmt, int64_t rows, int64_t cols)
     return g;
 }
 
-int sk_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x, float *y, const SkGeom &g,
-              const DevInfo &di, cudaStream_t st)
+// Fills the geometry fields of p and launches; the caller set the mode's
+// pointers, rows, cols and row_bytes.
+int sk_launch(int fmt, int mode, SkParams &p, const SkGeom &g, const DevInfo &di, cudaStream_t st)
 {
     const int bw = block_weights(fmt), bb = block_bytes(fmt);
-    SkParams p{};
-    p.W = static_cast<const uint8_t *>(W);
-    p.x = x;
-    p.y = y;
-    p.rows = rows;
-    p.row_bytes = cols / bw * bb;
-    const int64_t units = ceil_div(rows, (int64_t)g.gran);
+    const int64_t units = ceil_div(p.rows, (int64_t)g.R);
     const int64_t ctas = std::max<int64_t>(1, std::min<int64_t>(di.sm_count, units));
     p.units_q = units / ctas;
     p.units_r = (int32_t)(units % ctas);
-    p.gran = g.gran;
-    p.cols = (int32_t)cols;
+    p.gran = g.R;
     p.ksegs = g.ksegs;
     p.seg_bytes = (int32_t)(SK_SEG / bw * bb);
     p.tile_rows = g.T;
     p.n_stage = g.S;
     p.stage_pitch = (int32_t)g.pitch;
+    p.rs_bytes = (int32_t)g.rs_bytes;
     p.x_in_ring = g.x_in_ring;
     p.x_off = (int32_t)g.x_off;
     p.err = di.err;
@@ -510,11 +522,25 @@ int sk_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x
     t_last_kernel = QMV_KERNEL_STREAM;
     cudaError_t e;
     switch (fmt) {
-    case QMV_Q8_0: e = launch_sk<FMT_Q8_0>(p, g.R, dim3((unsigned)ctas), g.smem, st, pdl); break;
-    case QMV_Q4_K: e = launch_sk<FMT_Q4_K>(p, g.R, dim3((unsigned)ctas), g.smem, st, pdl); break;
-    default: e = launch_sk<FMT_Q6_K>(p, g.R, dim3((unsigned)ctas), g.smem, st, pdl); break;
+    case QMV_Q8_0: e = launch_sk<FMT_Q8_0>(p, mode, g.R, dim3((unsigned)ctas), g.smem, st, pdl); break;
+    case QMV_Q4_K: e = launch_sk<FMT_Q4_K>(p, mode, g.R, dim3((unsigned)ctas), g.smem, st, pdl); break;
+    default: e = launch_sk<FMT_Q6_K>(p, mode, g.R, dim3((unsigned)ctas), g.smem, st, pdl); break;
     }
     return e == cudaSuccess ? QMV_OK : cuda_fail(e);
+}
+
+int sk_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x, float *y, const SkGeom &g,
+              const DevInfo &di, cudaStream_t st)
+{
+    SkParams p{};
+    p.W = static_cast<const uint8_t *>(W);
+    p.x = x;
+    p.y = y;
+    p.rows = rows;
+    p.cols = (int32_t)cols;
+    p.row_bytes = cols / block_weights(fmt) * block_bytes(fmt);
+    p.n_sel = 1;
+    return sk_launch(fmt, SK_PLAIN, p, g, di, st);
 }
 
 // Several tokens of a Q8_0 or Q4_K matrix on the tensor-core kernel: one CTA of
@@ -600,6 +626,69 @@ int tc_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x
                           : fmt == QMV_Q4_K ? launch_tc<FMT_Q4_K>(p, g.x_smem, dim3((unsigned)ctas), g.smem, st, pdl)
                                             : launch_tc<FMT_Q6_K>(p, g.x_smem, dim3((unsigned)ctas), g.smem, st, pdl);
     return e == cudaSuccess ? QMV_OK : cuda_fail(e);
+}
+
+// In-order one-token matvecs on the chained streaming kernel, up to
+// SKC_MAX_TASKS per cooperative launch (one CTA per SM).  Returns
+// QMV_ERR_SHAPE (nothing launched) when some task does not fit its layout.
+int skc_chain(int fmt, const qmv_task *tasks, int n_tasks, const DevInfo &di, cudaStream_t st)
+{
+    const int bw = block_weights(fmt), bb = block_bytes(fmt);
+    const int R = 2;
+    int64_t max_stage = 0, max_x = 0;
+    for (int t = 0; t < n_tasks; ++t) {
+        const qmv_task &k = tasks[t];
+        const int64_t rb = k.cols / bw * bb;
+        const int nk = sk_ksegs(ceil_div(k.cols, SK_SEG));
+        if (nk == 0 || (fmt == QMV_Q8_0 && k.cols % 64 != 0) || (R * rb) % 16 != 0 || (k.rows * rb) % 16 != 0 ||
+            k.rows > INT32_MAX)
+            return QMV_ERR_SHAPE;
+        max_stage = std::max<int64_t>(max_stage, (int64_t)(SK_NC / nk) * R * rb);
+        max_x = std::max<int64_t>(max_x, ceil_div(k.cols * 4, 128) * 128);
+    }
+    const int64_t pitch = ceil_div(max_stage + 16, 128) * 128;
+    const int64_t budget = SK_CTA_SMEM - SK_HDR - SK_PART - max_x;
+    const int64_t S = std::min<int64_t>(SK_MAX_STAGES, budget / pitch);
+    if (max_x > SK_X_MAX_BYTES || S < 2) return QMV_ERR_SHAPE;
+    static thread_local SkChainParams p;
+    const int64_t ctas = di.sm_count;
+    t_last_kernel = QMV_KERNEL_STREAM;
+    for (int t0 = 0; t0 < n_tasks; t0 += SKC_MAX_TASKS) {
+        const int n = std::min(SKC_MAX_TASKS, n_tasks - t0);
+        p.n_tasks = n;
+        p.n_stage = (int)S;
+        p.stage_pitch = (int32_t)pitch;
+        p.x_off = (int32_t)(S * pitch);
+        p.sync = di.sync;
+        p.err = di.err;
+        p.debug_extra_tx = g_debug_extra_tx.load();
+        for (int i = 0; i < n; ++i) {
+            const qmv_task &k = tasks[t0 + i];
+            SkTask &tk = p.t[i];
+            tk = SkTask{};
+            tk.W = static_cast<const uint8_t *>(k.W_blocks);
+            tk.x = k.x;
+            tk.y = k.y;
+            tk.rows = k.rows;
+            tk.row_bytes = k.cols / bw * bb;
+            const int64_t units = ceil_div(k.rows, (int64_t)R);
+            tk.units_q = units / ctas;
+            tk.units_r = (int32_t)(units % ctas);
+            tk.cols = (int32_t)k.cols;
+            tk.ksegs = sk_ksegs(ceil_div(k.cols, SK_SEG));
+            tk.seg_bytes = SK_SEG / bw * bb;
+            tk.tile_rows = (SK_NC / tk.ksegs) * R;
+        }
+        const size_t smem = (size_t)(128 + SK_HDR + SK_PART + S * pitch + max_x);
+        cudaError_t e;
+        switch (fmt) {
+        case QMV_Q8_0: e = launch_skc<FMT_Q8_0>(p, R, dim3((unsigned)ctas), smem, st); break;
+        case QMV_Q4_K: e = launch_skc<FMT_Q4_K>(p, R, dim3((unsigned)ctas), smem, st); break;
+        default: e = launch_skc<FMT_Q6_K>(p, R, dim3((unsigned)ctas), smem, st); break;
+        }
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return QMV_OK;
 }
 
 // In-order one-token matvecs of one format on the warp-ring kernel, up to
@@ -709,7 +798,7 @@ int qmv_batched(int fmt, const void *W_blocks, int64_t rows, int64_t cols, const
     if (tc_preferred(fmt, rows, cols, n_tok) && tc_geom(fmt, cols, n_tok, di).ok)
         return tc_single(fmt, W_blocks, rows, cols, x, y, n_tok, di, reinterpret_cast<cudaStream_t>(stream));
     if (n_tok == 1) {
-        const SkGeom g = sk_geom(fmt, rows, cols);
+        const SkGeom g = sk_geom(fmt, SK_PLAIN, rows, cols);
         if (g.ok) return sk_single(fmt, W_blocks, rows, cols, x, y, g, di, reinterpret_cast<cudaStream_t>(stream));
     }
     if (n_tok == 1 ? rw_preferred(fmt, rows, cols) : rw_mt_preferred(fmt, rows, cols, n_tok))
@@ -816,6 +905,8 @@ int qmv_chain(int fmt, const qmv_task *tasks, int n_tasks, qmv_stream_t stream)
     int rc = get_dev(di);
     if (rc) return rc;
     const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    rc = skc_chain(fmt, tasks, n_tasks, di, st);
+    if (rc != QMV_ERR_SHAPE) return rc;
     if (all) return rw_chain(fmt, tasks, n_tasks, di, st);
     // a shape the chained kernel does not take: one launch per task, in order
     for (int t = 0; t < n_tasks; ++t) {
@@ -911,6 +1002,39 @@ int moe_ffn(int fmt_gu, const void *gate_blocks, const void *up_blocks, int64_t 
     DevInfo di;
     if ((rc = get_dev(di))) return rc;
     const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+    const SkGeom ga = sk_geom(fmt_gu, SK_SWIGLU, (int64_t)n_sel * inter, hidden, n_sel, inter);
+    const SkGeom gb = sk_geom(fmt_down, SK_GATHER, hidden, inter, n_sel);
+    if (ga.ok && gb.ok && (int64_t)n_sel * inter <= INT32_MAX) {
+        // h_k = silu(G_k x) * (U_k x), then y = sum_k g_k D_k h_k, on the streaming kernel
+        SkParams a{};
+        a.W = static_cast<const uint8_t *>(gate_blocks);
+        a.W2 = static_cast<const uint8_t *>(up_blocks);
+        a.expert_stride = gu_stride_bytes;
+        a.ids = expert_ids;
+        a.n_expert = n_expert;
+        a.n_sel = n_sel;
+        a.inter = (int32_t)inter;
+        a.cols = (int32_t)hidden;
+        a.x = x;
+        a.y = h_scratch;
+        a.rows = (int64_t)n_sel * inter;
+        a.row_bytes = hidden / block_weights(fmt_gu) * block_bytes(fmt_gu);
+        if ((rc = sk_launch(fmt_gu, SK_SWIGLU, a, ga, di, st))) return rc;
+        SkParams b{};
+        b.W = static_cast<const uint8_t *>(down_blocks);
+        b.expert_stride = down_stride_bytes;
+        b.ids = expert_ids;
+        b.gw = g;
+        b.n_expert = n_expert;
+        b.n_sel = n_sel;
+        b.cols = (int32_t)inter;
+        b.x = h_scratch;
+        b.y = y;
+        b.rows = hidden;
+        b.row_bytes = inter / block_weights(fmt_down) * block_bytes(fmt_down);
+        return sk_launch(fmt_down, SK_GATHER, b, gb, di, st);
+    }
 
     // h_k = silu(G_k x) * (U_k x): two groups (gate, up) per routed expert
     Plan a;

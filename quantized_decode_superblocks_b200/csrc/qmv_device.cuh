@@ -189,6 +189,28 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
     }
 }
 
+// As mbar_wait_bounded, polling with the blocking try_wait and no suspend-time
+// hint: the thread sleeps until the phase completes or the system's time
+// window ends.  Measured faster than the hinted form for the streaming
+// kernel, whose consumer warps often wait on data in flight.
+__device__ __forceinline__ bool mbar_wait_bounded_block(uint32_t bar, uint32_t parity)
+{
+    auto poll = [&]() {
+        uint32_t ok;
+        asm volatile("{\n\t.reg .pred p;\n\t"
+                     "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}"
+                     : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+        return ok != 0;
+    };
+    if (poll()) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (poll()) return true;
+        if ((i & 15u) == 0u && global_timer_ns() - t0 > 1000000000ull) return false;
+    }
+}
+
 // One 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
 // dst, src 16-byte aligned, bytes a multiple of 16.  Local memory only.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)

@@ -219,15 +219,43 @@ cudaError_t launch_multi(const MultiParams &mp, const KernelChoice &kc, int grid
     return pick<FMT>(kc, MultiLaunch{mp, dim3((unsigned)grid), smem, stream, kc.pdl});
 }
 
-// The one-token streaming kernel, R rows per consumer warp.
-template <int FMT>
-cudaError_t launch_sk(const SkParams &p, int R, dim3 grid, size_t smem, cudaStream_t st, bool pdl)
+// The one-token streaming kernel: form (plain, SwiGLU, gathered experts) and
+// rows per consumer warp.
+template <int FMT, int MODE>
+static cudaError_t launch_sk_mode(const SkParams &p, int R, dim3 grid, size_t smem, cudaStream_t st, bool pdl)
 {
     static SmemCfg c1, c2, c4;
     switch (R) {
-    case 1: return launch_with(qmv_sk_kernel<FMT, 1>, c1, p, grid, smem, st, pdl, false, SK_THREADS);
-    case 2: return launch_with(qmv_sk_kernel<FMT, 2>, c2, p, grid, smem, st, pdl, false, SK_THREADS);
-    case 4: return launch_with(qmv_sk_kernel<FMT, 4>, c4, p, grid, smem, st, pdl, false, SK_THREADS);
+    case 1: return launch_with(qmv_sk_kernel<FMT, 1, MODE>, c1, p, grid, smem, st, pdl, false, SK_THREADS);
+    case 2: return launch_with(qmv_sk_kernel<FMT, 2, MODE>, c2, p, grid, smem, st, pdl, false, SK_THREADS);
+    case 4:
+        if constexpr (MODE == SK_PLAIN)
+            return launch_with(qmv_sk_kernel<FMT, 4, MODE>, c4, p, grid, smem, st, pdl, false, SK_THREADS);
+        return cudaErrorInvalidValue;
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int FMT>
+cudaError_t launch_sk(const SkParams &p, int mode, int R, dim3 grid, size_t smem, cudaStream_t st, bool pdl)
+{
+    switch (mode) {
+    case SK_PLAIN: return launch_sk_mode<FMT, SK_PLAIN>(p, R, grid, smem, st, pdl);
+    case SK_SWIGLU: return launch_sk_mode<FMT, SK_SWIGLU>(p, R, grid, smem, st, pdl);
+    case SK_GATHER: return launch_sk_mode<FMT, SK_GATHER>(p, R, grid, smem, st, pdl);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+// The chained streaming kernel (cooperative: one CTA per SM, all resident).
+template <int FMT>
+cudaError_t launch_skc(const SkChainParams &p, int R, dim3 grid, size_t smem, cudaStream_t st)
+{
+    static SmemCfg c1, c2, c4;
+    switch (R) {
+    case 1: return launch_with(qmv_skc_kernel<FMT, 1>, c1, p, grid, smem, st, false, true, SK_THREADS);
+    case 2: return launch_with(qmv_skc_kernel<FMT, 2>, c2, p, grid, smem, st, false, true, SK_THREADS);
+    case 4: return launch_with(qmv_skc_kernel<FMT, 4>, c4, p, grid, smem, st, false, true, SK_THREADS);
     default: return cudaErrorInvalidValue;
     }
 }

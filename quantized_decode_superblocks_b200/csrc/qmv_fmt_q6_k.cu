@@ -9,5 +9,6 @@ template cudaError_t launch_rw<FMT_Q6_K, RW_MAX_TASKS>(const RwParams &, int, di
 template cudaError_t rw_occupancy<FMT_Q6_K>(int, size_t, int *);
 template cudaError_t launch_rw_mt<FMT_Q6_K>(const RwParams1 &, int, int, dim3, size_t, cudaStream_t, bool);
 template cudaError_t launch_tc<FMT_Q6_K>(const TcParams &, bool, dim3, size_t, cudaStream_t, bool);
-template cudaError_t launch_sk<FMT_Q6_K>(const SkParams &, int, dim3, size_t, cudaStream_t, bool);
+template cudaError_t launch_sk<FMT_Q6_K>(const SkParams &, int, int, dim3, size_t, cudaStream_t, bool);
+template cudaError_t launch_skc<FMT_Q6_K>(const SkChainParams &, int, dim3, size_t, cudaStream_t);
 }  // namespace qmv

@@ -9,5 +9,6 @@ template cudaError_t launch_rw<FMT_Q8_0, RW_MAX_TASKS>(const RwParams &, int, di
 template cudaError_t rw_occupancy<FMT_Q8_0>(int, size_t, int *);
 template cudaError_t launch_rw_mt<FMT_Q8_0>(const RwParams1 &, int, int, dim3, size_t, cudaStream_t, bool);
 template cudaError_t launch_tc<FMT_Q8_0>(const TcParams &, bool, dim3, size_t, cudaStream_t, bool);
-template cudaError_t launch_sk<FMT_Q8_0>(const SkParams &, int, dim3, size_t, cudaStream_t, bool);
+template cudaError_t launch_sk<FMT_Q8_0>(const SkParams &, int, int, dim3, size_t, cudaStream_t, bool);
+template cudaError_t launch_skc<FMT_Q8_0>(const SkChainParams &, int, dim3, size_t, cudaStream_t);
 }  // namespace qmv

@@ -117,6 +117,18 @@ __device__ __forceinline__ void fence_proxy_async_smem()
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Slices (64 weights for the K-quants, 32 for Q8_0) of one K-segment: a row's
+// n1 slices split over wpr warps.  For the K-quants a segment starts on a
+// superblock boundary (a multiple of 4 slices), so that slice s and lane
+// (s mod 32) agree on which quarter of the superblock they hold: the Q4_K
+// scale selectors are built from the lane.
+template <int FMT>
+__device__ __forceinline__ int seg_slices(int n1, int wpr)
+{
+    const int P = (n1 + wpr - 1) / wpr;
+    return FMT == FMT_Q8_0 ? P : (P + 3) & ~3;
+}
+
 // One-token slice dot product (factored form) of one row at rowp.
 template <int FMT, bool XSUM_INLINE, class XP>
 __device__ __forceinline__ float dot1(uint32_t rowp, int s, const Q4kSel &sel, XP &&xp, float xsa, float xsb)
@@ -276,7 +288,7 @@ __device__ __forceinline__ void qmv_pipeline_body(const Params &p, const int cta
     float xsa[XREG ? SPL1 : 1], xsb[XREG ? SPL1 : 1];
     if (XREG) {
         const int n1 = p.cols / Slice1<FMT>::W;
-        const int P = (n1 + p.wpr - 1) / p.wpr;
+        const int P = seg_slices<FMT>(n1, p.wpr);
 #pragma unroll
         for (int q = 0; q < SPL1; ++q) {
             const int j = lane + 32 * q;
@@ -312,8 +324,8 @@ __device__ __forceinline__ void qmv_pipeline_body(const Params &p, const int cta
     // slice geometry of a full and of the last K-chunk
     const int n1_full = p.chunk_cols / Slice1<FMT>::W;
     const int n1_last = p.last_chunk_cols / Slice1<FMT>::W;
-    const int P_full = (n1_full + p.wpr - 1) / p.wpr;
-    const int P_last = (n1_last + p.wpr - 1) / p.wpr;
+    const int P_full = seg_slices<FMT>(n1_full, p.wpr);
+    const int P_last = seg_slices<FMT>(n1_last, p.wpr);
 
     // tile i: stage slot, ring round, K-chunk, first row, row-group parity --
     // advanced incrementally (no divisions in the loop); f_*: the tile i + S

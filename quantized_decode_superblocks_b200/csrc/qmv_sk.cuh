@@ -1,5 +1,5 @@
 // qmv_sk.cuh -- the one-token streaming matvec: one producer warp, twelve
-// consumer warps, whole multi-row stages.
+// consumer warps, multi-row stages.
 //
 // A batch-1 decode matvec streams every weight once (BebeLM：纯Rust实现的端侧
 // 大模型推理引擎, §性能表现: decode is bound by memory bandwidth).  On B200 the
@@ -7,27 +7,36 @@
 // leaves about six issue slots per weight at full issue rate; the decode
 // itself takes three (Q8_0), so everything around it has to be nearly free.
 // This kernel is built for that:
-//   * each CTA owns one contiguous range of rows; its producer warp (one
-//     elected lane) moves T whole rows at a time -- one contiguous 1-D bulk
-//     async copy of T x row_bytes -- into a ring of S shared-memory stages,
-//     completing on the stage's "full" mbarrier, and refills a stage once all
-//     consumer warps have arrived on its "empty" mbarrier;
-//   * consumer warp w takes R rows of every stage (of its K-segment when rows
-//     are longer than 2048 columns): wait, decode, release, reduce -- no
-//     copies, cursors or 64-bit bookkeeping in the consumer loop;
+//   * each CTA owns one contiguous range of output rows; its producer warp
+//     (one elected lane) fills a ring of S shared-memory stages.  A stage
+//     holds T rows as nrs "row slots" of R rows; each row slot is filled by
+//     1-D bulk async copies of whole rows that complete on the row slot's own
+//     "full" mbarrier, so a consumer warp waits only for its own rows.  A
+//     stage is refilled once all twelve consumer warps have arrived on its
+//     "empty" mbarrier;
+//   * consumer warp w = (row slot, K-segment) takes its R rows of every stage
+//     (its 2048-column K-segment when rows are longer): wait, decode, release,
+//     reduce -- no copies, cursors or 64-bit bookkeeping in the consumer loop;
 //   * lane l's x values for its 64 columns of the K-segment sit in registers
 //     for the whole kernel (staged once per CTA through shared memory);
-//   * a multi-row butterfly reduces the warp's R partial sums; rows split over
+//   * a multi-row butterfly reduces the warp's partial sums; rows split over
 //     K-segments add their warps' partials in shared memory in a fixed order
 //     (deterministic, no atomics);
 //   * one CTA of 13 warps per SM (at most four warps per SM sub-partition, so
-//     128 registers a thread: x and R rows of decode stay in registers) with a
-//     ring of ~200 KB; with programmatic dependent launch the next matvec's
-//     CTA takes the SM as soon as this one's CTA exits and streams its first
-//     stages while the rest of this kernel finishes.
-// Every wait is bounded (about a second): a timeout records QMV_DEVERR_TIMEOUT,
-// the warp stops decoding but keeps releasing stages, and the producer drains
-// its copies before the CTA exits (QMV_DEVERR_DRAIN if that wait runs out too).
+//     128 registers a thread) with a ring of up to ~200 KB; with programmatic
+//     dependent launch the next kernel's CTA takes the SM as soon as this
+//     one's CTA exits and streams its first stages while the rest finishes.
+// Three forms share the body (BebeLM page, §核心算子, MoE前馈网络):
+//   SK_PLAIN   y = W x (a matrix, or a row-concatenated fused projection);
+//   SK_SWIGLU  h[k][r] = silu(G_{ids[k]} x)[r] * (U_{ids[k]} x)[r]: a row slot
+//              holds R gate rows and the same R up rows of one routed expert;
+//   SK_GATHER  y[r] = sum_k g[k] (D_{ids[k]} h_k)[r]: K-segment k of a row is
+//              row r of expert ids[k]'s matrix, weighted and summed in k order.
+// An expert id outside [0, n_expert) copies nothing, contributes zero and
+// records QMV_DEVERR_EXPERT_ID.  Every wait is bounded (about a second): a
+// timeout records QMV_DEVERR_TIMEOUT, the warp stops decoding but keeps
+// releasing stages, and the producer drains its copies before the CTA exits
+// (QMV_DEVERR_DRAIN if that wait runs out too).
 #pragma once
 
 #include "qmv_rw.cuh"
@@ -38,55 +47,126 @@ constexpr int SK_NC = 12;                     // consumer warps
 constexpr int SK_THREADS = (SK_NC + 1) * 32;  // + one producer warp
 constexpr int SK_MAX_STAGES = 8;
 constexpr int SK_SEG = 2048;                  // columns of one K-segment: 64 per lane
-constexpr int SK_MAX_KSEGS = 4;               // rows up to 8192 columns (ksegs divides SK_NC)
-constexpr int SK_HDR = 256;                   // mbarriers: full[8], empty[8], x_done
-constexpr int SK_PART = 2 * SK_NC * 4 * 4;    // K-segment partials (SK_NC * R <= 48 floats), double-buffered
+constexpr int SK_MAX_KSEGS = SK_NC;           // K-segments per row: a divisor of SK_NC
+constexpr int SK_MAX_RS = SK_NC;              // row slots per stage
+// header: full[stage][row slot], empty[stage], x_done, abort flag, segment weights
+constexpr int SK_FULL_OFF = 0;
+constexpr int SK_EMPTY_OFF = 8 * SK_MAX_STAGES * SK_MAX_RS;           // 768
+constexpr int SK_XDONE_OFF = SK_EMPTY_OFF + 8 * SK_MAX_STAGES;        // 832
+constexpr int SK_ABORT_OFF = SK_XDONE_OFF + 8;                        // 840
+constexpr int SK_WSEG_OFF = 896;                                      // float[SK_MAX_KSEGS]
+constexpr int SK_HDR = 1024;
+constexpr int SK_PART = 2 * SK_NC * 4 * 2 * 4;   // partials [row][group][segment] <= NC*R*G floats, double-buffered
+
+enum { SK_PLAIN = 0, SK_SWIGLU = 1, SK_GATHER = 2 };
+
+// SK_PLAIN: 1 = one bulk copy and one "full" mbarrier per stage (all row slots
+// wait for the whole stage), 0 = one of each per row slot.
+#ifndef QMV_SK_STAGE_BARRIER
+#define QMV_SK_STAGE_BARRIER 1      // measured faster on B200 (one copy per stage)
+#endif
 
 struct SkParams {
-    const uint8_t *W;
-    const float *x;          // [cols]
+    const uint8_t *W;        // PLAIN: the matrix; SWIGLU: gate matrices; GATHER: down matrices
+    const uint8_t *W2;       // SWIGLU: up matrices
+    int64_t expert_stride;   // SWIGLU / GATHER: bytes from one expert's matrix to the next
+    const int32_t *ids;      // SWIGLU / GATHER: routed expert ids [n_sel] (device)
+    const float *gw;         // GATHER: expert weights [n_sel] (device)
+    int32_t n_expert;
+    int32_t n_sel;
+    int32_t inter;           // SWIGLU: rows per expert (output row v = k * inter + r)
+    int32_t cols;            // columns of one matrix row (GATHER: of one expert's row = one K-segment)
+    const float *x;          // PLAIN / SWIGLU: x [cols]; GATHER: h [n_sel][cols]
     float *y;                // [rows]
-    int64_t rows;
-    int64_t row_bytes;
+    int64_t rows;            // output rows (SWIGLU: n_sel * inter)
+    int64_t row_bytes;       // bytes of one matrix row (GATHER: of one expert's row)
     int64_t units_q;         // CTA c owns units_q + (c < units_r) units of `gran` rows
     int32_t units_r;
-    int32_t gran;            // rows per unit: gran * row_bytes is a multiple of 16 bytes
-    int32_t cols;
-    int32_t ksegs;           // consumer warps per row (1, 2 or 4)
-    int32_t seg_bytes;       // bytes of one 2048-column K-segment of a row
+    int32_t gran;            // rows per unit: a multiple of R
+    int32_t ksegs;           // consumer warps per row (a divisor of SK_NC)
+    int32_t seg_bytes;       // PLAIN / SWIGLU: bytes of one 2048-column K-segment of a row
     int32_t tile_rows;       // T = (SK_NC / ksegs) * R rows per stage
     int32_t n_stage;         // S
-    int32_t stage_pitch;     // bytes per stage slot (multiple of 128, >= T * row_bytes + 16)
+    int32_t stage_pitch;     // bytes per stage slot (multiple of 128, >= a stage + 16)
+    int32_t rs_bytes;        // bytes of one row slot's region in a stage
     int32_t x_in_ring;       // 1: x is staged in ring slot S-1 before its first fill
     int32_t x_off;           // else: byte offset of the x area from the ring start
     int *err;
-    uint32_t debug_extra_tx; // test hook: bytes expected per stage beyond those copied (0 in use)
+    uint32_t debug_extra_tx; // test hook: bytes expected per row slot beyond those copied (0 in use)
 };
 
-// x value layout in registers for one lane's 64-column slice of a K-segment:
-// the same slice geometry and pairing as the warp-ring kernel.
-template <int FMT>
-__device__ __forceinline__ void sk_load_x(uint32_t xs, int seg, int ncols, int lane, float2 (&xr)[16][2],
-                                          float &xsa, float &xsb)
+__device__ __forceinline__ bool sk_valid(const SkParams &p, int k)
 {
-    rw_load_x_smem<FMT>(xs, seg, ncols, lane, xr, xsa, xsb);
+    const int e = p.ids[k];
+    return e >= 0 && e < p.n_expert;
 }
 
-template <int FMT, int R>
+// Starts moving `bytes` (a multiple of 16, 16-byte aligned) of global memory
+// into L2 without waiting.  Used on x before griddepcontrol.wait: if the
+// previous kernel writes x afterwards, L2 holds its writes all the same.
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(src), "r"(bytes) : "memory");
+}
+
+constexpr int SK_X_MAX_BYTES = 96 * 1024;    // largest x staged in shared memory (24576 floats)
+
+// Copies x into the swizzled x area of shared memory (float4 d at
+// 16 * rw_xswz(d)): n_rows rows of nr float4, row k from src + k * src_row
+// floats to float4 k * 512 of the area (SK_SEG columns per row).  A thread
+// issues up to eight loads before its first store, so staging up to 12288
+// floats costs one memory round trip (the loads queue behind the weight
+// copies in flight).
+// COHERENT: read through L2 only (x may have been written earlier in the same
+// launch by another SM).
+template <bool COHERENT>
+__device__ __forceinline__ void sk_stage_x(uint32_t xs, const float *src, int n_rows, int nr, int64_t src_row)
+{
+    constexpr int B = 8;                          // loads in flight per thread and pass
+    const int n = n_rows == 1 ? nr : n_rows * (SK_SEG / 4);
+#pragma unroll 1
+    for (int base = 0; base < n; base += B * SK_NC * 32) {
+        float4 v[B];
+#pragma unroll
+        for (int j = 0; j < B; ++j) {
+            const int d = base + (int)threadIdx.x + j * SK_NC * 32;
+            const int k = n_rows == 1 ? 0 : d >> 9, c = n_rows == 1 ? d : d & 511;
+            if (d < n && c < nr) {
+                const float4 *a = reinterpret_cast<const float4 *>(src + (int64_t)k * src_row) + c;
+                v[j] = COHERENT ? __ldcg(a) : __ldg(a);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < B; ++j) {
+            const int d = base + (int)threadIdx.x + j * SK_NC * 32;
+            const int c = n_rows == 1 ? d : d & 511;
+            if (d < n && c < nr) sts_f4(xs + 16u * rw_xswz((uint32_t)d), v[j]);
+        }
+    }
+}
+
+template <int FMT, int R, int MODE>
 __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_constant__ SkParams p)
 {
     static_assert(R == 1 || R == 2 || R == 4, "rows per consumer warp");
+    constexpr int G = MODE == SK_SWIGLU ? 2 : 1;      // matrices per row slot (gate and up)
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = (int)threadIdx.x >> 5, lane = (int)threadIdx.x & 31;
     const uint32_t sraw = smem_addr(smem);
     const uint32_t sbase = (sraw + 127u) & ~127u;          // the launch adds 128 spare bytes
-    const uint32_t full0 = sbase, empty0 = sbase + 8u * SK_MAX_STAGES, xdone = sbase + 16u * SK_MAX_STAGES;
-    volatile int *const abort_flag = reinterpret_cast<volatile int *>(smem + (sbase - sraw) + 16 * SK_MAX_STAGES + 8);
+    uint8_t *const sgen = smem + (sbase - sraw);
+    const uint32_t full0 = sbase + SK_FULL_OFF, empty0 = sbase + SK_EMPTY_OFF, xdone = sbase + SK_XDONE_OFF;
+    volatile int *const abort_flag = reinterpret_cast<volatile int *>(sgen + SK_ABORT_OFF);
+    float *const wseg = reinterpret_cast<float *>(sgen + SK_WSEG_OFF);
     const uint32_t part0 = sbase + (uint32_t)SK_HDR;
     const uint32_t ring = part0 + (uint32_t)SK_PART;
     const int S = p.n_stage;
+    const int nrs = SK_NC / p.ksegs;
     const uint32_t pitch = (uint32_t)p.stage_pitch;
     const uint32_t xs = p.x_in_ring ? ring + (uint32_t)(S - 1) * pitch : ring + (uint32_t)p.x_off;
+    // one "full" mbarrier per stage (plain copies of whole stages) or per row slot
+    constexpr bool STAGE_BAR = MODE == SK_PLAIN && QMV_SK_STAGE_BARRIER;
+    auto full_bar = [&](int s, int r) { return full0 + 8u * (uint32_t)(s * SK_MAX_RS + (STAGE_BAR ? 0 : r)); };
 
     // this CTA's rows
     const int c = (int)blockIdx.x;
@@ -98,7 +178,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_cons
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(full0 + 8u * (uint32_t)s, 1);
+            for (int r = 0; r < nrs; ++r) mbar_init(full_bar(s, r), 1);
             mbar_init(empty0 + 8u * (uint32_t)s, SK_NC);
         }
         mbar_init(xdone, SK_NC);
@@ -110,37 +190,77 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_cons
 
     if (warp == SK_NC) {
         // ------------------------------------------------------ producer --
-        // Weights do not depend on earlier kernels: no griddepcontrol.wait here.
-        if (lane == 0) {
-            const uint64_t row_bytes = (uint64_t)p.row_bytes;
-            const uint8_t *src = p.W + (uint64_t)r_begin * row_bytes;
-            const uint64_t stage_bytes = (uint64_t)T * row_bytes;
-            int issued = 0;
-            bool ok = true;
-            for (int i = 0; i < n_st && ok; ++i) {
-                const int slot = i % S;
-                const int round = i / S;
-                if (round > 0) ok = mbar_wait_bounded(empty0 + 8u * (uint32_t)slot, (uint32_t)((round - 1) & 1));
-                else if (p.x_in_ring && slot == S - 1) ok = mbar_wait_bounded(xdone, 0u);
-                if (!ok) {
-                    atomicOr(p.err, DEVERR_TIMEOUT);
-                    break;
-                }
-                if (*abort_flag) break;           // a consumer timed out: stop re-arming stages
-                const int64_t r0 = r_begin + (int64_t)i * T;
-                const uint32_t bytes = (uint32_t)(min((int64_t)T, r_end - r0) * p.row_bytes);
-                const uint32_t full = full0 + 8u * (uint32_t)slot;
-                // the slot was last read (and x, in slot S-1, written) through the generic proxy
-                if (round > 0 || (p.x_in_ring && slot == S - 1)) fence_proxy_async_smem();
-                mbar_arrive_expect_tx(full, bytes + p.debug_extra_tx);
-                bulk_g2s(ring + (uint32_t)slot * pitch, src, bytes, full);
-                src += stage_bytes;
-                ++issued;
+        if (lane != 0) return;
+        // plain weights do not depend on earlier kernels; routed experts do (ids)
+        if (MODE != SK_PLAIN) pdl_wait();
+        const uint64_t rb = (uint64_t)p.row_bytes;
+        int issued = 0;
+        bool ok = true;
+        for (int i = 0; i < n_st && ok; ++i) {
+            const int slot = i % S;
+            const int round = i / S;
+            if (round > 0) ok = mbar_wait_bounded_block(empty0 + 8u * (uint32_t)slot, (uint32_t)((round - 1) & 1));
+            else if (p.x_in_ring && slot == S - 1) ok = mbar_wait_bounded_block(xdone, 0u);
+            if (!ok) {
+                atomicOr(p.err, DEVERR_TIMEOUT);
+                break;
             }
-            // let every copy land before the CTA can exit
-            for (int i = max(0, issued - S); i < issued; ++i) {
-                if (!mbar_wait_bounded(full0 + 8u * (uint32_t)(i % S), (uint32_t)((i / S) & 1))) {
+            if (*abort_flag) break;           // a consumer timed out: stop re-arming stages
+            // the slot was last read (and x, in slot S-1, written) through the generic proxy
+            if (round > 0 || (p.x_in_ring && slot == S - 1)) fence_proxy_async_smem();
+            const int64_t r0 = r_begin + (int64_t)i * T;
+            const int tr = (int)min((int64_t)T, r_end - r0);
+            const uint32_t st = ring + (uint32_t)slot * pitch;
+            if (STAGE_BAR) {
+                const uint32_t bytes = (uint32_t)tr * (uint32_t)rb;
+                mbar_arrive_expect_tx(full_bar(slot, 0), bytes + p.debug_extra_tx);
+                bulk_g2s(st, p.W + (uint64_t)r0 * rb, bytes, full_bar(slot, 0));
+            }
+            for (int rs = 0; rs < nrs && rs * R < tr && !STAGE_BAR; ++rs) {
+                const int ra = min(R, tr - rs * R);
+                const int64_t v0 = r0 + rs * R;
+                const uint32_t full = full_bar(slot, rs);
+                const uint32_t dst = st + (uint32_t)(rs * p.rs_bytes);
+                const uint32_t bytes = (uint32_t)ra * (uint32_t)rb;
+                if (MODE == SK_PLAIN) {
+                    mbar_arrive_expect_tx(full, bytes + p.debug_extra_tx);
+                    bulk_g2s(dst, p.W + (uint64_t)v0 * rb, bytes, full);
+                } else if (MODE == SK_SWIGLU) {
+                    const int k = (int)(v0 / p.inter);
+                    const int64_t r = v0 - (int64_t)k * p.inter;
+                    const int e = p.ids[k];
+                    const bool valid = e >= 0 && e < p.n_expert;
+                    mbar_arrive_expect_tx(full, (valid ? 2u * bytes : 0u) + p.debug_extra_tx);
+                    if (valid) {
+                        const uint64_t off = (uint64_t)e * (uint64_t)p.expert_stride + (uint64_t)r * rb;
+                        bulk_g2s(dst, p.W + off, bytes, full);
+                        bulk_g2s(dst + (uint32_t)R * (uint32_t)rb, p.W2 + off, bytes, full);
+                    }
+                } else {
+                    const int n_seg = min(p.n_sel, p.ksegs);   // a row slot holds ksegs segments
+                    uint32_t total = 0;
+                    for (int k = 0; k < n_seg; ++k)
+                        if (sk_valid(p, k)) total += bytes;
+                    mbar_arrive_expect_tx(full, total + p.debug_extra_tx);
+                    for (int k = 0; k < n_seg; ++k) {
+                        const int e = p.ids[k];
+                        if (e < 0 || e >= p.n_expert) continue;
+                        bulk_g2s(dst + (uint32_t)(k * R) * (uint32_t)rb,
+                                 p.W + (uint64_t)e * (uint64_t)p.expert_stride + (uint64_t)v0 * rb, bytes, full);
+                    }
+                }
+            }
+            ++issued;
+        }
+        // let every copy land before the CTA can exit
+        bool drained = true;
+        for (int i = max(0, issued - S); i < issued && drained; ++i) {
+            const int64_t r0 = r_begin + (int64_t)i * T;
+            const int tr = (int)min((int64_t)T, r_end - r0);
+            for (int rs = 0; rs < (STAGE_BAR ? 1 : nrs) && rs * R < tr; ++rs) {
+                if (!mbar_wait_bounded_block(full_bar(i % S, rs), (uint32_t)((i / S) & 1))) {
                     atomicOr(p.err, DEVERR_DRAIN);
+                    drained = false;
                     break;
                 }
             }
@@ -149,85 +269,347 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_cons
     }
 
     // -------------------------------------------------------- consumers --
-    pdl_wait();                                    // x is the previous kernel's output
-    {
-        const float4 *src = reinterpret_cast<const float4 *>(p.x);
-        for (int f = (int)threadIdx.x; f < (p.cols >> 2); f += SK_NC * 32)
-            sts_f4(xs + 16u * rw_xswz((uint32_t)f), __ldg(src + f));
+    const int n_xrow = MODE == SK_GATHER ? min(p.n_sel, p.ksegs) : 1;
+    if (threadIdx.x == 0) prefetch_l2(p.x, (uint32_t)(n_xrow * p.cols * 4));
+    pdl_wait();                                    // x, h, ids and weights come from earlier kernels
+    if (MODE == SK_GATHER) {
+        // h_k at float offset k * SK_SEG of the x area (a K-segment per expert)
+        sk_stage_x<false>(xs, p.x, n_xrow, p.cols >> 2, p.cols);
+        if ((int)threadIdx.x < SK_MAX_KSEGS) {
+            const int k = (int)threadIdx.x;
+            float w = 0.f;
+            if (k < p.n_sel) {
+                if (sk_valid(p, k)) w = p.gw[k];
+                else atomicOr(p.err, DEVERR_EXPERT_ID);
+            }
+            wseg[k] = w;
+        }
+    } else {
+        sk_stage_x<false>(xs, p.x, 1, p.cols >> 2, 0);
+        if (MODE == SK_SWIGLU && (int)threadIdx.x < p.n_sel && !sk_valid(p, (int)threadIdx.x))
+            atomicOr(p.err, DEVERR_EXPERT_ID);
     }
     named_bar_sync(1, SK_NC * 32);
     const int ks = warp % p.ksegs, rs = warp / p.ksegs;
-    const int seg_cols = min(SK_SEG, p.cols - ks * SK_SEG);
+    int seg_cols;
+    if (MODE == SK_GATHER) seg_cols = ks < p.n_sel && sk_valid(p, ks) ? p.cols : 0;
+    else seg_cols = min(SK_SEG, p.cols - ks * SK_SEG);
     float2 xr[16][2];
     float xsa = 0.f, xsb = 0.f;
-    sk_load_x<FMT>(xs, ks, seg_cols, lane, xr, xsa, xsb);
+    rw_load_x_smem<FMT>(xs, ks, seg_cols, lane, xr, xsa, xsb);
     __syncwarp();
     if (lane == 0) mbar_arrive(xdone);             // the x area may now become ring slot S-1
 
     const bool have = 64 * (lane + 1) <= seg_cols;
     const Q4kSel sel = q4k_sel(lane & 3);
-    const uint32_t row_bytes = (uint32_t)p.row_bytes;
-    // this lane's slice within a row of a stage
-    uint32_t slice = (uint32_t)ks * (uint32_t)p.seg_bytes;
+    const uint32_t rb = (uint32_t)p.row_bytes;
+    // this lane's slice within the warp's part of a row slot
+    uint32_t slice = (uint32_t)rs * (uint32_t)p.rs_bytes;
+    slice += (uint32_t)ks * (MODE == SK_GATHER ? (uint32_t)R * rb : (uint32_t)p.seg_bytes);
     if (FMT == FMT_Q8_0) slice += 68u * (uint32_t)lane;
     else if (FMT == FMT_Q4_K) slice += 144u * (uint32_t)(lane >> 2);
     else slice += 210u * (uint32_t)(lane >> 2);
     const int q6h = (lane >> 1) & 1, q6l = 16 * (lane & 1);
-    constexpr int SH = 5 - Log2<R>::v;
+    constexpr int V = G * R;
+    constexpr int SH = 5 - Log2<V>::v;
     const bool leader = (lane & ((1 << SH) - 1)) == 0;
-    const int kl = lane >> SH;                     // row (of the warp's R) a leader holds after the butterfly
+    const int vi = lane >> SH;                     // value (group * R + row) a leader holds after the butterfly
+    const int vg = vi / R, vk = vi % R;
     auto xp = [&](int gq, float2 &x02, float2 &x13) {
         x02 = xr[gq][0];
         x13 = xr[gq][1];
     };
 
     bool dead = false;
+    int slot = 0;
+    uint32_t phase = 0, st = ring;
+    int64_t r0 = r_begin;
     for (int i = 0; i < n_st; ++i) {
-        const int slot = i % S;
-        const uint32_t st = ring + (uint32_t)slot * pitch;
-        if (!dead && !__all_sync(0xFFFFFFFFu, mbar_wait_bounded(full0 + 8u * (uint32_t)slot, (uint32_t)((i / S) & 1)))) {
+        const int ra = min(R, (int)min((int64_t)T, r_end - r0) - rs * R);     // rows of this row slot
+        bool rowok = ra > 0;
+        if (MODE == SK_SWIGLU && rowok) rowok = sk_valid(p, (int)((r0 + rs * R) / p.inter));
+        if (ra > 0 && !dead && !__all_sync(0xFFFFFFFFu, mbar_wait_bounded_block(full_bar(slot, rs), phase))) {
             if (lane == 0) {
                 atomicOr(p.err, DEVERR_TIMEOUT);
                 *abort_flag = 1;
             }
             dead = true;                          // no more waits; stages are still released
         }
-        const int64_t r0 = r_begin + (int64_t)i * T;
-        const int tr = (int)min((int64_t)T, r_end - r0);
-        float acc[R];
+        float acc[V];
 #pragma unroll
-        for (int k = 0; k < R; ++k) {
-            acc[k] = 0.f;
-            const int rl = rs * R + k;
-            if (!dead && have && rl < tr) {
-                const uint32_t a = st + (uint32_t)rl * row_bytes + slice;
-                if (FMT == FMT_Q8_0) acc[k] = q8_0_dot_pair(a, xp);
-                else if (FMT == FMT_Q4_K) acc[k] = q4_k_dot1<false>(a, lane & 3, sel, xp, xsa, xsb);
-                else acc[k] = q6_k_dot1(a, q6h, q6l, xp);
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int k = 0; k < R; ++k) {
+                acc[g * R + k] = 0.f;
+                if (!dead && rowok && have && k < ra) {
+                    const uint32_t a = st + slice + (uint32_t)(g * R + k) * rb;
+                    if (FMT == FMT_Q8_0) acc[g * R + k] = q8_0_dot_pair(a, xp);
+                    else if (FMT == FMT_Q4_K) acc[g * R + k] = q4_k_dot1<false>(a, lane & 3, sel, xp, xsa, xsb);
+                    else acc[g * R + k] = q6_k_dot1(a, q6h, q6l, xp);
+                }
             }
-        }
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8u * (uint32_t)slot);   // the stage may be refilled
-        warp_transpose_reduce<R>(acc, lane);
-        const int rl = rs * R + kl;
+        warp_transpose_reduce<V>(acc, lane);
+        const int64_t row = r0 + rs * R + vk;
         if (p.ksegs == 1) {
-            if (leader && rl < tr) p.y[r0 + rl] = acc[0];
+            if (MODE == SK_SWIGLU) {
+                const float u = __shfl_down_sync(0xFFFFFFFFu, acc[0], R << SH);    // the up value of row vk
+                if (leader && vg == 0 && vk < ra) p.y[row] = rowok ? acc[0] / (1.0f + expf(-acc[0])) * u : 0.f;
+            } else if (leader && vk < ra) {
+                p.y[row] = MODE == SK_GATHER ? wseg[0] * acc[0] : acc[0];
+            }
         } else {
-            // partials of the row's K-segments, added in K order by the first one
+            // partials of the row's K-segments, added in K order by segment 0
             const uint32_t pb = part0 + (uint32_t)(i & 1) * (uint32_t)(SK_PART / 2);
-            if (leader) sts_f32(pb + 4u * (uint32_t)(rl * p.ksegs + ks), acc[0]);
-            named_bar_sync(2 + rs, 32 * p.ksegs);
-            if (ks == 0 && leader && rl < tr) {
-                float v = 0.f;
-                for (int k2 = 0; k2 < p.ksegs; ++k2) v += lds_f32(pb + 4u * (uint32_t)(rl * p.ksegs + k2));
-                p.y[r0 + rl] = v;
+            const int nk = p.ksegs;
+            if (leader) sts_f32(pb + 4u * (uint32_t)(((rs * R + vk) * G + vg) * nk + ks), acc[0]);
+            named_bar_sync(2 + rs, 32 * nk);
+            if (ks == 0 && leader && vg == 0 && vk < ra) {
+                float s0 = 0.f, s1 = 0.f;
+                const uint32_t e0 = pb + 4u * (uint32_t)((rs * R + vk) * G * nk);
+                for (int k2 = 0; k2 < nk; ++k2) {
+                    const float v = lds_f32(e0 + 4u * (uint32_t)k2);
+                    if (MODE == SK_GATHER) s0 = fmaf(wseg[k2], v, s0);
+                    else s0 += v;
+                    if (MODE == SK_SWIGLU) s1 += lds_f32(e0 + 4u * (uint32_t)(nk + k2));
+                }
+                p.y[row] = MODE == SK_SWIGLU ? (rowok ? s0 / (1.0f + expf(-s0)) * s1 : 0.f) : s0;
             }
         }
+        if (++slot == S) {
+            slot = 0;
+            phase ^= 1u;
+        }
+        st = ring + (uint32_t)slot * pitch;
+        r0 += T;
     }
 }
 
 // Defined per format in qmv_fmt_*.cu.
 template <int FMT>
-cudaError_t launch_sk(const SkParams &p, int R, dim3 grid, size_t smem, cudaStream_t stream, bool pdl);
+cudaError_t launch_sk(const SkParams &p, int mode, int R, dim3 grid, size_t smem, cudaStream_t stream, bool pdl);
+
+// ---------------------------------------------------------------------------
+// Ordered chain of one-token matvecs in one persistent launch (the layer after
+// layer order of a decode step, BebeLM page, §核心算子 / §性能表现): task t+1
+// may read any earlier task's y.  One cooperative CTA per SM; for every task
+// each CTA takes its contiguous share of the rows.  The producer streams the
+// stages of all tasks in sequence and never waits for the grid, so while the
+// consumers cross the grid barrier between tasks the ring fills with the
+// next task's weights.  The consumers of every CTA finish task t (y written),
+// meet at a grid barrier, stage x of task t+1 through L2 (it may have been
+// written by another SM in this launch) and decode from an already filled
+// ring.
+constexpr int SKC_MAX_TASKS = 64;
+
+struct SkTask {
+    const uint8_t *W;
+    const float *x;          // [cols]
+    float *y;                // [rows]
+    int64_t rows;
+    int64_t row_bytes;
+    int64_t units_q;         // CTA c owns units_q + (c < units_r) units of R rows
+    int32_t units_r;
+    int32_t cols;
+    int32_t ksegs;           // consumer warps per row (a divisor of SK_NC)
+    int32_t seg_bytes;       // bytes of one 2048-column K-segment of a row
+    int32_t tile_rows;       // T = (SK_NC / ksegs) * R
+    int32_t pad_;
+};
+
+struct SkChainParams {
+    int32_t n_tasks;
+    int32_t n_stage;
+    int32_t stage_pitch;
+    int32_t x_off;           // byte offset of the x area from the ring start
+    unsigned *sync;          // {arrivals, exits} of the grid barrier, zero between launches
+    int *err;
+    uint32_t debug_extra_tx;
+    SkTask t[SKC_MAX_TASKS];
+};
+
+// This CTA's rows [a, b) of task tk (R rows per unit).
+template <int R>
+__device__ __forceinline__ void skc_rows(const SkTask &tk, int c, int64_t &a, int64_t &b)
+{
+    const int64_t u0 = (int64_t)c * tk.units_q + min(c, tk.units_r);
+    a = u0 * R;
+    b = min(tk.rows, (u0 + tk.units_q + (c < tk.units_r ? 1 : 0)) * R);
+}
+
+template <int FMT, int R>
+__global__ void __launch_bounds__(SK_THREADS, 1) qmv_skc_kernel(const __grid_constant__ SkChainParams p)
+{
+    static_assert(R == 1 || R == 2 || R == 4, "rows per consumer warp");
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int warp = (int)threadIdx.x >> 5, lane = (int)threadIdx.x & 31;
+    const uint32_t sraw = smem_addr(smem);
+    const uint32_t sbase = (sraw + 127u) & ~127u;          // the launch adds 128 spare bytes
+    uint8_t *const sgen = smem + (sbase - sraw);
+    const uint32_t full0 = sbase + SK_FULL_OFF, empty0 = sbase + SK_EMPTY_OFF;
+    volatile int *const abort_flag = reinterpret_cast<volatile int *>(sgen + SK_ABORT_OFF);
+    const uint32_t part0 = sbase + (uint32_t)SK_HDR;
+    const uint32_t ring = part0 + (uint32_t)SK_PART;
+    const uint32_t xs = ring + (uint32_t)p.x_off;
+    const int S = p.n_stage;
+    const uint32_t pitch = (uint32_t)p.stage_pitch;
+    const int c = (int)blockIdx.x;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full0 + 8u * (uint32_t)s, 1);
+            mbar_init(empty0 + 8u * (uint32_t)s, SK_NC);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == SK_NC) {
+        // ------------------------------------------------------ producer --
+        if (lane != 0) return;
+        int i = 0;                                     // stage sequence over all tasks
+        bool ok = true;
+        for (int t = 0; t < p.n_tasks && ok; ++t) {
+            const SkTask &tk = p.t[t];
+            int64_t a, b;
+            skc_rows<R>(tk, c, a, b);
+            const uint64_t rb = (uint64_t)tk.row_bytes;
+            for (int64_t r0 = a; r0 < b; r0 += tk.tile_rows, ++i) {
+                const int slot = i % S, round = i / S;
+                if (round > 0 && !mbar_wait_bounded_block(empty0 + 8u * (uint32_t)slot, (uint32_t)((round - 1) & 1))) {
+                    atomicOr(p.err, DEVERR_TIMEOUT);
+                    ok = false;
+                    break;
+                }
+                if (*abort_flag) {
+                    ok = false;
+                    break;
+                }
+                if (round > 0) fence_proxy_async_smem();
+                const uint32_t bytes = (uint32_t)(min((int64_t)tk.tile_rows, b - r0) * (int64_t)rb);
+                const uint32_t full = full0 + 8u * (uint32_t)slot;
+                mbar_arrive_expect_tx(full, bytes + p.debug_extra_tx);
+                bulk_g2s(ring + (uint32_t)slot * pitch, tk.W + (uint64_t)r0 * rb, bytes, full);
+            }
+        }
+        // let every copy land before the CTA can exit
+        for (int j = max(0, i - S); j < i; ++j) {
+            if (!mbar_wait_bounded_block(full0 + 8u * (uint32_t)(j % S), (uint32_t)((j / S) & 1))) {
+                atomicOr(p.err, DEVERR_DRAIN);
+                break;
+            }
+        }
+        return;
+    }
+
+    // -------------------------------------------------------- consumers --
+    const Q4kSel sel = q4k_sel(lane & 3);
+    const int q6h = (lane >> 1) & 1, q6l = 16 * (lane & 1);
+    constexpr int SH = 5 - Log2<R>::v;
+    const bool leader = (lane & ((1 << SH) - 1)) == 0;
+    const int vk = lane >> SH;
+    bool dead = false;
+    int i = 0;
+    for (int t = 0; t < p.n_tasks; ++t) {
+        const SkTask &tk = p.t[t];
+        if (t > 0) {
+            // every CTA has written task t-1's y
+            named_bar_sync(1, SK_NC * 32);
+            if (threadIdx.x == 0) {
+                // release: this CTA's y stores (ordered before by the CTA barrier)
+                // become visible before the arrival; acquire: every CTA's stores
+                // are visible after the last arrival is seen
+                asm volatile("red.release.gpu.global.add.u32 [%0], 1;" :: "l"(p.sync) : "memory");
+                const unsigned target = (unsigned)t * gridDim.x;
+                const uint64_t t0 = global_timer_ns();
+                for (uint32_t n = 0;; ++n) {
+                    unsigned v;
+                    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p.sync) : "memory");
+                    if ((int)(v - target) >= 0) break;
+                    if ((n & 63u) == 63u && global_timer_ns() - t0 > 1000000000ull) {
+                        atomicOr(p.err, DEVERR_TIMEOUT);
+                        break;
+                    }
+                }
+            }
+            named_bar_sync(1, SK_NC * 32);
+        }
+        // x of this task through L2 (written earlier in this launch, possibly by another SM)
+        sk_stage_x<true>(xs, tk.x, 1, tk.cols >> 2, 0);
+        named_bar_sync(1, SK_NC * 32);
+        const int nk = tk.ksegs;
+        const int ks = warp % nk, rs = warp / nk;
+        const int seg_cols = min(SK_SEG, tk.cols - ks * SK_SEG);
+        float2 xr[16][2];
+        float xsa = 0.f, xsb = 0.f;
+        rw_load_x_smem<FMT>(xs, ks, seg_cols, lane, xr, xsa, xsb);
+        auto xp = [&](int gq, float2 &x02, float2 &x13) {
+            x02 = xr[gq][0];
+            x13 = xr[gq][1];
+        };
+        const bool have = 64 * (lane + 1) <= seg_cols;
+        const uint32_t rb = (uint32_t)tk.row_bytes;
+        uint32_t slice = (uint32_t)(rs * R) * rb + (uint32_t)ks * (uint32_t)tk.seg_bytes;
+        if (FMT == FMT_Q8_0) slice += 68u * (uint32_t)lane;
+        else if (FMT == FMT_Q4_K) slice += 144u * (uint32_t)(lane >> 2);
+        else slice += 210u * (uint32_t)(lane >> 2);
+        int64_t a, b;
+        skc_rows<R>(tk, c, a, b);
+        for (int64_t r0 = a; r0 < b; r0 += tk.tile_rows, ++i) {
+            const int slot = i % S;
+            const uint32_t st = ring + (uint32_t)slot * pitch;
+            const int ra = min(R, (int)min((int64_t)tk.tile_rows, b - r0) - rs * R);
+            if (ra > 0 && !dead &&
+                !__all_sync(0xFFFFFFFFu, mbar_wait_bounded_block(full0 + 8u * (uint32_t)slot, (uint32_t)((i / S) & 1)))) {
+                if (lane == 0) {
+                    atomicOr(p.err, DEVERR_TIMEOUT);
+                    *abort_flag = 1;
+                }
+                dead = true;
+            }
+            float acc[R];
+#pragma unroll
+            for (int k = 0; k < R; ++k) {
+                acc[k] = 0.f;
+                if (!dead && have && k < ra) {
+                    const uint32_t ad = st + slice + (uint32_t)k * rb;
+                    if (FMT == FMT_Q8_0) acc[k] = q8_0_dot_pair(ad, xp);
+                    else if (FMT == FMT_Q4_K) acc[k] = q4_k_dot1<false>(ad, lane & 3, sel, xp, xsa, xsb);
+                    else acc[k] = q6_k_dot1(ad, q6h, q6l, xp);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty0 + 8u * (uint32_t)slot);
+            warp_transpose_reduce<R>(acc, lane);
+            const int64_t row = r0 + rs * R + vk;
+            if (nk == 1) {
+                if (leader && vk < ra) tk.y[row] = acc[0];
+            } else {
+                const uint32_t pb = part0 + (uint32_t)(i & 1) * (uint32_t)(SK_PART / 2);
+                if (leader) sts_f32(pb + 4u * (uint32_t)((rs * R + vk) * nk + ks), acc[0]);
+                named_bar_sync(2 + rs, 32 * nk);
+                if (ks == 0 && leader && vk < ra) {
+                    float s0 = 0.f;
+                    for (int k2 = 0; k2 < nk; ++k2) s0 += lds_f32(pb + 4u * (uint32_t)((rs * R + vk) * nk + k2));
+                    tk.y[row] = s0;
+                }
+            }
+        }
+    }
+    // the last CTA to leave puts the barrier words back to zero for the next launch
+    named_bar_sync(1, SK_NC * 32);
+    if (threadIdx.x == 0) {
+        const unsigned old = atomicAdd(p.sync + 1, 1u);
+        if (old == gridDim.x - 1u) {
+            atomicExch(p.sync, 0u);
+            atomicExch(p.sync + 1, 0u);
+        }
+    }
+}
+
+template <int FMT>
+cudaError_t launch_skc(const SkChainParams &p, int R, dim3 grid, size_t smem, cudaStream_t stream);
 
 }  // namespace qmv

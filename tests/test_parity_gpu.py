@@ -624,10 +624,15 @@ def test_moe_ffn_other_expert_counts(ids):
     _check_moe_ffn(8, 512, 768, 50 + len(ids), ids, g)
 
 
-@pytest.mark.parametrize("fmt,hidden,inter", [(Q4_K, 2048, 1792), (Q8_0, 1024, 512), (Q8_0, 4096, 1024)])
-def test_moe_ffn_formats_and_a_bad_expert_id(fmt, hidden, inter):
-    # Q8_0 experts, rows of more than one K-chunk (hidden 4096), and an expert id
-    # out of range: that expert contributes nothing (h row zero) and is reported
+@pytest.mark.parametrize("fmt,hidden,inter,kernel", [(Q4_K, 2048, 1792, q.KERNEL_STREAM),
+                                                     (Q8_0, 1024, 512, q.KERNEL_STREAM),
+                                                     (Q8_0, 4096, 1024, q.KERNEL_STREAM),
+                                                     (Q4_K, 512, 2304, q.KERNEL_GENERAL)])
+def test_moe_ffn_formats_and_a_bad_expert_id(fmt, hidden, inter, kernel):
+    # Q8_0 experts, rows of more than one K-segment (hidden 4096), expert rows
+    # longer than one K-segment (inter 2304: the general kernel), and an expert
+    # id out of range: that expert contributes nothing (h row zero) and is
+    # reported
     n_expert, ids, g32 = 6, [4, 1, 9, 3], np.array([0.4, 0.3, 0.2, 0.1], np.float32)
     gus, ds = synth.matrix_bytes(fmt, inter, hidden), synth.matrix_bytes(fmt, hidden, inter)
     gate = synth.gen_blocks(fmt, inter * n_expert, hidden, 61, 1)
@@ -638,6 +643,7 @@ def test_moe_ffn_formats_and_a_bad_expert_id(fmt, hidden, inter):
     y = torch.full((hidden,), float("nan"), device="cuda")
     q.moe_ffn(fmt, dev(gate), dev(up), gus, fmt, dev(down), ds, n_expert, dev(np.array(ids, np.int32)),
               dev(g32), 4, hidden, inter, dev(x), h, y)
+    assert q.qmv_debug_last_kernel() == kernel
     err = q.qmv_check()
     assert err & q.DEVERR_EXPERT_ID
     hh, yy = h.cpu().numpy(), y.cpu().numpy()
