@@ -390,7 +390,10 @@ def measure_matvec(torch, q, stream, fmt, rows, cols, n_tok, seed, reps=200, arg
             "single_launch_timing": "one launch, PDL off, CUDA events around it"}
 
 
-def measure_moe(torch, q, stream, reps=200):
+def measure_moe(torch, q, stream, reps=200, separate=False):
+    """The MoE FFN step of the 32-expert workload: moe_ffn_routed (router and
+    both products in one launch), or with separate=True moe_route followed by
+    moe_ffn (three launches)."""
     w = synth.workload_cfg3()
     E, hidden, inter, seed = w["n_expert"], w["hidden"], w["inter"], w["seed"]
     gus = synth.matrix_bytes(Q4_K, inter, hidden)
@@ -410,12 +413,16 @@ def measure_moe(torch, q, stream, reps=200):
     g = torch.empty(4, device="cuda")
     h = torch.empty((4, inter), device="cuda")
     y = torch.empty(hidden, device="cuda")
+    ws = torch.zeros(q.MOE_WS_BYTES // 8, dtype=torch.int64, device="cuda")
     per_graph = 2 * n_copies
 
     def one(i):
         G, U, D = sets[i % n_copies]
-        q.moe_route(lg, bs, E, 4, ids, g)
-        q.moe_ffn(Q4_K, G, U, gus, Q4_K, D, ds, E, ids, g, 4, hidden, inter, x, h, y)
+        if separate:
+            q.moe_route(lg, bs, E, 4, ids, g)
+            q.moe_ffn(Q4_K, G, U, gus, Q4_K, D, ds, E, ids, g, 4, hidden, inter, x, h, y)
+        else:
+            q.moe_ffn_routed(lg, bs, E, 4, Q4_K, G, U, gus, Q4_K, D, ds, hidden, inter, x, ids, g, h, y, ws)
 
     def body():
         for i in range(per_graph):
@@ -427,7 +434,8 @@ def measure_moe(torch, q, stream, reps=200):
     del gr
     us1 = single_launch_us(torch, q, stream, one, n_copies)
     return {"workload": "MoE FFN step: route top-4 of 32 + Q4_K gate/up 1792x2048 + down 2048x1792",
-            "us": sec * 1e6, "weight_gbs": touched / sec / 1e9, "launches_per_step": 3,
+            "calls": "moe_route + moe_ffn" if separate else "moe_ffn_routed",
+            "us": sec * 1e6, "weight_gbs": touched / sec / 1e9,
             "weight_bytes_touched": touched, "copies": n_copies,
             "timing": "graph of back-to-back steps, programmatic dependent launch on (pipelined)",
             "us_single_launch": round(us1, 3), "weight_gbs_single_launch": round(touched / us1 / 1e3, 1),
@@ -552,8 +560,8 @@ PROFILE_CASES = {
 
 
 def run_profile_moe(args):
-    """A few MoE FFN steps of the 32-expert workload (router, gate/up with the
-    SwiGLU epilogue, weighted down), 198 MB of experts on the device."""
+    """A few MoE FFN steps of the 32-expert workload, 198 MB of experts on the
+    device: moe_ffn_routed (one launch), then moe_route + moe_ffn (three)."""
     import torch
     import quantized_decode_superblocks_b200 as q
     torch.cuda.set_device(0)
@@ -570,6 +578,9 @@ def run_profile_moe(args):
     g = torch.empty(4, device="cuda")
     h = torch.empty((4, inter), device="cuda")
     y = torch.empty(hidden, device="cuda")
+    ws = torch.zeros(q.MOE_WS_BYTES // 8, dtype=torch.int64, device="cuda")
+    for _ in range(max(1, args.steps)):
+        q.moe_ffn_routed(lg, bs, E, 4, Q4_K, G, U, gus, Q4_K, D, ds, hidden, inter, x, ids, g, h, y, ws)
     for _ in range(max(1, args.steps)):
         q.moe_route(lg, bs, E, 4, ids, g)
         q.moe_ffn(Q4_K, G, U, gus, Q4_K, D, ds, E, ids, g, 4, hidden, inter, x, h, y)
@@ -682,6 +693,7 @@ def main():
             per_config["cfg2_q6_k_vocab_128000x2048_ntok1_greedy_argmax"] = measure_matvec(
                 torch, q, stream, Q6_K, 128000, 2048, 1, 2, reps=20, argmax=True)
             per_config["cfg3_moe_ffn_step"] = measure_moe(torch, q, stream)
+            per_config["cfg3_moe_route_then_ffn"] = measure_moe(torch, q, stream, separate=True)
             for nt in (1, 2, 4, 8):
                 sw = Sweep(torch, q, nt, cache)
                 for md in (("launches", "chain", "grouped") if nt == 1 else ("launches", "grouped")):

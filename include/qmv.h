@@ -47,7 +47,7 @@
  *     state: a per-device properties cache, the programmatic-dependent-launch
  *     switch (qmv_set_pdl), and per device the sticky error word read by
  *     qmv_check(), the two grid-barrier words of qmv_chain, qmv_argmax's
- *     per-token keys and the scratch array of moe_ffn_static.
+ *     workspace and the scratch array of moe_ffn_static.
  */
 #ifndef QMV_H
 #define QMV_H
@@ -188,6 +188,29 @@ int moe_ffn(int fmt_gu, const void *gate_blocks, const void *up_blocks,
             const float *g, int n_sel, int64_t hidden, int64_t inter,
             const float *x, float *h_scratch, float *y, qmv_stream_t stream);
 
+/* The MoE FFN step with its router, in one launch where the shapes allow
+ * (BebeLM page, §核心算子, MoE前馈网络): moe_route on (logits, bias, n_expert,
+ * top_k) -- ids_out, g_out as moe_route writes them, the same values -- then
+ * moe_ffn with those ids and weights (n_sel = top_k): h_scratch
+ * f32 [top_k][inter] holds the SwiGLU activations, y f32 [hidden] the result.
+ * When both matrices have one format, expert rows are at most 2048 columns,
+ * n_expert <= 256 and the rows are 16-byte multiples in pairs, one
+ * cooperative launch does it all: every CTA routes on its own, streams the
+ * routed gate/up rows and then the routed down rows through one pipeline, and
+ * the CTAs meet once, at a grid barrier, between the two products (h complete).
+ * Otherwise moe_route and moe_ffn run in turn.  `workspace`:
+ * QMV_MOE_WS_BYTES of caller-owned device memory (8-byte aligned) that must be
+ * zero before the first call and that every completed call leaves zero again
+ * (the barrier's counters); calls that may overlap on the GPU need workspaces
+ * of their own.  Errors as moe_route and moe_ffn. */
+#define QMV_MOE_WS_BYTES 16
+int moe_ffn_routed(const float *logits, const float *bias, int n_expert, int top_k,
+                   int fmt_gu, const void *gate_blocks, const void *up_blocks,
+                   int64_t gu_stride_bytes, int fmt_down, const void *down_blocks,
+                   int64_t down_stride_bytes, int64_t hidden, int64_t inter, const float *x,
+                   int32_t *ids_out, float *g_out, float *h_scratch, float *y, void *workspace,
+                   qmv_stream_t stream);
+
 /* moe_ffn without a caller-provided scratch buffer, for callers that cannot
  * allocate device memory: code running while a stream is being captured into
  * a CUDA graph (where cudaMalloc is not allowed), plugins and callbacks that
@@ -213,15 +236,30 @@ int moe_ffn_static(int fmt_gu, const void *gate_blocks, const void *up_blocks,
 
 /* Greedy next-token choice on the device (FlareLLM page, §推理层面的深度优化:
  * greedy decoding of the vocabulary projection): y = W x as qmv_batched (the
- * logits are kept in the caller's y, f32 [n_tok][rows]), then
+ * logits are kept in the caller's y, f32 [n_tok][rows]), and
  * idx_out[t] = the row of the largest y[t][row] -- IEEE > on f32, ties to
  * the lower row, NaN values skipped, -1 if every value of the token is NaN.
  * idx_out: device int32 [n_tok], 4-byte aligned.  rows <= INT32_MAX.
- * Two launches on `stream`; the choice is deterministic (the CTAs combine
- * their candidates with an order-independent 64-bit atomic max).  The
- * reduction keeps one key and one counter per token in device memory of the
- * library, back to zero after every call: do not run two qmv_argmax calls on
- * the same device at the same time.  Errors as qmv_batched. */
+ * With one token on the shapes the one-token streaming kernel takes (rows of
+ * at most 2048 columns) the choice is fused into the projection: every CTA
+ * folds the best of its rows into a 64-bit key while it writes them, and the
+ * last CTA writes idx -- one launch.  Otherwise a second launch scans y.
+ * Either way the choice is deterministic (an order-independent atomic max
+ * over keys: the value's order-preserving bits high, the complemented row
+ * low).
+ * The keys and arrival counters live in `workspace`, QMV_ARGMAX_WS_BYTES of
+ * caller-owned device memory (8-byte aligned) that must be zero before the
+ * first call and that every completed call leaves zero again; calls that may
+ * overlap on the GPU need workspaces of their own.  Errors as qmv_batched,
+ * QMV_ERR_NULL for a NULL workspace. */
+#define QMV_ARGMAX_WS_BYTES 128
+int qmv_argmax_ws(int fmt, const void *W_blocks, int64_t rows, int64_t cols,
+                  const float *x, float *y, int n_tok, int32_t *idx_out, void *workspace,
+                  qmv_stream_t stream);
+
+/* qmv_argmax_ws with the library's own workspace on the current device: do
+ * not run two qmv_argmax calls on one device at the same time (use
+ * qmv_argmax_ws with separate workspaces for that). */
 int qmv_argmax(int fmt, const void *W_blocks, int64_t rows, int64_t cols,
                const float *x, float *y, int n_tok, int32_t *idx_out, qmv_stream_t stream);
 

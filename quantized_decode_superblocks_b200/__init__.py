@@ -27,7 +27,7 @@ DEVERR_TIMEOUT = 2
 DEVERR_DRAIN = 4
 KERNEL_WARP_RING, KERNEL_GENERAL, KERNEL_TENSOR_CORE, KERNEL_STREAM = 1, 2, 3, 4
 
-EXPORTED = ("qmv_f32", "qmv_batched", "qmv_multi", "qmv_chain", "qmv_argmax", "moe_route", "moe_qmv", "moe_ffn", "moe_ffn_static",
+EXPORTED = ("qmv_f32", "qmv_batched", "qmv_multi", "qmv_chain", "qmv_argmax", "qmv_argmax_ws", "moe_route", "moe_qmv", "moe_ffn", "moe_ffn_routed", "moe_ffn_static",
             "qmv_dequant",
             "qmv_check", "qmv_strerror", "qmv_block_bytes", "qmv_block_weights",
             "qmv_debug_fail_next_launches", "qmv_debug_short_copies", "qmv_set_pdl", "qmv_get_pdl",
@@ -65,10 +65,13 @@ def lib() -> ctypes.CDLL:
         L.qmv_multi.argtypes = [c_int, c_int, ctypes.POINTER(QmvTask), c_int, vp]
         L.qmv_chain.argtypes = [c_int, ctypes.POINTER(QmvTask), c_int, vp]
         L.qmv_argmax.argtypes = [c_int, vp, i64, i64, vp, vp, c_int, vp, vp]
+        L.qmv_argmax_ws.argtypes = [c_int, vp, i64, i64, vp, vp, c_int, vp, vp, vp]
         L.moe_route.argtypes = [vp, vp, c_int, c_int, vp, vp, vp]
         L.moe_qmv.argtypes = [c_int, vp, i64, c_int, vp, c_int, i64, i64, vp, i64, vp, vp, vp]
         L.moe_ffn.argtypes = [c_int, vp, vp, i64, c_int, vp, i64, c_int, vp, vp, c_int, i64, i64,
                               vp, vp, vp, vp]
+        L.moe_ffn_routed.argtypes = [vp, vp, c_int, c_int, c_int, vp, vp, i64, c_int, vp, i64, i64, i64,
+                                     vp, vp, vp, vp, vp, vp, vp]
         L.moe_ffn_static.argtypes = [c_int, vp, vp, i64, c_int, vp, i64, c_int, vp, vp, c_int, i64, i64,
                                      vp, vp, vp]
         L.qmv_dequant.argtypes = [c_int, vp, i64, i64, vp, vp]
@@ -190,6 +193,16 @@ def qmv_argmax(fmt, W, rows, cols, x, y, n_tok, idx_out, stream=None):
                             _stream(stream)), "qmv_argmax")
 
 
+ARGMAX_WS_BYTES = 128
+
+
+def qmv_argmax_ws(fmt, W, rows, cols, x, y, n_tok, idx_out, workspace, stream=None):
+    """qmv_argmax with a caller-owned workspace of ARGMAX_WS_BYTES device bytes
+    (zero before the first call; every completed call leaves it zero)."""
+    _check(lib().qmv_argmax_ws(fmt, _ptr(W), rows, cols, _ptr(x), _ptr(y), n_tok, _ptr(idx_out),
+                               _ptr(workspace), _stream(stream)), "qmv_argmax_ws")
+
+
 def moe_route(logits, bias, n_expert, top_k, ids_out, g_out, stream=None):
     _check(lib().moe_route(_ptr(logits), _ptr(bias), n_expert, top_k, _ptr(ids_out), _ptr(g_out),
                            _stream(stream)), "moe_route")
@@ -209,6 +222,19 @@ def moe_ffn(fmt_gu, gate_blocks, up_blocks, gu_stride_bytes, fmt_down, down_bloc
                          _ptr(down_blocks), down_stride_bytes, n_expert, _ptr(expert_ids), _ptr(g),
                          n_sel, hidden, inter, _ptr(x), _ptr(h_scratch), _ptr(y), _stream(stream)),
            "moe_ffn")
+
+
+MOE_WS_BYTES = 16
+
+
+def moe_ffn_routed(logits, bias, n_expert, top_k, fmt_gu, gate_blocks, up_blocks, gu_stride_bytes,
+                   fmt_down, down_blocks, down_stride_bytes, hidden, inter, x, ids_out, g_out, h_scratch, y,
+                   workspace, stream=None):
+    """Router + MoE FFN step (one launch where the shapes allow; see include/qmv.h)."""
+    _check(lib().moe_ffn_routed(_ptr(logits), _ptr(bias), n_expert, top_k, fmt_gu, _ptr(gate_blocks),
+                                _ptr(up_blocks), gu_stride_bytes, fmt_down, _ptr(down_blocks), down_stride_bytes,
+                                hidden, inter, _ptr(x), _ptr(ids_out), _ptr(g_out), _ptr(h_scratch), _ptr(y),
+                                _ptr(workspace), _stream(stream)), "moe_ffn_routed")
 
 
 def moe_ffn_static(fmt_gu, gate_blocks, up_blocks, gu_stride_bytes, fmt_down, down_blocks,

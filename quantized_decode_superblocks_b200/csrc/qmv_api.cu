@@ -24,10 +24,10 @@ __device__ int g_dev_err;
 // at the end of every launch; qmv_check clears both after a device error.
 __device__ unsigned g_chain_sync[2];
 
-// Greedy argmax: one 64-bit key and one arrival counter per token, back to
-// zero at the end of every call; qmv_check clears them after a device error.
-__device__ unsigned long long g_amax_key[QMV_MAX_NTOK];
-__device__ unsigned g_amax_done[QMV_MAX_NTOK];
+// Greedy argmax workspace of qmv_argmax (the layout of qmv_argmax_ws's): one
+// 64-bit key per token, then one arrival counter per token; back to zero at
+// the end of every call; qmv_check clears it after a device error.
+__device__ unsigned long long g_amax_ws[QMV_ARGMAX_WS_BYTES / 8];
 
 // Scratch of moe_ffn_static: the SwiGLU activations h[n_sel][inter].  Every
 // device that loads the library holds one copy until the process exits.
@@ -50,8 +50,7 @@ struct DevInfo {
     int smem_optin = 0;
     int *err = nullptr;
     unsigned *sync = nullptr;
-    unsigned long long *amax_key = nullptr;
-    unsigned *amax_done = nullptr;
+    unsigned long long *amax_key = nullptr;   // device address of g_amax_ws
     float *static_h = nullptr;   // device address of g_static_h, set up by moe_ffn_static
     bool ok = false;
 };
@@ -105,8 +104,7 @@ int get_dev(DevInfo &out)
             cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaGetSymbolAddress(reinterpret_cast<void **>(&d.err), g_dev_err) != cudaSuccess ||
             cudaGetSymbolAddress(reinterpret_cast<void **>(&d.sync), g_chain_sync) != cudaSuccess ||
-            cudaGetSymbolAddress(reinterpret_cast<void **>(&d.amax_key), g_amax_key) != cudaSuccess ||
-            cudaGetSymbolAddress(reinterpret_cast<void **>(&d.amax_done), g_amax_done) != cudaSuccess) {
+            cudaGetSymbolAddress(reinterpret_cast<void **>(&d.amax_key), g_amax_ws) != cudaSuccess) {
             (void)cudaGetLastError();
             return QMV_ERR_DEVICE;
         }
@@ -530,9 +528,13 @@ int sk_launch(int fmt, int mode, SkParams &p, const SkGeom &g, const DevInfo &di
 }
 
 int sk_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x, float *y, const SkGeom &g,
-              const DevInfo &di, cudaStream_t st)
+              const DevInfo &di, cudaStream_t st, int32_t *amax_idx = nullptr,
+              unsigned long long *amax_key = nullptr, unsigned *amax_done = nullptr)
 {
     SkParams p{};
+    p.amax_idx = amax_idx;
+    p.amax_key = amax_key;
+    p.amax_done = amax_done;
     p.W = static_cast<const uint8_t *>(W);
     p.x = x;
     p.y = y;
@@ -743,6 +745,18 @@ int check_matrix(int fmt, int64_t rows, int64_t cols)
     if (!fmt_ok(fmt)) return QMV_ERR_FMT;
     if (rows < 1 || cols < 1 || rows > QMV_MAX_ROWS || cols > QMV_MAX_COLS || cols % block_weights(fmt) != 0)
         return QMV_ERR_SHAPE;
+    return QMV_OK;
+}
+
+int argmax_check(int fmt, const void *W, int64_t rows, int64_t cols, const float *x, const float *y, int n_tok,
+                 const int32_t *idx_out)
+{
+    if (!W || !x || !y || !idx_out) return QMV_ERR_NULL;
+    const int rc = check_matrix(fmt, rows, cols);
+    if (rc) return rc;
+    if (rows > INT32_MAX) return QMV_ERR_SHAPE;
+    if (n_tok < 1 || n_tok > QMV_MAX_NTOK) return QMV_ERR_NTOK;
+    if (!aligned(W, 16) || !aligned(x, 16) || !aligned(y, 4) || !aligned(idx_out, 4)) return QMV_ERR_ALIGN;
     return QMV_OK;
 }
 
@@ -1070,6 +1084,105 @@ int moe_ffn(int fmt_gu, const void *gate_blocks, const void *up_blocks, int64_t 
     return launch_plan(fmt_down, b, st);
 }
 
+int moe_ffn_routed(const float *logits, const float *bias, int n_expert, int top_k, int fmt_gu,
+                   const void *gate_blocks, const void *up_blocks, int64_t gu_stride_bytes, int fmt_down,
+                   const void *down_blocks, int64_t down_stride_bytes, int64_t hidden, int64_t inter,
+                   const float *x, int32_t *ids_out, float *g_out, float *h_scratch, float *y, void *workspace,
+                   qmv_stream_t stream)
+{
+    if (!logits || !bias || !gate_blocks || !up_blocks || !down_blocks || !x || !ids_out || !g_out ||
+        !h_scratch || !y || !workspace)
+        return QMV_ERR_NULL;
+    int rc = check_matrix(fmt_gu, inter, hidden);
+    if (rc) return rc;
+    if ((rc = check_matrix(fmt_down, hidden, inter))) return rc;
+    if (n_expert < 1 || n_expert > QMV_MAX_EXPERTS || top_k < 1 || top_k > QMV_MAX_SEL || top_k > n_expert)
+        return QMV_ERR_NSEL;
+    const int64_t gu_bytes = inter * (hidden / block_weights(fmt_gu)) * block_bytes(fmt_gu);
+    const int64_t dn_bytes = hidden * (inter / block_weights(fmt_down)) * block_bytes(fmt_down);
+    if (gu_stride_bytes < gu_bytes || down_stride_bytes < dn_bytes) return QMV_ERR_SHAPE;
+    if (!aligned(logits, 4) || !aligned(bias, 4) || !aligned(gate_blocks, 16) || !aligned(up_blocks, 16) ||
+        !aligned(down_blocks, 16) || gu_stride_bytes % 16 != 0 || down_stride_bytes % 16 != 0 || !aligned(x, 16) ||
+        !aligned(ids_out, 4) || !aligned(g_out, 4) || !aligned(h_scratch, 16) || !aligned(y, 4) ||
+        !aligned(workspace, 8))
+        return QMV_ERR_ALIGN;
+    if (injected_failure()) return QMV_ERR_CUDA;
+    DevInfo di;
+    if ((rc = get_dev(di))) return rc;
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+    // the one-launch form: both matrices of one format, expert rows of at most
+    // one K-segment, the router on the device in every CTA
+    const int bw = block_weights(fmt_gu), bb = block_bytes(fmt_gu);
+    const int R = 2;
+    const int64_t rba = hidden / bw * bb, rbb = inter / bw * bb;
+    const int ka = sk_ksegs(ceil_div(hidden, SK_SEG)), kb = sk_ksegs(top_k);
+    bool fused = fmt_gu == fmt_down && n_expert <= SKM_MAX_EXPERTS && inter <= SK_SEG && ka > 0 && kb >= top_k &&
+                 inter % R == 0 && (R * rba) % 16 == 0 && (R * rbb) % 16 == 0 &&
+                 (fmt_gu != QMV_Q8_0 || (hidden % 64 == 0 && inter % 64 == 0));
+    SkMoeParams p{};
+    size_t smem = 0;
+    if (fused) {
+        const int64_t stage_a = (int64_t)(SK_NC / ka) * 2 * R * rba, stage_b = (int64_t)(SK_NC / kb) * kb * R * rbb;
+        const int64_t pitch = ceil_div(std::max(stage_a, stage_b) + 16, 128) * 128;
+        const int64_t x_bytes = ceil_div(std::max<int64_t>(hidden * 4, (int64_t)kb * SK_SEG * 4), 128) * 128;
+        const int64_t S = std::min<int64_t>(SK_MAX_STAGES, (SK_CTA_SMEM - SK_HDR - SK_PART - x_bytes) / pitch);
+        fused = S >= 2 && x_bytes <= SK_X_MAX_BYTES;
+        const int64_t ctas = di.sm_count;
+        const int64_t ua = ceil_div((int64_t)top_k * inter, (int64_t)R), ub = ceil_div(hidden, (int64_t)R);
+        p.logits = logits;
+        p.bias = bias;
+        p.ids_out = ids_out;
+        p.g_out = g_out;
+        p.n_expert = n_expert;
+        p.n_sel = top_k;
+        p.G = static_cast<const uint8_t *>(gate_blocks);
+        p.U = static_cast<const uint8_t *>(up_blocks);
+        p.gu_stride = gu_stride_bytes;
+        p.gu_row_bytes = rba;
+        p.D = static_cast<const uint8_t *>(down_blocks);
+        p.d_stride = down_stride_bytes;
+        p.d_row_bytes = rbb;
+        p.hidden = (int32_t)hidden;
+        p.inter = (int32_t)inter;
+        p.x = x;
+        p.h = h_scratch;
+        p.y = y;
+        p.a_ksegs = ka;
+        p.a_seg_bytes = SK_SEG / bw * bb;
+        p.a_T = (SK_NC / ka) * R;
+        p.a_rs_bytes = (int32_t)(2 * R * rba);
+        p.a_units_q = ua / ctas;
+        p.a_units_r = (int32_t)(ua % ctas);
+        p.b_ksegs = kb;
+        p.b_T = (SK_NC / kb) * R;
+        p.b_rs_bytes = (int32_t)(kb * R * rbb);
+        p.b_units_q = ub / ctas;
+        p.b_units_r = (int32_t)(ub % ctas);
+        p.n_stage = (int32_t)S;
+        p.stage_pitch = (int32_t)pitch;
+        p.x_off = (int32_t)(S * pitch);
+        p.sync = static_cast<unsigned *>(workspace);
+        p.err = di.err;
+        p.debug_extra_tx = g_debug_extra_tx.load();
+        smem = (size_t)(128 + SK_HDR + SK_PART + S * pitch + x_bytes);
+    }
+    if (fused) {
+        t_last_kernel = QMV_KERNEL_STREAM;
+        cudaError_t e;
+        switch (fmt_gu) {
+        case QMV_Q8_0: e = launch_skm<FMT_Q8_0>(p, R, dim3((unsigned)di.sm_count), smem, st); break;
+        case QMV_Q4_K: e = launch_skm<FMT_Q4_K>(p, R, dim3((unsigned)di.sm_count), smem, st); break;
+        default: e = launch_skm<FMT_Q6_K>(p, R, dim3((unsigned)di.sm_count), smem, st); break;
+        }
+        return e == cudaSuccess ? QMV_OK : cuda_fail(e);
+    }
+    // other shapes: the router, then the two-launch FFN step
+    if ((rc = moe_route(logits, bias, n_expert, top_k, ids_out, g_out, stream))) return rc;
+    return moe_ffn(fmt_gu, gate_blocks, up_blocks, gu_stride_bytes, fmt_down, down_blocks, down_stride_bytes,
+                   n_expert, ids_out, g_out, top_k, hidden, inter, x, h_scratch, y, stream);
+}
+
 int moe_ffn_static(int fmt_gu, const void *gate_blocks, const void *up_blocks, int64_t gu_stride_bytes,
                    int fmt_down, const void *down_blocks, int64_t down_stride_bytes, int n_expert,
                    const int32_t *expert_ids, const float *g, int n_sel, int64_t hidden, int64_t inter,
@@ -1099,24 +1212,42 @@ int moe_ffn_static(int fmt_gu, const void *gate_blocks, const void *up_blocks, i
                    n_expert, expert_ids, g, n_sel, hidden, inter, x, h, y, stream);
 }
 
-int qmv_argmax(int fmt, const void *W_blocks, int64_t rows, int64_t cols, const float *x, float *y, int n_tok,
-               int32_t *idx_out, qmv_stream_t stream)
+int qmv_argmax_ws(int fmt, const void *W_blocks, int64_t rows, int64_t cols, const float *x, float *y, int n_tok,
+                  int32_t *idx_out, void *workspace, qmv_stream_t stream)
 {
-    if (!W_blocks || !x || !y || !idx_out) return QMV_ERR_NULL;
-    int rc = check_matrix(fmt, rows, cols);
+    int rc = argmax_check(fmt, W_blocks, rows, cols, x, y, n_tok, idx_out);
     if (rc) return rc;
-    if (rows > INT32_MAX) return QMV_ERR_SHAPE;
-    if (n_tok < 1 || n_tok > QMV_MAX_NTOK) return QMV_ERR_NTOK;
-    if (!aligned(W_blocks, 16) || !aligned(x, 16) || !aligned(y, 4) || !aligned(idx_out, 4)) return QMV_ERR_ALIGN;
+    if (!workspace) return QMV_ERR_NULL;
+    if (!aligned(workspace, 8)) return QMV_ERR_ALIGN;
     DevInfo di;
     if ((rc = get_dev(di))) return rc;
+    unsigned long long *keys = static_cast<unsigned long long *>(workspace);
+    unsigned *done = reinterpret_cast<unsigned *>(keys + QMV_MAX_NTOK);
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (n_tok == 1) {
+        // one launch: the streaming kernel folds each CTA's best row into the key
+        const SkGeom g = sk_geom(fmt, SK_PLAIN, rows, cols);
+        if (g.ok && g.ksegs == 1) {
+            if (injected_failure()) return QMV_ERR_CUDA;
+            return sk_single(fmt, W_blocks, rows, cols, x, y, g, di, st, idx_out, keys, done);
+        }
+    }
     if ((rc = qmv_batched(fmt, W_blocks, rows, cols, x, y, n_tok, stream))) return rc;
     const dim3 grid((unsigned)ceil_div(rows, ARGMAX_ROWS_PER_CTA), (unsigned)n_tok);
-    argmax_rows_kernel<<<grid, ARGMAX_THREADS, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        y, rows, rows, idx_out, di.amax_key, di.amax_done);
+    argmax_rows_kernel<<<grid, ARGMAX_THREADS, 0, st>>>(y, rows, rows, idx_out, keys, done);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e);
     return QMV_OK;
+}
+
+int qmv_argmax(int fmt, const void *W_blocks, int64_t rows, int64_t cols, const float *x, float *y, int n_tok,
+               int32_t *idx_out, qmv_stream_t stream)
+{
+    int rc = argmax_check(fmt, W_blocks, rows, cols, x, y, n_tok, idx_out);
+    if (rc) return rc;
+    DevInfo di;
+    if ((rc = get_dev(di))) return rc;
+    return qmv_argmax_ws(fmt, W_blocks, rows, cols, x, y, n_tok, idx_out, di.amax_key, stream);
 }
 
 int qmv_dequant(int fmt, const void *W_blocks, int64_t rows, int64_t cols, float *out, qmv_stream_t stream)
@@ -1158,8 +1289,7 @@ int qmv_check(qmv_stream_t stream, int *dev_err_out)
         return QMV_ERR_CUDA;
     }
     if (word && (cudaMemset(di.sync, 0, 2 * sizeof(unsigned)) != cudaSuccess ||
-                 cudaMemset(di.amax_key, 0, QMV_MAX_NTOK * sizeof(unsigned long long)) != cudaSuccess ||
-                 cudaMemset(di.amax_done, 0, QMV_MAX_NTOK * sizeof(unsigned)) != cudaSuccess ||
+                 cudaMemset(di.amax_key, 0, QMV_ARGMAX_WS_BYTES) != cudaSuccess ||
                  cudaDeviceSynchronize() != cudaSuccess)) {
         (void)cudaGetLastError();
         return QMV_ERR_CUDA;

@@ -229,6 +229,28 @@ __device__ __forceinline__ float half_bits_to_float(uint32_t bits)
     return __half2float(__ushort_as_half(static_cast<unsigned short>(bits & 0xFFFFu)));
 }
 
+// ------------------------------------------------------- greedy argmax --
+// Candidate (value, row) pairs: IEEE > on f32, ties to the lower row; bi < 0
+// means no candidate.  A 64-bit key orders candidates the same way: the
+// value's bits mapped to an order-preserving unsigned in the high word, the
+// complement of the row in the low word, so an atomic max over keys picks the
+// same winner in any order.
+__device__ __forceinline__ void argmax_merge(float &bv, int &bi, float ov, int oi)
+{
+    if (oi < 0) return;
+    if (bi < 0 || ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+    }
+}
+
+__device__ __forceinline__ unsigned long long argmax_key(float v, int row)
+{
+    const uint32_t u = v == 0.f ? 0u : __float_as_uint(v);            // -0 and +0 compare equal
+    const uint32_t hi = (u & 0x80000000u) ? ~u : (u | 0x80000000u);   // order-preserving for non-NaN
+    return ((unsigned long long)hi << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)row);
+}
+
 // ------------------------------------------------- multi-row warp reduction --
 // v[V] (V a power of two <= 32) holds this lane's partial sums of V different
 // outputs.  Each butterfly step halves the number of values a lane carries by

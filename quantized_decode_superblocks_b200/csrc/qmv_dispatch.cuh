@@ -260,6 +260,18 @@ cudaError_t launch_skc(const SkChainParams &p, int R, dim3 grid, size_t smem, cu
     }
 }
 
+// The one-launch MoE FFN step (cooperative: one CTA per SM, all resident).
+template <int FMT>
+cudaError_t launch_skm(const SkMoeParams &p, int R, dim3 grid, size_t smem, cudaStream_t st)
+{
+    static SmemCfg c1, c2;
+    switch (R) {
+    case 1: return launch_with(qmv_skm_kernel<FMT, 1>, c1, p, grid, smem, st, false, true, SK_THREADS);
+    case 2: return launch_with(qmv_skm_kernel<FMT, 2>, c2, p, grid, smem, st, false, true, SK_THREADS);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
 // The tensor-core several-token kernel (Q8_0): x in shared memory or through L2.
 template <int FMT>
 cudaError_t launch_tc(const TcParams &p, bool x_smem, dim3 grid, size_t smem, cudaStream_t st, bool pdl)

@@ -11,4 +11,5 @@ template cudaError_t launch_rw_mt<FMT_Q6_K>(const RwParams1 &, int, int, dim3, s
 template cudaError_t launch_tc<FMT_Q6_K>(const TcParams &, bool, dim3, size_t, cudaStream_t, bool);
 template cudaError_t launch_sk<FMT_Q6_K>(const SkParams &, int, int, dim3, size_t, cudaStream_t, bool);
 template cudaError_t launch_skc<FMT_Q6_K>(const SkChainParams &, int, dim3, size_t, cudaStream_t);
+template cudaError_t launch_skm<FMT_Q6_K>(const SkMoeParams &, int, dim3, size_t, cudaStream_t);
 }  // namespace qmv

@@ -18,22 +18,6 @@ namespace qmv {
 // row: the result does not depend on the order of the atomics.  The last CTA
 // of the token (an arrival counter) writes idx and puts the key and the
 // counter back to zero for the next call.
-__device__ __forceinline__ void argmax_merge(float &bv, int &bi, float ov, int oi)
-{
-    if (oi < 0) return;
-    if (bi < 0 || ov > bv || (ov == bv && oi < bi)) {
-        bv = ov;
-        bi = oi;
-    }
-}
-
-__device__ __forceinline__ unsigned long long argmax_key(float v, int row)
-{
-    const uint32_t u = v == 0.f ? 0u : __float_as_uint(v);            // -0 and +0 compare equal
-    const uint32_t hi = (u & 0x80000000u) ? ~u : (u | 0x80000000u);   // order-preserving for non-NaN
-    return ((unsigned long long)hi << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)row);
-}
-
 constexpr int ARGMAX_THREADS = 256;
 constexpr int ARGMAX_ROWS_PER_CTA = 2048;
 

@@ -60,6 +60,19 @@ constexpr int SK_PART = 2 * SK_NC * 4 * 2 * 4;   // partials [row][group][segmen
 
 enum { SK_PLAIN = 0, SK_SWIGLU = 1, SK_GATHER = 2 };
 
+// 1: the rows (and gate / up groups) of a row slot are decoded by one copy of
+// the decode body in a loop, keeping the kernels' code small (a kernel that
+// runs a few stages per launch spends much of its time fetching cold
+// instructions); 0: fully unrolled.
+#ifndef QMV_SK_ROW_LOOP
+#define QMV_SK_ROW_LOOP 0
+#endif
+#if QMV_SK_ROW_LOOP
+#define QMV_SK_ROWS_PRAGMA _Pragma("unroll 1")
+#else
+#define QMV_SK_ROWS_PRAGMA _Pragma("unroll")
+#endif
+
 // SK_PLAIN: 1 = one bulk copy and one "full" mbarrier per stage (all row slots
 // wait for the whole stage), 0 = one of each per row slot.
 #ifndef QMV_SK_STAGE_BARRIER
@@ -91,6 +104,13 @@ struct SkParams {
     int32_t rs_bytes;        // bytes of one row slot's region in a stage
     int32_t x_in_ring;       // 1: x is staged in ring slot S-1 before its first fill
     int32_t x_off;           // else: byte offset of the x area from the ring start
+    // PLAIN with a single K-segment: greedy argmax of y fused into the epilogue
+    // (amax_idx != NULL).  Every CTA folds its best (value, row) into *amax_key;
+    // the last CTA to arrive on *amax_done writes *amax_idx and puts both back
+    // to zero.
+    unsigned long long *amax_key;
+    unsigned *amax_done;
+    int32_t *amax_idx;
     int *err;
     uint32_t debug_extra_tx; // test hook: bytes expected per row slot beyond those copied (0 in use)
 };
@@ -324,6 +344,8 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_cons
     int slot = 0;
     uint32_t phase = 0, st = ring;
     int64_t r0 = r_begin;
+    float best_v = 0.f;                            // fused argmax: this lane's candidate
+    int best_i = -1;
     for (int i = 0; i < n_st; ++i) {
         const int ra = min(R, (int)min((int64_t)T, r_end - r0) - rs * R);     // rows of this row slot
         bool rowok = ra > 0;
@@ -337,17 +359,21 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_cons
         }
         float acc[V];
 #pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-            for (int k = 0; k < R; ++k) {
-                acc[g * R + k] = 0.f;
-                if (!dead && rowok && have && k < ra) {
-                    const uint32_t a = st + slice + (uint32_t)(g * R + k) * rb;
-                    if (FMT == FMT_Q8_0) acc[g * R + k] = q8_0_dot_pair(a, xp);
-                    else if (FMT == FMT_Q4_K) acc[g * R + k] = q4_k_dot1<false>(a, lane & 3, sel, xp, xsa, xsb);
-                    else acc[g * R + k] = q6_k_dot1(a, q6h, q6l, xp);
-                }
+        for (int j = 0; j < V; ++j) acc[j] = 0.f;
+        QMV_SK_ROWS_PRAGMA
+        for (int j = 0; j < V; ++j) {                // j = g * R + k
+            const int k = j % R;
+            float d = 0.f;
+            if (!dead && rowok && have && k < ra) {
+                const uint32_t a = st + slice + (uint32_t)j * rb;
+                if (FMT == FMT_Q8_0) d = q8_0_dot_pair(a, xp);
+                else if (FMT == FMT_Q4_K) d = q4_k_dot1<false>(a, lane & 3, sel, xp, xsa, xsb);
+                else d = q6_k_dot1(a, q6h, q6l, xp);
             }
+#pragma unroll
+            for (int j2 = 0; j2 < V; ++j2)
+                if (j2 == j) acc[j2] = d;
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8u * (uint32_t)slot);   // the stage may be refilled
         warp_transpose_reduce<V>(acc, lane);
@@ -357,7 +383,9 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_cons
                 const float u = __shfl_down_sync(0xFFFFFFFFu, acc[0], R << SH);    // the up value of row vk
                 if (leader && vg == 0 && vk < ra) p.y[row] = rowok ? acc[0] / (1.0f + expf(-acc[0])) * u : 0.f;
             } else if (leader && vk < ra) {
-                p.y[row] = MODE == SK_GATHER ? wseg[0] * acc[0] : acc[0];
+                const float v = MODE == SK_GATHER ? wseg[0] * acc[0] : acc[0];
+                p.y[row] = v;
+                if (MODE == SK_PLAIN && v == v) argmax_merge(best_v, best_i, v, (int)row);
             }
         } else {
             // partials of the row's K-segments, added in K order by segment 0
@@ -383,6 +411,40 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_cons
         }
         st = ring + (uint32_t)slot * pitch;
         r0 += T;
+    }
+    if (MODE == SK_PLAIN && p.amax_idx != nullptr) {
+        // CTA's best candidate (warp butterfly, then warp 0 over the warps'
+        // results in the partials area), one atomic per CTA
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1)
+            argmax_merge(best_v, best_i, __shfl_xor_sync(0xFFFFFFFFu, best_v, o), __shfl_xor_sync(0xFFFFFFFFu, best_i, o));
+        named_bar_sync(1, SK_NC * 32);            // every warp is past its last partials
+        if (lane == 0) {
+            sts_f32(part0 + 8u * (uint32_t)warp, best_v);
+            sts_f32(part0 + 8u * (uint32_t)warp + 4u, __int_as_float(best_i));
+        }
+        named_bar_sync(1, SK_NC * 32);
+        if (warp == 0) {
+            float v = 0.f;
+            int bi = -1;
+            if (lane < SK_NC) {
+                v = lds_f32(part0 + 8u * (uint32_t)lane);
+                bi = __float_as_int(lds_f32(part0 + 8u * (uint32_t)lane + 4u));
+            }
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1)
+                argmax_merge(v, bi, __shfl_xor_sync(0xFFFFFFFFu, v, o), __shfl_xor_sync(0xFFFFFFFFu, bi, o));
+            if (lane == 0) {
+                if (bi >= 0) atomicMax(p.amax_key, argmax_key(v, bi));
+                __threadfence();
+                if (atomicAdd(p.amax_done, 1u) == gridDim.x - 1u) {     // the last CTA
+                    __threadfence();
+                    const unsigned long long k = atomicExch(p.amax_key, 0ull);
+                    atomicExch(p.amax_done, 0u);
+                    *p.amax_idx = k ? (int32_t)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFull)) : -1;
+                }
+            }
+        }
     }
 }
 
@@ -571,14 +633,19 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skc_kernel(const __grid_con
             }
             float acc[R];
 #pragma unroll
+            for (int k = 0; k < R; ++k) acc[k] = 0.f;
+            QMV_SK_ROWS_PRAGMA
             for (int k = 0; k < R; ++k) {
-                acc[k] = 0.f;
+                float d = 0.f;
                 if (!dead && have && k < ra) {
                     const uint32_t ad = st + slice + (uint32_t)k * rb;
-                    if (FMT == FMT_Q8_0) acc[k] = q8_0_dot_pair(ad, xp);
-                    else if (FMT == FMT_Q4_K) acc[k] = q4_k_dot1<false>(ad, lane & 3, sel, xp, xsa, xsb);
-                    else acc[k] = q6_k_dot1(ad, q6h, q6l, xp);
+                    if (FMT == FMT_Q8_0) d = q8_0_dot_pair(ad, xp);
+                    else if (FMT == FMT_Q4_K) d = q4_k_dot1<false>(ad, lane & 3, sel, xp, xsa, xsb);
+                    else d = q6_k_dot1(ad, q6h, q6l, xp);
                 }
+#pragma unroll
+                for (int k2 = 0; k2 < R; ++k2)
+                    if (k2 == k) acc[k2] = d;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(empty0 + 8u * (uint32_t)slot);
@@ -611,5 +678,412 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skc_kernel(const __grid_con
 
 template <int FMT>
 cudaError_t launch_skc(const SkChainParams &p, int R, dim3 grid, size_t smem, cudaStream_t stream);
+
+// ---------------------------------------------------------------------------
+// The whole MoE FFN step in one cooperative launch (BebeLM page, §核心算子,
+// MoE前馈网络: sigmoid router, top-k by the biased score, weights normalised
+// over the unbiased scores; SwiGLU experts):
+//   1. every CTA routes on its own (the same f32 arithmetic as moe_route, so
+//      the same ids and weights) or reads given ids / weights; CTA 0 writes
+//      them out;
+//   2. h_k = silu(G_{ids[k]} x) * (U_{ids[k]} x) over this CTA's share of the
+//      n_sel * inter rows (the SK_SWIGLU form), stored to h;
+//   3. a grid barrier (h complete), then y = sum_k g_k D_{ids[k]} h_k over this
+//      CTA's share of the hidden rows (the SK_GATHER form).
+// The producer streams the stages of step 2 and then of step 3 without
+// waiting for the grid, so the routed down weights are already in shared
+// memory when the consumers cross the barrier.
+constexpr int SKM_MAX_EXPERTS = 256;          // routed on the device: eight per lane
+
+struct SkMoeParams {
+    const float *logits;     // [n_expert]: route on the device; NULL: ids / gw given
+    const float *bias;       // [n_expert]
+    int32_t *ids_out;        // routed: [n_sel] written by CTA 0 (or NULL)
+    float *g_out;            // routed: [n_sel] (or NULL)
+    const int32_t *ids;      // given ids [n_sel] (logits == NULL)
+    const float *gw;         // given weights [n_sel]
+    int32_t n_expert;
+    int32_t n_sel;
+    const uint8_t *G, *U;    // gate / up experts: [inter x hidden] each
+    int64_t gu_stride;
+    int64_t gu_row_bytes;
+    const uint8_t *D;        // down experts: [hidden x inter]
+    int64_t d_stride;
+    int64_t d_row_bytes;
+    int32_t hidden, inter;
+    const float *x;          // [hidden]
+    float *h;                // [n_sel][inter]
+    float *y;                // [hidden]
+    // step 2 (gate/up): K-segments of hidden, rows per stage, row slot bytes, CTA split
+    int32_t a_ksegs, a_seg_bytes, a_T, a_rs_bytes;
+    int64_t a_units_q;
+    int32_t a_units_r;
+    // step 3 (down): one K-segment per routed expert
+    int32_t b_ksegs, b_T, b_rs_bytes;
+    int64_t b_units_q;
+    int32_t b_units_r;
+    int32_t n_stage, stage_pitch, x_off;
+    unsigned *sync;          // {arrivals, exits} of the grid barrier (caller workspace), zero between launches
+    int *err;
+    uint32_t debug_extra_tx;
+};
+
+// Top-k routing by one warp, n_expert <= SKM_MAX_EXPERTS: the arithmetic and
+// tie rule of moe_route_kernel (sigmoid score s, biased b = s + bias, k rounds
+// of a warp argmax over b with ties to the lower index, g = s / sum of the
+// chosen s in k order).  Results in sids / sg (shared memory).
+__device__ __forceinline__ void skm_route(const float *logits, const float *bias, int n_expert, int top_k, int lane,
+                                          int *sids, float *sg)
+{
+    float sc[SKM_MAX_EXPERTS / 32], bb[SKM_MAX_EXPERTS / 32];
+    unsigned taken = 0;
+#pragma unroll
+    for (int j = 0; j < SKM_MAX_EXPERTS / 32; ++j) {
+        const int e = lane + 32 * j;
+        sc[j] = 0.f;
+        bb[j] = 0.f;
+        if (e < n_expert) {
+            const float s = 1.0f / (1.0f + expf(-logits[e]));
+            sc[j] = s;
+            bb[j] = s + bias[e];
+        }
+    }
+    float total = 0.f;
+    for (int k = 0; k < top_k; ++k) {
+        float bv = 0.f, sv = 0.f;
+        int bi = -1;
+#pragma unroll
+        for (int j = 0; j < SKM_MAX_EXPERTS / 32; ++j) {
+            const int e = lane + 32 * j;
+            if (e < n_expert && !((taken >> j) & 1u) && (bi < 0 || bb[j] > bv)) {
+                bv = bb[j];
+                bi = e;
+                sv = sc[j];
+            }
+        }
+        for (int o = 16; o >= 1; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, o);
+            const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
+            const float os = __shfl_xor_sync(0xFFFFFFFFu, sv, o);
+            if ((oi >= 0) && (bi < 0 || ov > bv || (ov == bv && oi < bi))) {
+                bv = ov;
+                bi = oi;
+                sv = os;
+            }
+        }
+        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+        if (lane == 0) {
+            sids[k] = bi;
+            sg[k] = sv;
+        }
+        total += sv;
+    }
+    __syncwarp();
+    if (lane < top_k) sg[lane] = sg[lane] / total;
+    __syncwarp();
+}
+
+template <int FMT, int R>
+__global__ void __launch_bounds__(SK_THREADS, 1) qmv_skm_kernel(const __grid_constant__ SkMoeParams p)
+{
+    static_assert(R == 1 || R == 2, "rows per consumer warp");
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int warp = (int)threadIdx.x >> 5, lane = (int)threadIdx.x & 31;
+    const uint32_t sraw = smem_addr(smem);
+    const uint32_t sbase = (sraw + 127u) & ~127u;          // the launch adds 128 spare bytes
+    uint8_t *const sgen = smem + (sbase - sraw);
+    const uint32_t full0 = sbase + SK_FULL_OFF, empty0 = sbase + SK_EMPTY_OFF;
+    volatile int *const abort_flag = reinterpret_cast<volatile int *>(sgen + SK_ABORT_OFF);
+    int *const sids = reinterpret_cast<int *>(sgen + SK_WSEG_OFF);              // [8]
+    float *const sg = reinterpret_cast<float *>(sgen + SK_WSEG_OFF + 32);      // [8] routed weights
+    float *const wseg = reinterpret_cast<float *>(sgen + SK_WSEG_OFF + 64);    // [12] segment weights (0: invalid)
+    const uint32_t part0 = sbase + (uint32_t)SK_HDR;
+    const uint32_t ring = part0 + (uint32_t)SK_PART;
+    const uint32_t xs = ring + (uint32_t)p.x_off;
+    const int S = p.n_stage;
+    const uint32_t pitch = (uint32_t)p.stage_pitch;
+    const int c = (int)blockIdx.x;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full0 + 8u * (uint32_t)s, 1);
+            mbar_init(empty0 + 8u * (uint32_t)s, SK_NC);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        if (p.logits) {
+            skm_route(p.logits, p.bias, p.n_expert, p.n_sel, lane, sids, sg);
+            if (c == 0 && lane < p.n_sel) {
+                if (p.ids_out) p.ids_out[lane] = sids[lane];
+                if (p.g_out) p.g_out[lane] = sg[lane];
+            }
+        } else if (lane < p.n_sel) {
+            sids[lane] = p.ids[lane];
+            sg[lane] = p.gw[lane];
+        }
+        __syncwarp();
+        if (lane < SK_MAX_KSEGS) {
+            const bool v = lane < p.n_sel && sids[lane] >= 0 && sids[lane] < p.n_expert;
+            wseg[lane] = v ? sg[lane] : 0.f;
+            if (lane < p.n_sel && !v && c == 0) atomicOr(p.err, DEVERR_EXPERT_ID);
+        }
+    }
+    __syncthreads();
+    auto valid = [&](int k) { return sids[k] >= 0 && sids[k] < p.n_expert; };
+
+    // this CTA's rows of step 2 (gate/up: n_sel * inter) and step 3 (down: hidden)
+    const int64_t a_u0 = (int64_t)c * p.a_units_q + min(c, p.a_units_r);
+    const int64_t a_begin = a_u0 * R;
+    const int64_t a_end = min((int64_t)p.n_sel * p.inter, (a_u0 + p.a_units_q + (c < p.a_units_r ? 1 : 0)) * R);
+    const int64_t b_u0 = (int64_t)c * p.b_units_q + min(c, p.b_units_r);
+    const int64_t b_begin = b_u0 * R;
+    const int64_t b_end = min((int64_t)p.hidden, (b_u0 + p.b_units_q + (c < p.b_units_r ? 1 : 0)) * R);
+    const int na = a_end > a_begin ? (int)((a_end - a_begin + p.a_T - 1) / p.a_T) : 0;
+    const int nb = b_end > b_begin ? (int)((b_end - b_begin + p.b_T - 1) / p.b_T) : 0;
+
+    if (warp == SK_NC) {
+        // ------------------------------------------------------ producer --
+        if (lane != 0) return;
+        bool ok = true;
+        int i = 0;
+        const uint64_t rga = (uint64_t)p.gu_row_bytes, rgb = (uint64_t)p.d_row_bytes;
+        for (; i < na + nb && ok; ++i) {
+            const int slot = i % S, round = i / S;
+            if (round > 0 && !mbar_wait_bounded_block(empty0 + 8u * (uint32_t)slot, (uint32_t)((round - 1) & 1))) {
+                atomicOr(p.err, DEVERR_TIMEOUT);
+                ok = false;
+                break;
+            }
+            if (*abort_flag) {
+                ok = false;
+                break;
+            }
+            if (round > 0) fence_proxy_async_smem();
+            const uint32_t st = ring + (uint32_t)slot * pitch;
+            const uint32_t full = full0 + 8u * (uint32_t)slot;
+            if (i < na) {
+                // step 2: R gate rows then the same R up rows of one expert per row slot
+                const int64_t r0 = a_begin + (int64_t)i * p.a_T;
+                const int tr = (int)min((int64_t)p.a_T, a_end - r0);
+                uint32_t total = 0;
+                for (int rs = 0; rs * R < tr; ++rs) {
+                    const int64_t v0 = r0 + rs * R;
+                    if (valid((int)(v0 / p.inter))) total += 2u * (uint32_t)min(R, tr - rs * R) * (uint32_t)rga;
+                }
+                mbar_arrive_expect_tx(full, total + p.debug_extra_tx);
+                for (int rs = 0; rs * R < tr; ++rs) {
+                    const int64_t v0 = r0 + rs * R;
+                    const int k = (int)(v0 / p.inter);
+                    if (!valid(k)) continue;
+                    const uint32_t bytes = (uint32_t)min(R, tr - rs * R) * (uint32_t)rga;
+                    const uint64_t off = (uint64_t)sids[k] * (uint64_t)p.gu_stride + (uint64_t)(v0 - (int64_t)k * p.inter) * rga;
+                    const uint32_t dst = st + (uint32_t)(rs * p.a_rs_bytes);
+                    bulk_g2s(dst, p.G + off, bytes, full);
+                    bulk_g2s(dst + (uint32_t)R * (uint32_t)rga, p.U + off, bytes, full);
+                }
+            } else {
+                // step 3: per row slot, R rows of every routed expert's down matrix
+                const int64_t r0 = b_begin + (int64_t)(i - na) * p.b_T;
+                const int tr = (int)min((int64_t)p.b_T, b_end - r0);
+                const int n_seg = min(p.n_sel, p.b_ksegs);
+                uint32_t total = 0;
+                for (int rs = 0; rs * R < tr; ++rs)
+                    for (int k = 0; k < n_seg; ++k)
+                        if (valid(k)) total += (uint32_t)min(R, tr - rs * R) * (uint32_t)rgb;
+                mbar_arrive_expect_tx(full, total + p.debug_extra_tx);
+                for (int rs = 0; rs * R < tr; ++rs) {
+                    const int64_t v0 = r0 + rs * R;
+                    const uint32_t bytes = (uint32_t)min(R, tr - rs * R) * (uint32_t)rgb;
+                    for (int k = 0; k < n_seg; ++k) {
+                        if (!valid(k)) continue;
+                        bulk_g2s(st + (uint32_t)(rs * p.b_rs_bytes) + (uint32_t)(k * R) * (uint32_t)rgb,
+                                 p.D + (uint64_t)sids[k] * (uint64_t)p.d_stride + (uint64_t)v0 * rgb, bytes, full);
+                    }
+                }
+            }
+        }
+        for (int j = max(0, i - S); j < i; ++j) {
+            if (!mbar_wait_bounded_block(full0 + 8u * (uint32_t)(j % S), (uint32_t)((j / S) & 1))) {
+                atomicOr(p.err, DEVERR_DRAIN);
+                break;
+            }
+        }
+        return;
+    }
+
+    // -------------------------------------------------------- consumers --
+    const Q4kSel sel = q4k_sel(lane & 3);
+    const int q6h = (lane >> 1) & 1, q6l = 16 * (lane & 1);
+    bool dead = false;
+    int i = 0;
+    auto wait_stage = [&](int slot, int i_) {
+        if (!dead && !__all_sync(0xFFFFFFFFu, mbar_wait_bounded_block(full0 + 8u * (uint32_t)slot, (uint32_t)((i_ / S) & 1)))) {
+            if (lane == 0) {
+                atomicOr(p.err, DEVERR_TIMEOUT);
+                *abort_flag = 1;
+            }
+            dead = true;
+        }
+    };
+    {
+        // ---- step 2: SwiGLU rows
+        sk_stage_x<false>(xs, p.x, 1, p.hidden >> 2, 0);
+        named_bar_sync(1, SK_NC * 32);
+        const int nk = p.a_ksegs;
+        const int ks = warp % nk, rs = warp / nk;
+        const int seg_cols = min(SK_SEG, p.hidden - ks * SK_SEG);
+        float2 xr[16][2];
+        float xsa = 0.f, xsb = 0.f;
+        rw_load_x_smem<FMT>(xs, ks, seg_cols, lane, xr, xsa, xsb);
+        auto xp = [&](int gq, float2 &x02, float2 &x13) {
+            x02 = xr[gq][0];
+            x13 = xr[gq][1];
+        };
+        const bool have = 64 * (lane + 1) <= seg_cols;
+        const uint32_t rb = (uint32_t)p.gu_row_bytes;
+        uint32_t slice = (uint32_t)(rs * p.a_rs_bytes) + (uint32_t)ks * (uint32_t)p.a_seg_bytes;
+        if (FMT == FMT_Q8_0) slice += 68u * (uint32_t)lane;
+        else if (FMT == FMT_Q4_K) slice += 144u * (uint32_t)(lane >> 2);
+        else slice += 210u * (uint32_t)(lane >> 2);
+        constexpr int V = 2 * R;
+        constexpr int SH = 5 - Log2<V>::v;
+        const bool leader = (lane & ((1 << SH) - 1)) == 0;
+        const int vg = (lane >> SH) / R, vk = (lane >> SH) % R;
+        for (int64_t r0 = a_begin; r0 < a_end; r0 += p.a_T, ++i) {
+            const int slot = i % S;
+            const uint32_t st = ring + (uint32_t)slot * pitch;
+            const int ra = min(R, (int)min((int64_t)p.a_T, a_end - r0) - rs * R);
+            const bool rowok = ra > 0 && valid((int)((r0 + rs * R) / p.inter));
+            wait_stage(slot, i);
+            float acc[V];
+#pragma unroll
+            for (int j = 0; j < V; ++j) acc[j] = 0.f;
+            QMV_SK_ROWS_PRAGMA
+            for (int j = 0; j < V; ++j) {            // j = g * R + k
+                const int k = j % R;
+                float d = 0.f;
+                if (!dead && rowok && have && k < ra) {
+                    const uint32_t a = st + slice + (uint32_t)j * rb;
+                    if (FMT == FMT_Q8_0) d = q8_0_dot_pair(a, xp);
+                    else if (FMT == FMT_Q4_K) d = q4_k_dot1<false>(a, lane & 3, sel, xp, xsa, xsb);
+                    else d = q6_k_dot1(a, q6h, q6l, xp);
+                }
+#pragma unroll
+                for (int j2 = 0; j2 < V; ++j2)
+                    if (j2 == j) acc[j2] = d;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty0 + 8u * (uint32_t)slot);
+            warp_transpose_reduce<V>(acc, lane);
+            const int64_t row = r0 + rs * R + vk;
+            if (nk == 1) {
+                const float u = __shfl_down_sync(0xFFFFFFFFu, acc[0], R << SH);
+                if (leader && vg == 0 && vk < ra) p.h[row] = rowok ? acc[0] / (1.0f + expf(-acc[0])) * u : 0.f;
+            } else {
+                const uint32_t pb = part0 + (uint32_t)(i & 1) * (uint32_t)(SK_PART / 2);
+                if (leader) sts_f32(pb + 4u * (uint32_t)(((rs * R + vk) * 2 + vg) * nk + ks), acc[0]);
+                named_bar_sync(2 + rs, 32 * nk);
+                if (ks == 0 && leader && vg == 0 && vk < ra) {
+                    float s0 = 0.f, s1 = 0.f;
+                    const uint32_t e0 = pb + 4u * (uint32_t)((rs * R + vk) * 2 * nk);
+                    for (int k2 = 0; k2 < nk; ++k2) {
+                        s0 += lds_f32(e0 + 4u * (uint32_t)k2);
+                        s1 += lds_f32(e0 + 4u * (uint32_t)(nk + k2));
+                    }
+                    p.h[row] = rowok ? s0 / (1.0f + expf(-s0)) * s1 : 0.f;
+                }
+            }
+        }
+    }
+    // ---- grid barrier: every CTA's h rows are written
+    named_bar_sync(1, SK_NC * 32);
+    if (threadIdx.x == 0) {
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" :: "l"(p.sync) : "memory");
+        const uint64_t t0 = global_timer_ns();
+        for (uint32_t n = 0;; ++n) {
+            unsigned v;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p.sync) : "memory");
+            if (v >= gridDim.x) break;
+            if ((n & 63u) == 63u && global_timer_ns() - t0 > 1000000000ull) {
+                atomicOr(p.err, DEVERR_TIMEOUT);
+                break;
+            }
+        }
+    }
+    named_bar_sync(1, SK_NC * 32);
+    {
+        // ---- step 3: y = sum_k g_k D_k h_k; K-segment ks is routed expert ks
+        const int n_xrow = min(p.n_sel, p.b_ksegs);
+        sk_stage_x<true>(xs, p.h, n_xrow, p.inter >> 2, p.inter);
+        named_bar_sync(1, SK_NC * 32);
+        const int nk = p.b_ksegs;
+        const int ks = warp % nk, rs = warp / nk;
+        const int seg_cols = ks < p.n_sel && valid(ks) ? p.inter : 0;
+        float2 xr[16][2];
+        float xsa = 0.f, xsb = 0.f;
+        rw_load_x_smem<FMT>(xs, ks, seg_cols, lane, xr, xsa, xsb);
+        auto xp = [&](int gq, float2 &x02, float2 &x13) {
+            x02 = xr[gq][0];
+            x13 = xr[gq][1];
+        };
+        const bool have = 64 * (lane + 1) <= seg_cols;
+        const uint32_t rb = (uint32_t)p.d_row_bytes;
+        uint32_t slice = (uint32_t)(rs * p.b_rs_bytes) + (uint32_t)(ks * R) * rb;
+        if (FMT == FMT_Q8_0) slice += 68u * (uint32_t)lane;
+        else if (FMT == FMT_Q4_K) slice += 144u * (uint32_t)(lane >> 2);
+        else slice += 210u * (uint32_t)(lane >> 2);
+        constexpr int SH = 5 - Log2<R>::v;
+        const bool leader = (lane & ((1 << SH) - 1)) == 0;
+        const int vk = lane >> SH;
+        for (int64_t r0 = b_begin; r0 < b_end; r0 += p.b_T, ++i) {
+            const int slot = i % S;
+            const uint32_t st = ring + (uint32_t)slot * pitch;
+            const int ra = min(R, (int)min((int64_t)p.b_T, b_end - r0) - rs * R);
+            wait_stage(slot, i);
+            float acc[R];
+#pragma unroll
+            for (int k = 0; k < R; ++k) acc[k] = 0.f;
+            QMV_SK_ROWS_PRAGMA
+            for (int k = 0; k < R; ++k) {
+                float d = 0.f;
+                if (!dead && have && k < ra) {
+                    const uint32_t a = st + slice + (uint32_t)k * rb;
+                    if (FMT == FMT_Q8_0) d = q8_0_dot_pair(a, xp);
+                    else if (FMT == FMT_Q4_K) d = q4_k_dot1<false>(a, lane & 3, sel, xp, xsa, xsb);
+                    else d = q6_k_dot1(a, q6h, q6l, xp);
+                }
+#pragma unroll
+                for (int k2 = 0; k2 < R; ++k2)
+                    if (k2 == k) acc[k2] = d;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty0 + 8u * (uint32_t)slot);
+            warp_transpose_reduce<R>(acc, lane);
+            const int64_t row = r0 + rs * R + vk;
+            const uint32_t pb = part0 + (uint32_t)(i & 1) * (uint32_t)(SK_PART / 2);
+            if (leader) sts_f32(pb + 4u * (uint32_t)((rs * R + vk) * nk + ks), acc[0]);
+            named_bar_sync(2 + rs, 32 * nk);
+            if (ks == 0 && leader && vk < ra) {
+                float s0 = 0.f;
+                for (int k2 = 0; k2 < nk; ++k2) s0 = fmaf(wseg[k2], lds_f32(pb + 4u * (uint32_t)((rs * R + vk) * nk + k2)), s0);
+                p.y[row] = s0;
+            }
+        }
+    }
+    // the last CTA to leave puts the barrier words back to zero for the next launch
+    named_bar_sync(1, SK_NC * 32);
+    if (threadIdx.x == 0) {
+        const unsigned old = atomicAdd(p.sync + 1, 1u);
+        if (old == gridDim.x - 1u) {
+            atomicExch(p.sync, 0u);
+            atomicExch(p.sync + 1, 0u);
+        }
+    }
+}
+
+template <int FMT>
+cudaError_t launch_skm(const SkMoeParams &p, int R, dim3 grid, size_t smem, cudaStream_t stream);
 
 }  // namespace qmv

@@ -88,6 +88,20 @@ def test_moe_argument_validation(L):
     assert ffn(gus=16) == SHAPE and ffn(h=A + 4) == ALIGN
 
 
+def test_moe_ffn_routed_argument_validation(L):
+    args = [A, A, 32, 4, 1, A, A, 1792 * 8 * 144, 1, A, 2048 * 7 * 144, 2048, 1792, A, A, A, A, A, A, None]
+    assert L.moe_ffn_routed(*args[:-2], None, None) == NULL          # no workspace
+    bad = list(args)
+    bad[3] = 9
+    assert L.moe_ffn_routed(*bad) == NSEL                             # top_k above 8
+    bad = list(args)
+    bad[12] = 1000
+    assert L.moe_ffn_routed(*bad) == SHAPE                            # inter not a multiple of 256
+    bad = list(args)
+    bad[18] = A + 4
+    assert L.moe_ffn_routed(*bad) == ALIGN                            # workspace alignment
+
+
 def test_multi_argument_validation(L):
     T = q.make_tasks([(A, 4, 256, A, A), (A, 8, 512, A, A)])
     assert L.qmv_multi(1, 1, None, 2, None) == NULL
@@ -132,6 +146,10 @@ def test_argmax_argument_validation(L):
     assert L.qmv_argmax(0, A, 4, 64, A, A, 9, A, None) == NTOK
     assert L.qmv_argmax(0, A + 8, 4, 64, A, A, 1, A, None) == ALIGN
     assert L.qmv_argmax(0, A, 4, 64, A, A, 1, A + 2, None) == ALIGN
+    # the workspace form: the same checks, then the workspace itself
+    assert L.qmv_argmax_ws(0, A, 4, 64, A, A, 1, A, None, None) == NULL
+    assert L.qmv_argmax_ws(0, A, 4, 64, A, A, 1, A, A + 4, None) == ALIGN
+    assert L.qmv_argmax_ws(0, A, 4, 64, A, A, 9, A, A, None) == NTOK
 
 
 def test_injected_launch_failure_is_reported(L):

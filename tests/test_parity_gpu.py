@@ -354,11 +354,40 @@ def _argmax_check(fmt, W, rows, cols, x, seed_note=""):
 
 
 @pytest.mark.parametrize("fmt,rows,cols,n_tok", [(Q6_K, 128000, 2048, 1), (Q6_K, 128000, 2048, 4),
-                                                 (Q8_0, 5000, 1024, 1), (Q4_K, 777, 512, 8)])
+                                                 (Q8_0, 5000, 1024, 1), (Q4_K, 777, 512, 8),
+                                                 (Q4_K, 3000, 2048, 1), (Q8_0, 300, 8192, 1)])
 def test_argmax_matches_logits_and_oracle(fmt, rows, cols, n_tok):
     W = synth.gen_blocks(fmt, rows, cols, 40 + n_tok, fmt)
     x = synth.gen_x(n_tok, cols, 41, n_tok)
     _argmax_check(fmt, W, rows, cols, x)
+    # one token on rows of <= 2048 columns: fused into the streaming kernel's epilogue
+    if n_tok == 1 and cols <= 2048:
+        assert q.qmv_debug_last_kernel() == q.KERNEL_STREAM
+
+
+def test_argmax_workspaces_on_two_streams():
+    # two argmax calls in flight at once on two streams, each with its own
+    # workspace: both choices correct, workspaces back to zero
+    shapes = [(Q6_K, 64000, 2048, 60), (Q8_0, 70000, 2048, 61)]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    ws = [torch.zeros(q.ARGMAX_WS_BYTES // 8, dtype=torch.int64, device="cuda") for _ in range(2)]
+    data = []
+    for fmt, rows, cols, seed in shapes:
+        W = synth.gen_blocks(fmt, rows, cols, seed, 0)
+        x = synth.gen_x(1, cols, seed, 1)
+        data.append((fmt, W, rows, cols, x, dev(W), dev(x), torch.empty((1, rows), device="cuda"),
+                     torch.full((1,), -7, dtype=torch.int32, device="cuda")))
+    torch.cuda.synchronize()
+    for rep in range(3):
+        for k, (fmt, W, rows, cols, x, Wd, xd, yd, idx) in enumerate(data):
+            q.qmv_argmax_ws(fmt, Wd, rows, cols, xd, yd, 1, idx, ws[k], streams[k])
+    torch.cuda.synchronize()
+    for k, (fmt, W, rows, cols, x, Wd, xd, yd, idx) in enumerate(data):
+        y = yd.cpu().numpy()
+        assert int(idx.cpu()[0]) == int(np.argmax(y[0]))
+        ref, bound = oracle.qmv_rows(fmt, W, rows, cols, np.array([int(idx.cpu()[0])]), x)
+        within(y[:, [int(idx.cpu()[0])]], ref, bound)
+        assert int(ws[k].abs().sum().cpu()) == 0
 
 
 def test_argmax_ties_go_to_the_lower_row_and_nan_is_skipped():
@@ -670,3 +699,43 @@ def test_moe_ffn_formats_and_a_bad_expert_id(fmt, hidden, inter, kernel):
         bnd += abs(float(g32[k])) * b[0]
     within(yy[None, :], yref[None, :], bnd[None, :])
     assert np.isfinite(ref["y"]).all()
+
+
+@pytest.mark.parametrize("fmt,n_expert,hidden,inter,top_k,seed", [(Q4_K, 32, 2048, 1792, 4, 3),
+                                                                  (Q8_0, 16, 1024, 512, 3, 71),
+                                                                  (Q4_K, 8, 4096, 768, 6, 72),
+                                                                  (Q4_K, 8, 512, 2304, 4, 73)])
+def test_moe_ffn_routed_matches_route_then_ffn(fmt, n_expert, hidden, inter, top_k, seed):
+    # the one-launch step (router in every CTA, grid barrier between the two
+    # products) against moe_route followed by moe_ffn: the same ids and
+    # weights, and bit-identical h and y (the same decode and reduction order);
+    # expert rows of 2304 columns take the two-launch path instead
+    gus, ds = synth.matrix_bytes(fmt, inter, hidden), synth.matrix_bytes(fmt, hidden, inter)
+    gate = dev(synth.gen_blocks(fmt, inter * n_expert, hidden, seed, 1))
+    up = dev(synth.gen_blocks(fmt, inter * n_expert, hidden, seed, 2))
+    down = dev(synth.gen_blocks(fmt, hidden * n_expert, inter, seed, 3))
+    ws = torch.zeros(q.MOE_WS_BYTES // 8, dtype=torch.int64, device="cuda")
+    for call in range(2):
+        logits, bias = synth.gen_router(n_expert, seed + call, 5)
+        lg, bs = dev(logits), dev(bias)
+        x = dev(synth.gen_x(1, hidden, seed + call, 4)[0])
+        ids_a = torch.empty(top_k, dtype=torch.int32, device="cuda")
+        g_a = torch.empty(top_k, device="cuda")
+        h_a = torch.empty((top_k, inter), device="cuda")
+        y_a = torch.empty(hidden, device="cuda")
+        q.moe_route(lg, bs, n_expert, top_k, ids_a, g_a)
+        q.moe_ffn(fmt, gate, up, gus, fmt, down, ds, n_expert, ids_a, g_a, top_k, hidden, inter, x, h_a, y_a)
+        ids_b = torch.full((top_k,), -9, dtype=torch.int32, device="cuda")
+        g_b = torch.full((top_k,), float("nan"), device="cuda")
+        h_b = torch.full((top_k, inter), float("nan"), device="cuda")
+        y_b = torch.full((hidden,), float("nan"), device="cuda")
+        q.moe_ffn_routed(lg, bs, n_expert, top_k, fmt, gate, up, gus, fmt, down, ds, hidden, inter, x,
+                         ids_b, g_b, h_b, y_b, ws)
+        assert q.qmv_debug_last_kernel() == (q.KERNEL_STREAM if inter <= 2048 else q.KERNEL_GENERAL)
+        torch.cuda.synchronize()
+        assert ids_b.cpu().tolist() == ids_a.cpu().tolist()
+        assert np.array_equal(g_b.cpu().numpy().view(np.uint32), g_a.cpu().numpy().view(np.uint32))
+        assert np.array_equal(h_b.cpu().numpy().view(np.uint32), h_a.cpu().numpy().view(np.uint32))
+        assert np.array_equal(y_b.cpu().numpy().view(np.uint32), y_a.cpu().numpy().view(np.uint32))
+        assert int(ws.abs().sum().cpu()) == 0
+    assert q.qmv_check() == 0
