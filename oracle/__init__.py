@@ -17,7 +17,7 @@ import numpy as np
 
 from .build import build_oracle, library_path
 
-Q8_0, Q4_K, Q6_K = 0, 1, 2
+Q8_0, Q4_K, Q6_K, Q4_0, Q5_K = 0, 1, 2, 3, 4
 
 _lib = None
 
@@ -40,7 +40,8 @@ def lib() -> ctypes.CDLL:
         L.orc_half_to_float.restype = ctypes.c_float
         L.orc_block_weights.argtypes = [c_int]
         L.orc_block_bytes.argtypes = [c_int]
-        for name in ("orc_dequant_block_q8_0", "orc_dequant_block_q4_k", "orc_dequant_block_q6_k"):
+        for name in ("orc_dequant_block_q8_0", "orc_dequant_block_q4_k", "orc_dequant_block_q6_k",
+                     "orc_dequant_block_q4_0", "orc_dequant_block_q5_k"):
             getattr(L, name).argtypes = [u8p, f32p]
             getattr(L, name).restype = None
         L.orc_dequant.argtypes = [c_int, u8p, i64, i64, f32p]
@@ -87,7 +88,8 @@ def dequant_block(fmt: int, blk: np.ndarray) -> np.ndarray:
     assert blk.size == block_bytes(fmt)
     out = np.empty(block_weights(fmt), dtype=np.float32)
     fn = {Q8_0: lib().orc_dequant_block_q8_0, Q4_K: lib().orc_dequant_block_q4_k,
-          Q6_K: lib().orc_dequant_block_q6_k}[fmt]
+          Q6_K: lib().orc_dequant_block_q6_k, Q4_0: lib().orc_dequant_block_q4_0,
+          Q5_K: lib().orc_dequant_block_q5_k}[fmt]
     fn(_p(blk, ctypes.c_uint8), _p(out, ctypes.c_float))
     return out
 

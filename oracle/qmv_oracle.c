@@ -65,6 +65,8 @@ int orc_block_weights(int fmt)
     case ORC_Q8_0: return 32;
     case ORC_Q4_K: return 256;
     case ORC_Q6_K: return 256;
+    case ORC_Q4_0: return 32;
+    case ORC_Q5_K: return 256;
     default: return 0;
     }
 }
@@ -75,6 +77,8 @@ int orc_block_bytes(int fmt)
     case ORC_Q8_0: return 2 + 32;            /* d, q[32]                   */
     case ORC_Q4_K: return 2 + 2 + 12 + 128;  /* d, dmin, scales[12], qs[128] */
     case ORC_Q6_K: return 128 + 64 + 16 + 2; /* ql, qh, scales[16], d      */
+    case ORC_Q4_0: return 2 + 16;            /* d, qs[16]                  */
+    case ORC_Q5_K: return 2 + 2 + 12 + 32 + 128; /* d, dmin, scales[12], qh[32], qs[128] */
     default: return 0;
     }
 }
@@ -189,6 +193,86 @@ void orc_dequant_block_q6_k(const uint8_t *blk, float *w)
     }
 }
 
+/* ---------------------------------------------------------------- Q4_0 -- */
+
+/* Q4_0 block, 18 bytes ([Flare] §量化技术的全面支持: the Q4_0 .. Q8_1 family):
+ *   bytes 0-1   fp16 d
+ *   bytes 2-17  qs[16]: byte qs[j] holds weight j in its low nibble and
+ *               weight j + 16 in its high nibble (j = 0..15)
+ *   w_i = d * (q_i - 8)                      (q_i = 0..15, so -8..7)
+ * 11 + 4 significant bits: exact in f32.
+ * Pinned by: per-slot round trips (every position x all 16 values), second
+ * decoder, a hand-worked block, closed forms. */
+void orc_dequant_block_q4_0(const uint8_t *blk, float *w)
+{
+    float d = half_at(blk);
+    const uint8_t *qs = blk + 2;
+    for (int j = 0; j < 16; ++j) {
+        int lo = qs[j] & 15;
+        int hi = qs[j] >> 4;
+        w[j] = d * (float)(lo - 8);
+        w[j + 16] = d * (float)(hi - 8);
+    }
+}
+
+/* ---------------------------------------------------------------- Q5_K -- */
+
+/* Q5_K superblock, 176 bytes ([Flare] §量化技术的全面支持: K-quants Q2K .. Q6K):
+ *   bytes 0-1     fp16 d
+ *   bytes 2-3     fp16 dmin
+ *   bytes 4-15    scales[12]: the eight 6-bit scales sc_j and mins m_j, packed
+ *                 exactly as in Q4_K
+ *   bytes 16-47   qh[32]: the fifth bit of every quant
+ *   bytes 48-175  qs[128]: the low four bits, laid out as the Q4_K nibbles
+ * For chunk c = 0..3 and l = 0..31:
+ *   weight 64c + l      : low nibble of qs[32c + l], fifth bit = bit 2c   of qh[l]
+ *   weight 64c + 32 + l : high nibble of qs[32c + l], fifth bit = bit 2c+1 of qh[l]
+ *   q_i = low4 + 16 * bit5                  (0..31)
+ * Weight i lies in sub-block j = i / 32 and
+ *   w_i = d * sc_j * q_i - dmin * m_j.
+ * d*sc_j (17 bits), (d*sc_j)*q_i (22 bits) and dmin*m_j (17 bits) are exact in
+ * f32; only the final subtraction rounds (to nearest even).
+ * Pinned by: per-slot round trips (every sc/m slot x all 64 values, every
+ * position x all 32 quants), second decoder, hand-worked blocks, closed
+ * forms. */
+void orc_dequant_block_q5_k(const uint8_t *blk, float *w)
+{
+    float d = half_at(blk + 0);
+    float dmin = half_at(blk + 2);
+    const uint8_t *scales = blk + 4;
+    const uint8_t *qh = blk + 16;
+    const uint8_t *qs = blk + 48;
+
+    int sc[8], m[8];
+    for (int j = 0; j < 8; ++j) {
+        if (j < 4) {
+            sc[j] = scales[j] & 63;
+            m[j] = scales[j + 4] & 63;
+        } else {
+            sc[j] = (scales[j + 4] & 15) | ((scales[j - 4] >> 6) << 4);
+            m[j] = (scales[j + 4] >> 4) | ((scales[j] >> 6) << 4);
+        }
+    }
+
+    int q[256];
+    for (int c = 0; c < 4; ++c) {
+        for (int l = 0; l < 32; ++l) {
+            uint8_t b = qs[32 * c + l];
+            int b5lo = (qh[l] >> (2 * c)) & 1;
+            int b5hi = (qh[l] >> (2 * c + 1)) & 1;
+            q[64 * c + l] = (b & 15) + 16 * b5lo;
+            q[64 * c + 32 + l] = (b >> 4) + 16 * b5hi;
+        }
+    }
+
+    for (int i = 0; i < 256; ++i) {
+        int j = i / 32;
+        float t1 = d * (float)sc[j];
+        float t2 = dmin * (float)m[j];
+        w[i] = t1 * (float)q[i] - t2;
+    }
+}
+
 /* ----------------------------------------------------------- matrices -- */
 
 static int shape_ok(int fmt, int64_t rows, int64_t cols)
@@ -210,7 +294,9 @@ static void dequant_row(int fmt, const uint8_t *W, int64_t cols, int64_t r, floa
         float *o = out + b * bw;
         if (fmt == ORC_Q8_0) orc_dequant_block_q8_0(blk, o);
         else if (fmt == ORC_Q4_K) orc_dequant_block_q4_k(blk, o);
-        else orc_dequant_block_q6_k(blk, o);
+        else if (fmt == ORC_Q6_K) orc_dequant_block_q6_k(blk, o);
+        else if (fmt == ORC_Q4_0) orc_dequant_block_q4_0(blk, o);
+        else orc_dequant_block_q5_k(blk, o);
     }
 }
 

@@ -5,8 +5,9 @@
  * shares no source, header, table or helper with the CUDA library.
  *
  * What it computes, and where that is stated:
- *   - GGUF block formats Q8_0 / Q4_K / Q6_K, dequantized at run time to f32,
- *     activations kept in f32:
+ *   - GGUF block formats Q8_0 / Q4_K / Q6_K (and Q4_0 / Q5_K, named among the
+ *     formats FlareLLM supports), dequantized at run time to f32, activations
+ *     kept in f32:
  *       BebeLM：纯Rust实现的端侧大模型推理引擎, §量化格式支持 (Q4_K: 256
  *       weights per superblock in 144 bytes; Q6_K for sensitive tensors;
  *       dequantization at run time, f32 activations);
@@ -34,7 +35,7 @@
 extern "C" {
 #endif
 
-enum { ORC_Q8_0 = 0, ORC_Q4_K = 1, ORC_Q6_K = 2 };
+enum { ORC_Q8_0 = 0, ORC_Q4_K = 1, ORC_Q6_K = 2, ORC_Q4_0 = 3, ORC_Q5_K = 4 };
 
 /* IEEE binary16 bit pattern -> f32, decoded bit by bit (exact). */
 float orc_half_to_float(uint16_t h);
@@ -48,6 +49,8 @@ int orc_block_bytes(int fmt);
 void orc_dequant_block_q8_0(const uint8_t *blk, float *w);
 void orc_dequant_block_q4_k(const uint8_t *blk, float *w);
 void orc_dequant_block_q6_k(const uint8_t *blk, float *w);
+void orc_dequant_block_q4_0(const uint8_t *blk, float *w);
+void orc_dequant_block_q5_k(const uint8_t *blk, float *w);
 
 /* Dequantize a dense row-major matrix of rows x cols weights (row r starts at
  * byte r * (cols / block_weights) * block_bytes) into out[rows][cols].

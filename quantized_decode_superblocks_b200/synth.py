@@ -17,6 +17,13 @@ Field byte ranges per block (GGUF layout, little-endian):
   Q6_K (210 B): [0,192) ql / qh: uniform random bytes, so the 6-bit quants are
                 U{0..63}; [192,208) int8 scales ~ U{-64..63};
                 [208,210) fp16 d ~ U[1e-4, 2e-3].
+  Q4_0 (18 B):  [0,2) fp16 d ~ U[1e-3, 2e-2]; [2,18) packed nibbles: uniform
+                random bytes, so q ~ U{0..15}.
+  Q5_K (176 B): [0,2) fp16 d, [2,4) fp16 dmin, both ~ U[1e-3, 1e-2];
+                [4,16) scales, [16,48) fifth bits, [48,176) nibbles: uniform
+                random bytes, so sc, m ~ U{0..63} and q ~ U{0..31}.
+No page or workload fixes distributions for Q4_0 and Q5_K; these mirror Q8_0
+and Q4_K.
 Uniform reals are drawn in f64 and rounded to fp16 by numpy (round to nearest
 even).  Activations and router logits are f32 N(0, 1); the expert bias is
 f32 N(0, 0.1).
@@ -25,10 +32,10 @@ from __future__ import annotations
 
 import numpy as np
 
-Q8_0, Q4_K, Q6_K = 0, 1, 2
-FORMAT_NAMES = {Q8_0: "Q8_0", Q4_K: "Q4_K", Q6_K: "Q6_K"}
-BLOCK_WEIGHTS = {Q8_0: 32, Q4_K: 256, Q6_K: 256}
-BLOCK_BYTES = {Q8_0: 34, Q4_K: 144, Q6_K: 210}
+Q8_0, Q4_K, Q6_K, Q4_0, Q5_K = 0, 1, 2, 3, 4
+FORMAT_NAMES = {Q8_0: "Q8_0", Q4_K: "Q4_K", Q6_K: "Q6_K", Q4_0: "Q4_0", Q5_K: "Q5_K"}
+BLOCK_WEIGHTS = {Q8_0: 32, Q4_K: 256, Q6_K: 256, Q4_0: 32, Q5_K: 256}
+BLOCK_BYTES = {Q8_0: 34, Q4_K: 144, Q6_K: 210, Q4_0: 18, Q5_K: 176}
 
 
 def rng(seed: int, tensor_id: int) -> np.random.Generator:
@@ -64,6 +71,11 @@ def gen_blocks(fmt: int, rows: int, cols: int, seed: int, tensor_id: int) -> np.
         sc = g.integers(-64, 64, size=(nblk, 16), dtype=np.int8)
         buf[:, 192:208] = sc.view(np.uint8)
         buf[:, 208:210] = _fp16_uniform(g, nblk, 1e-4, 2e-3)
+    elif fmt == Q4_0:
+        buf[:, 0:2] = _fp16_uniform(g, nblk, 1e-3, 2e-2)
+    elif fmt == Q5_K:
+        buf[:, 0:2] = _fp16_uniform(g, nblk, 1e-3, 1e-2)
+        buf[:, 2:4] = _fp16_uniform(g, nblk, 1e-3, 1e-2)
     else:
         raise ValueError("unknown format")
     return buf.reshape(-1)

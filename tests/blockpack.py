@@ -67,6 +67,33 @@ def pack_q6_k(d_bits: int, scales, q) -> np.ndarray:
     return out
 
 
+def pack_q4_0(d_bits: int, q) -> np.ndarray:
+    q = [int(v) for v in q]
+    assert len(q) == 32 and all(0 <= v < 16 for v in q)
+    out = np.zeros(18, dtype=np.uint8)
+    out[0], out[1] = d_bits & 0xFF, d_bits >> 8
+    for i, v in enumerate(q):
+        # weights 0..15 in the low nibbles of bytes 2..17, weights 16..31 in the high ones
+        out[2 + (i % 16)] |= v << (4 * (i // 16))
+    return out
+
+
+def pack_q5_k(d_bits: int, dmin_bits: int, sc, m, q) -> np.ndarray:
+    """Q5_K: the Q4_K header and scale packing, 32 bytes of fifth bits, then the
+    low nibbles in the Q4_K arrangement."""
+    q = [int(v) for v in q]
+    assert len(q) == 256 and all(0 <= v < 32 for v in q)
+    lo4 = pack_q4_k(d_bits, dmin_bits, sc, m, [v & 15 for v in q])
+    out = np.zeros(176, dtype=np.uint8)
+    out[0:16] = lo4[0:16]
+    out[48:176] = lo4[16:144]
+    for i, v in enumerate(q):
+        c, r = divmod(i, 64)
+        hi, l = divmod(r, 32)
+        out[16 + l] |= (v >> 4) << (2 * c + hi)
+    return out
+
+
 # ----------------------------------------------------------- second decoder
 
 def _bits(blk: np.ndarray, start: int, n: int) -> int:
@@ -125,6 +152,23 @@ def fields_q6_k(blk):
             "q": q}
 
 
+def fields_q4_0(blk):
+    return {"d": _half(_bits(blk, 0, 16)),
+            "q": [_bits(blk, 16 + 8 * (i % 16) + 4 * (i // 16), 4) for i in range(32)]}
+
+
+def fields_q5_k(blk):
+    # the scale / min fields sit where Q4_K has them; the nibbles start at byte 48
+    f = fields_q4_k(np.concatenate([blk[0:16], blk[48:176]]))
+    q = []
+    for i in range(256):
+        c, r = divmod(i, 64)
+        hi, l = divmod(r, 32)
+        q.append(f["q"][i] + 16 * _bits(blk, 8 * (16 + l) + 2 * c + hi, 1))
+    f["q"] = q
+    return f
+
+
 def decode2(fmt: int, blk) -> np.ndarray:
     """Second decoder: fields by bit index, then the weight formula evaluated in
     f64 and rounded once to f32 (the products are exact, see the oracle)."""
@@ -133,6 +177,13 @@ def decode2(fmt: int, blk) -> np.ndarray:
         return np.array([f["d"] * q for q in f["q"]], dtype=np.float64).astype(np.float32)
     if fmt == 1:
         f = fields_q4_k(blk)
+        return np.array([f["d"] * f["sc"][i // 32] * f["q"][i] - f["dmin"] * f["m"][i // 32]
+                         for i in range(256)], dtype=np.float64).astype(np.float32)
+    if fmt == 3:
+        f = fields_q4_0(blk)
+        return np.array([f["d"] * (q - 8) for q in f["q"]], dtype=np.float64).astype(np.float32)
+    if fmt == 4:
+        f = fields_q5_k(blk)
         return np.array([f["d"] * f["sc"][i // 32] * f["q"][i] - f["dmin"] * f["m"][i // 32]
                          for i in range(256)], dtype=np.float64).astype(np.float32)
     f = fields_q6_k(blk)
@@ -195,4 +246,30 @@ def pack_q6_k_many(d_bits, scales, q) -> np.ndarray:
             out[:, 128 + 32 * h:160 + 32 * h] |= (qq[:, h, t, :] >> 4) << (2 * t)
     out[:, 192:208] = scales & 0xFF
     out[:, 208], out[:, 209] = d_bits & 0xFF, d_bits >> 8
+    return out.astype(np.uint8).reshape(-1)
+
+
+def pack_q4_0_many(d_bits, q) -> np.ndarray:
+    d_bits = np.asarray(d_bits, dtype=np.uint16)
+    q = np.asarray(q, dtype=np.int64)
+    n = d_bits.shape[0]
+    assert q.shape == (n, 32) and q.min() >= 0 and q.max() < 16
+    out = np.zeros((n, 18), dtype=np.int64)
+    out[:, 0], out[:, 1] = d_bits & 0xFF, d_bits >> 8
+    out[:, 2:] = q[:, :16] | (q[:, 16:] << 4)
+    return out.astype(np.uint8).reshape(-1)
+
+
+def pack_q5_k_many(d_bits, dmin_bits, sc, m, q) -> np.ndarray:
+    q = np.asarray(q, dtype=np.int64)
+    n = q.shape[0]
+    assert q.shape == (n, 256) and q.min() >= 0 and q.max() < 32
+    lo4 = pack_q4_k_many(d_bits, dmin_bits, sc, m, q & 15).reshape(n, 144)
+    out = np.zeros((n, 176), dtype=np.int64)
+    out[:, 0:16] = lo4[:, 0:16]
+    out[:, 48:176] = lo4[:, 16:144]
+    qq = (q >> 4).reshape(n, 4, 2, 32)            # [chunk c][low / high nibble][l]
+    for c in range(4):
+        for hi in range(2):
+            out[:, 16:48] |= qq[:, c, hi, :] << (2 * c + hi)
     return out.astype(np.uint8).reshape(-1)
