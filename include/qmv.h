@@ -1,7 +1,7 @@
 /*
  * qmv.h -- C ABI of libqmv.so: the decode-step matrix-vector product of a
- * GGUF block-quantized weight matrix (Q8_0, Q4_K, Q6_K) with f32 activations,
- * dequantized on the fly, on one NVIDIA B200 (sm_100a).
+ * GGUF block-quantized weight matrix (Q8_0, Q4_0, Q4_K, Q5_K, Q6_K) with f32
+ * activations, dequantized on the fly, on one NVIDIA B200 (sm_100a).
  *
  * Sources (page title, section):
  *   BebeLM：纯Rust实现的端侧大模型推理引擎
@@ -15,7 +15,7 @@
  *     §推理层面的深度优化 -- fused QKV and gate/up matvecs (43% fewer matvec
  *       calls per layer); n-gram speculative decoding (several tokens checked
  *       in one pass over the weights); zero-allocation forward pass.
- *     §计算路径的智能选择, §量化技术的全面支持 -- Q8_0 and the K-quants.
+ *     §计算路径的智能选择, §量化技术的全面支持 -- Q8_0, Q4_0 and the K-quants.
  *     §生态对比与定位 -- standard GGUF files.
  *
  * Block layouts (GGUF, little-endian, fp16 = IEEE binary16):
@@ -24,6 +24,12 @@
  *                             w = d*sc_j*q - dmin*m_j, j = sub-block of 32
  *   Q6_K 256 weights / 210 B: ql[128] | qh[64] | scales[16] int8 | d
  *                             w = d*scales[i/16]*(q - 32), q = 6 bits
+ *   Q4_0  32 weights / 18 B : d | qs[16]; byte j holds weight j (low nibble)
+ *                             and weight j+16 (high nibble);  w = d*(q - 8)
+ *   Q5_K 256 weights / 176 B: d | dmin | scales[12] (as Q4_K) | qh[32] | qs[128]
+ *                             (as Q4_K); the fifth bit of weight 64c + l is
+ *                             bit 2c of qh[l], of weight 64c + 32 + l bit 2c+1;
+ *                             w = d*sc_j*q - dmin*m_j
  * A matrix is rows x cols weights stored densely row-major: row r starts at
  * byte r * (cols / block_weights) * block_bytes; no padding.
  *
@@ -62,7 +68,7 @@ extern "C" {
 /* Same type as cudaStream_t, without including the CUDA headers. */
 typedef struct CUstream_st *qmv_stream_t;
 
-typedef enum { QMV_Q8_0 = 0, QMV_Q4_K = 1, QMV_Q6_K = 2 } qmv_fmt;
+typedef enum { QMV_Q8_0 = 0, QMV_Q4_K = 1, QMV_Q6_K = 2, QMV_Q4_0 = 3, QMV_Q5_K = 4 } qmv_fmt;
 
 typedef enum {
     QMV_OK = 0,
@@ -265,7 +271,7 @@ int qmv_argmax(int fmt, const void *W_blocks, int64_t rows, int64_t cols,
 
 /* Dequantize the whole matrix to f32: out[rows][cols].  The values are
  * bit-exact f32 evaluations of the block formulas above (every product in
- * them is exact in f32; Q4_K rounds once, in the subtraction). */
+ * them is exact in f32; Q4_K and Q5_K round once, in the subtraction). */
 int qmv_dequant(int fmt, const void *W_blocks, int64_t rows, int64_t cols,
                 float *out, qmv_stream_t stream);
 

@@ -1,7 +1,7 @@
 """quantized_decode_superblocks_b200 -- Python binding of libqmv.so.
 
-The decode-step matvec of GGUF block-quantized weights (Q8_0, Q4_K, Q6_K) with
-f32 activations, dequantized on the fly, on an NVIDIA B200 (sm_100a).  Every
+The decode-step matvec of GGUF block-quantized weights (Q8_0, Q4_0, Q4_K, Q5_K,
+Q6_K) with f32 activations, dequantized on the fly, on an NVIDIA B200 (sm_100a).  Every
 step runs in the library's CUDA kernels; this module only marshals arguments
 (tensor data pointers, sizes, the current CUDA stream) through ctypes to the C
 ABI declared in ``include/qmv.h``, with the same function names.  PyTorch
@@ -13,7 +13,7 @@ from __future__ import annotations
 import ctypes
 import os
 
-from .synth import Q4_K, Q6_K, Q8_0  # noqa: F401  (format ids)
+from .synth import Q4_0, Q4_K, Q5_K, Q6_K, Q8_0  # noqa: F401  (format ids)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libqmv.so")

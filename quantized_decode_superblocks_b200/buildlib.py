@@ -18,7 +18,7 @@ ROOT = os.path.dirname(HERE)
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libqmv.so")
 
-SOURCES = ["qmv_api.cu", "qmv_fmt_q8_0.cu", "qmv_fmt_q4_k.cu", "qmv_fmt_q6_k.cu"]
+SOURCES = ["qmv_api.cu", "qmv_fmt_q8_0.cu", "qmv_fmt_q4_k.cu", "qmv_fmt_q6_k.cu", "qmv_fmt_q4_0.cu", "qmv_fmt_q5_k.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
                      "-I", os.path.join(ROOT, "include"), "--expt-relaxed-constexpr"]

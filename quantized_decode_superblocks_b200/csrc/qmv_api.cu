@@ -5,6 +5,7 @@
 #include <climits>
 #include <atomic>
 #include <mutex>
+#include <type_traits>
 #include <vector>
 
 #include "../../include/qmv.h"
@@ -72,9 +73,40 @@ int cuda_fail(cudaError_t e)
     return QMV_ERR_CUDA;
 }
 
-int block_weights(int fmt) { return fmt == QMV_Q8_0 ? 32 : (fmt == QMV_Q4_K || fmt == QMV_Q6_K) ? 256 : 0; }
-int block_bytes(int fmt) { return fmt == QMV_Q8_0 ? 34 : fmt == QMV_Q4_K ? 144 : fmt == QMV_Q6_K ? 210 : 0; }
-bool fmt_ok(int fmt) { return fmt == QMV_Q8_0 || fmt == QMV_Q4_K || fmt == QMV_Q6_K; }
+int block_weights(int fmt)
+{
+    return (fmt == QMV_Q8_0 || fmt == QMV_Q4_0) ? 32 : (fmt == QMV_Q4_K || fmt == QMV_Q5_K || fmt == QMV_Q6_K) ? 256 : 0;
+}
+int block_bytes(int fmt)
+{
+    switch (fmt) {
+    case QMV_Q8_0: return 34;
+    case QMV_Q4_0: return 18;
+    case QMV_Q4_K: return 144;
+    case QMV_Q5_K: return 176;
+    case QMV_Q6_K: return 210;
+    default: return 0;
+    }
+}
+bool fmt_ok(int fmt) { return block_bytes(fmt) != 0; }
+// 32-weight blocks: a one-token lane slice of 64 columns is a block pair
+bool small_blk(int fmt) { return fmt == QMV_Q8_0 || fmt == QMV_Q4_0; }
+// the formats the warp-ring and tensor-core kernels are built for
+bool rw_tc_fmt(int fmt) { return fmt == QMV_Q8_0 || fmt == QMV_Q4_K || fmt == QMV_Q6_K; }
+
+// Calls f(std::integral_constant<int, FMT>) for block format fmt (validated:
+// the QMV_* ids equal the kernels' FMT_* ids).
+template <class F>
+auto by_fmt(int fmt, F &&f)
+{
+    switch (fmt) {
+    case QMV_Q8_0: return f(std::integral_constant<int, FMT_Q8_0>{});
+    case QMV_Q4_0: return f(std::integral_constant<int, FMT_Q4_0>{});
+    case QMV_Q4_K: return f(std::integral_constant<int, FMT_Q4_K>{});
+    case QMV_Q5_K: return f(std::integral_constant<int, FMT_Q5_K>{});
+    default: return f(std::integral_constant<int, FMT_Q6_K>{});
+    }
+}
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 int pow2ceil(int v) { int p = 1; while (p < v) p <<= 1; return p; }
@@ -131,8 +163,8 @@ int make_plan(int fmt, int64_t rows, int64_t cols, int n_tok, int G, int n_jobs,
     const int64_t rb = cols / bw * bb;
     const int ntp = pow2ceil(n_tok);
     const int gp = pow2ceil(G);
-    const int sw = fmt == QMV_Q8_0 ? 32 : 64;          // weights per lane slice
-    const int64_t xcap = fmt == QMV_Q8_0 ? 64 : 32;    // register-resident slices per lane x 32
+    const int sw = small_blk(fmt) ? 32 : 64;           // weights per lane slice
+    const int64_t xcap = small_blk(fmt) ? 64 : 32;     // register-resident slices per lane x 32
     const int64_t n1 = cols / sw;
     const bool tma = (rb % 16) == 0;
     // Two CTAs per SM hide memory latency for large matrices.  A small matrix
@@ -176,7 +208,7 @@ int make_plan(int fmt, int64_t rows, int64_t cols, int n_tok, int G, int n_jobs,
 
     int64_t chunk_cols = cols, chunk_bytes = rb;
     if ((int64_t)G * T * rb > STAGE_MAX) {
-        const int64_t align = tma ? (fmt == QMV_Q6_K ? 2048 : 256) : (fmt == QMV_Q8_0 ? 32 : 256);
+        const int64_t align = tma ? (fmt == QMV_Q6_K ? 2048 : 256) : (small_blk(fmt) ? 32 : 256);
         const int64_t per_row = STAGE_MAX / ((int64_t)G * T);
         const int64_t n_ch = ceil_div(rb, per_row);
         chunk_cols = ceil_div(ceil_div(cols, n_ch), align) * align;
@@ -237,11 +269,7 @@ int launch_plan(int fmt, const Plan &pl, cudaStream_t stream)
 {
     t_last_kernel = QMV_KERNEL_GENERAL;
     cudaError_t e;
-    switch (fmt) {
-    case QMV_Q8_0: e = launch_pipeline<FMT_Q8_0>(pl.p, pl.kc, pl.grid, pl.smem, stream); break;
-    case QMV_Q4_K: e = launch_pipeline<FMT_Q4_K>(pl.p, pl.kc, pl.grid, pl.smem, stream); break;
-    default: e = launch_pipeline<FMT_Q6_K>(pl.p, pl.kc, pl.grid, pl.smem, stream); break;
-    }
+    e = by_fmt(fmt, [&](auto f) { return launch_pipeline<decltype(f)::value>(pl.p, pl.kc, pl.grid, pl.smem, stream); });
     if (e != cudaSuccess) return cuda_fail(e);
     return QMV_OK;
 }
@@ -310,6 +338,7 @@ RwGeom rw_geom(int fmt, int64_t x_floats, int n_tasks, int n_tok = 1)
 bool rw_ok(int fmt, int64_t cols)
 {
     const int bw = block_weights(fmt), bb = block_bytes(fmt);
+    if (!rw_tc_fmt(fmt)) return false;
     if (fmt == QMV_Q8_0 && cols % 64 != 0) return false;
     if (cols > RW_CK && cols > RW_X_SMEM_MAX) return false;     // x of a long row must fit in shared memory
     const int64_t rb = cols / bw * bb;
@@ -379,7 +408,8 @@ cudaError_t rw_launch(int fmt, const RwParamsT<NT> &p, int R, dim3 grid, size_t 
     switch (fmt) {
     case QMV_Q8_0: return launch_rw<FMT_Q8_0, NT>(p, R, grid, smem, st, pdl, coop);
     case QMV_Q4_K: return launch_rw<FMT_Q4_K, NT>(p, R, grid, smem, st, pdl, coop);
-    default: return launch_rw<FMT_Q6_K, NT>(p, R, grid, smem, st, pdl, coop);
+    case QMV_Q6_K: return launch_rw<FMT_Q6_K, NT>(p, R, grid, smem, st, pdl, coop);
+    default: return cudaErrorInvalidValue;
     }
 }
 
@@ -388,7 +418,8 @@ cudaError_t rw_occ(int fmt, int R, size_t smem, int *n)
     switch (fmt) {
     case QMV_Q8_0: return rw_occupancy<FMT_Q8_0>(R, smem, n);
     case QMV_Q4_K: return rw_occupancy<FMT_Q4_K>(R, smem, n);
-    default: return rw_occupancy<FMT_Q6_K>(R, smem, n);
+    case QMV_Q6_K: return rw_occupancy<FMT_Q6_K>(R, smem, n);
+    default: return cudaErrorInvalidValue;
     }
 }
 
@@ -425,7 +456,8 @@ int rw_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x
         switch (fmt) {
         case QMV_Q8_0: e = launch_rw_mt<FMT_Q8_0>(p, n_tok, g.R, dim3((unsigned)ctas), g.smem, st, pdl); break;
         case QMV_Q4_K: e = launch_rw_mt<FMT_Q4_K>(p, n_tok, g.R, dim3((unsigned)ctas), g.smem, st, pdl); break;
-        default: e = launch_rw_mt<FMT_Q6_K>(p, n_tok, g.R, dim3((unsigned)ctas), g.smem, st, pdl); break;
+        case QMV_Q6_K: e = launch_rw_mt<FMT_Q6_K>(p, n_tok, g.R, dim3((unsigned)ctas), g.smem, st, pdl); break;
+        default: e = cudaErrorInvalidValue; break;
         }
     }
     return e == cudaSuccess ? QMV_OK : cuda_fail(e);
@@ -461,7 +493,7 @@ SkGeom sk_geom(int fmt, int mode, int64_t rows, int64_t cols, int n_sel = 1, int
 {
     SkGeom g;
     const int bw = block_weights(fmt), bb = block_bytes(fmt);
-    if (fmt == QMV_Q8_0 && cols % 64 != 0) return g;     // a Q8_0 lane slice is a 4-byte-aligned block pair
+    if (small_blk(fmt) && cols % 64 != 0) return g;      // a Q8_0 / Q4_0 lane slice is a 4-byte-aligned block pair
     const int64_t rb = cols / bw * bb;
     // GATHER: one K-segment per routed expert, each expert row at most one segment long
     const int64_t nseg = mode == SK_GATHER ? (cols <= SK_SEG ? n_sel : 0) : ceil_div(cols, SK_SEG);
@@ -472,7 +504,7 @@ SkGeom sk_geom(int fmt, int mode, int64_t rows, int64_t cols, int n_sel = 1, int
     const int64_t x_bytes = mode == SK_GATHER ? (int64_t)g.ksegs * SK_SEG * 4 : ceil_div(cols * 4, 128) * 128;
     if (x_bytes > SK_X_MAX_BYTES) return g;
     const int64_t budget = SK_CTA_SMEM - SK_HDR - SK_PART;
-    const int r_pref = mode == SK_PLAIN && fmt == QMV_Q4_K ? 4 : 2;
+    const int r_pref = mode == SK_PLAIN && (fmt == QMV_Q4_K || fmt == QMV_Q5_K) ? 4 : 2;
     for (int R = r_pref; R >= 1; R >>= 1) {
         if ((R * rb) % 16 != 0) continue;                 // every row slot's copies 16-byte aligned
         if (mode == SK_SWIGLU && inter % R != 0) continue; // a row slot never straddles two experts
@@ -519,11 +551,9 @@ int sk_launch(int fmt, int mode, SkParams &p, const SkGeom &g, const DevInfo &di
     const bool pdl = g_pdl.load() != 0;
     t_last_kernel = QMV_KERNEL_STREAM;
     cudaError_t e;
-    switch (fmt) {
-    case QMV_Q8_0: e = launch_sk<FMT_Q8_0>(p, mode, g.R, dim3((unsigned)ctas), g.smem, st, pdl); break;
-    case QMV_Q4_K: e = launch_sk<FMT_Q4_K>(p, mode, g.R, dim3((unsigned)ctas), g.smem, st, pdl); break;
-    default: e = launch_sk<FMT_Q6_K>(p, mode, g.R, dim3((unsigned)ctas), g.smem, st, pdl); break;
-    }
+    e = by_fmt(fmt, [&](auto f) {
+        return launch_sk<decltype(f)::value>(p, mode, g.R, dim3((unsigned)ctas), g.smem, st, pdl);
+    });
     return e == cudaSuccess ? QMV_OK : cuda_fail(e);
 }
 
@@ -592,7 +622,9 @@ TcGeom tc_geom(int fmt, int64_t cols, int n_tok, const DevInfo &di)
 // superblock's offset in its 16-byte-aligned slot is the same in every row).
 bool tc_preferred(int fmt, int64_t rows, int64_t cols, int n_tok)
 {
-    const bool shape = fmt == QMV_Q6_K ? cols % 2048 == 0 : (fmt == QMV_Q8_0 || fmt == QMV_Q4_K) && cols % TC_KCOLS == 0;
+    const bool shape = fmt == QMV_Q6_K                        ? cols % 2048 == 0
+                       : (fmt == QMV_Q8_0 || fmt == QMV_Q4_K) ? cols % TC_KCOLS == 0
+                                                              : false;
     return shape && n_tok >= 3 && n_tok <= 8 && cols <= (int64_t)1 << 24 && rows <= (int64_t)INT_MAX;
 }
 
@@ -642,7 +674,7 @@ int skc_chain(int fmt, const qmv_task *tasks, int n_tasks, const DevInfo &di, cu
         const qmv_task &k = tasks[t];
         const int64_t rb = k.cols / bw * bb;
         const int nk = sk_ksegs(ceil_div(k.cols, SK_SEG));
-        if (nk == 0 || (fmt == QMV_Q8_0 && k.cols % 64 != 0) || (R * rb) % 16 != 0 || (k.rows * rb) % 16 != 0 ||
+        if (nk == 0 || (small_blk(fmt) && k.cols % 64 != 0) || (R * rb) % 16 != 0 || (k.rows * rb) % 16 != 0 ||
             k.rows > INT32_MAX)
             return QMV_ERR_SHAPE;
         max_stage = std::max<int64_t>(max_stage, (int64_t)(SK_NC / nk) * R * rb);
@@ -683,11 +715,7 @@ int skc_chain(int fmt, const qmv_task *tasks, int n_tasks, const DevInfo &di, cu
         }
         const size_t smem = (size_t)(128 + SK_HDR + SK_PART + S * pitch + max_x);
         cudaError_t e;
-        switch (fmt) {
-        case QMV_Q8_0: e = launch_skc<FMT_Q8_0>(p, R, dim3((unsigned)ctas), smem, st); break;
-        case QMV_Q4_K: e = launch_skc<FMT_Q4_K>(p, R, dim3((unsigned)ctas), smem, st); break;
-        default: e = launch_skc<FMT_Q6_K>(p, R, dim3((unsigned)ctas), smem, st); break;
-        }
+        e = by_fmt(fmt, [&](auto f) { return launch_skc<decltype(f)::value>(p, R, dim3((unsigned)ctas), smem, st); });
         if (e != cudaSuccess) return cuda_fail(e);
     }
     return QMV_OK;
@@ -890,11 +918,7 @@ int qmv_multi(int fmt, int n_tok, const qmv_task *tasks, int n_tasks, qmv_stream
         }
         mp.cta_begin[mp.n] = ctas;
         cudaError_t e;
-        switch (fmt) {
-        case QMV_Q8_0: e = launch_multi<FMT_Q8_0>(mp, kc, ctas, smem, st); break;
-        case QMV_Q4_K: e = launch_multi<FMT_Q4_K>(mp, kc, ctas, smem, st); break;
-        default: e = launch_multi<FMT_Q6_K>(mp, kc, ctas, smem, st); break;
-        }
+        e = by_fmt(fmt, [&](auto f) { return launch_multi<decltype(f)::value>(mp, kc, ctas, smem, st); });
         if (e != cudaSuccess) return cuda_fail(e);
     }
     return QMV_OK;
@@ -1119,7 +1143,7 @@ int moe_ffn_routed(const float *logits, const float *bias, int n_expert, int top
     const int ka = sk_ksegs(ceil_div(hidden, SK_SEG)), kb = sk_ksegs(top_k);
     bool fused = fmt_gu == fmt_down && n_expert <= SKM_MAX_EXPERTS && inter <= SK_SEG && ka > 0 && kb >= top_k &&
                  inter % R == 0 && (R * rba) % 16 == 0 && (R * rbb) % 16 == 0 &&
-                 (fmt_gu != QMV_Q8_0 || (hidden % 64 == 0 && inter % 64 == 0));
+                 (!small_blk(fmt_gu) || (hidden % 64 == 0 && inter % 64 == 0));
     SkMoeParams p{};
     size_t smem = 0;
     if (fused) {
@@ -1170,11 +1194,9 @@ int moe_ffn_routed(const float *logits, const float *bias, int n_expert, int top
     if (fused) {
         t_last_kernel = QMV_KERNEL_STREAM;
         cudaError_t e;
-        switch (fmt_gu) {
-        case QMV_Q8_0: e = launch_skm<FMT_Q8_0>(p, R, dim3((unsigned)di.sm_count), smem, st); break;
-        case QMV_Q4_K: e = launch_skm<FMT_Q4_K>(p, R, dim3((unsigned)di.sm_count), smem, st); break;
-        default: e = launch_skm<FMT_Q6_K>(p, R, dim3((unsigned)di.sm_count), smem, st); break;
-        }
+        e = by_fmt(fmt_gu, [&](auto f) {
+            return launch_skm<decltype(f)::value>(p, R, dim3((unsigned)di.sm_count), smem, st);
+        });
         return e == cudaSuccess ? QMV_OK : cuda_fail(e);
     }
     // other shapes: the router, then the two-launch FFN step
@@ -1264,11 +1286,7 @@ int qmv_dequant(int fmt, const void *W_blocks, int64_t rows, int64_t cols, float
     const unsigned grid = (unsigned)std::min<int64_t>(ceil_div(nblk, 256), (int64_t)di.sm_count * 16);
     const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const uint8_t *W = static_cast<const uint8_t *>(W_blocks);
-    switch (fmt) {
-    case QMV_Q8_0: dequant_kernel<FMT_Q8_0><<<grid, 256, 0, st>>>(W, nblk, bpr, cols, out); break;
-    case QMV_Q4_K: dequant_kernel<FMT_Q4_K><<<grid, 256, 0, st>>>(W, nblk, bpr, cols, out); break;
-    default: dequant_kernel<FMT_Q6_K><<<grid, 256, 0, st>>>(W, nblk, bpr, cols, out); break;
-    }
+    by_fmt(fmt, [&](auto f) { dequant_kernel<decltype(f)::value><<<grid, 256, 0, st>>>(W, nblk, bpr, cols, out); });
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e);
     return QMV_OK;

@@ -210,9 +210,9 @@ __device__ __forceinline__ float q6_k_dot1(uint32_t sb, int h, int l0, XP &&xp)
 template <int FMT>
 __device__ __forceinline__ int slice1_group_col(int s, int gq)
 {
-    if (FMT == FMT_Q8_0) {
+    if (small_block<FMT>()) {
         return 32 * s + 4 * gq;
-    } else if (FMT == FMT_Q4_K) {
+    } else if (q4k_like<FMT>()) {
         const int sb = s >> 2, c = s & 3;
         return 256 * sb + 64 * c + (gq < 8 ? 4 * gq : 32 + 4 * (gq - 8));
     } else {
@@ -222,7 +222,7 @@ __device__ __forceinline__ int slice1_group_col(int s, int gq)
 }
 
 template <int FMT> struct Slice1 {
-    static constexpr int W = (FMT == FMT_Q8_0) ? 32 : 64;   // weights per lane slice
+    static constexpr int W = small_block<FMT>() ? 32 : 64;   // weights per lane slice
     static constexpr int G = W / 4;                          // groups of four columns
 };
 

@@ -16,12 +16,19 @@
 
 namespace qmv {
 
-enum { FMT_Q8_0 = 0, FMT_Q4_K = 1, FMT_Q6_K = 2 };
+enum { FMT_Q8_0 = 0, FMT_Q4_K = 1, FMT_Q6_K = 2, FMT_Q4_0 = 3, FMT_Q5_K = 4 };
 
 template <int FMT> struct Fmt;
 template <> struct Fmt<FMT_Q8_0> { static constexpr int BW = 32;  static constexpr int BB = 34; };
 template <> struct Fmt<FMT_Q4_K> { static constexpr int BW = 256; static constexpr int BB = 144; };
 template <> struct Fmt<FMT_Q6_K> { static constexpr int BW = 256; static constexpr int BB = 210; };
+template <> struct Fmt<FMT_Q4_0> { static constexpr int BW = 32;  static constexpr int BB = 18; };
+template <> struct Fmt<FMT_Q5_K> { static constexpr int BW = 256; static constexpr int BB = 176; };
+
+// Formats whose one-token slice is one 32-weight block (else 64 weights of a
+// 256-weight superblock), and the K-quants that share Q4_K's scale packing.
+template <int FMT> constexpr bool small_block() { return FMT == FMT_Q8_0 || FMT == FMT_Q4_0; }
+template <int FMT> constexpr bool q4k_like() { return FMT == FMT_Q4_K || FMT == FMT_Q5_K; }
 
 // ------------------------------------------------------------ PTX wrappers --
 

@@ -1,5 +1,5 @@
 // qmv_dispatch.cuh -- runtime (n_tok, R, x-in-registers) -> kernel instance,
-// instantiated once per format by qmv_fmt_*.cu so the three formats compile in
+// instantiated once per format by qmv_fmt_*.cu so the formats compile in
 // parallel.
 #pragma once
 

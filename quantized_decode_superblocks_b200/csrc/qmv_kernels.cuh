@@ -34,6 +34,7 @@
 
 #include <cuda_runtime.h>
 
+#include "qmv_decode45.cuh"
 #include "qmv_decodemt.cuh"
 #include "qmv_device.cuh"
 
@@ -117,7 +118,7 @@ __device__ __forceinline__ void fence_proxy_async_smem()
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// Slices (64 weights for the K-quants, 32 for Q8_0) of one K-segment: a row's
+// Slices (64 weights for the K-quants, 32 for Q8_0 / Q4_0) of one K-segment: a row's
 // n1 slices split over wpr warps.  For the K-quants a segment starts on a
 // superblock boundary (a multiple of 4 slices), so that slice s and lane
 // (s mod 32) agree on which quarter of the superblock they hold: the Q4_K
@@ -126,7 +127,7 @@ template <int FMT>
 __device__ __forceinline__ int seg_slices(int n1, int wpr)
 {
     const int P = (n1 + wpr - 1) / wpr;
-    return FMT == FMT_Q8_0 ? P : (P + 3) & ~3;
+    return small_block<FMT>() ? P : (P + 3) & ~3;
 }
 
 // One-token slice dot product (factored form) of one row at rowp.
@@ -135,8 +136,12 @@ __device__ __forceinline__ float dot1(uint32_t rowp, int s, const Q4kSel &sel, X
 {
     if (FMT == FMT_Q8_0) {
         return q8_0_dot1(rowp + 34u * (uint32_t)s, xp);
+    } else if (FMT == FMT_Q4_0) {
+        return q4_0_dot1(rowp + 18u * (uint32_t)s, xp);
     } else if (FMT == FMT_Q4_K) {
         return q4_k_dot1<XSUM_INLINE>(rowp + 144u * (uint32_t)(s >> 2), s & 3, sel, xp, xsa, xsb);
+    } else if (FMT == FMT_Q5_K) {
+        return q5_k_dot1<XSUM_INLINE>(rowp + 176u * (uint32_t)(s >> 2), s & 3, sel, xp, xsa, xsb);
     } else {
         return q6_k_dot1(rowp + 210u * (uint32_t)(s >> 2), (s >> 1) & 1, 16 * (s & 1), xp);
     }
@@ -195,7 +200,7 @@ __device__ __forceinline__ void qmv_pipeline_body(const Params &p, const int cta
     constexpr int V = R * NTP;
     static_assert(V <= 32, "R * NTOK too large");
     static_assert(!XREG || NTOK == 1, "register-resident x is for one token");
-    constexpr int SPL1 = (FMT == FMT_Q8_0) ? 2 : 1;            // register-resident slices per lane
+    constexpr int SPL1 = small_block<FMT>() ? 2 : 1;           // register-resident slices per lane
     constexpr int NG1 = Slice1<FMT>::G;
 
     extern __shared__ __align__(128) uint8_t smem[];
@@ -401,10 +406,18 @@ __device__ __forceinline__ void qmv_pipeline_body(const Params &p, const int cta
 #pragma unroll
                             for (int k = 0; k < R; ++k) bp[k] = rowp[k] + 34u * (uint32_t)s;
                             q8_0_slice_mt<NTOK, R>(bp, 32 * s, xl, accmt);
+                        } else if (FMT == FMT_Q4_0) {
+#pragma unroll
+                            for (int k = 0; k < R; ++k) bp[k] = rowp[k] + 18u * (uint32_t)s;
+                            q4_0_slice_mt<NTOK, R>(bp, 32 * s, xl, accmt);
                         } else if (FMT == FMT_Q4_K) {
 #pragma unroll
                             for (int k = 0; k < R; ++k) bp[k] = rowp[k] + 144u * (uint32_t)(s >> 2);
                             q4_k_slice_mt<NTOK, R>(bp, s & 3, sel, 256 * (s >> 2) + 64 * (s & 3), xl, accmt);
+                        } else if (FMT == FMT_Q5_K) {
+#pragma unroll
+                            for (int k = 0; k < R; ++k) bp[k] = rowp[k] + 176u * (uint32_t)(s >> 2);
+                            q5_k_slice_mt<NTOK, R>(bp, s & 3, sel, 256 * (s >> 2) + 64 * (s & 3), xl, accmt);
                         } else {
 #pragma unroll
                             for (int k = 0; k < R; ++k) bp[k] = rowp[k] + 210u * (uint32_t)(s >> 2);

@@ -132,7 +132,9 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t *W, int64_t 
         float *o = out + r * cols + b * BW;
         const uint8_t *blk = W + bi * BB;
         if (FMT == FMT_Q8_0) dequant_block_q8_0(blk, o);
+        else if (FMT == FMT_Q4_0) dequant_block_q4_0(blk, o);
         else if (FMT == FMT_Q4_K) dequant_block_q4_k(blk, o);
+        else if (FMT == FMT_Q5_K) dequant_block_q5_k(blk, o);
         else dequant_block_q6_k(blk, o);
     }
 }

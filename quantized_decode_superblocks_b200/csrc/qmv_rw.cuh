@@ -198,21 +198,41 @@ __device__ __forceinline__ float q8_0_dot_pair(uint32_t a, XP &&xp)
     return fmaf(d1, hsum2(t0, t1), r);
 }
 
+// One token: lane l's 64-weight slice at shared address a against the x
+// groups xp holds (rw_group_col order); xsa / xsb are the sums of groups 0..7
+// and 8..15 (the K-quant min terms).
+template <int FMT, class XP>
+__device__ __forceinline__ float lane_dot(uint32_t a, int l, const Q4kSel &sel, XP &&xp, float xsa, float xsb)
+{
+    if (FMT == FMT_Q8_0) return q8_0_dot_pair(a, xp);
+    if (FMT == FMT_Q4_0) return q4_0_dot_pair(a, xp);
+    if (FMT == FMT_Q4_K) return q4_k_dot1<false>(a, l & 3, sel, xp, xsa, xsb);
+    if (FMT == FMT_Q5_K) return q5_k_dot1<false>(a, l & 3, sel, xp, xsa, xsb);
+    return q6_k_dot1(a, (l >> 1) & 1, 16 * (l & 1), xp);
+}
+
 // Column (within the K-chunk) of x group gq of lane l's 64-weight slice.
 template <int FMT>
 __device__ __forceinline__ int rw_group_col(int l, int gq)
 {
-    if (FMT == FMT_Q8_0) return 64 * l + 4 * gq;
+    if (small_block<FMT>()) return 64 * l + 4 * gq;
     return slice1_group_col<FMT>(l, gq);
+}
+
+// Byte offset of lane l's 64-weight slice within a row: two 32-weight blocks,
+// or a quarter of a superblock.
+template <int FMT>
+__device__ __forceinline__ uint32_t lane_slice_off(int l)
+{
+    if (small_block<FMT>()) return 2u * (uint32_t)Fmt<FMT>::BB * (uint32_t)l;
+    return (uint32_t)Fmt<FMT>::BB * (uint32_t)(l >> 2);
 }
 
 // Shared address of lane l's slice within one row of a stage.
 template <int FMT>
 __device__ __forceinline__ uint32_t rw_slice_addr(uint32_t rowp, int l)
 {
-    if (FMT == FMT_Q8_0) return rowp + 68u * (uint32_t)l;
-    if (FMT == FMT_Q4_K) return rowp + 144u * (uint32_t)(l >> 2);
-    return rowp + 210u * (uint32_t)(l >> 2);
+    return rowp + lane_slice_off<FMT>(l);
 }
 
 // A task's x sits in shared memory for the whole task; a lane loads its 64
@@ -438,9 +458,7 @@ __global__ void __launch_bounds__(NTHREADS, (NTOK > 2 ? 1 : 2)) qmv_rw_kernel(co
                     uint32_t sa = rw_slice_addr<FMT>(st, lane);
 #pragma unroll
                     for (int k = 0; k < R; ++k, sa += cb) {
-                        if (FMT == FMT_Q8_0) acc.v[k] += q8_0_dot_pair(sa, xp);
-                        else if (FMT == FMT_Q4_K) acc.v[k] += q4_k_dot1<false>(sa, lane & 3, sel, xp, xsa, xsb);
-                        else acc.v[k] += q6_k_dot1(sa, (lane >> 1) & 1, 16 * (lane & 1), xp);
+                        acc.v[k] += lane_dot<FMT>(sa, lane, sel, xp, xsa, xsb);
                     }
                 } else {
                     // several tokens: weights decoded once per step, each token's

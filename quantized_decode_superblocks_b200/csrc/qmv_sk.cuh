@@ -326,10 +326,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_cons
     // this lane's slice within the warp's part of a row slot
     uint32_t slice = (uint32_t)rs * (uint32_t)p.rs_bytes;
     slice += (uint32_t)ks * (MODE == SK_GATHER ? (uint32_t)R * rb : (uint32_t)p.seg_bytes);
-    if (FMT == FMT_Q8_0) slice += 68u * (uint32_t)lane;
-    else if (FMT == FMT_Q4_K) slice += 144u * (uint32_t)(lane >> 2);
-    else slice += 210u * (uint32_t)(lane >> 2);
-    const int q6h = (lane >> 1) & 1, q6l = 16 * (lane & 1);
+    slice += lane_slice_off<FMT>(lane);
     constexpr int V = G * R;
     constexpr int SH = 5 - Log2<V>::v;
     const bool leader = (lane & ((1 << SH) - 1)) == 0;
@@ -366,9 +363,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_cons
             float d = 0.f;
             if (!dead && rowok && have && k < ra) {
                 const uint32_t a = st + slice + (uint32_t)j * rb;
-                if (FMT == FMT_Q8_0) d = q8_0_dot_pair(a, xp);
-                else if (FMT == FMT_Q4_K) d = q4_k_dot1<false>(a, lane & 3, sel, xp, xsa, xsb);
-                else d = q6_k_dot1(a, q6h, q6l, xp);
+                d = lane_dot<FMT>(a, lane, sel, xp, xsa, xsb);
             }
 #pragma unroll
             for (int j2 = 0; j2 < V; ++j2)
@@ -568,7 +563,6 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skc_kernel(const __grid_con
 
     // -------------------------------------------------------- consumers --
     const Q4kSel sel = q4k_sel(lane & 3);
-    const int q6h = (lane >> 1) & 1, q6l = 16 * (lane & 1);
     constexpr int SH = 5 - Log2<R>::v;
     const bool leader = (lane & ((1 << SH) - 1)) == 0;
     const int vk = lane >> SH;
@@ -614,9 +608,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skc_kernel(const __grid_con
         const bool have = 64 * (lane + 1) <= seg_cols;
         const uint32_t rb = (uint32_t)tk.row_bytes;
         uint32_t slice = (uint32_t)(rs * R) * rb + (uint32_t)ks * (uint32_t)tk.seg_bytes;
-        if (FMT == FMT_Q8_0) slice += 68u * (uint32_t)lane;
-        else if (FMT == FMT_Q4_K) slice += 144u * (uint32_t)(lane >> 2);
-        else slice += 210u * (uint32_t)(lane >> 2);
+        slice += lane_slice_off<FMT>(lane);
         int64_t a, b;
         skc_rows<R>(tk, c, a, b);
         for (int64_t r0 = a; r0 < b; r0 += tk.tile_rows, ++i) {
@@ -639,9 +631,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skc_kernel(const __grid_con
                 float d = 0.f;
                 if (!dead && have && k < ra) {
                     const uint32_t ad = st + slice + (uint32_t)k * rb;
-                    if (FMT == FMT_Q8_0) d = q8_0_dot_pair(ad, xp);
-                    else if (FMT == FMT_Q4_K) d = q4_k_dot1<false>(ad, lane & 3, sel, xp, xsa, xsb);
-                    else d = q6_k_dot1(ad, q6h, q6l, xp);
+                    d = lane_dot<FMT>(ad, lane, sel, xp, xsa, xsb);
                 }
 #pragma unroll
                 for (int k2 = 0; k2 < R; ++k2)
@@ -915,7 +905,6 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skm_kernel(const __grid_con
 
     // -------------------------------------------------------- consumers --
     const Q4kSel sel = q4k_sel(lane & 3);
-    const int q6h = (lane >> 1) & 1, q6l = 16 * (lane & 1);
     bool dead = false;
     int i = 0;
     auto wait_stage = [&](int slot, int i_) {
@@ -944,9 +933,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skm_kernel(const __grid_con
         const bool have = 64 * (lane + 1) <= seg_cols;
         const uint32_t rb = (uint32_t)p.gu_row_bytes;
         uint32_t slice = (uint32_t)(rs * p.a_rs_bytes) + (uint32_t)ks * (uint32_t)p.a_seg_bytes;
-        if (FMT == FMT_Q8_0) slice += 68u * (uint32_t)lane;
-        else if (FMT == FMT_Q4_K) slice += 144u * (uint32_t)(lane >> 2);
-        else slice += 210u * (uint32_t)(lane >> 2);
+        slice += lane_slice_off<FMT>(lane);
         constexpr int V = 2 * R;
         constexpr int SH = 5 - Log2<V>::v;
         const bool leader = (lane & ((1 << SH) - 1)) == 0;
@@ -966,9 +953,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skm_kernel(const __grid_con
                 float d = 0.f;
                 if (!dead && rowok && have && k < ra) {
                     const uint32_t a = st + slice + (uint32_t)j * rb;
-                    if (FMT == FMT_Q8_0) d = q8_0_dot_pair(a, xp);
-                    else if (FMT == FMT_Q4_K) d = q4_k_dot1<false>(a, lane & 3, sel, xp, xsa, xsb);
-                    else d = q6_k_dot1(a, q6h, q6l, xp);
+                    d = lane_dot<FMT>(a, lane, sel, xp, xsa, xsb);
                 }
 #pragma unroll
                 for (int j2 = 0; j2 < V; ++j2)
@@ -1031,9 +1016,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skm_kernel(const __grid_con
         const bool have = 64 * (lane + 1) <= seg_cols;
         const uint32_t rb = (uint32_t)p.d_row_bytes;
         uint32_t slice = (uint32_t)(rs * p.b_rs_bytes) + (uint32_t)(ks * R) * rb;
-        if (FMT == FMT_Q8_0) slice += 68u * (uint32_t)lane;
-        else if (FMT == FMT_Q4_K) slice += 144u * (uint32_t)(lane >> 2);
-        else slice += 210u * (uint32_t)(lane >> 2);
+        slice += lane_slice_off<FMT>(lane);
         constexpr int SH = 5 - Log2<R>::v;
         const bool leader = (lane & ((1 << SH) - 1)) == 0;
         const int vk = lane >> SH;
@@ -1050,9 +1033,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skm_kernel(const __grid_con
                 float d = 0.f;
                 if (!dead && have && k < ra) {
                     const uint32_t a = st + slice + (uint32_t)k * rb;
-                    if (FMT == FMT_Q8_0) d = q8_0_dot_pair(a, xp);
-                    else if (FMT == FMT_Q4_K) d = q4_k_dot1<false>(a, lane & 3, sel, xp, xsa, xsb);
-                    else d = q6_k_dot1(a, q6h, q6l, xp);
+                    d = lane_dot<FMT>(a, lane, sel, xp, xsa, xsb);
                 }
 #pragma unroll
                 for (int k2 = 0; k2 < R; ++k2)

@@ -42,9 +42,9 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_block_sizes_and_strerror(L):
-    assert [q.qmv_block_weights(f) for f in (0, 1, 2)] == [32, 256, 256]
-    assert [q.qmv_block_bytes(f) for f in (0, 1, 2)] == [34, 144, 210]
-    assert q.qmv_block_bytes(3) == 0 and q.qmv_block_weights(-1) == 0
+    assert [q.qmv_block_weights(f) for f in (0, 1, 2, 3, 4)] == [32, 256, 256, 32, 256]
+    assert [q.qmv_block_bytes(f) for f in (0, 1, 2, 3, 4)] == [34, 144, 210, 18, 176]
+    assert q.qmv_block_bytes(5) == 0 and q.qmv_block_weights(-1) == 0
     for s in (OK, NULL, FMT, SHAPE, ALIGN, NTOK, NSEL, CUDA, DEVICE, 42):
         assert isinstance(q.strerror(s), str) and q.strerror(s)
 
@@ -55,10 +55,12 @@ def qb(L, fmt=1, W=A, rows=4, cols=256, x=A, y=A, n_tok=1):
 
 def test_qmv_argument_validation(L):
     assert qb(L, W=None) == NULL and qb(L, x=None) == NULL and qb(L, y=None) == NULL
-    assert qb(L, fmt=3) == FMT and qb(L, fmt=-1) == FMT
+    assert qb(L, fmt=5) == FMT and qb(L, fmt=-1) == FMT
     assert qb(L, rows=0) == SHAPE and qb(L, cols=0) == SHAPE
     assert qb(L, cols=128) == SHAPE            # Q4_K needs multiples of 256
     assert qb(L, fmt=0, cols=48) == SHAPE       # Q8_0 needs multiples of 32
+    assert qb(L, fmt=3, cols=48) == SHAPE       # so does Q4_0
+    assert qb(L, fmt=4, cols=128) == SHAPE      # Q5_K needs multiples of 256
     assert qb(L, cols=2 ** 21) == SHAPE
     assert qb(L, n_tok=0) == NTOK and qb(L, n_tok=9) == NTOK
     assert qb(L, W=A + 8) == ALIGN and qb(L, x=A + 4) == ALIGN and qb(L, y=A + 2) == ALIGN
