@@ -10,7 +10,8 @@ decode order (each matvec reads its x only after the previous one is complete,
 as its input would be the previous output in a model): 64 library calls with
 programmatic dependent launch (each launch may copy its weights while the
 previous one finishes; --no-pdl turns it off), or with --mode chain one
-qmv_chain call (a persistent launch with a grid barrier between matvecs).  The
+qmv_chain call (the same launches, each also moving the next matvec's
+weights into L2 once its own copies are issued).  The
 step is captured once as a CUDA graph of the library's C-ABI calls and
 replayed.
 Metric: weight bytes streamed per second (GB/s), with the fraction of the
@@ -270,7 +271,7 @@ class Sweep:
         if mode == "chain" and self.n_tok != 1:
             raise ValueError("the chained step is one-token")
         self.mode = mode
-        self.launches = {"launches": len(self.mats), "chain": -(-len(self.mats) // 64),
+        self.launches = {"launches": len(self.mats), "chain": len(self.mats),
                          "grouped": None}[mode]
 
     def launch(self, i, stream=None):
@@ -621,8 +622,8 @@ def main():
     ap.add_argument("--n-tok", type=int, default=1)
     ap.add_argument("--mode", choices=["launches", "chain"], default="launches",
                     help="how the step runs, in decode order either way: 'launches' = one library "
-                         "call per matvec (default), 'chain' = qmv_chain (one persistent launch with a "
-                         "grid barrier between matvecs; one token)")
+                         "call per matvec (default), 'chain' = one qmv_chain call (the same launches, "
+                         "each moving the next matvec's weights into L2; one token)")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch without programmatic dependent launch (qmv_set_pdl(0))")
     ap.add_argument("--headline-only", action="store_true",
@@ -667,10 +668,7 @@ def main():
         dist.barrier(torch)
         sec = dist.max(torch, sec)
         # the dominant kernel: every launch of the step, event-timed on its stream
-        if mode == "launches":
-            durs, kinds = per_kind_durations(torch, q, sweep, stream)
-        else:
-            durs, kinds = {"chain": (time_graph(torch, graph, 20, stream) / 20, 1)}, {}
+        durs, kinds = per_kind_durations(torch, q, sweep, stream)
         # end to end: pinned x -> device, the step's library calls, y -> pinned host
         e2e_reps = max(3, min(200, args.steps // 5))
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -724,13 +722,9 @@ def main():
     dom_launch_sec, dom_n = durs[dom_name]
     dom_share = dom_launch_sec * dom_n / total_kernel_sec
     shares = {k: round(v[0] * v[1] / total_kernel_sec, 4) for k, v in durs.items()}
-    if mode == "launches":
-        rows, cols = shapes[dom_name]
-        dom_bytes = algo_bytes(Q8_0, rows, cols, args.n_tok)
-        dom_kernel = f"Q8_0 {dom_name} matvec {rows}x{cols} ({kinds[dom_name]}), {dom_n} launches per step"
-    else:
-        dom_bytes = sweep.algo
-        dom_kernel = "qmv_rw_kernel, chained: the whole step in one launch"
+    rows, cols = shapes[dom_name]
+    dom_bytes = algo_bytes(Q8_0, rows, cols, args.n_tok)
+    dom_kernel = f"Q8_0 {dom_name} matvec {rows}x{cols} ({kinds[dom_name]}), {dom_n} launches per step"
     achieved = dom_bytes / dom_launch_sec / 1e9
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "ncu_traffic.json")

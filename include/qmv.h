@@ -52,8 +52,8 @@
  *   - Thread safety: calls may be made from several host threads.  Global
  *     state: a per-device properties cache, the programmatic-dependent-launch
  *     switch (qmv_set_pdl), and per device the sticky error word read by
- *     qmv_check(), the two grid-barrier words of qmv_chain, qmv_argmax's
- *     workspace and the scratch array of moe_ffn_static.
+ *     qmv_check(), qmv_argmax's workspace and the scratch array of
+ *     moe_ffn_static.
  */
 #ifndef QMV_H
 #define QMV_H
@@ -135,15 +135,14 @@ int qmv_multi(int fmt, int n_tok, const qmv_task *tasks, int n_tasks, qmv_stream
  * §核心算子 and §性能表现: every layer's matvecs each decode step): task t+1
  * starts only after every row of task t is written, so a task's x may be the
  * y of any earlier task of the same call (tasks' n_tok is 1: x f32 [cols],
- * y f32 [rows]).  The library runs up to 64 tasks in one persistent
- * cooperative launch with a grid barrier between tasks, and keeps copying the
- * next tasks' weights into shared memory while the GPU waits at a barrier;
- * longer lists take several consecutive launches.  A task shape that the
- * persistent kernel does not take turns the whole call into one launch per
- * task, in order.  The grid barrier's state is one per device: do not run two
- * qmv_chain calls on the same device at the same time (different streams);
- * a barrier that waits about a second reports QMV_DEVERR_TIMEOUT through
- * qmv_check, which also resets the barrier.  `tasks` is a host array of
+ * y f32 [rows]).  Each task is one streaming-kernel launch, ordered by
+ * programmatic dependent launch (a kernel reads its x only after the previous
+ * one has finished), and each launch, once its own weight copies are issued,
+ * starts moving the next task's weights into L2, so the next launch reads them
+ * from there while HBM already streams the one after.  The call keeps no
+ * state between calls: calls on different streams may overlap.  A task shape
+ * that the streaming kernel does not take turns the whole call into one
+ * qmv_f32 call per task, in order.  `tasks` is a host array of
  * n_tasks entries (1 <= n_tasks <= QMV_MAX_TASKS), read during the call only.
  * Errors as qmv_multi. */
 int qmv_chain(int fmt, const qmv_task *tasks, int n_tasks, qmv_stream_t stream);

@@ -21,10 +21,6 @@ using namespace qmv;
 // Sticky device error word (QMV_DEVERR_* bits), read and cleared by qmv_check.
 __device__ int g_dev_err;
 
-// Grid barrier of ordered chained launches: {arrivals, exits}, back to zero
-// at the end of every launch; qmv_check clears both after a device error.
-__device__ unsigned g_chain_sync[2];
-
 // Greedy argmax workspace of qmv_argmax (the layout of qmv_argmax_ws's): one
 // 64-bit key per token, then one arrival counter per token; back to zero at
 // the end of every call; qmv_check clears it after a device error.
@@ -50,7 +46,6 @@ struct DevInfo {
     int sm_count = 0;
     int smem_optin = 0;
     int *err = nullptr;
-    unsigned *sync = nullptr;
     unsigned long long *amax_key = nullptr;   // device address of g_amax_ws
     float *static_h = nullptr;   // device address of g_static_h, set up by moe_ffn_static
     bool ok = false;
@@ -135,7 +130,6 @@ int get_dev(DevInfo &out)
             cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaGetSymbolAddress(reinterpret_cast<void **>(&d.err), g_dev_err) != cudaSuccess ||
-            cudaGetSymbolAddress(reinterpret_cast<void **>(&d.sync), g_chain_sync) != cudaSuccess ||
             cudaGetSymbolAddress(reinterpret_cast<void **>(&d.amax_key), g_amax_ws) != cudaSuccess) {
             (void)cudaGetLastError();
             return QMV_ERR_DEVICE;
@@ -413,16 +407,6 @@ cudaError_t rw_launch(int fmt, const RwParamsT<NT> &p, int R, dim3 grid, size_t 
     }
 }
 
-cudaError_t rw_occ(int fmt, int R, size_t smem, int *n)
-{
-    switch (fmt) {
-    case QMV_Q8_0: return rw_occupancy<FMT_Q8_0>(R, smem, n);
-    case QMV_Q4_K: return rw_occupancy<FMT_Q4_K>(R, smem, n);
-    case QMV_Q6_K: return rw_occupancy<FMT_Q6_K>(R, smem, n);
-    default: return cudaErrorInvalidValue;
-    }
-}
-
 // One matvec on the warp-ring kernel: enough CTAs that every warp has a row
 // group, at most two per SM.
 int rw_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x, float *y, int n_tok,
@@ -433,12 +417,9 @@ int rw_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x
     if (g.R == 0) return QMV_ERR_SHAPE;
     RwParams1 p{};
     p.n_tasks = 1;
-    p.chain = 0;
-    p.ordered = 0;
     p.n_stage = g.S;
     p.stage_pitch = g.pitch;
     p.x_floats = (int32_t)x_floats;
-    p.sync = di.sync;
     p.err = di.err;
     p.debug_extra_tx = g_debug_extra_tx.load();
     p.t[0] = rw_task(fmt, g.R, W, rows, cols, x, y);
@@ -476,13 +457,13 @@ struct SkGeom {
     size_t smem = 0;
 };
 
-// K-segments per row: the smallest divisor of the twelve consumer warps that
-// covers nseg segments (0 if none does).
+// K-segments per row: the smallest divisor of the consumer warps (twelve)
+// that covers nseg segments (0 if none does).
 int sk_ksegs(int64_t nseg)
 {
     if (nseg < 1) return 0;
-    for (int d : {1, 2, 3, 4, 6, 12})
-        if (d >= nseg) return d;
+    for (int d = 1; d <= SK_NC; ++d)
+        if (SK_NC % d == 0 && d >= nseg) return d;
     return 0;
 }
 
@@ -559,9 +540,12 @@ int sk_launch(int fmt, int mode, SkParams &p, const SkGeom &g, const DevInfo &di
 
 int sk_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x, float *y, const SkGeom &g,
               const DevInfo &di, cudaStream_t st, int32_t *amax_idx = nullptr,
-              unsigned long long *amax_key = nullptr, unsigned *amax_done = nullptr)
+              unsigned long long *amax_key = nullptr, unsigned *amax_done = nullptr,
+              const void *pf = nullptr, int64_t pf_bytes = 0)
 {
     SkParams p{};
+    p.pf = static_cast<const uint8_t *>(pf);
+    p.pf_bytes = pf_bytes;
     p.amax_idx = amax_idx;
     p.amax_key = amax_key;
     p.amax_done = amax_done;
@@ -662,111 +646,29 @@ int tc_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x
     return e == cudaSuccess ? QMV_OK : cuda_fail(e);
 }
 
-// In-order one-token matvecs on the chained streaming kernel, up to
-// SKC_MAX_TASKS per cooperative launch (one CTA per SM).  Returns
-// QMV_ERR_SHAPE (nothing launched) when some task does not fit its layout.
-int skc_chain(int fmt, const qmv_task *tasks, int n_tasks, const DevInfo &di, cudaStream_t st)
+
+// In-order one-token matvecs as one streaming-kernel launch each, ordered by
+// programmatic dependent launch (each kernel reads its x only after the
+// previous one has finished).  Each launch, once its own weight copies are
+// issued, moves the next task's weights into L2: the next launch's copies then
+// come from L2 while HBM already streams the one after.  Returns QMV_ERR_SHAPE
+// (nothing launched) when some task does not fit the streaming kernel.
+int sk_seq(int fmt, const qmv_task *tasks, int n_tasks, const DevInfo &di, cudaStream_t st)
 {
+    for (int t = 0; t < n_tasks; ++t)
+        if (!sk_geom(fmt, SK_PLAIN, tasks[t].rows, tasks[t].cols).ok) return QMV_ERR_SHAPE;
     const int bw = block_weights(fmt), bb = block_bytes(fmt);
-    const int R = 2;
-    int64_t max_stage = 0, max_x = 0;
     for (int t = 0; t < n_tasks; ++t) {
         const qmv_task &k = tasks[t];
-        const int64_t rb = k.cols / bw * bb;
-        const int nk = sk_ksegs(ceil_div(k.cols, SK_SEG));
-        if (nk == 0 || (small_blk(fmt) && k.cols % 64 != 0) || (R * rb) % 16 != 0 || (k.rows * rb) % 16 != 0 ||
-            k.rows > INT32_MAX)
-            return QMV_ERR_SHAPE;
-        max_stage = std::max<int64_t>(max_stage, (int64_t)(SK_NC / nk) * R * rb);
-        max_x = std::max<int64_t>(max_x, ceil_div(k.cols * 4, 128) * 128);
-    }
-    const int64_t pitch = ceil_div(max_stage + 16, 128) * 128;
-    const int64_t budget = SK_CTA_SMEM - SK_HDR - SK_PART - max_x;
-    const int64_t S = std::min<int64_t>(SK_MAX_STAGES, budget / pitch);
-    if (max_x > SK_X_MAX_BYTES || S < 2) return QMV_ERR_SHAPE;
-    static thread_local SkChainParams p;
-    const int64_t ctas = di.sm_count;
-    t_last_kernel = QMV_KERNEL_STREAM;
-    for (int t0 = 0; t0 < n_tasks; t0 += SKC_MAX_TASKS) {
-        const int n = std::min(SKC_MAX_TASKS, n_tasks - t0);
-        p.n_tasks = n;
-        p.n_stage = (int)S;
-        p.stage_pitch = (int32_t)pitch;
-        p.x_off = (int32_t)(S * pitch);
-        p.sync = di.sync;
-        p.err = di.err;
-        p.debug_extra_tx = g_debug_extra_tx.load();
-        for (int i = 0; i < n; ++i) {
-            const qmv_task &k = tasks[t0 + i];
-            SkTask &tk = p.t[i];
-            tk = SkTask{};
-            tk.W = static_cast<const uint8_t *>(k.W_blocks);
-            tk.x = k.x;
-            tk.y = k.y;
-            tk.rows = k.rows;
-            tk.row_bytes = k.cols / bw * bb;
-            const int64_t units = ceil_div(k.rows, (int64_t)R);
-            tk.units_q = units / ctas;
-            tk.units_r = (int32_t)(units % ctas);
-            tk.cols = (int32_t)k.cols;
-            tk.ksegs = sk_ksegs(ceil_div(k.cols, SK_SEG));
-            tk.seg_bytes = SK_SEG / bw * bb;
-            tk.tile_rows = (SK_NC / tk.ksegs) * R;
-        }
-        const size_t smem = (size_t)(128 + SK_HDR + SK_PART + S * pitch + max_x);
-        cudaError_t e;
-        e = by_fmt(fmt, [&](auto f) { return launch_skc<decltype(f)::value>(p, R, dim3((unsigned)ctas), smem, st); });
-        if (e != cudaSuccess) return cuda_fail(e);
+        const qmv_task *nx = t + 1 < n_tasks ? &tasks[t + 1] : nullptr;
+        const SkGeom g = sk_geom(fmt, SK_PLAIN, k.rows, k.cols);
+        const int rc = sk_single(fmt, k.W_blocks, k.rows, k.cols, k.x, k.y, g, di, st, nullptr, nullptr, nullptr,
+                                 nx ? nx->W_blocks : nullptr, nx ? nx->rows * (nx->cols / bw * bb) : 0);
+        if (rc) return rc;
     }
     return QMV_OK;
 }
 
-// In-order one-token matvecs of one format on the warp-ring kernel, up to
-// RW_MAX_TASKS per launch.  Every CTA works on every task, in order, each
-// task's row groups spread over all warps (so small and large tasks alike use
-// the whole GPU), with a grid barrier between consecutive tasks (cooperative
-// launch).
-int rw_chain(int fmt, const qmv_task *tasks, int n_tasks, const DevInfo &di, cudaStream_t st)
-{
-    int64_t x_floats = 0;
-    for (int t = 0; t < n_tasks; ++t) x_floats = std::max<int64_t>(x_floats, tasks[t].cols);
-    const RwGeom g = rw_geom(fmt, x_floats, std::min(n_tasks, RW_MAX_TASKS));
-    if (g.R == 0) return QMV_ERR_SHAPE;
-    static thread_local RwParams p;
-    int ctas_per_sm = 2;
-    {
-        const cudaError_t e = rw_occ(fmt, g.R, g.smem, &ctas_per_sm);
-        if (e != cudaSuccess) return cuda_fail(e);
-        if (ctas_per_sm < 1) return QMV_ERR_SHAPE;
-    }
-    const int64_t ctas = (int64_t)ctas_per_sm * di.sm_count;
-    t_last_kernel = QMV_KERNEL_WARP_RING;
-    for (int t0 = 0; t0 < n_tasks; t0 += RW_MAX_TASKS) {
-        const int n = std::min(RW_MAX_TASKS, n_tasks - t0);
-        p.n_tasks = n;
-        p.chain = 1;
-        p.ordered = 1;
-        p.n_stage = g.S;
-        p.stage_pitch = g.pitch;
-        p.x_floats = (int32_t)x_floats;
-        p.sync = di.sync;
-        p.err = di.err;
-        p.debug_extra_tx = g_debug_extra_tx.load();
-        // each task starts on the warp after the previous task's last row group
-        int64_t rot = 0;
-        for (int i = 0; i < n; ++i) {
-            const qmv_task &k = tasks[t0 + i];
-            p.t[i] = rw_task(fmt, g.R, k.W_blocks, k.rows, k.cols, k.x, k.y);
-            rw_split(p.t[i], ctas * NW, rot);
-            rot = (rot + p.t[i].n_rg) % (ctas * NW);
-        }
-        p.cta_begin[0] = 0;
-        p.cta_begin[1] = (int32_t)ctas;
-        const cudaError_t e = rw_launch(fmt, p, g.R, dim3((unsigned)ctas), g.smem, st, false, true);
-        if (e != cudaSuccess) return cuda_fail(e);
-    }
-    return QMV_OK;
-}
 
 int check_matrix(int fmt, int64_t rows, int64_t cols)
 {
@@ -929,24 +831,20 @@ int qmv_chain(int fmt, const qmv_task *tasks, int n_tasks, qmv_stream_t stream)
     if (!tasks) return QMV_ERR_NULL;
     if (!fmt_ok(fmt)) return QMV_ERR_FMT;
     if (n_tasks < 1 || n_tasks > QMV_MAX_TASKS) return QMV_ERR_SHAPE;
-    bool all = true;
     for (int t = 0; t < n_tasks; ++t) {
         const qmv_task &k = tasks[t];
         if (!k.W_blocks || !k.x || !k.y) return QMV_ERR_NULL;
         const int rc = check_matrix(fmt, k.rows, k.cols);
         if (rc) return rc;
         if (!aligned(k.W_blocks, 16) || !aligned(k.x, 16) || !aligned(k.y, 4)) return QMV_ERR_ALIGN;
-        all = all && rw_ok(fmt, k.cols);
     }
     if (injected_failure()) return QMV_ERR_CUDA;
     DevInfo di;
     int rc = get_dev(di);
     if (rc) return rc;
-    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    rc = skc_chain(fmt, tasks, n_tasks, di, st);
+    rc = sk_seq(fmt, tasks, n_tasks, di, reinterpret_cast<cudaStream_t>(stream));
     if (rc != QMV_ERR_SHAPE) return rc;
-    if (all) return rw_chain(fmt, tasks, n_tasks, di, st);
-    // a shape the chained kernel does not take: one launch per task, in order
+    // a shape the streaming kernel does not take: one call per task, in order
     for (int t = 0; t < n_tasks; ++t) {
         const qmv_task &k = tasks[t];
         if ((rc = qmv_batched(fmt, k.W_blocks, k.rows, k.cols, k.x, k.y, 1, stream))) return rc;
@@ -1306,8 +1204,7 @@ int qmv_check(qmv_stream_t stream, int *dev_err_out)
         (void)cudaGetLastError();
         return QMV_ERR_CUDA;
     }
-    if (word && (cudaMemset(di.sync, 0, 2 * sizeof(unsigned)) != cudaSuccess ||
-                 cudaMemset(di.amax_key, 0, QMV_ARGMAX_WS_BYTES) != cudaSuccess ||
+    if (word && (cudaMemset(di.amax_key, 0, QMV_ARGMAX_WS_BYTES) != cudaSuccess ||
                  cudaDeviceSynchronize() != cudaSuccess)) {
         (void)cudaGetLastError();
         return QMV_ERR_CUDA;

@@ -153,12 +153,6 @@ struct RwInstance {
     {
         return launch_with(qmv_rw_kernel<FMT, R, NT, NTOK>, configured(), p, grid, smem, st, pdl, coop);
     }
-    static cudaError_t occupancy(size_t smem, int *n)
-    {
-        const cudaError_t e = ensure_smem(qmv_rw_kernel<FMT, R, NT, NTOK>, configured(), smem);
-        if (e != cudaSuccess) return e;
-        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(n, qmv_rw_kernel<FMT, R, NT, NTOK>, NTHREADS, smem);
-    }
 };
 
 template <int FMT, int NT>
@@ -191,17 +185,6 @@ cudaError_t launch_rw_mt(const RwParams1 &p, int n_tok, int R, dim3 grid, size_t
     case 3: return launch_rw_mt_r<FMT, 3>(p, R, grid, smem, stream, pdl);
     case 4: return launch_rw_mt_r<FMT, 4>(p, R, grid, smem, stream, pdl);
     default: return cudaErrorInvalidValue;      // 5..8 tokens take the general kernel
-    }
-}
-
-template <int FMT>
-cudaError_t rw_occupancy(int R, size_t smem, int *ctas_per_sm)
-{
-    switch (R) {
-    case 1: return RwInstance<FMT, 1, RW_MAX_TASKS>::occupancy(smem, ctas_per_sm);
-    case 2: return RwInstance<FMT, 2, RW_MAX_TASKS>::occupancy(smem, ctas_per_sm);
-    case 4: return RwInstance<FMT, 4, RW_MAX_TASKS>::occupancy(smem, ctas_per_sm);
-    default: return cudaErrorInvalidValue;
     }
 }
 
@@ -243,19 +226,6 @@ cudaError_t launch_sk(const SkParams &p, int mode, int R, dim3 grid, size_t smem
     case SK_PLAIN: return launch_sk_mode<FMT, SK_PLAIN>(p, R, grid, smem, st, pdl);
     case SK_SWIGLU: return launch_sk_mode<FMT, SK_SWIGLU>(p, R, grid, smem, st, pdl);
     case SK_GATHER: return launch_sk_mode<FMT, SK_GATHER>(p, R, grid, smem, st, pdl);
-    default: return cudaErrorInvalidValue;
-    }
-}
-
-// The chained streaming kernel (cooperative: one CTA per SM, all resident).
-template <int FMT>
-cudaError_t launch_skc(const SkChainParams &p, int R, dim3 grid, size_t smem, cudaStream_t st)
-{
-    static SmemCfg c1, c2, c4;
-    switch (R) {
-    case 1: return launch_with(qmv_skc_kernel<FMT, 1>, c1, p, grid, smem, st, false, true, SK_THREADS);
-    case 2: return launch_with(qmv_skc_kernel<FMT, 2>, c2, p, grid, smem, st, false, true, SK_THREADS);
-    case 4: return launch_with(qmv_skc_kernel<FMT, 4>, c4, p, grid, smem, st, false, true, SK_THREADS);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -5,11 +5,8 @@ namespace qmv {
 template cudaError_t launch_pipeline<FMT_Q6_K>(const Params &, const KernelChoice &, dim3, size_t, cudaStream_t);
 template cudaError_t launch_multi<FMT_Q6_K>(const MultiParams &, const KernelChoice &, int, size_t, cudaStream_t);
 template cudaError_t launch_rw<FMT_Q6_K, 1>(const RwParams1 &, int, dim3, size_t, cudaStream_t, bool, bool);
-template cudaError_t launch_rw<FMT_Q6_K, RW_MAX_TASKS>(const RwParams &, int, dim3, size_t, cudaStream_t, bool, bool);
-template cudaError_t rw_occupancy<FMT_Q6_K>(int, size_t, int *);
 template cudaError_t launch_rw_mt<FMT_Q6_K>(const RwParams1 &, int, int, dim3, size_t, cudaStream_t, bool);
 template cudaError_t launch_tc<FMT_Q6_K>(const TcParams &, bool, dim3, size_t, cudaStream_t, bool);
 template cudaError_t launch_sk<FMT_Q6_K>(const SkParams &, int, int, dim3, size_t, cudaStream_t, bool);
-template cudaError_t launch_skc<FMT_Q6_K>(const SkChainParams &, int, dim3, size_t, cudaStream_t);
 template cudaError_t launch_skm<FMT_Q6_K>(const SkMoeParams &, int, dim3, size_t, cudaStream_t);
 }  // namespace qmv

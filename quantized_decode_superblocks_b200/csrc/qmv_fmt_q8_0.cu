@@ -5,11 +5,8 @@ namespace qmv {
 template cudaError_t launch_pipeline<FMT_Q8_0>(const Params &, const KernelChoice &, dim3, size_t, cudaStream_t);
 template cudaError_t launch_multi<FMT_Q8_0>(const MultiParams &, const KernelChoice &, int, size_t, cudaStream_t);
 template cudaError_t launch_rw<FMT_Q8_0, 1>(const RwParams1 &, int, dim3, size_t, cudaStream_t, bool, bool);
-template cudaError_t launch_rw<FMT_Q8_0, RW_MAX_TASKS>(const RwParams &, int, dim3, size_t, cudaStream_t, bool, bool);
-template cudaError_t rw_occupancy<FMT_Q8_0>(int, size_t, int *);
 template cudaError_t launch_rw_mt<FMT_Q8_0>(const RwParams1 &, int, int, dim3, size_t, cudaStream_t, bool);
 template cudaError_t launch_tc<FMT_Q8_0>(const TcParams &, bool, dim3, size_t, cudaStream_t, bool);
 template cudaError_t launch_sk<FMT_Q8_0>(const SkParams &, int, int, dim3, size_t, cudaStream_t, bool);
-template cudaError_t launch_skc<FMT_Q8_0>(const SkChainParams &, int, dim3, size_t, cudaStream_t);
 template cudaError_t launch_skm<FMT_Q8_0>(const SkMoeParams &, int, dim3, size_t, cudaStream_t);
 }  // namespace qmv

@@ -18,14 +18,8 @@
 // 端侧大模型推理引擎, §性能表现); on this one the decode arithmetic is the
 // tighter limit, which is what the layout above optimises for.
 //
-// The same body serves three launch forms:
-//   * one matvec (one task, all CTAs);
-//   * several independent matvecs (each task owns a range of CTAs);
-//   * a chain: every CTA works on every task in order, with a grid-wide
-//     barrier between consecutive tasks, so task t+1 may read task t's output
-//     (the layer-after-layer order of a decode step).  Weights do not depend on
-//     earlier tasks, so each warp's ring keeps prefetching the next tasks'
-//     tiles while the CTA waits at the barrier.
+// The same body serves one matvec (one task, all CTAs) and several
+// independent matvecs (each task owns a range of CTAs).
 #pragma once
 
 #include "qmv_kernels.cuh"
@@ -72,19 +66,15 @@ __host__ __device__ constexpr int rw_hdr_bytes(int n_tasks)
 template <int NT>
 struct RwParamsT {
     int32_t n_tasks;
-    int32_t chain;            // 1: every CTA works on every task, in order
-    int32_t ordered;          // chained: grid barrier between consecutive tasks (cooperative launch)
     int32_t n_stage;          // ring stages per warp
     int32_t stage_pitch;      // bytes per stage (multiple of 128)
     int32_t x_floats;         // shared-memory x: the longest task row (floats), one such row per token
-    int32_t cta_begin[NT + 1];   // not chained: task t owns CTAs [cta_begin[t], cta_begin[t+1])
-    unsigned *sync;           // ordered: {arrivals, exits} of the grid barrier, zero between launches
+    int32_t cta_begin[NT + 1];   // task t owns CTAs [cta_begin[t], cta_begin[t+1])
     int *err;
     uint32_t debug_extra_tx;  // test hook: bytes expected per tile beyond those copied (0 in use)
     RwTask t[NT];
 };
 using RwParams1 = RwParamsT<1>;
-using RwParams = RwParamsT<RW_MAX_TASKS>;
 
 // Row groups [a, b) of a task that warp wg takes: contiguous, balanced, split
 // on the host (no divisions here).
@@ -271,50 +261,6 @@ __device__ __forceinline__ void rw_load_x_smem(uint32_t xs, int kc, int ncols, i
     xsb = sb.x + sb.y;
 }
 
-// Grid-wide barrier of an ordered chained launch (all CTAs co-resident:
-// cooperative launch).  sync[0] counts arrivals and only grows within a
-// launch: barrier k is passed once it reaches (k + 1) * n_ctas.  One thread
-// per CTA fences the CTA's writes, adds its arrival, polls with relaxed loads
-// and fences once more on the way out; the last CTA to leave the kernel
-// (sync[1]) puts both words back to zero for the next launch.  A wait gives
-// up after about a second and returns false (the caller records the error;
-// the kernel still finishes).
-__device__ __forceinline__ bool rw_grid_barrier(unsigned *sync, unsigned target)
-{
-    bool ok = true;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        asm volatile("fence.acq_rel.gpu;" ::: "memory");
-        asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" :: "l"(sync) : "memory");
-        // bounded by the SM cycle counter (cheap to read): about a second at 2 GHz
-        const long long c0 = clock64();
-        for (;;) {
-            unsigned c;
-            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(sync) : "memory");
-            if ((int)(c - target) >= 0) break;
-            if (clock64() - c0 > 2000000000LL) {
-                ok = false;
-                break;
-            }
-        }
-        asm volatile("fence.acq_rel.gpu;" ::: "memory");
-    }
-    __syncthreads();
-    return ok;
-}
-
-__device__ __forceinline__ void rw_grid_exit(unsigned *sync, unsigned n_ctas)
-{
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const unsigned old = atomicAdd(sync + 1, 1u);
-        if (old == n_ctas - 1u) {       // every CTA has passed its last barrier
-            atomicExch(sync, 0u);
-            atomicExch(sync + 1, 0u);
-        }
-    }
-}
-
 // Accumulators of one row group: one token -> a float per row (factored
 // decode); several tokens -> a packed pair per (row, token) (weight-stationary
 // decode units of qmv_decodemt.cuh).
@@ -357,18 +303,10 @@ __global__ void __launch_bounds__(NTHREADS, (NTOK > 2 ? 1 : 2)) qmv_rw_kernel(co
     const uint32_t x_area = (uint32_t)NTOK * (uint32_t)(((p.x_floats * 4) + 127) & ~127);   // one row per token
     const uint32_t stage0 = xs + x_area + (uint32_t)(warp * S) * (uint32_t)p.stage_pitch;
 
-    int t_begin, t_end, wg;
-    if (p.chain) {
-        t_begin = 0;
-        t_end = p.n_tasks;
-        wg = (int)blockIdx.x * NW + warp;
-    } else {
-        int t = 0;
-        while (t + 1 < p.n_tasks && (int)blockIdx.x >= p.cta_begin[t + 1]) ++t;
-        t_begin = t;
-        t_end = t + 1;
-        wg = ((int)blockIdx.x - p.cta_begin[t]) * NW + warp;
-    }
+    int tt = 0;
+    while (tt + 1 < p.n_tasks && (int)blockIdx.x >= p.cta_begin[tt + 1]) ++tt;
+    const int t_begin = tt, t_end = tt + 1;
+    const int wg = ((int)blockIdx.x - p.cta_begin[tt]) * NW + warp;
 
     {
         const uint4 *src = reinterpret_cast<const uint4 *>(&p.t[0]);
@@ -402,7 +340,6 @@ __global__ void __launch_bounds__(NTHREADS, (NTOK > 2 ? 1 : 2)) qmv_rw_kernel(co
 
     pdl_wait();                                    // x is the previous kernel's output
     const Q4kSel sel = q4k_sel(lane & 3);
-    const bool coherent = p.ordered != 0;
     bool dead = false;
     int slot = 0;
     uint32_t phase = 0;
@@ -411,10 +348,6 @@ __global__ void __launch_bounds__(NTHREADS, (NTOK > 2 ? 1 : 2)) qmv_rw_kernel(co
     float2 xr[16][2];
     float xsa = 0.f, xsb = 0.f;
     for (int t = t_begin; t < t_end; ++t) {
-        if (p.ordered && t > t_begin) {
-            if (!rw_grid_barrier(p.sync, (unsigned)(t - t_begin) * gridDim.x) && threadIdx.x == 0)
-                atomicOr(p.err, DEVERR_TIMEOUT);
-        }
         const RwTask &tk = tasks[t];
         const int nch = tk.n_chunks;
         // The CTA copies the task's x into shared memory once (every thread a
@@ -424,7 +357,7 @@ __global__ void __launch_bounds__(NTHREADS, (NTOK > 2 ? 1 : 2)) qmv_rw_kernel(co
         const int cols_t = (nch - 1) * RW_CK + tk.last_cols;
         const uint32_t xrow = (uint32_t)((cols_t * 4 + 127) & ~127);   // bytes per token row of staged x
 #pragma unroll 1
-        for (int n = 0; n < NTOK; ++n) rw_stage_x(xs + (uint32_t)n * xrow, tk.x + (int64_t)n * cols_t, cols_t, coherent);
+        for (int n = 0; n < NTOK; ++n) rw_stage_x(xs + (uint32_t)n * xrow, tk.x + (int64_t)n * cols_t, cols_t, false);
         __syncthreads();
         int64_t a, b;
         rw_range(tk, wg, a, b);
@@ -550,7 +483,6 @@ __global__ void __launch_bounds__(NTHREADS, (NTOK > 2 ? 1 : 2)) qmv_rw_kernel(co
         }
         __syncthreads();                          // x stays until every warp is done with it
     }
-    if (p.ordered) rw_grid_exit(p.sync, gridDim.x);
     // after a timeout: let the copies still in flight land before the CTA
     // exits; if that wait runs out too, DEVERR_DRAIN marks the device's later
     // results as suspect (copies may land in shared memory after the exit)
@@ -576,7 +508,5 @@ cudaError_t launch_rw(const RwParamsT<NT> &p, int R, dim3 grid, size_t smem, cud
 // Several tokens (2..4), single launches (3 and 4: one CTA per SM).
 template <int FMT>
 cudaError_t launch_rw_mt(const RwParams1 &p, int n_tok, int R, dim3 grid, size_t smem, cudaStream_t stream, bool pdl);
-template <int FMT>
-cudaError_t rw_occupancy(int R, size_t smem, int *ctas_per_sm);
 
 }  // namespace qmv

@@ -50,12 +50,14 @@ constexpr int SK_SEG = 2048;                  // columns of one K-segment: 64 pe
 constexpr int SK_MAX_KSEGS = SK_NC;           // K-segments per row: a divisor of SK_NC
 constexpr int SK_MAX_RS = SK_NC;              // row slots per stage
 // header: full[stage][row slot], empty[stage], x_done, abort flag, segment weights
+// (the fused MoE kernel keeps its routed ids and weights, 64 bytes, in front
+// of the segment weights)
 constexpr int SK_FULL_OFF = 0;
-constexpr int SK_EMPTY_OFF = 8 * SK_MAX_STAGES * SK_MAX_RS;           // 768
-constexpr int SK_XDONE_OFF = SK_EMPTY_OFF + 8 * SK_MAX_STAGES;        // 832
-constexpr int SK_ABORT_OFF = SK_XDONE_OFF + 8;                        // 840
-constexpr int SK_WSEG_OFF = 896;                                      // float[SK_MAX_KSEGS]
-constexpr int SK_HDR = 1024;
+constexpr int SK_EMPTY_OFF = 8 * SK_MAX_STAGES * SK_MAX_RS;           // 768 for 12 consumer warps
+constexpr int SK_XDONE_OFF = SK_EMPTY_OFF + 8 * SK_MAX_STAGES;
+constexpr int SK_ABORT_OFF = SK_XDONE_OFF + 8;
+constexpr int SK_WSEG_OFF = (SK_ABORT_OFF + 8 + 63) / 64 * 64;       // [64 B of MoE routing] float[SK_MAX_KSEGS]
+constexpr int SK_HDR = (SK_WSEG_OFF + 64 + 4 * SK_MAX_KSEGS + 127) / 128 * 128;
 constexpr int SK_PART = 2 * SK_NC * 4 * 2 * 4;   // partials [row][group][segment] <= NC*R*G floats, double-buffered
 
 enum { SK_PLAIN = 0, SK_SWIGLU = 1, SK_GATHER = 2 };
@@ -111,6 +113,11 @@ struct SkParams {
     unsigned long long *amax_key;
     unsigned *amax_done;
     int32_t *amax_idx;
+    // weights of the next matvec in stream order (NULL: none): once its last
+    // copy is issued, CTA c starts moving its share of them into L2, so the
+    // next launch finds them there and HBM stays busy across the boundary
+    const uint8_t *pf;
+    int64_t pf_bytes;
     int *err;
     uint32_t debug_extra_tx; // test hook: bytes expected per row slot beyond those copied (0 in use)
 };
@@ -130,6 +137,7 @@ __device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes)
 }
 
 constexpr int SK_X_MAX_BYTES = 96 * 1024;    // largest x staged in shared memory (24576 floats)
+constexpr uint32_t SK_PF_PIECE = 64 * 1024;  // bytes per L2 prefetch request
 
 // Copies x into the swizzled x area of shared memory (float4 d at
 // 16 * rw_xswz(d)): n_rows rows of nr float4, row k from src + k * src_row
@@ -196,14 +204,78 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_cons
     const int T = p.tile_rows;
     const int n_st = r_end > r_begin ? (int)((r_end - r_begin + T - 1) / T) : 0;
 
-    if (threadIdx.x == 0) {
+    const uint64_t rbw = (uint64_t)p.row_bytes;   // bytes of one matrix row
+    const int n_xrow = MODE == SK_GATHER ? min(p.n_sel, p.ksegs) : 1;
+    // weights are read once per decode step: evict them from L2 first
+    const uint64_t wpol = l2_evict_first_policy();
+    auto wcopy = [&](uint32_t dst, const uint8_t *src, uint32_t bytes, uint32_t bar) {
+        bulk_g2s_hint(dst, src, bytes, bar, wpol);
+    };
+    // the copies of stage i into ring slot `slot` (producer lane 0)
+    auto issue = [&](int i, int slot) {
+        const int64_t r0 = r_begin + (int64_t)i * T;
+        const int tr = (int)min((int64_t)T, r_end - r0);
+        const uint32_t st = ring + (uint32_t)slot * pitch;
+        if (STAGE_BAR) {
+            const uint32_t bytes = (uint32_t)tr * (uint32_t)rbw;
+            mbar_arrive_expect_tx(full_bar(slot, 0), bytes + p.debug_extra_tx);
+            wcopy(st, p.W + (uint64_t)r0 * rbw, bytes, full_bar(slot, 0));
+        }
+        for (int rs = 0; rs < nrs && rs * R < tr && !STAGE_BAR; ++rs) {
+            const int ra = min(R, tr - rs * R);
+            const int64_t v0 = r0 + rs * R;
+            const uint32_t full = full_bar(slot, rs);
+            const uint32_t dst = st + (uint32_t)(rs * p.rs_bytes);
+            const uint32_t bytes = (uint32_t)ra * (uint32_t)rbw;
+            if (MODE == SK_PLAIN) {
+                mbar_arrive_expect_tx(full, bytes + p.debug_extra_tx);
+                wcopy(dst, p.W + (uint64_t)v0 * rbw, bytes, full);
+            } else if (MODE == SK_SWIGLU) {
+                const int k = (int)(v0 / p.inter);
+                const int64_t r = v0 - (int64_t)k * p.inter;
+                const int e = p.ids[k];
+                const bool valid = e >= 0 && e < p.n_expert;
+                mbar_arrive_expect_tx(full, (valid ? 2u * bytes : 0u) + p.debug_extra_tx);
+                if (valid) {
+                    const uint64_t off = (uint64_t)e * (uint64_t)p.expert_stride + (uint64_t)r * rbw;
+                    wcopy(dst, p.W + off, bytes, full);
+                    wcopy(dst + (uint32_t)R * (uint32_t)rbw, p.W2 + off, bytes, full);
+                }
+            } else {
+                const int n_seg = min(p.n_sel, p.ksegs);   // a row slot holds ksegs segments
+                uint32_t total = 0;
+                for (int k = 0; k < n_seg; ++k)
+                    if (sk_valid(p, k)) total += bytes;
+                mbar_arrive_expect_tx(full, total + p.debug_extra_tx);
+                for (int k = 0; k < n_seg; ++k) {
+                    const int e = p.ids[k];
+                    if (e < 0 || e >= p.n_expert) continue;
+                    wcopy(dst + (uint32_t)(k * R) * (uint32_t)rbw,
+                             p.W + (uint64_t)e * (uint64_t)p.expert_stride + (uint64_t)v0 * rbw, bytes, full);
+                }
+            }
+        }
+    };
+
+    // The producer initialises the barriers and, for a plain matrix (whose
+    // weights depend on no earlier kernel), issues the first stages before the
+    // CTA-wide barrier: the copies are in flight from the CTA's start.  The
+    // other threads meanwhile start x on its way into L2.
+    int pre = 0;
+    if (warp == SK_NC && lane == 0) {
         for (int s = 0; s < S; ++s) {
-            for (int r = 0; r < nrs; ++r) mbar_init(full_bar(s, r), 1);
+            for (int r = 0; r < (STAGE_BAR ? 1 : nrs); ++r) mbar_init(full_bar(s, r), 1);
             mbar_init(empty0 + 8u * (uint32_t)s, SK_NC);
         }
         mbar_init(xdone, SK_NC);
         *abort_flag = 0;
         fence_mbar_init();
+        if (MODE == SK_PLAIN) {
+            pre = min(n_st, p.x_in_ring ? S - 1 : S);
+            for (int i = 0; i < pre; ++i) issue(i, i);
+        }
+    } else if (threadIdx.x == 0) {
+        prefetch_l2(p.x, (uint32_t)(n_xrow * p.cols * 4));
     }
     __syncthreads();
     pdl_launch_dependents();
@@ -211,12 +283,11 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_cons
     if (warp == SK_NC) {
         // ------------------------------------------------------ producer --
         if (lane != 0) return;
-        // plain weights do not depend on earlier kernels; routed experts do (ids)
+        // routed experts depend on the previous kernel (ids)
         if (MODE != SK_PLAIN) pdl_wait();
-        const uint64_t rb = (uint64_t)p.row_bytes;
-        int issued = 0;
+        int issued = pre;
         bool ok = true;
-        for (int i = 0; i < n_st && ok; ++i) {
+        for (int i = pre; i < n_st && ok; ++i) {
             const int slot = i % S;
             const int round = i / S;
             if (round > 0) ok = mbar_wait_bounded_block(empty0 + 8u * (uint32_t)slot, (uint32_t)((round - 1) & 1));
@@ -228,49 +299,17 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_cons
             if (*abort_flag) break;           // a consumer timed out: stop re-arming stages
             // the slot was last read (and x, in slot S-1, written) through the generic proxy
             if (round > 0 || (p.x_in_ring && slot == S - 1)) fence_proxy_async_smem();
-            const int64_t r0 = r_begin + (int64_t)i * T;
-            const int tr = (int)min((int64_t)T, r_end - r0);
-            const uint32_t st = ring + (uint32_t)slot * pitch;
-            if (STAGE_BAR) {
-                const uint32_t bytes = (uint32_t)tr * (uint32_t)rb;
-                mbar_arrive_expect_tx(full_bar(slot, 0), bytes + p.debug_extra_tx);
-                bulk_g2s(st, p.W + (uint64_t)r0 * rb, bytes, full_bar(slot, 0));
-            }
-            for (int rs = 0; rs < nrs && rs * R < tr && !STAGE_BAR; ++rs) {
-                const int ra = min(R, tr - rs * R);
-                const int64_t v0 = r0 + rs * R;
-                const uint32_t full = full_bar(slot, rs);
-                const uint32_t dst = st + (uint32_t)(rs * p.rs_bytes);
-                const uint32_t bytes = (uint32_t)ra * (uint32_t)rb;
-                if (MODE == SK_PLAIN) {
-                    mbar_arrive_expect_tx(full, bytes + p.debug_extra_tx);
-                    bulk_g2s(dst, p.W + (uint64_t)v0 * rb, bytes, full);
-                } else if (MODE == SK_SWIGLU) {
-                    const int k = (int)(v0 / p.inter);
-                    const int64_t r = v0 - (int64_t)k * p.inter;
-                    const int e = p.ids[k];
-                    const bool valid = e >= 0 && e < p.n_expert;
-                    mbar_arrive_expect_tx(full, (valid ? 2u * bytes : 0u) + p.debug_extra_tx);
-                    if (valid) {
-                        const uint64_t off = (uint64_t)e * (uint64_t)p.expert_stride + (uint64_t)r * rb;
-                        bulk_g2s(dst, p.W + off, bytes, full);
-                        bulk_g2s(dst + (uint32_t)R * (uint32_t)rb, p.W2 + off, bytes, full);
-                    }
-                } else {
-                    const int n_seg = min(p.n_sel, p.ksegs);   // a row slot holds ksegs segments
-                    uint32_t total = 0;
-                    for (int k = 0; k < n_seg; ++k)
-                        if (sk_valid(p, k)) total += bytes;
-                    mbar_arrive_expect_tx(full, total + p.debug_extra_tx);
-                    for (int k = 0; k < n_seg; ++k) {
-                        const int e = p.ids[k];
-                        if (e < 0 || e >= p.n_expert) continue;
-                        bulk_g2s(dst + (uint32_t)(k * R) * (uint32_t)rb,
-                                 p.W + (uint64_t)e * (uint64_t)p.expert_stride + (uint64_t)v0 * rb, bytes, full);
-                    }
-                }
-            }
+            issue(i, slot);
             ++issued;
+        }
+        if (ok && p.pf != nullptr) {
+            // this CTA's share of the next matvec's weights (16-byte granules)
+            const uint64_t total = (uint64_t)p.pf_bytes & ~15ull;
+            const uint64_t share = ((total / gridDim.x) + 15u) & ~15ull;
+            const uint64_t b0 = share * blockIdx.x;
+            const uint64_t b1 = min(b0 + share, total);
+            for (uint64_t o = b0; o < b1; o += SK_PF_PIECE)
+                prefetch_l2(p.pf + o, (uint32_t)min((uint64_t)SK_PF_PIECE, b1 - o));
         }
         // let every copy land before the CTA can exit
         bool drained = true;
@@ -289,8 +328,6 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_cons
     }
 
     // -------------------------------------------------------- consumers --
-    const int n_xrow = MODE == SK_GATHER ? min(p.n_sel, p.ksegs) : 1;
-    if (threadIdx.x == 0) prefetch_l2(p.x, (uint32_t)(n_xrow * p.cols * 4));
     pdl_wait();                                    // x, h, ids and weights come from earlier kernels
     if (MODE == SK_GATHER) {
         // h_k at float offset k * SK_SEG of the x area (a K-segment per expert)
@@ -448,228 +485,6 @@ template <int FMT>
 cudaError_t launch_sk(const SkParams &p, int mode, int R, dim3 grid, size_t smem, cudaStream_t stream, bool pdl);
 
 // ---------------------------------------------------------------------------
-// Ordered chain of one-token matvecs in one persistent launch (the layer after
-// layer order of a decode step, BebeLM page, §核心算子 / §性能表现): task t+1
-// may read any earlier task's y.  One cooperative CTA per SM; for every task
-// each CTA takes its contiguous share of the rows.  The producer streams the
-// stages of all tasks in sequence and never waits for the grid, so while the
-// consumers cross the grid barrier between tasks the ring fills with the
-// next task's weights.  The consumers of every CTA finish task t (y written),
-// meet at a grid barrier, stage x of task t+1 through L2 (it may have been
-// written by another SM in this launch) and decode from an already filled
-// ring.
-constexpr int SKC_MAX_TASKS = 64;
-
-struct SkTask {
-    const uint8_t *W;
-    const float *x;          // [cols]
-    float *y;                // [rows]
-    int64_t rows;
-    int64_t row_bytes;
-    int64_t units_q;         // CTA c owns units_q + (c < units_r) units of R rows
-    int32_t units_r;
-    int32_t cols;
-    int32_t ksegs;           // consumer warps per row (a divisor of SK_NC)
-    int32_t seg_bytes;       // bytes of one 2048-column K-segment of a row
-    int32_t tile_rows;       // T = (SK_NC / ksegs) * R
-    int32_t pad_;
-};
-
-struct SkChainParams {
-    int32_t n_tasks;
-    int32_t n_stage;
-    int32_t stage_pitch;
-    int32_t x_off;           // byte offset of the x area from the ring start
-    unsigned *sync;          // {arrivals, exits} of the grid barrier, zero between launches
-    int *err;
-    uint32_t debug_extra_tx;
-    SkTask t[SKC_MAX_TASKS];
-};
-
-// This CTA's rows [a, b) of task tk (R rows per unit).
-template <int R>
-__device__ __forceinline__ void skc_rows(const SkTask &tk, int c, int64_t &a, int64_t &b)
-{
-    const int64_t u0 = (int64_t)c * tk.units_q + min(c, tk.units_r);
-    a = u0 * R;
-    b = min(tk.rows, (u0 + tk.units_q + (c < tk.units_r ? 1 : 0)) * R);
-}
-
-template <int FMT, int R>
-__global__ void __launch_bounds__(SK_THREADS, 1) qmv_skc_kernel(const __grid_constant__ SkChainParams p)
-{
-    static_assert(R == 1 || R == 2 || R == 4, "rows per consumer warp");
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int warp = (int)threadIdx.x >> 5, lane = (int)threadIdx.x & 31;
-    const uint32_t sraw = smem_addr(smem);
-    const uint32_t sbase = (sraw + 127u) & ~127u;          // the launch adds 128 spare bytes
-    uint8_t *const sgen = smem + (sbase - sraw);
-    const uint32_t full0 = sbase + SK_FULL_OFF, empty0 = sbase + SK_EMPTY_OFF;
-    volatile int *const abort_flag = reinterpret_cast<volatile int *>(sgen + SK_ABORT_OFF);
-    const uint32_t part0 = sbase + (uint32_t)SK_HDR;
-    const uint32_t ring = part0 + (uint32_t)SK_PART;
-    const uint32_t xs = ring + (uint32_t)p.x_off;
-    const int S = p.n_stage;
-    const uint32_t pitch = (uint32_t)p.stage_pitch;
-    const int c = (int)blockIdx.x;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(full0 + 8u * (uint32_t)s, 1);
-            mbar_init(empty0 + 8u * (uint32_t)s, SK_NC);
-        }
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    __syncthreads();
-
-    if (warp == SK_NC) {
-        // ------------------------------------------------------ producer --
-        if (lane != 0) return;
-        int i = 0;                                     // stage sequence over all tasks
-        bool ok = true;
-        for (int t = 0; t < p.n_tasks && ok; ++t) {
-            const SkTask &tk = p.t[t];
-            int64_t a, b;
-            skc_rows<R>(tk, c, a, b);
-            const uint64_t rb = (uint64_t)tk.row_bytes;
-            for (int64_t r0 = a; r0 < b; r0 += tk.tile_rows, ++i) {
-                const int slot = i % S, round = i / S;
-                if (round > 0 && !mbar_wait_bounded_block(empty0 + 8u * (uint32_t)slot, (uint32_t)((round - 1) & 1))) {
-                    atomicOr(p.err, DEVERR_TIMEOUT);
-                    ok = false;
-                    break;
-                }
-                if (*abort_flag) {
-                    ok = false;
-                    break;
-                }
-                if (round > 0) fence_proxy_async_smem();
-                const uint32_t bytes = (uint32_t)(min((int64_t)tk.tile_rows, b - r0) * (int64_t)rb);
-                const uint32_t full = full0 + 8u * (uint32_t)slot;
-                mbar_arrive_expect_tx(full, bytes + p.debug_extra_tx);
-                bulk_g2s(ring + (uint32_t)slot * pitch, tk.W + (uint64_t)r0 * rb, bytes, full);
-            }
-        }
-        // let every copy land before the CTA can exit
-        for (int j = max(0, i - S); j < i; ++j) {
-            if (!mbar_wait_bounded_block(full0 + 8u * (uint32_t)(j % S), (uint32_t)((j / S) & 1))) {
-                atomicOr(p.err, DEVERR_DRAIN);
-                break;
-            }
-        }
-        return;
-    }
-
-    // -------------------------------------------------------- consumers --
-    const Q4kSel sel = q4k_sel(lane & 3);
-    constexpr int SH = 5 - Log2<R>::v;
-    const bool leader = (lane & ((1 << SH) - 1)) == 0;
-    const int vk = lane >> SH;
-    bool dead = false;
-    int i = 0;
-    for (int t = 0; t < p.n_tasks; ++t) {
-        const SkTask &tk = p.t[t];
-        if (t > 0) {
-            // every CTA has written task t-1's y
-            named_bar_sync(1, SK_NC * 32);
-            if (threadIdx.x == 0) {
-                // release: this CTA's y stores (ordered before by the CTA barrier)
-                // become visible before the arrival; acquire: every CTA's stores
-                // are visible after the last arrival is seen
-                asm volatile("red.release.gpu.global.add.u32 [%0], 1;" :: "l"(p.sync) : "memory");
-                const unsigned target = (unsigned)t * gridDim.x;
-                const uint64_t t0 = global_timer_ns();
-                for (uint32_t n = 0;; ++n) {
-                    unsigned v;
-                    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p.sync) : "memory");
-                    if ((int)(v - target) >= 0) break;
-                    if ((n & 63u) == 63u && global_timer_ns() - t0 > 1000000000ull) {
-                        atomicOr(p.err, DEVERR_TIMEOUT);
-                        break;
-                    }
-                }
-            }
-            named_bar_sync(1, SK_NC * 32);
-        }
-        // x of this task through L2 (written earlier in this launch, possibly by another SM)
-        sk_stage_x<true>(xs, tk.x, 1, tk.cols >> 2, 0);
-        named_bar_sync(1, SK_NC * 32);
-        const int nk = tk.ksegs;
-        const int ks = warp % nk, rs = warp / nk;
-        const int seg_cols = min(SK_SEG, tk.cols - ks * SK_SEG);
-        float2 xr[16][2];
-        float xsa = 0.f, xsb = 0.f;
-        rw_load_x_smem<FMT>(xs, ks, seg_cols, lane, xr, xsa, xsb);
-        auto xp = [&](int gq, float2 &x02, float2 &x13) {
-            x02 = xr[gq][0];
-            x13 = xr[gq][1];
-        };
-        const bool have = 64 * (lane + 1) <= seg_cols;
-        const uint32_t rb = (uint32_t)tk.row_bytes;
-        uint32_t slice = (uint32_t)(rs * R) * rb + (uint32_t)ks * (uint32_t)tk.seg_bytes;
-        slice += lane_slice_off<FMT>(lane);
-        int64_t a, b;
-        skc_rows<R>(tk, c, a, b);
-        for (int64_t r0 = a; r0 < b; r0 += tk.tile_rows, ++i) {
-            const int slot = i % S;
-            const uint32_t st = ring + (uint32_t)slot * pitch;
-            const int ra = min(R, (int)min((int64_t)tk.tile_rows, b - r0) - rs * R);
-            if (ra > 0 && !dead &&
-                !__all_sync(0xFFFFFFFFu, mbar_wait_bounded_block(full0 + 8u * (uint32_t)slot, (uint32_t)((i / S) & 1)))) {
-                if (lane == 0) {
-                    atomicOr(p.err, DEVERR_TIMEOUT);
-                    *abort_flag = 1;
-                }
-                dead = true;
-            }
-            float acc[R];
-#pragma unroll
-            for (int k = 0; k < R; ++k) acc[k] = 0.f;
-            QMV_SK_ROWS_PRAGMA
-            for (int k = 0; k < R; ++k) {
-                float d = 0.f;
-                if (!dead && have && k < ra) {
-                    const uint32_t ad = st + slice + (uint32_t)k * rb;
-                    d = lane_dot<FMT>(ad, lane, sel, xp, xsa, xsb);
-                }
-#pragma unroll
-                for (int k2 = 0; k2 < R; ++k2)
-                    if (k2 == k) acc[k2] = d;
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(empty0 + 8u * (uint32_t)slot);
-            warp_transpose_reduce<R>(acc, lane);
-            const int64_t row = r0 + rs * R + vk;
-            if (nk == 1) {
-                if (leader && vk < ra) tk.y[row] = acc[0];
-            } else {
-                const uint32_t pb = part0 + (uint32_t)(i & 1) * (uint32_t)(SK_PART / 2);
-                if (leader) sts_f32(pb + 4u * (uint32_t)((rs * R + vk) * nk + ks), acc[0]);
-                named_bar_sync(2 + rs, 32 * nk);
-                if (ks == 0 && leader && vk < ra) {
-                    float s0 = 0.f;
-                    for (int k2 = 0; k2 < nk; ++k2) s0 += lds_f32(pb + 4u * (uint32_t)((rs * R + vk) * nk + k2));
-                    tk.y[row] = s0;
-                }
-            }
-        }
-    }
-    // the last CTA to leave puts the barrier words back to zero for the next launch
-    named_bar_sync(1, SK_NC * 32);
-    if (threadIdx.x == 0) {
-        const unsigned old = atomicAdd(p.sync + 1, 1u);
-        if (old == gridDim.x - 1u) {
-            atomicExch(p.sync, 0u);
-            atomicExch(p.sync + 1, 0u);
-        }
-    }
-}
-
-template <int FMT>
-cudaError_t launch_skc(const SkChainParams &p, int R, dim3 grid, size_t smem, cudaStream_t stream);
-
-// ---------------------------------------------------------------------------
 // The whole MoE FFN step in one cooperative launch (BebeLM page, §核心算子,
 // MoE前馈网络: sigmoid router, top-k by the biased score, weights normalised
 // over the unbiased scores; SwiGLU experts):
@@ -786,7 +601,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skm_kernel(const __grid_con
     volatile int *const abort_flag = reinterpret_cast<volatile int *>(sgen + SK_ABORT_OFF);
     int *const sids = reinterpret_cast<int *>(sgen + SK_WSEG_OFF);              // [8]
     float *const sg = reinterpret_cast<float *>(sgen + SK_WSEG_OFF + 32);      // [8] routed weights
-    float *const wseg = reinterpret_cast<float *>(sgen + SK_WSEG_OFF + 64);    // [12] segment weights (0: invalid)
+    float *const wseg = reinterpret_cast<float *>(sgen + SK_WSEG_OFF + 64);    // [ksegs] segment weights (0: invalid)
     const uint32_t part0 = sbase + (uint32_t)SK_HDR;
     const uint32_t ring = part0 + (uint32_t)SK_PART;
     const uint32_t xs = ring + (uint32_t)p.x_off;

@@ -285,16 +285,14 @@ def _chain_case(fmt, dims, seed):
 
 @pytest.mark.parametrize("fmt", [Q8_0, Q4_K, Q6_K])
 def test_qmv_chain_dependent_tasks(fmt):
-    # x of every task is the previous task's y: the grid barrier must order them
+    # x of every task is the previous task's y: the launches must be ordered
     dims = [2048, 3072, 2048, 16384, 2048, 8192, 2048] if fmt != Q6_K else [2048, 4096, 2048, 6144, 2048]
     _chain_case(fmt, dims, 80 + fmt)
 
 
-def test_qmv_chain_crosses_launch_split():
-    # 70 tasks (more than one persistent launch holds) on 512 x 512 Q4_K
-    # matrices; task t reads task t-1's output unless t % 3 == 0 (then a fresh
-    # x), so activations stay finite and task 64 depends on task 63 across the
-    # launch boundary
+def test_qmv_chain_long():
+    # 70 tasks on 512 x 512 Q4_K matrices; task t reads task t-1's output
+    # unless t % 3 == 0 (then a fresh x), so activations stay finite
     fmt, n, T = Q4_K, 512, 70
     x0 = synth.gen_x(1, n, 93, 0)[0]
     x0d = dev(x0)
@@ -320,9 +318,31 @@ def test_qmv_chain_fallback_shape_keeps_order():
     _chain_case(Q8_0, dims, 91)
 
 
-def test_qmv_chain_repeated_calls_reuse_the_barrier():
+def test_qmv_chain_repeated_calls():
     for rep in range(3):
         _chain_case(Q8_0, [1024, 2048, 512, 1024], 92 + rep)
+
+
+def test_qmv_chain_on_two_streams_at_once():
+    # the call keeps no state between calls: two chains may overlap
+    dims = [2048, 4096, 2048, 8192, 2048]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    cases = []
+    for s_i, st in enumerate(streams):
+        bufs = [dev(synth.gen_x(1, dims[0], 94 + s_i, 0)[0])] + [torch.full((d,), float("nan"), device="cuda")
+                                                                 for d in dims[1:]]
+        Ws = [synth.gen_blocks(Q8_0, dims[t + 1], dims[t], 94 + s_i, t) for t in range(len(dims) - 1)]
+        args = [(dev(W), dims[t + 1], dims[t], bufs[t], bufs[t + 1]) for t, W in enumerate(Ws)]
+        cases.append((st, bufs, Ws, args))
+    torch.cuda.synchronize()
+    for st, _, _, args in cases:
+        q.qmv_chain(Q8_0, args, st)
+    torch.cuda.synchronize()
+    for _, bufs, Ws, _ in cases:
+        outs = [b.cpu().numpy() for b in bufs]
+        for t in range(len(dims) - 1):
+            ref, bound = oracle.qmv(Q8_0, Ws[t], dims[t + 1], dims[t], outs[t][None, :])
+            within(outs[t + 1][None, :], ref, bound)
 
 
 # ------------------------------------------------------------ greedy argmax --
