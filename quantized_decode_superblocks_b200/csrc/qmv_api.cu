@@ -453,7 +453,7 @@ constexpr int64_t SK_CTA_SMEM = 210 * 1024;
 struct SkGeom {
     bool ok = false;
     int R = 0, T = 0, S = 0, ksegs = 1, x_in_ring = 0;
-    int64_t pitch = 0, rs_bytes = 0, x_off = 0;
+    int64_t pitch = 0, x_off = 0;
     size_t smem = 0;
 };
 
@@ -499,7 +499,6 @@ SkGeom sk_geom(int fmt, int mode, int64_t rows, int64_t cols, int n_sel = 1, int
         g.T = nrs * R;
         g.S = (int)S;
         g.pitch = pitch;
-        g.rs_bytes = rs_bytes;
         g.x_in_ring = in_ring ? 1 : 0;
         g.x_off = in_ring ? 0 : S * pitch;
         g.smem = (size_t)(128 + SK_HDR + SK_PART + S * pitch + (in_ring ? 0 : x_bytes));
@@ -524,7 +523,6 @@ int sk_launch(int fmt, int mode, SkParams &p, const SkGeom &g, const DevInfo &di
     p.tile_rows = g.T;
     p.n_stage = g.S;
     p.stage_pitch = (int32_t)g.pitch;
-    p.rs_bytes = (int32_t)g.rs_bytes;
     p.x_in_ring = g.x_in_ring;
     p.x_off = (int32_t)g.x_off;
     p.err = di.err;
@@ -1073,12 +1071,10 @@ int moe_ffn_routed(const float *logits, const float *bias, int n_expert, int top
         p.a_ksegs = ka;
         p.a_seg_bytes = SK_SEG / bw * bb;
         p.a_T = (SK_NC / ka) * R;
-        p.a_rs_bytes = (int32_t)(2 * R * rba);
         p.a_units_q = ua / ctas;
         p.a_units_r = (int32_t)(ua % ctas);
         p.b_ksegs = kb;
         p.b_T = (SK_NC / kb) * R;
-        p.b_rs_bytes = (int32_t)(kb * R * rbb);
         p.b_units_q = ub / ctas;
         p.b_units_r = (int32_t)(ub % ctas);
         p.n_stage = (int32_t)S;

@@ -9,11 +9,12 @@
 // This kernel is built for that:
 //   * each CTA owns one contiguous range of output rows; its producer warp
 //     (one elected lane) fills a ring of S shared-memory stages.  A stage
-//     holds T rows as nrs "row slots" of R rows; each row slot is filled by
-//     1-D bulk async copies of whole rows that complete on the row slot's own
-//     "full" mbarrier, so a consumer warp waits only for its own rows.  A
-//     stage is refilled once all twelve consumer warps have arrived on its
-//     "empty" mbarrier;
+//     holds T rows, contiguous per matrix, filled by a few 1-D bulk async
+//     copies of whole rows (one per matrix and run of rows of one expert)
+//     that complete on the stage's "full" mbarrier; the producer issues the
+//     first stages of a plain matrix before the CTA-wide barrier, and tags
+//     the copies to leave L2 first.  A stage is refilled once all twelve
+//     consumer warps have arrived on its "empty" mbarrier;
 //   * consumer warp w = (row slot, K-segment) takes its R rows of every stage
 //     (its 2048-column K-segment when rows are longer): wait, decode, release,
 //     reduce -- no copies, cursors or 64-bit bookkeeping in the consumer loop;
@@ -28,10 +29,11 @@
 //     one's CTA exits and streams its first stages while the rest finishes.
 // Three forms share the body (BebeLM page, §核心算子, MoE前馈网络):
 //   SK_PLAIN   y = W x (a matrix, or a row-concatenated fused projection);
-//   SK_SWIGLU  h[k][r] = silu(G_{ids[k]} x)[r] * (U_{ids[k]} x)[r]: a row slot
-//              holds R gate rows and the same R up rows of one routed expert;
+//   SK_SWIGLU  h[k][r] = silu(G_{ids[k]} x)[r] * (U_{ids[k]} x)[r]: a stage
+//              holds T gate rows, then the same T up rows;
 //   SK_GATHER  y[r] = sum_k g[k] (D_{ids[k]} h_k)[r]: K-segment k of a row is
-//              row r of expert ids[k]'s matrix, weighted and summed in k order.
+//              row r of expert ids[k]'s matrix (a stage holds T rows of each
+//              routed expert in turn), weighted and summed in k order.
 // An expert id outside [0, n_expert) copies nothing, contributes zero and
 // records QMV_DEVERR_EXPERT_ID.  Every wait is bounded (about a second): a
 // timeout records QMV_DEVERR_TIMEOUT, the warp stops decoding but keeps
@@ -75,12 +77,6 @@ enum { SK_PLAIN = 0, SK_SWIGLU = 1, SK_GATHER = 2 };
 #define QMV_SK_ROWS_PRAGMA _Pragma("unroll")
 #endif
 
-// SK_PLAIN: 1 = one bulk copy and one "full" mbarrier per stage (all row slots
-// wait for the whole stage), 0 = one of each per row slot.
-#ifndef QMV_SK_STAGE_BARRIER
-#define QMV_SK_STAGE_BARRIER 1      // measured faster on B200 (one copy per stage)
-#endif
-
 struct SkParams {
     const uint8_t *W;        // PLAIN: the matrix; SWIGLU: gate matrices; GATHER: down matrices
     const uint8_t *W2;       // SWIGLU: up matrices
@@ -103,7 +99,6 @@ struct SkParams {
     int32_t tile_rows;       // T = (SK_NC / ksegs) * R rows per stage
     int32_t n_stage;         // S
     int32_t stage_pitch;     // bytes per stage slot (multiple of 128, >= a stage + 16)
-    int32_t rs_bytes;        // bytes of one row slot's region in a stage
     int32_t x_in_ring;       // 1: x is staged in ring slot S-1 before its first fill
     int32_t x_off;           // else: byte offset of the x area from the ring start
     // PLAIN with a single K-segment: greedy argmax of y fused into the epilogue
@@ -189,12 +184,10 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_cons
     const uint32_t part0 = sbase + (uint32_t)SK_HDR;
     const uint32_t ring = part0 + (uint32_t)SK_PART;
     const int S = p.n_stage;
-    const int nrs = SK_NC / p.ksegs;
     const uint32_t pitch = (uint32_t)p.stage_pitch;
     const uint32_t xs = p.x_in_ring ? ring + (uint32_t)(S - 1) * pitch : ring + (uint32_t)p.x_off;
-    // one "full" mbarrier per stage (plain copies of whole stages) or per row slot
-    constexpr bool STAGE_BAR = MODE == SK_PLAIN && QMV_SK_STAGE_BARRIER;
-    auto full_bar = [&](int s, int r) { return full0 + 8u * (uint32_t)(s * SK_MAX_RS + (STAGE_BAR ? 0 : r)); };
+    // one "full" mbarrier per stage: every consumer waits for the whole stage
+    auto full_bar = [&](int s) { return full0 + 8u * (uint32_t)s; };
 
     // this CTA's rows
     const int c = (int)blockIdx.x;
@@ -211,48 +204,53 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_cons
     auto wcopy = [&](uint32_t dst, const uint8_t *src, uint32_t bytes, uint32_t bar) {
         bulk_g2s_hint(dst, src, bytes, bar, wpol);
     };
-    // the copies of stage i into ring slot `slot` (producer lane 0)
+    // The copies of stage i into ring slot `slot` (producer lane 0), all
+    // completing on the slot's one "full" barrier.  A stage's T rows are
+    // contiguous in shared memory per matrix: PLAIN one copy; SWIGLU the gate
+    // rows then (at T rows) the up rows, one copy of each per run of rows of
+    // one expert; GATHER expert k's rows at k T rows, one copy per expert.
     auto issue = [&](int i, int slot) {
         const int64_t r0 = r_begin + (int64_t)i * T;
         const int tr = (int)min((int64_t)T, r_end - r0);
         const uint32_t st = ring + (uint32_t)slot * pitch;
-        if (STAGE_BAR) {
+        const uint32_t full = full_bar(slot);
+        if (MODE == SK_PLAIN) {
             const uint32_t bytes = (uint32_t)tr * (uint32_t)rbw;
-            mbar_arrive_expect_tx(full_bar(slot, 0), bytes + p.debug_extra_tx);
-            wcopy(st, p.W + (uint64_t)r0 * rbw, bytes, full_bar(slot, 0));
-        }
-        for (int rs = 0; rs < nrs && rs * R < tr && !STAGE_BAR; ++rs) {
-            const int ra = min(R, tr - rs * R);
-            const int64_t v0 = r0 + rs * R;
-            const uint32_t full = full_bar(slot, rs);
-            const uint32_t dst = st + (uint32_t)(rs * p.rs_bytes);
-            const uint32_t bytes = (uint32_t)ra * (uint32_t)rbw;
-            if (MODE == SK_PLAIN) {
-                mbar_arrive_expect_tx(full, bytes + p.debug_extra_tx);
-                wcopy(dst, p.W + (uint64_t)v0 * rbw, bytes, full);
-            } else if (MODE == SK_SWIGLU) {
-                const int k = (int)(v0 / p.inter);
-                const int64_t r = v0 - (int64_t)k * p.inter;
-                const int e = p.ids[k];
-                const bool valid = e >= 0 && e < p.n_expert;
-                mbar_arrive_expect_tx(full, (valid ? 2u * bytes : 0u) + p.debug_extra_tx);
-                if (valid) {
-                    const uint64_t off = (uint64_t)e * (uint64_t)p.expert_stride + (uint64_t)r * rbw;
+            mbar_arrive_expect_tx(full, bytes + p.debug_extra_tx);
+            wcopy(st, p.W + (uint64_t)r0 * rbw, bytes, full);
+        } else if (MODE == SK_SWIGLU) {
+            // output row v = k * inter + r (expert slot k, row r of its matrices)
+            int k = (int)(r0 / p.inter);
+            int r = (int)(r0 - (int64_t)k * p.inter);
+            uint32_t total = 0;
+            for (int done = 0, kk = k, rr = r; done < tr; ++kk, rr = 0) {
+                const int run = min(tr - done, p.inter - rr);
+                if (sk_valid(p, kk)) total += 2u * (uint32_t)run * (uint32_t)rbw;
+                done += run;
+            }
+            mbar_arrive_expect_tx(full, total + p.debug_extra_tx);
+            for (int done = 0; done < tr; ++k, r = 0) {
+                const int run = min(tr - done, p.inter - r);
+                if (sk_valid(p, k)) {
+                    const uint64_t off = (uint64_t)p.ids[k] * (uint64_t)p.expert_stride + (uint64_t)r * rbw;
+                    const uint32_t dst = st + (uint32_t)done * (uint32_t)rbw;
+                    const uint32_t bytes = (uint32_t)run * (uint32_t)rbw;
                     wcopy(dst, p.W + off, bytes, full);
-                    wcopy(dst + (uint32_t)R * (uint32_t)rbw, p.W2 + off, bytes, full);
+                    wcopy(dst + (uint32_t)T * (uint32_t)rbw, p.W2 + off, bytes, full);
                 }
-            } else {
-                const int n_seg = min(p.n_sel, p.ksegs);   // a row slot holds ksegs segments
-                uint32_t total = 0;
-                for (int k = 0; k < n_seg; ++k)
-                    if (sk_valid(p, k)) total += bytes;
-                mbar_arrive_expect_tx(full, total + p.debug_extra_tx);
-                for (int k = 0; k < n_seg; ++k) {
-                    const int e = p.ids[k];
-                    if (e < 0 || e >= p.n_expert) continue;
-                    wcopy(dst + (uint32_t)(k * R) * (uint32_t)rbw,
-                             p.W + (uint64_t)e * (uint64_t)p.expert_stride + (uint64_t)v0 * rbw, bytes, full);
-                }
+                done += run;
+            }
+        } else {
+            const int n_seg = min(p.n_sel, p.ksegs);   // a stage holds ksegs experts' rows
+            const uint32_t bytes = (uint32_t)tr * (uint32_t)rbw;
+            uint32_t total = 0;
+            for (int k = 0; k < n_seg; ++k)
+                if (sk_valid(p, k)) total += bytes;
+            mbar_arrive_expect_tx(full, total + p.debug_extra_tx);
+            for (int k = 0; k < n_seg; ++k) {
+                if (!sk_valid(p, k)) continue;
+                wcopy(st + (uint32_t)(k * T) * (uint32_t)rbw,
+                      p.W + (uint64_t)p.ids[k] * (uint64_t)p.expert_stride + (uint64_t)r0 * rbw, bytes, full);
             }
         }
     };
@@ -264,7 +262,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_cons
     int pre = 0;
     if (warp == SK_NC && lane == 0) {
         for (int s = 0; s < S; ++s) {
-            for (int r = 0; r < (STAGE_BAR ? 1 : nrs); ++r) mbar_init(full_bar(s, r), 1);
+            mbar_init(full_bar(s), 1);
             mbar_init(empty0 + 8u * (uint32_t)s, SK_NC);
         }
         mbar_init(xdone, SK_NC);
@@ -314,14 +312,9 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_cons
         // let every copy land before the CTA can exit
         bool drained = true;
         for (int i = max(0, issued - S); i < issued && drained; ++i) {
-            const int64_t r0 = r_begin + (int64_t)i * T;
-            const int tr = (int)min((int64_t)T, r_end - r0);
-            for (int rs = 0; rs < (STAGE_BAR ? 1 : nrs) && rs * R < tr; ++rs) {
-                if (!mbar_wait_bounded_block(full_bar(i % S, rs), (uint32_t)((i / S) & 1))) {
-                    atomicOr(p.err, DEVERR_DRAIN);
-                    drained = false;
-                    break;
-                }
+            if (!mbar_wait_bounded_block(full_bar(i % S), (uint32_t)((i / S) & 1))) {
+                atomicOr(p.err, DEVERR_DRAIN);
+                drained = false;
             }
         }
         return;
@@ -360,10 +353,12 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_cons
     const bool have = 64 * (lane + 1) <= seg_cols;
     const Q4kSel sel = q4k_sel(lane & 3);
     const uint32_t rb = (uint32_t)p.row_bytes;
-    // this lane's slice within the warp's part of a row slot
-    uint32_t slice = (uint32_t)rs * (uint32_t)p.rs_bytes;
-    slice += (uint32_t)ks * (MODE == SK_GATHER ? (uint32_t)R * rb : (uint32_t)p.seg_bytes);
+    // this lane's slice of the warp's first row in a stage (layout: issue());
+    // SWIGLU's up rows follow the gate rows at gst
+    uint32_t slice = (uint32_t)(rs * R) * rb;
+    slice += (uint32_t)ks * (MODE == SK_GATHER ? (uint32_t)T * rb : (uint32_t)p.seg_bytes);
     slice += lane_slice_off<FMT>(lane);
+    const uint32_t gst = (uint32_t)T * rb;
     constexpr int V = G * R;
     constexpr int SH = 5 - Log2<V>::v;
     const bool leader = (lane & ((1 << SH) - 1)) == 0;
@@ -383,8 +378,8 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_cons
     for (int i = 0; i < n_st; ++i) {
         const int ra = min(R, (int)min((int64_t)T, r_end - r0) - rs * R);     // rows of this row slot
         bool rowok = ra > 0;
-        if (MODE == SK_SWIGLU && rowok) rowok = sk_valid(p, (int)((r0 + rs * R) / p.inter));
-        if (ra > 0 && !dead && !__all_sync(0xFFFFFFFFu, mbar_wait_bounded_block(full_bar(slot, rs), phase))) {
+        if (MODE == SK_SWIGLU && rowok) rowok = sk_valid(p, (int)(r0 + rs * R) / p.inter);
+        if (ra > 0 && !dead && !__all_sync(0xFFFFFFFFu, mbar_wait_bounded_block(full_bar(slot), phase))) {
             if (lane == 0) {
                 atomicOr(p.err, DEVERR_TIMEOUT);
                 *abort_flag = 1;
@@ -399,7 +394,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_cons
             const int k = j % R;
             float d = 0.f;
             if (!dead && rowok && have && k < ra) {
-                const uint32_t a = st + slice + (uint32_t)j * rb;
+                const uint32_t a = st + slice + (uint32_t)(j / R) * gst + (uint32_t)k * rb;
                 d = lane_dot<FMT>(a, lane, sel, xp, xsa, xsb);
             }
 #pragma unroll
@@ -519,12 +514,12 @@ struct SkMoeParams {
     const float *x;          // [hidden]
     float *h;                // [n_sel][inter]
     float *y;                // [hidden]
-    // step 2 (gate/up): K-segments of hidden, rows per stage, row slot bytes, CTA split
-    int32_t a_ksegs, a_seg_bytes, a_T, a_rs_bytes;
+    // step 2 (gate/up): K-segments of hidden, rows per stage, CTA split
+    int32_t a_ksegs, a_seg_bytes, a_T;
     int64_t a_units_q;
     int32_t a_units_r;
     // step 3 (down): one K-segment per routed expert
-    int32_t b_ksegs, b_T, b_rs_bytes;
+    int32_t b_ksegs, b_T;
     int64_t b_units_q;
     int32_t b_units_r;
     int32_t n_stage, stage_pitch, x_off;
@@ -669,43 +664,44 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skm_kernel(const __grid_con
             const uint32_t st = ring + (uint32_t)slot * pitch;
             const uint32_t full = full0 + 8u * (uint32_t)slot;
             if (i < na) {
-                // step 2: R gate rows then the same R up rows of one expert per row slot
-                const int64_t r0 = a_begin + (int64_t)i * p.a_T;
-                const int tr = (int)min((int64_t)p.a_T, a_end - r0);
+                // step 2: the stage's a_T gate rows, then the same up rows (at
+                // a_T rows), one copy of each per run of rows of one expert
+                const int r0 = (int)(a_begin + (int64_t)i * p.a_T);
+                const int tr = min(p.a_T, (int)(a_end - r0));
+                const int k0 = r0 / p.inter, q0 = r0 - k0 * p.inter;
                 uint32_t total = 0;
-                for (int rs = 0; rs * R < tr; ++rs) {
-                    const int64_t v0 = r0 + rs * R;
-                    if (valid((int)(v0 / p.inter))) total += 2u * (uint32_t)min(R, tr - rs * R) * (uint32_t)rga;
+                for (int done = 0, k = k0, rr = q0; done < tr; ++k, rr = 0) {
+                    const int run = min(tr - done, p.inter - rr);
+                    if (valid(k)) total += 2u * (uint32_t)run * (uint32_t)rga;
+                    done += run;
                 }
                 mbar_arrive_expect_tx(full, total + p.debug_extra_tx);
-                for (int rs = 0; rs * R < tr; ++rs) {
-                    const int64_t v0 = r0 + rs * R;
-                    const int k = (int)(v0 / p.inter);
-                    if (!valid(k)) continue;
-                    const uint32_t bytes = (uint32_t)min(R, tr - rs * R) * (uint32_t)rga;
-                    const uint64_t off = (uint64_t)sids[k] * (uint64_t)p.gu_stride + (uint64_t)(v0 - (int64_t)k * p.inter) * rga;
-                    const uint32_t dst = st + (uint32_t)(rs * p.a_rs_bytes);
-                    bulk_g2s(dst, p.G + off, bytes, full);
-                    bulk_g2s(dst + (uint32_t)R * (uint32_t)rga, p.U + off, bytes, full);
+                for (int done = 0, k = k0, rr = q0; done < tr; ++k, rr = 0) {
+                    const int run = min(tr - done, p.inter - rr);
+                    if (valid(k)) {
+                        const uint64_t off = (uint64_t)sids[k] * (uint64_t)p.gu_stride + (uint64_t)rr * rga;
+                        const uint32_t dst = st + (uint32_t)done * (uint32_t)rga;
+                        const uint32_t bytes = (uint32_t)run * (uint32_t)rga;
+                        bulk_g2s(dst, p.G + off, bytes, full);
+                        bulk_g2s(dst + (uint32_t)p.a_T * (uint32_t)rga, p.U + off, bytes, full);
+                    }
+                    done += run;
                 }
             } else {
-                // step 3: per row slot, R rows of every routed expert's down matrix
+                // step 3: the stage's b_T rows of every routed expert's down
+                // matrix, expert k at k * b_T rows: one copy per expert
                 const int64_t r0 = b_begin + (int64_t)(i - na) * p.b_T;
                 const int tr = (int)min((int64_t)p.b_T, b_end - r0);
                 const int n_seg = min(p.n_sel, p.b_ksegs);
+                const uint32_t bytes = (uint32_t)tr * (uint32_t)rgb;
                 uint32_t total = 0;
-                for (int rs = 0; rs * R < tr; ++rs)
-                    for (int k = 0; k < n_seg; ++k)
-                        if (valid(k)) total += (uint32_t)min(R, tr - rs * R) * (uint32_t)rgb;
+                for (int k = 0; k < n_seg; ++k)
+                    if (valid(k)) total += bytes;
                 mbar_arrive_expect_tx(full, total + p.debug_extra_tx);
-                for (int rs = 0; rs * R < tr; ++rs) {
-                    const int64_t v0 = r0 + rs * R;
-                    const uint32_t bytes = (uint32_t)min(R, tr - rs * R) * (uint32_t)rgb;
-                    for (int k = 0; k < n_seg; ++k) {
-                        if (!valid(k)) continue;
-                        bulk_g2s(st + (uint32_t)(rs * p.b_rs_bytes) + (uint32_t)(k * R) * (uint32_t)rgb,
-                                 p.D + (uint64_t)sids[k] * (uint64_t)p.d_stride + (uint64_t)v0 * rgb, bytes, full);
-                    }
+                for (int k = 0; k < n_seg; ++k) {
+                    if (!valid(k)) continue;
+                    bulk_g2s(st + (uint32_t)(k * p.b_T) * (uint32_t)rgb,
+                             p.D + (uint64_t)sids[k] * (uint64_t)p.d_stride + (uint64_t)r0 * rgb, bytes, full);
                 }
             }
         }
@@ -747,8 +743,9 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skm_kernel(const __grid_con
         };
         const bool have = 64 * (lane + 1) <= seg_cols;
         const uint32_t rb = (uint32_t)p.gu_row_bytes;
-        uint32_t slice = (uint32_t)(rs * p.a_rs_bytes) + (uint32_t)ks * (uint32_t)p.a_seg_bytes;
+        uint32_t slice = (uint32_t)(rs * R) * rb + (uint32_t)ks * (uint32_t)p.a_seg_bytes;
         slice += lane_slice_off<FMT>(lane);
+        const uint32_t gst = (uint32_t)p.a_T * rb;        // the up rows follow the gate rows
         constexpr int V = 2 * R;
         constexpr int SH = 5 - Log2<V>::v;
         const bool leader = (lane & ((1 << SH) - 1)) == 0;
@@ -757,7 +754,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skm_kernel(const __grid_con
             const int slot = i % S;
             const uint32_t st = ring + (uint32_t)slot * pitch;
             const int ra = min(R, (int)min((int64_t)p.a_T, a_end - r0) - rs * R);
-            const bool rowok = ra > 0 && valid((int)((r0 + rs * R) / p.inter));
+            const bool rowok = ra > 0 && valid((int)(r0 + rs * R) / p.inter);
             wait_stage(slot, i);
             float acc[V];
 #pragma unroll
@@ -767,7 +764,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skm_kernel(const __grid_con
                 const int k = j % R;
                 float d = 0.f;
                 if (!dead && rowok && have && k < ra) {
-                    const uint32_t a = st + slice + (uint32_t)j * rb;
+                    const uint32_t a = st + slice + (uint32_t)(j / R) * gst + (uint32_t)k * rb;
                     d = lane_dot<FMT>(a, lane, sel, xp, xsa, xsb);
                 }
 #pragma unroll
@@ -830,7 +827,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skm_kernel(const __grid_con
         };
         const bool have = 64 * (lane + 1) <= seg_cols;
         const uint32_t rb = (uint32_t)p.d_row_bytes;
-        uint32_t slice = (uint32_t)(rs * p.b_rs_bytes) + (uint32_t)(ks * R) * rb;
+        uint32_t slice = (uint32_t)(rs * R) * rb + (uint32_t)(ks * p.b_T) * rb;
         slice += lane_slice_off<FMT>(lane);
         constexpr int SH = 5 - Log2<R>::v;
         const bool leader = (lane & ((1 << SH) - 1)) == 0;
