@@ -83,6 +83,14 @@ def source_hash():
     return h.hexdigest()[:16]
 
 
+def step_config(n_tok):
+    """The workload of a bench line, the same for both arms."""
+    weight_bytes = sum(synth.matrix_bytes(Q8_0, rows, cols) for (_, _, _, rows, cols) in sweep_layers())
+    return {"workload": WORKLOAD, "n_tok": n_tok, "layers": synth.CFG4_LAYERS,
+            "weight_bytes_per_step": weight_bytes,
+            "l2": "inputs larger than L2 (1.03 GB of weights per step, L2 126 MB)"}
+
+
 def sweep_layers():
     return [(l, m, name, rows, cols) for l in range(synth.CFG4_LAYERS)
             for m, (name, rows, cols) in enumerate(synth.workload_cfg4_layer())]
@@ -443,6 +451,91 @@ def measure_moe(torch, q, stream, reps=200, separate=False):
             "single_launch_timing": "one step alone, PDL off, CUDA events around it"}
 
 
+def measure_lfm_mix(torch, q, stream, reps=10):
+    """One decode token of the LFM2.5-style 24-layer mix (synth.workload_lfm_mix):
+    per layer the attention (fused QK, V, O) or short-convolution (in / out
+    projection) matvecs, then the routed MoE FFN step (moe_ffn_routed, its own
+    router logits per layer), and finally the vocabulary projection with greedy
+    argmax -- 79 library calls in decode order, captured as one CUDA graph.
+    Every layer has its own weights on the device (4.9 GB in all, each layer's
+    a block-rotated copy of one generated set, so no two layers share data);
+    a token streams about 1 GB of them.  Activations chain from call to call
+    (each call reads the previous output) without norms or the convolution
+    and attention arithmetic, which are not matvecs: a bandwidth workload, not
+    a forward pass."""
+    w = synth.workload_lfm_mix()
+    seed, L, mo = w["seed"], w["layers"], w["moe"]
+    E, hidden, inter, top_k = mo["n_expert"], mo["hidden"], mo["inter"], mo["top_k"]
+
+    def rotated(host, fmt, layer):
+        t = torch.from_numpy(host).cuda()
+        nb = host.size // synth.BLOCK_BYTES[fmt]
+        return torch.roll(t, shifts=int((layer * 7919) % nb) * synth.BLOCK_BYTES[fmt]) if layer else t
+
+    base = {}
+    for name, fmt, rows, cols in w["attention"] + w["conv"]:
+        base[name] = (fmt, rows, cols, synth.gen_blocks(fmt, rows, cols, seed, len(base) + 1))
+    gus, ds = synth.matrix_bytes(Q4_K, inter, hidden), synth.matrix_bytes(Q4_K, hidden, inter)
+    ex_host = [synth.gen_blocks(Q4_K, inter * E, hidden, seed, 10), synth.gen_blocks(Q4_K, inter * E, hidden, seed, 11),
+               synth.gen_blocks(Q4_K, hidden * E, inter, seed, 12)]
+    vf, vrows, vcols = w["vocab"]
+    vocab = torch.from_numpy(synth.gen_blocks(vf, vrows, vcols, seed, 13)).cuda()
+    layers = []
+    touched = synth.matrix_bytes(vf, vrows, vcols)
+    for l in range(L):
+        kind = "attention" if synth.lfm_attention_layer(l) else "conv"
+        mats = [(base[n][0], base[n][1], base[n][2], rotated(base[n][3], base[n][0], l)) for n, *_ in w[kind]]
+        experts = [rotated(h, Q4_K, l) for h in ex_host]
+        logits, bias = synth.gen_router(E, seed, 100 + l)
+        layers.append((kind, mats, experts, torch.from_numpy(logits).cuda(), torch.from_numpy(bias).cuda()))
+        touched += sum(synth.matrix_bytes(f, r, c) for f, r, c, _ in mats) + top_k * (2 * gus + ds)
+    h = torch.from_numpy(synth.gen_x(1, hidden, seed, 20)[0]).cuda()
+    h2 = torch.empty(hidden, device="cuda")
+    y_big = torch.empty(3 * hidden, device="cuda")
+    y_v = torch.empty(512, device="cuda")
+    ids = torch.empty(top_k, dtype=torch.int32, device="cuda")
+    g = torch.empty(top_k, device="cuda")
+    hs = torch.empty((top_k, inter), device="cuda")
+    ws = torch.zeros(q.MOE_WS_BYTES // 8, dtype=torch.int64, device="cuda")
+    vlog = torch.empty(vrows, device="cuda")
+    idx = torch.empty(1, dtype=torch.int32, device="cuda")
+    n_calls = 0
+
+    def token():
+        nonlocal n_calls
+        n_calls = 0
+        for kind, mats, (G, U, D), lg, bs in layers:
+            if kind == "attention":
+                (fq, rq, cq, Wq), (fv, rv, cv, Wv), (fo, ro, co, Wo) = mats
+                q.qmv_f32(fq, Wq, rq, cq, h, y_big)
+                q.qmv_f32(fv, Wv, rv, cv, h, y_v)
+                q.qmv_f32(fo, Wo, ro, co, y_big, h2)           # stand-in for the attention output
+                n_calls += 3
+            else:
+                (fi, ri, ci, Wi), (fo, ro, co, Wo) = mats
+                q.qmv_f32(fi, Wi, ri, ci, h, y_big)
+                q.qmv_f32(fo, Wo, ro, co, y_big, h2)           # stand-in for the gated convolution output
+                n_calls += 2
+            q.moe_ffn_routed(lg, bs, E, top_k, Q4_K, G, U, gus, Q4_K, D, ds, hidden, inter, h2, ids, g, hs, h, ws)
+            n_calls += 1
+        q.qmv_argmax(vf, vocab, vrows, vcols, h, vlog, 1, idx)
+        n_calls += 1
+
+    gr = capture(torch, token, stream)
+    time_graph(torch, gr, 3, stream)
+    sec = time_graph(torch, gr, reps, stream) / reps
+    del gr
+    assert q.qmv_check(stream) == 0
+    return {"workload": "LFM2.5-style decode token: 24 layers (6 attention: QK 2560x2048 Q4_K, V 512x2048 Q6_K, "
+                        "O 2048x2048 Q4_K; 18 short convolution: in 6144x2048, out 2048x2048 Q4_K), a top-4-of-32 "
+                        "Q4_K MoE FFN (1792) per layer, Q6_K vocabulary 128000x2048 with greedy argmax",
+            "calls": f"{n_calls} library calls per token (qmv_f32, moe_ffn_routed, qmv_argmax) in one CUDA graph",
+            "us": sec * 1e6, "tokens_per_s": round(1.0 / sec, 1), "weight_gbs": touched / sec / 1e9,
+            "weight_bytes_per_token": touched,
+            "timing": "graph of one token's calls, replayed; CUDA events; weights of all 24 layers resident "
+                      "(no L2 reuse across layers)"}
+
+
 # ----------------------------------------------------------- reference arm --
 
 def cpu_info():
@@ -541,7 +634,8 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(dt / args.steps * 1e3, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "n_tok": 1, "parallelism": "host cores (oracle)"},
+            "config": step_config(args.n_tok),
+            "run": {"parallelism": "host cores (oracle)"},
             "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -692,6 +786,8 @@ def main():
                 torch, q, stream, Q6_K, 128000, 2048, 1, 2, reps=20, argmax=True)
             per_config["cfg3_moe_ffn_step"] = measure_moe(torch, q, stream)
             per_config["cfg3_moe_route_then_ffn"] = measure_moe(torch, q, stream, separate=True)
+            per_config["lfm2_5_style_mix_token"] = measure_lfm_mix(torch, q, stream)
+            torch.cuda.empty_cache()
             for nt in (1, 2, 4, 8):
                 sw = Sweep(torch, q, nt, cache)
                 for md in (("launches", "chain", "grouped") if nt == 1 else ("launches", "grouped")):
@@ -752,14 +848,13 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "n_tok": args.n_tok, "layers": synth.CFG4_LAYERS,
-                   "weight_bytes_per_step": sweep.weight_bytes, "launches_per_step": sweep.launches,
-                   "l2": "inputs larger than L2 (1.03 GB of weights per step, L2 126 MB)",
-                   "timing": "CUDA graph of the step's C-ABI calls, replayed; CUDA events on the launch stream",
-                   "mode": mode,
-                   "pdl": not args.no_pdl,
-                   "order": "decode order: every matvec reads its x after the previous one has finished",
-                   "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"},
+        "config": step_config(args.n_tok),
+        "run": {"launches_per_step": sweep.launches,
+                "timing": "CUDA graph of the step's C-ABI calls, replayed; CUDA events on the launch stream",
+                "mode": mode,
+                "pdl": not args.no_pdl,
+                "order": "decode order: every matvec reads its x after the previous one has finished",
+                "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"},
         "frac_of_hbm_peak": round(value / dist.world / hbm_peak, 4),
         "us_per_step": round(ms_per_step * 1e3, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",

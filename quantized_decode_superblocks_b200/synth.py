@@ -128,3 +128,28 @@ def workload_cfg4_layer():
 
 CFG4_LAYERS = 16
 CFG4_SEED = 4
+
+LFM_LAYERS = 24
+LFM_SEED = 5
+
+
+def lfm_attention_layer(layer: int) -> bool:
+    """Six of the 24 layers are attention layers, spread evenly: every fourth,
+    from layer 3 (the pages say only that they are sparsely distributed)."""
+    return layer % 4 == 3
+
+
+def workload_lfm_mix():
+    """One decode token of an LFM2.5-style decoder (BebeLM：纯Rust实现的端侧大模型
+    推理引擎, §独特的层设计, §门控短卷积, §量化格式支持, §核心算子): hidden 2048,
+    24 layers -- 6 GQA attention layers (32 query / 8 KV heads of 64) and 18
+    gated short-convolution layers -- each followed by a top-4-of-32 MoE FFN,
+    then the 128000-row vocabulary projection with greedy argmax.  Weights are
+    Q4_K except the sensitive tensors the page names, which are Q6_K (the
+    attention V projection and the vocabulary).  The weight matvecs of one
+    layer kind, in order, as (name, fmt, rows, cols):"""
+    return dict(
+        attention=[("qk", Q4_K, 2560, 2048), ("v", Q6_K, 512, 2048), ("o", Q4_K, 2048, 2048)],
+        conv=[("in_proj", Q4_K, 3 * 2048, 2048), ("out_proj", Q4_K, 2048, 2048)],
+        moe=dict(fmt=Q4_K, n_expert=32, top_k=4, hidden=2048, inter=1792),
+        vocab=(Q6_K, 128000, 2048), layers=LFM_LAYERS, seed=LFM_SEED)
