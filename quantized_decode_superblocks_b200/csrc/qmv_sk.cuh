@@ -133,6 +133,10 @@ __device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes)
 
 constexpr int SK_X_MAX_BYTES = 96 * 1024;    // largest x staged in shared memory (24576 floats)
 constexpr uint32_t SK_PF_PIECE = 64 * 1024;  // bytes per L2 prefetch request
+// Stages of a plain matrix issued before x is loaded (measured on B200: two
+// beat one, three and the whole ring -- the Q8_0 gate/up 16384x2048 matvec
+// 9.0 against 9.7 us with the whole ring).
+constexpr int SK_HEAD_START = 2;
 
 // Copies x into the swizzled x area of shared memory (float4 d at
 // 16 * rw_xswz(d)): n_rows rows of nr float4, row k from src + k * src_row
@@ -256,9 +260,9 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_cons
     };
 
     // The producer initialises the barriers and, for a plain matrix (whose
-    // weights depend on no earlier kernel), issues the first stages before the
-    // CTA-wide barrier: the copies are in flight from the CTA's start.  The
-    // other threads meanwhile start x on its way into L2.
+    // weights depend on no earlier kernel), issues the first SK_HEAD_START
+    // stages before the CTA-wide barrier: the copies are in flight from the
+    // CTA's start.  The other threads meanwhile start x on its way into L2.
     int pre = 0;
     if (warp == SK_NC && lane == 0) {
         for (int s = 0; s < S; ++s) {
@@ -269,7 +273,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_cons
         *abort_flag = 0;
         fence_mbar_init();
         if (MODE == SK_PLAIN) {
-            pre = min(n_st, p.x_in_ring ? S - 1 : S);
+            pre = min(n_st, min(p.x_in_ring ? S - 1 : S, SK_HEAD_START));
             for (int i = 0; i < pre; ++i) issue(i, i);
         }
     } else if (threadIdx.x == 0) {
@@ -285,6 +289,13 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_sk_kernel(const __grid_cons
         if (MODE != SK_PLAIN) pdl_wait();
         int issued = pre;
         bool ok = true;
+        // after the head start, the rest of the ring waits until x is in the
+        // warps' registers: x's loads then do not queue behind a whole ring of
+        // weight copies (the head start keeps HBM busy meanwhile)
+        if (MODE == SK_PLAIN && pre < n_st && !mbar_wait_bounded_block(xdone, 0u)) {
+            atomicOr(p.err, DEVERR_TIMEOUT);
+            ok = false;
+        }
         for (int i = pre; i < n_st && ok; ++i) {
             const int slot = i % S;
             const int round = i / S;
