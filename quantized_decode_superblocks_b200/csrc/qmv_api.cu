@@ -12,6 +12,7 @@
 #include "qmv_misc.cuh"
 #include "qmv_rw.cuh"
 #include "qmv_sk.cuh"
+#include "qmv_skt.cuh"
 #include "qmv_tc.cuh"
 
 namespace {
@@ -467,10 +468,11 @@ int sk_ksegs(int64_t nseg)
     return 0;
 }
 
-// Geometry of a streaming-kernel launch.  mode SK_PLAIN: rows x cols; SK_SWIGLU:
+// Geometry of a streaming-kernel launch.  mode SK_PLAIN: rows x cols (n_tok
+// tokens: every token's x stays in shared memory after the ring); SK_SWIGLU:
 // n_sel experts of inter rows x cols (gate and up); SK_GATHER: rows of n_sel
 // expert segments of cols columns each.
-SkGeom sk_geom(int fmt, int mode, int64_t rows, int64_t cols, int n_sel = 1, int64_t inter = 0)
+SkGeom sk_geom(int fmt, int mode, int64_t rows, int64_t cols, int n_sel = 1, int64_t inter = 0, int n_tok = 1)
 {
     SkGeom g;
     const int bw = block_weights(fmt), bb = block_bytes(fmt);
@@ -482,17 +484,17 @@ SkGeom sk_geom(int fmt, int mode, int64_t rows, int64_t cols, int n_sel = 1, int
     if (g.ksegs == 0 || (mode == SK_GATHER && g.ksegs < n_sel)) return g;
     if (mode != SK_SWIGLU && (rows * rb) % 16 != 0) return g;   // the last copy ends on a 16-byte boundary
     // x staged in shared memory (GATHER: one 2048-column row per expert)
-    const int64_t x_bytes = mode == SK_GATHER ? (int64_t)g.ksegs * SK_SEG * 4 : ceil_div(cols * 4, 128) * 128;
-    if (x_bytes > SK_X_MAX_BYTES) return g;
+    const int64_t x_bytes = mode == SK_GATHER ? (int64_t)g.ksegs * SK_SEG * 4 : n_tok * ceil_div(cols * 4, 128) * 128;
+    if (x_bytes > SK_X_MAX_BYTES || (n_tok > 1 && mode != SK_PLAIN)) return g;
     const int64_t budget = SK_CTA_SMEM - SK_HDR - SK_PART;
-    const int r_pref = mode == SK_PLAIN && (fmt == QMV_Q4_K || fmt == QMV_Q5_K) ? 4 : 2;
+    const int r_pref = mode == SK_PLAIN && n_tok == 1 && (fmt == QMV_Q4_K || fmt == QMV_Q5_K) ? 4 : 2;
     for (int R = r_pref; R >= 1; R >>= 1) {
         if ((R * rb) % 16 != 0) continue;                 // every row slot's copies 16-byte aligned
         if (mode == SK_SWIGLU && inter % R != 0) continue; // a row slot never straddles two experts
         const int nrs = SK_NC / g.ksegs;
         const int64_t rs_bytes = (mode == SK_SWIGLU ? 2 : mode == SK_GATHER ? g.ksegs : 1) * R * rb;
         const int64_t pitch = ceil_div(nrs * rs_bytes + 16, 128) * 128;
-        const bool in_ring = x_bytes <= pitch;
+        const bool in_ring = n_tok == 1 && x_bytes <= pitch;
         const int64_t S = std::min<int64_t>(SK_MAX_STAGES, (budget - (in_ring ? 0 : x_bytes)) / pitch);
         if (S < (R > 1 ? 3 : 2)) continue;
         g.R = R;
@@ -532,6 +534,43 @@ int sk_launch(int fmt, int mode, SkParams &p, const SkGeom &g, const DevInfo &di
     cudaError_t e;
     e = by_fmt(fmt, [&](auto f) {
         return launch_sk<decltype(f)::value>(p, mode, g.R, dim3((unsigned)ctas), g.smem, st, pdl);
+    });
+    return e == cudaSuccess ? QMV_OK : cuda_fail(e);
+}
+
+// Several tokens (2..SKT_MAX_NTOK) of a plain matrix on the streaming kernel's
+// several-token form (qmv_skt.cuh); g from sk_geom(..., n_tok).
+int skt_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x, float *y, int n_tok,
+               const SkGeom &g, const DevInfo &di, cudaStream_t st)
+{
+    const int bw = block_weights(fmt), bb = block_bytes(fmt);
+    SkParams p{};
+    p.W = static_cast<const uint8_t *>(W);
+    p.x = x;
+    p.y = y;
+    p.rows = rows;
+    p.cols = (int32_t)cols;
+    p.row_bytes = cols / bw * bb;
+    p.n_sel = 1;
+    p.x_row = (int32_t)(ceil_div(cols * 4, 128) * 128);
+    const int64_t units = ceil_div(p.rows, (int64_t)g.R);
+    const int64_t ctas = std::max<int64_t>(1, std::min<int64_t>(di.sm_count, units));
+    p.units_q = units / ctas;
+    p.units_r = (int32_t)(units % ctas);
+    p.gran = g.R;
+    p.ksegs = g.ksegs;
+    p.seg_bytes = (int32_t)(SK_SEG / bw * bb);
+    p.tile_rows = g.T;
+    p.n_stage = g.S;
+    p.stage_pitch = (int32_t)g.pitch;
+    p.x_in_ring = 0;
+    p.x_off = (int32_t)g.x_off;
+    p.err = di.err;
+    p.debug_extra_tx = g_debug_extra_tx.load();
+    const bool pdl = g_pdl.load() != 0;
+    t_last_kernel = QMV_KERNEL_STREAM;
+    const cudaError_t e = by_fmt(fmt, [&](auto f) {
+        return launch_skt<decltype(f)::value>(p, n_tok, g.R, dim3((unsigned)ctas), g.smem, st, pdl);
     });
     return e == cudaSuccess ? QMV_OK : cuda_fail(e);
 }
@@ -742,6 +781,10 @@ int qmv_batched(int fmt, const void *W_blocks, int64_t rows, int64_t cols, const
     if (n_tok == 1) {
         const SkGeom g = sk_geom(fmt, SK_PLAIN, rows, cols);
         if (g.ok) return sk_single(fmt, W_blocks, rows, cols, x, y, g, di, reinterpret_cast<cudaStream_t>(stream));
+    } else if (n_tok <= SKT_MAX_NTOK) {
+        const SkGeom g = sk_geom(fmt, SK_PLAIN, rows, cols, 1, 0, n_tok);
+        if (g.ok)
+            return skt_single(fmt, W_blocks, rows, cols, x, y, n_tok, g, di, reinterpret_cast<cudaStream_t>(stream));
     }
     if (n_tok == 1 ? rw_preferred(fmt, rows, cols) : rw_mt_preferred(fmt, rows, cols, n_tok))
         return rw_single(fmt, W_blocks, rows, cols, x, y, n_tok, di, reinterpret_cast<cudaStream_t>(stream));

@@ -8,6 +8,7 @@
 
 #include "qmv_rw.cuh"
 #include "qmv_sk.cuh"
+#include "qmv_skt.cuh"
 #include "qmv_tc.cuh"
 
 namespace qmv {
@@ -226,6 +227,29 @@ cudaError_t launch_sk(const SkParams &p, int mode, int R, dim3 grid, size_t smem
     case SK_PLAIN: return launch_sk_mode<FMT, SK_PLAIN>(p, R, grid, smem, st, pdl);
     case SK_SWIGLU: return launch_sk_mode<FMT, SK_SWIGLU>(p, R, grid, smem, st, pdl);
     case SK_GATHER: return launch_sk_mode<FMT, SK_GATHER>(p, R, grid, smem, st, pdl);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+// The streaming kernel's several-token form (plain matrices).
+template <int FMT, int NTOK>
+static cudaError_t launch_skt_r(const SkParams &p, int R, dim3 grid, size_t smem, cudaStream_t st, bool pdl)
+{
+    static SmemCfg c1, c2;
+    switch (R) {
+    case 1: return launch_with(qmv_skt_kernel<FMT, 1, NTOK>, c1, p, grid, smem, st, pdl, false, SK_THREADS);
+    case 2: return launch_with(qmv_skt_kernel<FMT, 2, NTOK>, c2, p, grid, smem, st, pdl, false, SK_THREADS);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int FMT>
+cudaError_t launch_skt(const SkParams &p, int n_tok, int R, dim3 grid, size_t smem, cudaStream_t st, bool pdl)
+{
+    switch (n_tok) {
+    case 2: return launch_skt_r<FMT, 2>(p, R, grid, smem, st, pdl);
+    case 3: return launch_skt_r<FMT, 3>(p, R, grid, smem, st, pdl);
+    case 4: return launch_skt_r<FMT, 4>(p, R, grid, smem, st, pdl);
     default: return cudaErrorInvalidValue;
     }
 }

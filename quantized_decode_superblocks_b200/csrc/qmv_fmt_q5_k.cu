@@ -7,5 +7,6 @@ namespace qmv {
 template cudaError_t launch_pipeline<FMT_Q5_K>(const Params &, const KernelChoice &, dim3, size_t, cudaStream_t);
 template cudaError_t launch_multi<FMT_Q5_K>(const MultiParams &, const KernelChoice &, int, size_t, cudaStream_t);
 template cudaError_t launch_sk<FMT_Q5_K>(const SkParams &, int, int, dim3, size_t, cudaStream_t, bool);
+template cudaError_t launch_skt<FMT_Q5_K>(const SkParams &, int, int, dim3, size_t, cudaStream_t, bool);
 template cudaError_t launch_skm<FMT_Q5_K>(const SkMoeParams &, int, dim3, size_t, cudaStream_t);
 }  // namespace qmv

@@ -101,6 +101,7 @@ struct SkParams {
     int32_t stage_pitch;     // bytes per stage slot (multiple of 128, >= a stage + 16)
     int32_t x_in_ring;       // 1: x is staged in ring slot S-1 before its first fill
     int32_t x_off;           // else: byte offset of the x area from the ring start
+    int32_t x_row;           // several tokens: bytes from one token's staged x row to the next
     // PLAIN with a single K-segment: greedy argmax of y fused into the epilogue
     // (amax_idx != NULL).  Every CTA folds its best (value, row) into *amax_key;
     // the last CTA to arrive on *amax_done writes *amax_idx and puts both back

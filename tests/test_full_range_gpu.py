@@ -110,7 +110,9 @@ PATHS = [
     (Q6_K, 24, 1792, 1, GEN),                                                          # rows not 16-byte multiples
     (Q8_0, 33, 12288, 1, SK), (Q6_K, 8, 10240, 1, SK),                                 # streaming, 6 / 5 K-segments
     (Q4_K, 5, 12288, 1, SK), (Q8_0, 37, 96, 1, GEN),                                   # 6 K-segments; general
-    (Q8_0, 300, 2048, 2, WR), (Q4_K, 300, 2048, 2, WR), (Q6_K, 300, 2048, 2, WR),     # warp-ring, two tokens
+    (Q8_0, 300, 2048, 2, SK), (Q4_K, 300, 2048, 2, SK), (Q6_K, 300, 2048, 2, SK),     # streaming, two tokens
+    (Q8_0, 70, 8192, 2, SK), (Q4_K, 9, 12288, 2, SK), (Q6_K, 36, 1024, 3, SK),       # K-split rows; Q6_K 3 tokens
+    (Q6_K, 300, 8192, 4, WR),                                                          # warp-ring: 128 KB of x
     (Q8_0, 300, 2048, 3, TC), (Q4_K, 300, 2048, 3, TC), (Q6_K, 300, 2048, 3, TC),     # tensor cores
     (Q8_0, 300, 2048, 8, TC), (Q4_K, 300, 2048, 8, TC), (Q6_K, 300, 2048, 8, TC),
     (Q4_K, 9, 512, 5, TC),                                                             # a partial tensor-core tile

@@ -111,8 +111,9 @@ PATHS = [
     (Q5_K, 3, 256, 1, SK), (Q5_K, 20, 768, 1, SK),               # fewer rows than a row slot
     (Q4_0, 37, 96, 1, GEN),                                      # rows not whole block pairs
     (Q4_0, 9, 32768, 1, GEN), (Q5_K, 9, 32768, 1, GEN),          # x beyond the streaming kernel's
-    (Q4_0, 300, 2048, 2, GEN), (Q5_K, 300, 2048, 2, GEN),        # several tokens
-    (Q4_0, 300, 2048, 3, GEN), (Q5_K, 300, 2048, 5, GEN),
+    (Q4_0, 300, 2048, 2, SK), (Q5_K, 300, 2048, 2, SK),          # several tokens: streaming (2-4)
+    (Q4_0, 300, 2048, 3, SK), (Q5_K, 37, 4096, 4, SK),
+    (Q5_K, 300, 2048, 5, GEN),                                   # general (5-8)
     (Q4_0, 300, 2048, 8, GEN), (Q5_K, 300, 2048, 8, GEN),
     (Q4_0, 37, 96, 5, GEN), (Q5_K, 20, 768, 7, GEN),
     (Q4_0, 40, 16384, 4, GEN), (Q5_K, 40, 16384, 4, GEN),        # K-chunked rows

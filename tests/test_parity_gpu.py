@@ -140,15 +140,21 @@ def test_tensor_core_tiles(fmt, rows, cols, n_tok):
     within(y, ref, bound)
 
 
-# Q6_K takes it when rows are whole 2048-column runs: superblocks at every
-# 2-byte offset within their 16-byte-aligned slots, the last row's copy cut at
-# the end of the matrix
-@pytest.mark.parametrize("rows,cols", [(5, 2048), (16 * 148 * 2 + 7, 2048), (300, 4096), (16, 6144)])
-@pytest.mark.parametrize("n_tok", [3, 4, 8])
-def test_tensor_core_q6_k_tiles(rows, cols, n_tok):
+# Q6_K takes it when rows are whole 2048-column runs and every token's x fits
+# in shared memory beside two-stage rings: superblocks at every 2-byte offset
+# within their 16-byte-aligned slots, the last row's copy cut at the end of the
+# matrix.  The kernel that served each case is asserted; 8 tokens of 4096
+# columns (131 KB of split x) do not fit and take the general kernel.
+@pytest.mark.parametrize("rows,cols,n_tok,kernel", [
+    (5, 2048, 3, q.KERNEL_TENSOR_CORE), (5, 2048, 4, q.KERNEL_TENSOR_CORE), (5, 2048, 8, q.KERNEL_TENSOR_CORE),
+    (16 * 148 * 2 + 7, 2048, 3, q.KERNEL_TENSOR_CORE), (16 * 148 * 2 + 7, 2048, 8, q.KERNEL_TENSOR_CORE),
+    (300, 4096, 3, q.KERNEL_TENSOR_CORE), (300, 4096, 4, q.KERNEL_TENSOR_CORE), (16, 6144, 3, q.KERNEL_TENSOR_CORE),
+    (300, 4096, 8, q.KERNEL_GENERAL)])
+def test_tensor_core_q6_k_tiles(rows, cols, n_tok, kernel):
     W = synth.gen_blocks(Q6_K, rows, cols, seed=14, tensor_id=rows)
     x = synth.gen_x(n_tok, cols, seed=14, tensor_id=cols + n_tok)
     y = run_qmv(Q6_K, W, rows, cols, x)
+    assert q.qmv_debug_last_kernel() == kernel
     ref, bound = oracle.qmv(Q6_K, W, rows, cols, x, nthreads=8)
     within(y, ref, bound)
 
@@ -579,13 +585,15 @@ def test_moe_bad_expert_id_is_dropped_and_reported():
     assert np.array_equal(yh[1], np.zeros(rows, np.float32))
 
 
-@pytest.mark.parametrize("n_tok,kernel", [(1, q.KERNEL_STREAM), (2, q.KERNEL_WARP_RING), (8, q.KERNEL_TENSOR_CORE)])
-def test_stage_wait_timeout_is_reported_and_the_gpu_stays_usable(n_tok, kernel):
+@pytest.mark.parametrize("fmt,rows,cols,n_tok,kernel", [(Q8_0, 512, 2048, 1, q.KERNEL_STREAM),
+                                                     (Q8_0, 512, 2048, 2, q.KERNEL_STREAM),
+                                                     (Q6_K, 300, 8192, 4, q.KERNEL_WARP_RING),
+                                                     (Q8_0, 512, 2048, 8, q.KERNEL_TENSOR_CORE)])
+def test_stage_wait_timeout_is_reported_and_the_gpu_stays_usable(fmt, rows, cols, n_tok, kernel):
     # the test hook makes every tile expect 16 bytes more than are copied
-    # (one token: the streaming kernel; two: the warp-ring kernel; eight: the
+    # (the streaming kernel at one and two tokens, the warp-ring kernel, the
     # tensor-core kernel): each stage wait runs out (about a second), the
     # kernel records the timeout and finishes, and the context stays usable
-    fmt, rows, cols = Q8_0, 512, 2048
     W = synth.gen_blocks(fmt, rows, cols, 45, 0)
     x = synth.gen_x(n_tok, cols, 45, 1)
     y = torch.empty((n_tok, rows), device="cuda")
