@@ -76,6 +76,7 @@ struct Q4kSel {
     uint32_t sel_lo;    // c < 2: [s[j0], s[j1], s[j0+4], s[j1+4]] from (s0, s1); c >= 2: low-nibble bytes from (s2, s2)
     uint32_t sel_hi;    // c >= 2: [s[j0-4], s[j1-4], s[j0], s[j1]] from (s0, s1)
     bool upper;         // c >= 2
+    uint32_t magic;     // 0x4B000000 (the bits of 2^23), held in a register
 };
 
 __device__ __forceinline__ Q4kSel q4k_sel(int c)
@@ -83,6 +84,7 @@ __device__ __forceinline__ Q4kSel q4k_sel(int c)
     Q4kSel s;
     const uint32_t j0 = 2u * (uint32_t)c, j1 = j0 + 1u;
     s.upper = c >= 2;
+    asm volatile("mov.u32 %0, 0x4B000000;" : "=r"(s.magic));
     if (!s.upper) {
         s.sel_lo = j0 | (j1 << 4) | ((j0 + 4u) << 8) | ((j1 + 4u) << 12);
         s.sel_hi = 0;
@@ -152,6 +154,83 @@ __device__ __forceinline__ float q4_k_dot1(uint32_t sb, int c, const Q4kSel &sel
     const float d = half_bits_to_float(hdr.x);
     const float dmin = half_bits_to_float(hdr.x >> 16);
     // d*sc0*sa + d*sc1*sb - dmin*m0*xsa - dmin*m1*xsb
+    float r = (d * sc0_m0.x) * sa;
+    r = fmaf(d * sc1_m1.x, sbv, r);
+    r = fmaf(-dmin * sc0_m0.y, xsa, r);
+    r = fmaf(-dmin * sc1_m1.y, xsb, r);
+    return r;
+}
+
+// Q4_K slice against x whose groups are pre-scaled by the powers of two that
+// q4k_prescale_x applies.  Every nibble becomes a float with one bitwise op:
+// a nibble at bit s of a 32-bit word, s <= 16, masked and placed under the
+// exponent of 2^23 reads 2^23 + q 2^s, and one subtraction leaves q 2^s
+// exactly; x carries the matching 2^-s, so each product is the same q x as
+// with unscaled values (the masks replace the nibble split and the byte
+// permutes of q4_k_dot1: 9 integer ops per 8 weights instead of 11).  The
+// nibbles at bits 20..31 are read from v = w >> 16.
+//   low nibbles (sub-block 2c):  byte 0 at bit 0, byte 1 at bit 8, byte 2 at
+//     bit 16 (from w), byte 3 at bit 8 (from v)
+//   high nibbles (2c + 1):      bytes 0 / 1 at bits 4 / 12 of w, bytes 2 / 3
+//     at bits 4 / 12 of v
+template <uint32_t MASK>
+__device__ __forceinline__ float nib_f(uint32_t w, uint32_t magic)
+{
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(w), "n"(MASK), "r"(magic));   // (w & MASK) | magic
+    return __uint_as_float(r);
+}
+
+__device__ __forceinline__ void q4k_prescale_x(float2 (&xr)[16][2])
+{
+#pragma unroll
+    for (int gq = 0; gq < 16; ++gq) {
+        if (gq < 8) {
+            xr[gq][0].y *= 0x1p-16f;
+            xr[gq][1].x *= 0x1p-8f;
+            xr[gq][1].y *= 0x1p-8f;
+        } else {
+            xr[gq][0].x *= 0x1p-4f;
+            xr[gq][0].y *= 0x1p-4f;
+            xr[gq][1].x *= 0x1p-12f;
+            xr[gq][1].y *= 0x1p-12f;
+        }
+    }
+}
+
+template <class XP>
+__device__ __forceinline__ float q4_k_dot1s(uint32_t sb, int c, const Q4kSel &sel, XP &&xp, float xsa, float xsb)
+{
+    const uint4 qa = lds_v4(sb + 16u + 32u * (uint32_t)c);
+    const uint4 qb = lds_v4(sb + 32u + 32u * (uint32_t)c);
+    const uint32_t qw[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+    const float2 nb = make_float2(-8388608.0f, -8388608.0f);
+    const uint32_t mg = sel.magic;
+    float2 a0 = make_float2(0.f, 0.f), a1 = a0, b0 = a0, b1 = a0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t w = qw[i];
+        const uint32_t v = w >> 16;
+        const float2 lo02 = f2add(make_float2(nib_f<0x0000000Fu>(w, mg), nib_f<0x000F0000u>(w, mg)), nb);
+        const float2 lo13 = f2add(make_float2(nib_f<0x00000F00u>(w, mg), nib_f<0x00000F00u>(v, mg)), nb);
+        const float2 hi02 = f2add(make_float2(nib_f<0x000000F0u>(w, mg), nib_f<0x000000F0u>(v, mg)), nb);
+        const float2 hi13 = f2add(make_float2(nib_f<0x0000F000u>(w, mg), nib_f<0x0000F000u>(v, mg)), nb);
+        float2 xl02, xl13, xh02, xh13;
+        xp(i, xl02, xl13);
+        xp(8 + i, xh02, xh13);
+        a0 = f2fma(lo02, xl02, a0);
+        a1 = f2fma(lo13, xl13, a1);
+        b0 = f2fma(hi02, xh02, b0);
+        b1 = f2fma(hi13, xh13, b1);
+    }
+    const float2 sa2 = f2add(a0, a1), sb2 = f2add(b0, b1);
+    const float sa = sa2.x + sa2.y, sbv = sb2.x + sb2.y;
+    const uint4 hdr = lds_v4(sb);
+    const uint32_t sv = q4k_scales_mins(hdr.y, hdr.z, hdr.w, sel);  // bytes [sc0, sc1, m0, m1]
+    float2 sc0_m0, sc1_m1;
+    bytes4_to_f2(sv, 0.0f, sc0_m0, sc1_m1);
+    const float d = half_bits_to_float(hdr.x);
+    const float dmin = half_bits_to_float(hdr.x >> 16);
     float r = (d * sc0_m0.x) * sa;
     r = fmaf(d * sc1_m1.x, sbv, r);
     r = fmaf(-dmin * sc0_m0.y, xsa, r);

@@ -191,12 +191,13 @@ __device__ __forceinline__ float q8_0_dot_pair(uint32_t a, XP &&xp)
 // One token: lane l's 64-weight slice at shared address a against the x
 // groups xp holds (rw_group_col order); xsa / xsb are the sums of groups 0..7
 // and 8..15 (the K-quant min terms).
-template <int FMT, class XP>
+// PS: x holds the Q4_K groups pre-scaled by q4k_prescale_x (rw_load_x_smem<FMT, true>).
+template <int FMT, bool PS = true, class XP>
 __device__ __forceinline__ float lane_dot(uint32_t a, int l, const Q4kSel &sel, XP &&xp, float xsa, float xsb)
 {
     if (FMT == FMT_Q8_0) return q8_0_dot_pair(a, xp);
     if (FMT == FMT_Q4_0) return q4_0_dot_pair(a, xp);
-    if (FMT == FMT_Q4_K) return q4_k_dot1<false>(a, l & 3, sel, xp, xsa, xsb);
+    if (FMT == FMT_Q4_K) return PS ? q4_k_dot1s(a, l & 3, sel, xp, xsa, xsb) : q4_k_dot1<false>(a, l & 3, sel, xp, xsa, xsb);
     if (FMT == FMT_Q5_K) return q5_k_dot1<false>(a, l & 3, sel, xp, xsa, xsb);
     return q6_k_dot1(a, (l >> 1) & 1, 16 * (l & 1), xp);
 }
@@ -242,7 +243,7 @@ __device__ __forceinline__ void rw_stage_x(uint32_t xs, const float *x, int cols
     }
 }
 
-template <int FMT>
+template <int FMT, bool PS = true>
 __device__ __forceinline__ void rw_load_x_smem(uint32_t xs, int kc, int ncols, int lane, float2 (&xr)[16][2],
                                                float &xsa, float &xsb)
 {
@@ -259,6 +260,7 @@ __device__ __forceinline__ void rw_load_x_smem(uint32_t xs, int kc, int ncols, i
     }
     xsa = sa.x + sa.y;
     xsb = sb.x + sb.y;
+    if (FMT == FMT_Q4_K && PS) q4k_prescale_x(xr);     // the groups lane_dot<FMT, true> expects
 }
 
 // Accumulators of one row group: one token -> a float per row (factored
@@ -391,7 +393,7 @@ __global__ void __launch_bounds__(NTHREADS, (NTOK > 2 ? 1 : 2)) qmv_rw_kernel(co
                     uint32_t sa = rw_slice_addr<FMT>(st, lane);
 #pragma unroll
                     for (int k = 0; k < R; ++k, sa += cb) {
-                        acc.v[k] += lane_dot<FMT>(sa, lane, sel, xp, xsa, xsb);
+                        acc.v[k] += lane_dot<FMT, false>(sa, lane, sel, xp, xsa, xsb);
                     }
                 } else {
                     // several tokens: weights decoded once per step, each token's
@@ -455,7 +457,7 @@ __global__ void __launch_bounds__(NTHREADS, (NTOK > 2 ? 1 : 2)) qmv_rw_kernel(co
         };
         if (nch == 1) {
             // one token: x stays in registers for the whole task
-            if constexpr (NTOK == 1) rw_load_x_smem<FMT>(xs, 0, last_cols, lane, xr, xsa, xsb);
+            if constexpr (NTOK == 1) rw_load_x_smem<FMT, false>(xs, 0, last_cols, lane, xr, xsa, xsb);
             for (int64_t rg = a; rg < b; ++rg) {
                 RwAcc<R, NTOK> acc;
                 acc.zero();
@@ -472,7 +474,7 @@ __global__ void __launch_bounds__(NTHREADS, (NTOK > 2 ? 1 : 2)) qmv_rw_kernel(co
                 for (int kc = 0; kc < nch; ++kc) {
                     const bool lastc = kc == nch - 1;
                     const int ncols = lastc ? last_cols : RW_CK;
-                    if constexpr (NTOK == 1) rw_load_x_smem<FMT>(xs, kc, ncols, lane, xr, xsa, xsb);
+                    if constexpr (NTOK == 1) rw_load_x_smem<FMT, false>(xs, kc, ncols, lane, xr, xsa, xsb);
                     if (!tile(acc, ncols, lastc ? last_bytes : chunk_bytes, kc)) {
                         dead = true;
                         break;
