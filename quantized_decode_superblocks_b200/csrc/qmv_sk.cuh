@@ -755,9 +755,14 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skm_kernel(const __grid_con
         };
         const bool have = 64 * (lane + 1) <= seg_cols;
         const uint32_t rb = (uint32_t)p.gu_row_bytes;
-        uint32_t slice = (uint32_t)(rs * R) * rb + (uint32_t)ks * (uint32_t)p.a_seg_bytes;
+        uint32_t slice = (uint32_t)ks * (uint32_t)p.a_seg_bytes;
         slice += lane_slice_off<FMT>(lane);
         const uint32_t gst = (uint32_t)p.a_T * rb;        // the up rows follow the gate rows
+        // a stage gives row slot rs rows rs*R..; a short stage (no more rows
+        // than row slots: the last one of a CTA with a remainder unit) one row
+        // each, so that one warp does not decode R rows while the others wait
+        // at the grid barrier.  K-segment partials stay indexed by slot.
+        const int nrs = p.a_T / R;                         // row slots
         constexpr int V = 2 * R;
         constexpr int SH = 5 - Log2<V>::v;
         const bool leader = (lane & ((1 << SH) - 1)) == 0;
@@ -765,8 +770,11 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skm_kernel(const __grid_con
         for (int64_t r0 = a_begin; r0 < a_end; r0 += p.a_T, ++i) {
             const int slot = i % S;
             const uint32_t st = ring + (uint32_t)slot * pitch;
-            const int ra = min(R, (int)min((int64_t)p.a_T, a_end - r0) - rs * R);
-            const bool rowok = ra > 0 && valid((int)(r0 + rs * R) / p.inter);
+            const int tr = (int)min((int64_t)p.a_T, a_end - r0);
+            const bool spread = tr <= nrs;
+            const int rl = spread ? rs : rs * R;
+            const int ra = spread ? (rs < tr ? 1 : 0) : min(R, tr - rl);
+            const bool rowok = ra > 0 && valid((int)(r0 + rl) / p.inter);
             wait_stage(slot, i);
             float acc[V];
 #pragma unroll
@@ -776,7 +784,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skm_kernel(const __grid_con
                 const int k = j % R;
                 float d = 0.f;
                 if (!dead && rowok && have && k < ra) {
-                    const uint32_t a = st + slice + (uint32_t)(j / R) * gst + (uint32_t)k * rb;
+                    const uint32_t a = st + slice + (uint32_t)(rl + k) * rb + (uint32_t)(j / R) * gst;
                     d = lane_dot<FMT>(a, lane, sel, xp, xsa, xsb);
                 }
 #pragma unroll
@@ -786,7 +794,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skm_kernel(const __grid_con
             __syncwarp();
             if (lane == 0) mbar_arrive(empty0 + 8u * (uint32_t)slot);
             warp_transpose_reduce<V>(acc, lane);
-            const int64_t row = r0 + rs * R + vk;
+            const int64_t row = r0 + rl + vk;
             if (nk == 1) {
                 const float u = __shfl_down_sync(0xFFFFFFFFu, acc[0], R << SH);
                 if (leader && vg == 0 && vk < ra) p.h[row] = rowok ? acc[0] / (1.0f + expf(-acc[0])) * u : 0.f;
@@ -839,15 +847,19 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skm_kernel(const __grid_con
         };
         const bool have = 64 * (lane + 1) <= seg_cols;
         const uint32_t rb = (uint32_t)p.d_row_bytes;
-        uint32_t slice = (uint32_t)(rs * R) * rb + (uint32_t)(ks * p.b_T) * rb;
+        uint32_t slice = (uint32_t)(ks * p.b_T) * rb;
         slice += lane_slice_off<FMT>(lane);
+        const int nrs = p.b_T / R;
         constexpr int SH = 5 - Log2<R>::v;
         const bool leader = (lane & ((1 << SH) - 1)) == 0;
         const int vk = lane >> SH;
         for (int64_t r0 = b_begin; r0 < b_end; r0 += p.b_T, ++i) {
             const int slot = i % S;
             const uint32_t st = ring + (uint32_t)slot * pitch;
-            const int ra = min(R, (int)min((int64_t)p.b_T, b_end - r0) - rs * R);
+            const int tr = (int)min((int64_t)p.b_T, b_end - r0);
+            const bool spread = tr <= nrs;
+            const int rl = spread ? rs : rs * R;
+            const int ra = spread ? (rs < tr ? 1 : 0) : min(R, tr - rl);
             wait_stage(slot, i);
             float acc[R];
 #pragma unroll
@@ -856,7 +868,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skm_kernel(const __grid_con
             for (int k = 0; k < R; ++k) {
                 float d = 0.f;
                 if (!dead && have && k < ra) {
-                    const uint32_t a = st + slice + (uint32_t)k * rb;
+                    const uint32_t a = st + slice + (uint32_t)(rl + k) * rb;
                     d = lane_dot<FMT>(a, lane, sel, xp, xsa, xsb);
                 }
 #pragma unroll
@@ -866,7 +878,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skm_kernel(const __grid_con
             __syncwarp();
             if (lane == 0) mbar_arrive(empty0 + 8u * (uint32_t)slot);
             warp_transpose_reduce<R>(acc, lane);
-            const int64_t row = r0 + rs * R + vk;
+            const int64_t row = r0 + rl + vk;
             const uint32_t pb = part0 + (uint32_t)(i & 1) * (uint32_t)(SK_PART / 2);
             if (leader) sts_f32(pb + 4u * (uint32_t)((rs * R + vk) * nk + ks), acc[0]);
             named_bar_sync(2 + rs, 32 * nk);
