@@ -447,9 +447,9 @@ int rw_single(int fmt, const void *W, int64_t rows, int64_t cols, const float *x
 
 // ---------------------------------------------------------------------------
 // One-token streaming kernel (qmv_sk.cuh): one CTA of 12 consumer warps and a
-// producer warp per SM, stages of T whole rows in up to ~210 KB of shared
+// producer warp per SM, stages of T whole rows in up to ~226 KB of shared
 // memory.
-constexpr int64_t SK_CTA_SMEM = 210 * 1024;
+constexpr int64_t SK_CTA_SMEM = 226 * 1024;       // + the 128-byte alignment pad <= the 227 KB opt-in
 
 struct SkGeom {
     bool ok = false;

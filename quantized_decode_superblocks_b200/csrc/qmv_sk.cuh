@@ -136,7 +136,7 @@ constexpr int SK_X_MAX_BYTES = 96 * 1024;    // largest x staged in shared memor
 constexpr uint32_t SK_PF_PIECE = 64 * 1024;  // bytes per L2 prefetch request
 // Stages of a plain matrix issued before x is loaded (measured on B200: two
 // beat one, three and the whole ring -- the Q8_0 gate/up 16384x2048 matvec
-// 9.0 against 9.7 us with the whole ring).
+// 9.0 against 9.7 us with three of a four-stage ring or the whole ring).
 constexpr int SK_HEAD_START = 2;
 
 // Copies x into the swizzled x area of shared memory (float4 d at
