@@ -472,7 +472,8 @@ int sk_ksegs(int64_t nseg)
 // tokens: every token's x stays in shared memory after the ring); SK_SWIGLU:
 // n_sel experts of inter rows x cols (gate and up); SK_GATHER: rows of n_sel
 // expert segments of cols columns each.
-SkGeom sk_geom(int fmt, int mode, int64_t rows, int64_t cols, int n_sel = 1, int64_t inter = 0, int n_tok = 1)
+SkGeom sk_geom(int fmt, int mode, int64_t rows, int64_t cols, int n_sel = 1, int64_t inter = 0, int n_tok = 1,
+               int sms = 0)
 {
     SkGeom g;
     const int bw = block_weights(fmt), bb = block_bytes(fmt);
@@ -487,16 +488,24 @@ SkGeom sk_geom(int fmt, int mode, int64_t rows, int64_t cols, int n_sel = 1, int
     const int64_t x_bytes = mode == SK_GATHER ? (int64_t)g.ksegs * SK_SEG * 4 : n_tok * ceil_div(cols * 4, 128) * 128;
     if (x_bytes > SK_X_MAX_BYTES || (n_tok > 1 && mode != SK_PLAIN)) return g;
     const int64_t budget = SK_CTA_SMEM - SK_HDR - SK_PART;
-    const int r_pref = mode == SK_PLAIN && n_tok == 1 && (fmt == QMV_Q4_K || fmt == QMV_Q5_K) ? 4 : 2;
-    for (int R = r_pref; R >= 1; R >>= 1) {
-        if ((R * rb) % 16 != 0) continue;                 // every row slot's copies 16-byte aligned
-        if (mode == SK_SWIGLU && inter % R != 0) continue; // a row slot never straddles two experts
+    const int r_max = mode == SK_PLAIN && n_tok == 1 && (fmt == QMV_Q4_K || fmt == QMV_Q5_K) ? 4 : 2;
+    int r_pref = r_max;
+    if (sms > 0 && mode == SK_PLAIN && n_tok == 1) {
+        // a matrix whose share per CTA fills at most half of one stage: fewer
+        // rows per warp, so that every warp gets some (Q4_K 3072x2048: 21 rows
+        // a CTA on 12 warps of 2 rows rather than 6 warps of 4)
+        const int64_t per_cta = ceil_div(rows, (int64_t)sms);
+        while (r_pref > 1 && 2 * per_cta <= (int64_t)(SK_NC / g.ksegs) * r_pref) r_pref >>= 1;
+    }
+    auto fits = [&](int R) {
+        if ((R * rb) % 16 != 0) return false;             // every row slot's copies 16-byte aligned
+        if (mode == SK_SWIGLU && inter % R != 0) return false;   // a row slot never straddles two experts
         const int nrs = SK_NC / g.ksegs;
         const int64_t rs_bytes = (mode == SK_SWIGLU ? 2 : mode == SK_GATHER ? g.ksegs : 1) * R * rb;
         const int64_t pitch = ceil_div(nrs * rs_bytes + 16, 128) * 128;
         const bool in_ring = n_tok == 1 && x_bytes <= pitch;
         const int64_t S = std::min<int64_t>(SK_MAX_STAGES, (budget - (in_ring ? 0 : x_bytes)) / pitch);
-        if (S < (R > 1 ? 3 : 2)) continue;
+        if (S < (R > 1 ? 3 : 2)) return false;
         g.R = R;
         g.T = nrs * R;
         g.S = (int)S;
@@ -505,8 +514,12 @@ SkGeom sk_geom(int fmt, int mode, int64_t rows, int64_t cols, int n_sel = 1, int
         g.x_off = in_ring ? 0 : S * pitch;
         g.smem = (size_t)(128 + SK_HDR + SK_PART + S * pitch + (in_ring ? 0 : x_bytes));
         g.ok = true;
-        return g;
-    }
+        return true;
+    };
+    for (int R = r_pref; R >= 1; R >>= 1)
+        if (fits(R)) return g;
+    for (int R = 2 * r_pref; R <= r_max; R <<= 1)       // the preferred R does not fit: a larger one may
+        if (fits(R)) return g;
     return g;
 }
 
@@ -698,7 +711,7 @@ int sk_seq(int fmt, const qmv_task *tasks, int n_tasks, const DevInfo &di, cudaS
     for (int t = 0; t < n_tasks; ++t) {
         const qmv_task &k = tasks[t];
         const qmv_task *nx = t + 1 < n_tasks ? &tasks[t + 1] : nullptr;
-        const SkGeom g = sk_geom(fmt, SK_PLAIN, k.rows, k.cols);
+        const SkGeom g = sk_geom(fmt, SK_PLAIN, k.rows, k.cols, 1, 0, 1, di.sm_count);
         const int rc = sk_single(fmt, k.W_blocks, k.rows, k.cols, k.x, k.y, g, di, st, nullptr, nullptr, nullptr,
                                  nx ? nx->W_blocks : nullptr, nx ? nx->rows * (nx->cols / bw * bb) : 0);
         if (rc) return rc;
@@ -779,7 +792,7 @@ int qmv_batched(int fmt, const void *W_blocks, int64_t rows, int64_t cols, const
     if (tc_preferred(fmt, rows, cols, n_tok) && tc_geom(fmt, cols, n_tok, di).ok)
         return tc_single(fmt, W_blocks, rows, cols, x, y, n_tok, di, reinterpret_cast<cudaStream_t>(stream));
     if (n_tok == 1) {
-        const SkGeom g = sk_geom(fmt, SK_PLAIN, rows, cols);
+        const SkGeom g = sk_geom(fmt, SK_PLAIN, rows, cols, 1, 0, 1, di.sm_count);
         if (g.ok) return sk_single(fmt, W_blocks, rows, cols, x, y, g, di, reinterpret_cast<cudaStream_t>(stream));
     } else if (n_tok <= SKT_MAX_NTOK) {
         const SkGeom g = sk_geom(fmt, SK_PLAIN, rows, cols, 1, 0, n_tok);
@@ -1185,7 +1198,7 @@ int qmv_argmax_ws(int fmt, const void *W_blocks, int64_t rows, int64_t cols, con
     const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (n_tok == 1) {
         // one launch: the streaming kernel folds each CTA's best row into the key
-        const SkGeom g = sk_geom(fmt, SK_PLAIN, rows, cols);
+        const SkGeom g = sk_geom(fmt, SK_PLAIN, rows, cols, 1, 0, 1, di.sm_count);
         if (g.ok && g.ksegs == 1) {
             if (injected_failure()) return QMV_ERR_CUDA;
             return sk_single(fmt, W_blocks, rows, cols, x, y, g, di, st, idx_out, keys, done);
