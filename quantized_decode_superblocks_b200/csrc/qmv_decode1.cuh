@@ -254,9 +254,9 @@ __device__ __forceinline__ float q6_k_dot1(uint32_t sb, int h, int l0, XP &&xp)
     lds_words_a2<4>(sb + 128u + (uint32_t)(32 * h + l0), H);
     lds_words_a2<2>(sb + 192u + 8u * (uint32_t)h, S);       // scales[8h .. 8h+7]
     const float d = half_bits_to_float(lds_u16(sb + 208u));
-    float2 acc[4][2];
+    float2 acc[4];                                   // one packed accumulator per scale group
 #pragma unroll
-    for (int t = 0; t < 4; ++t) acc[t][0] = acc[t][1] = make_float2(0.f, 0.f);
+    for (int t = 0; t < 4; ++t) acc[t] = make_float2(0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const uint32_t q[4] = {
@@ -269,8 +269,7 @@ __device__ __forceinline__ float q6_k_dot1(uint32_t sb, int h, int l0, XP &&xp)
             float2 p02, p13, x02, x13;
             bytes4_to_f2(q[t], 32.0f, p02, p13);
             xp(4 * t + i, x02, x13);
-            acc[t][0] = f2fma(p02, x02, acc[t][0]);
-            acc[t][1] = f2fma(p13, x13, acc[t][1]);
+            acc[t] = f2fma(p13, x13, f2fma(p02, x02, acc[t]));
         }
     }
     // scales for t = 0..3: bytes (l0/16) + {0, 2, 4, 6} of S
@@ -278,10 +277,10 @@ __device__ __forceinline__ float q6_k_dot1(uint32_t sb, int h, int l0, XP &&xp)
     const uint32_t sv = __byte_perm(S[0], S[1], o | ((o + 2u) << 4) | ((o + 4u) << 8) | ((o + 6u) << 12));
     float2 s02, s13;
     bytes4_to_f2(sv ^ 0x80808080u, 128.0f, s02, s13);        // int8 scales (t0, t2), (t1, t3)
-    float r = s02.x * hsum2(acc[0][0], acc[0][1]);
-    r = fmaf(s13.x, hsum2(acc[1][0], acc[1][1]), r);
-    r = fmaf(s02.y, hsum2(acc[2][0], acc[2][1]), r);
-    r = fmaf(s13.y, hsum2(acc[3][0], acc[3][1]), r);
+    float r = s02.x * (acc[0].x + acc[0].y);
+    r = fmaf(s13.x, acc[1].x + acc[1].y, r);
+    r = fmaf(s02.y, acc[2].x + acc[2].y, r);
+    r = fmaf(s13.y, acc[3].x + acc[3].y, r);
     return d * r;
 }
 

@@ -142,10 +142,7 @@ __device__ __forceinline__ float q5_k_dot1(uint32_t sb, int c, const Q4kSel &sel
     const uint4 qa = lds_v4(sb + 48u + 32u * (uint32_t)c), qb = lds_v4(sb + 64u + 32u * (uint32_t)c);
     const uint32_t qh[8] = {ha.x, ha.y, ha.z, ha.w, hb.x, hb.y, hb.z, hb.w};
     const uint32_t qw[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
-    float2 a[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-    float2 b[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-    float2 a2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-    float2 b2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+    float2 a0 = make_float2(0.f, 0.f), a1 = a0, b0 = a0, b1 = a0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         uint32_t lo, hi;
@@ -159,16 +156,11 @@ __device__ __forceinline__ float q5_k_dot1(uint32_t sb, int c, const Q4kSel &sel
             xs_a = f2add(xs_a, f2add(xl02, xl13));
             xs_b = f2add(xs_b, f2add(xh02, xh13));
         }
-        if (i & 1) {
-            a2[0] = f2fma(lo02, xl02, a2[0]); a2[1] = f2fma(lo13, xl13, a2[1]);
-            b2[0] = f2fma(hi02, xh02, b2[0]); b2[1] = f2fma(hi13, xh13, b2[1]);
-        } else {
-            a[0] = f2fma(lo02, xl02, a[0]); a[1] = f2fma(lo13, xl13, a[1]);
-            b[0] = f2fma(hi02, xh02, b[0]); b[1] = f2fma(hi13, xh13, b[1]);
-        }
+        a0 = f2fma(lo02, xl02, a0); a1 = f2fma(lo13, xl13, a1);
+        b0 = f2fma(hi02, xh02, b0); b1 = f2fma(hi13, xh13, b1);
     }
-    const float sa = hsum2(a[0], a[1]) + hsum2(a2[0], a2[1]);
-    const float sbv = hsum2(b[0], b[1]) + hsum2(b2[0], b2[1]);
+    const float2 sa2 = f2add(a0, a1), sb2 = f2add(b0, b1);
+    const float sa = sa2.x + sa2.y, sbv = sb2.x + sb2.y;
     if (XSUM_INLINE) {
         xsa = xs_a.x + xs_a.y;
         xsb = xs_b.x + xs_b.y;

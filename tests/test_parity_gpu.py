@@ -111,6 +111,23 @@ def test_qmv_small_shapes(fmt, rows, cols, n_tok):
     within(y, ref, bound)
 
 
+# Small one-token matrices: when a CTA's share of rows fills at most half of
+# one stage the streaming kernel takes fewer rows per warp (Q4_K 3072x2048:
+# 2 instead of 4; 700 rows: 1); Q8_0 1000x128 prefers one row per warp, whose
+# 136-byte copies are not 16-byte multiples, and falls back to two.  The
+# streaming kernel must serve every case.
+@pytest.mark.parametrize("fmt,rows,cols", [(Q4_K, 3072, 2048), (Q4_K, 700, 2048), (Q8_0, 1024, 1024),
+                                           (Q8_0, 1000, 128), (Q6_K, 500, 2048), (Q8_0, 148 * 12 + 5, 2048),
+                                           (Q4_K, 148 * 24 + 3, 2048)])
+def test_small_matrices_rows_per_warp(fmt, rows, cols):
+    W = synth.gen_blocks(fmt, rows, cols, seed=31, tensor_id=rows)
+    x = synth.gen_x(1, cols, seed=31, tensor_id=cols)
+    y = run_qmv(fmt, W, rows, cols, x)
+    assert q.qmv_debug_last_kernel() == q.KERNEL_STREAM
+    ref, bound = oracle.qmv(fmt, W, rows, cols, x)
+    within(y, ref, bound)
+
+
 @pytest.mark.parametrize("fmt,rows,cols", [(Q8_0, 300, 8192), (Q8_0, 9, 16384), (Q4_K, 40, 16384),
                                            (Q6_K, 33, 8192), (Q8_0, 17, 8224), (Q6_K, 5, 4352),
                                            (Q8_0, 5, 65536), (Q4_K, 3, 65536), (Q6_K, 4, 34816),
