@@ -488,11 +488,14 @@ SkGeom sk_geom(int fmt, int mode, int64_t rows, int64_t cols, int n_sel = 1, int
     const int64_t x_bytes = mode == SK_GATHER ? (int64_t)g.ksegs * SK_SEG * 4 : n_tok * ceil_div(cols * 4, 128) * 128;
     if (x_bytes > SK_X_MAX_BYTES || (n_tok > 1 && mode != SK_PLAIN)) return g;
     const int64_t budget = SK_CTA_SMEM - SK_HDR - SK_PART;
-    // one token, plain: four rows per warp (Q8_0 2048x8192 6.9 -> 6.0 us, Q6_K
-    // 128000x2048 53.3 -> 50.4 us against two), fewer for small matrices
-    const int r_max = mode == SK_PLAIN && n_tok == 1 ? 4 : 2;
+    // plain: four rows per warp for one token (Q8_0 2048x8192 6.9 -> 6.0 us,
+    // Q6_K 128000x2048 53.3 -> 50.4 us against two) and for two tokens of a
+    // K-quant, whose decode the four rows' shared x loads pay for (Q6_K
+    // 128000x2048 92.3 -> 77.3 us; Q8_0 gate/up 13.0 -> 13.8 us, so not Q8_0);
+    // fewer for small matrices
+    const int r_max = mode == SK_PLAIN && (n_tok == 1 || (n_tok == 2 && !small_blk(fmt))) ? 4 : 2;
     int r_pref = r_max;
-    if (sms > 0 && mode == SK_PLAIN && n_tok == 1) {
+    if (sms > 0 && mode == SK_PLAIN && n_tok <= 2) {
         // a matrix whose share per CTA fills at most half of one stage: fewer
         // rows per warp, so that every warp gets some (Q4_K 3072x2048: 21 rows
         // a CTA on 12 warps of 2 rows rather than 6 warps of 4)
@@ -797,7 +800,7 @@ int qmv_batched(int fmt, const void *W_blocks, int64_t rows, int64_t cols, const
         const SkGeom g = sk_geom(fmt, SK_PLAIN, rows, cols, 1, 0, 1, di.sm_count);
         if (g.ok) return sk_single(fmt, W_blocks, rows, cols, x, y, g, di, reinterpret_cast<cudaStream_t>(stream));
     } else if (n_tok <= SKT_MAX_NTOK) {
-        const SkGeom g = sk_geom(fmt, SK_PLAIN, rows, cols, 1, 0, n_tok);
+        const SkGeom g = sk_geom(fmt, SK_PLAIN, rows, cols, 1, 0, n_tok, di.sm_count);
         if (g.ok)
             return skt_single(fmt, W_blocks, rows, cols, x, y, n_tok, g, di, reinterpret_cast<cudaStream_t>(stream));
     }

@@ -235,10 +235,14 @@ cudaError_t launch_sk(const SkParams &p, int mode, int R, dim3 grid, size_t smem
 template <int FMT, int NTOK>
 static cudaError_t launch_skt_r(const SkParams &p, int R, dim3 grid, size_t smem, cudaStream_t st, bool pdl)
 {
-    static SmemCfg c1, c2;
+    static SmemCfg c1, c2, c4;
     switch (R) {
     case 1: return launch_with(qmv_skt_kernel<FMT, 1, NTOK>, c1, p, grid, smem, st, pdl, false, SK_THREADS);
     case 2: return launch_with(qmv_skt_kernel<FMT, 2, NTOK>, c2, p, grid, smem, st, pdl, false, SK_THREADS);
+    case 4:
+        if constexpr (NTOK == 2)
+            return launch_with(qmv_skt_kernel<FMT, 4, NTOK>, c4, p, grid, smem, st, pdl, false, SK_THREADS);
+        return cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
     }
 }

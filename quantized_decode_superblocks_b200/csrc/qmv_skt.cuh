@@ -85,7 +85,7 @@ __device__ __forceinline__ void lane_slice_mt(const uint32_t (&rowp)[R], int l, 
 template <int FMT, int R, int NTOK>
 __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skt_kernel(const __grid_constant__ SkParams p)
 {
-    static_assert(R == 1 || R == 2, "rows per consumer warp");
+    static_assert(R == 1 || R == 2 || (R == 4 && NTOK == 2), "rows per consumer warp (four: two tokens)");
     static_assert(NTOK >= 2 && NTOK <= SKT_MAX_NTOK, "tokens");
     constexpr int NTP = Pow2Ceil<NTOK>::v;
     constexpr int V = R * NTP;                    // values a warp reduces per stage: (row, token)
