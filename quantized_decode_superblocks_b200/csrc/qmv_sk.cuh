@@ -624,6 +624,32 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skm_kernel(const __grid_con
         *abort_flag = 0;
         fence_mbar_init();
     }
+    // this CTA's rows of step 2 (gate/up: n_sel * inter) and step 3 (down: hidden)
+    const int64_t a_u0 = (int64_t)c * p.a_units_q + min(c, p.a_units_r);
+    const int64_t a_begin = a_u0 * R;
+    const int64_t a_end = min((int64_t)p.n_sel * p.inter, (a_u0 + p.a_units_q + (c < p.a_units_r ? 1 : 0)) * R);
+    const int64_t b_u0 = (int64_t)c * p.b_units_q + min(c, p.b_units_r);
+    const int64_t b_begin = b_u0 * R;
+    const int64_t b_end = min((int64_t)p.hidden, (b_u0 + p.b_units_q + (c < p.b_units_r ? 1 : 0)) * R);
+    const int na = a_end > a_begin ? (int)((a_end - a_begin + p.a_T - 1) / p.a_T) : 0;
+    const int nb = b_end > b_begin ? (int)((b_end - b_begin + p.b_T - 1) / p.b_T) : 0;
+    // The producer's parameters, read while warp 0 routes and kept opaque so
+    // that they are not read again from the parameter bank after the barrier:
+    // a constant-cache miss there would sit between the routing and the first
+    // weight copy.
+    int n_expert = p.n_expert;
+    const uint8_t *pG = nullptr, *pU = nullptr, *pD = nullptr;
+    uint64_t gus = 0, dstr = 0, rga = 0, rgb = 0;
+    int aT = 0, bT = 0, inter = 0, nsel = 0, bks = 0;
+    uint32_t xtx = 0;
+    if (warp == SK_NC && lane == 0) {
+        pG = p.G; pU = p.U; pD = p.D;
+        gus = (uint64_t)p.gu_stride; dstr = (uint64_t)p.d_stride;
+        rga = (uint64_t)p.gu_row_bytes; rgb = (uint64_t)p.d_row_bytes;
+        aT = p.a_T; bT = p.b_T; inter = p.inter; nsel = p.n_sel; bks = p.b_ksegs; xtx = p.debug_extra_tx;
+        asm volatile("" : "+l"(pG), "+l"(pU), "+l"(pD), "+l"(gus), "+l"(dstr), "+l"(rga), "+l"(rgb));
+        asm volatile("" : "+r"(aT), "+r"(bT), "+r"(inter), "+r"(nsel), "+r"(bks), "+r"(xtx), "+r"(n_expert));
+    }
     if (warp == 0) {
         if (p.logits) {
             skm_route(p.logits, p.bias, p.n_expert, p.n_sel, lane, sids, sg);
@@ -643,24 +669,13 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skm_kernel(const __grid_con
         }
     }
     __syncthreads();
-    auto valid = [&](int k) { return sids[k] >= 0 && sids[k] < p.n_expert; };
-
-    // this CTA's rows of step 2 (gate/up: n_sel * inter) and step 3 (down: hidden)
-    const int64_t a_u0 = (int64_t)c * p.a_units_q + min(c, p.a_units_r);
-    const int64_t a_begin = a_u0 * R;
-    const int64_t a_end = min((int64_t)p.n_sel * p.inter, (a_u0 + p.a_units_q + (c < p.a_units_r ? 1 : 0)) * R);
-    const int64_t b_u0 = (int64_t)c * p.b_units_q + min(c, p.b_units_r);
-    const int64_t b_begin = b_u0 * R;
-    const int64_t b_end = min((int64_t)p.hidden, (b_u0 + p.b_units_q + (c < p.b_units_r ? 1 : 0)) * R);
-    const int na = a_end > a_begin ? (int)((a_end - a_begin + p.a_T - 1) / p.a_T) : 0;
-    const int nb = b_end > b_begin ? (int)((b_end - b_begin + p.b_T - 1) / p.b_T) : 0;
+    auto valid = [&](int k) { return sids[k] >= 0 && sids[k] < n_expert; };
 
     if (warp == SK_NC) {
         // ------------------------------------------------------ producer --
         if (lane != 0) return;
         bool ok = true;
         int i = 0;
-        const uint64_t rga = (uint64_t)p.gu_row_bytes, rgb = (uint64_t)p.d_row_bytes;
         for (; i < na + nb && ok; ++i) {
             const int slot = i % S, round = i / S;
             if (round > 0 && !mbar_wait_bounded_block(empty0 + 8u * (uint32_t)slot, (uint32_t)((round - 1) & 1))) {
@@ -678,42 +693,42 @@ __global__ void __launch_bounds__(SK_THREADS, 1) qmv_skm_kernel(const __grid_con
             if (i < na) {
                 // step 2: the stage's a_T gate rows, then the same up rows (at
                 // a_T rows), one copy of each per run of rows of one expert
-                const int r0 = (int)(a_begin + (int64_t)i * p.a_T);
-                const int tr = min(p.a_T, (int)(a_end - r0));
-                const int k0 = r0 / p.inter, q0 = r0 - k0 * p.inter;
+                const int r0 = (int)(a_begin + (int64_t)i * aT);
+                const int tr = min(aT, (int)(a_end - r0));
+                const int k0 = r0 / inter, q0 = r0 - k0 * inter;
                 uint32_t total = 0;
                 for (int done = 0, k = k0, rr = q0; done < tr; ++k, rr = 0) {
-                    const int run = min(tr - done, p.inter - rr);
+                    const int run = min(tr - done, inter - rr);
                     if (valid(k)) total += 2u * (uint32_t)run * (uint32_t)rga;
                     done += run;
                 }
-                mbar_arrive_expect_tx(full, total + p.debug_extra_tx);
+                mbar_arrive_expect_tx(full, total + xtx);
                 for (int done = 0, k = k0, rr = q0; done < tr; ++k, rr = 0) {
-                    const int run = min(tr - done, p.inter - rr);
+                    const int run = min(tr - done, inter - rr);
                     if (valid(k)) {
-                        const uint64_t off = (uint64_t)sids[k] * (uint64_t)p.gu_stride + (uint64_t)rr * rga;
+                        const uint64_t off = (uint64_t)sids[k] * gus + (uint64_t)rr * rga;
                         const uint32_t dst = st + (uint32_t)done * (uint32_t)rga;
                         const uint32_t bytes = (uint32_t)run * (uint32_t)rga;
-                        bulk_g2s(dst, p.G + off, bytes, full);
-                        bulk_g2s(dst + (uint32_t)p.a_T * (uint32_t)rga, p.U + off, bytes, full);
+                        bulk_g2s(dst, pG + off, bytes, full);
+                        bulk_g2s(dst + (uint32_t)aT * (uint32_t)rga, pU + off, bytes, full);
                     }
                     done += run;
                 }
             } else {
                 // step 3: the stage's b_T rows of every routed expert's down
                 // matrix, expert k at k * b_T rows: one copy per expert
-                const int64_t r0 = b_begin + (int64_t)(i - na) * p.b_T;
-                const int tr = (int)min((int64_t)p.b_T, b_end - r0);
-                const int n_seg = min(p.n_sel, p.b_ksegs);
+                const int64_t r0 = b_begin + (int64_t)(i - na) * bT;
+                const int tr = (int)min((int64_t)bT, b_end - r0);
+                const int n_seg = min(nsel, bks);
                 const uint32_t bytes = (uint32_t)tr * (uint32_t)rgb;
                 uint32_t total = 0;
                 for (int k = 0; k < n_seg; ++k)
                     if (valid(k)) total += bytes;
-                mbar_arrive_expect_tx(full, total + p.debug_extra_tx);
+                mbar_arrive_expect_tx(full, total + xtx);
                 for (int k = 0; k < n_seg; ++k) {
                     if (!valid(k)) continue;
-                    bulk_g2s(st + (uint32_t)(k * p.b_T) * (uint32_t)rgb,
-                             p.D + (uint64_t)sids[k] * (uint64_t)p.d_stride + (uint64_t)r0 * rgb, bytes, full);
+                    bulk_g2s(st + (uint32_t)(k * bT) * (uint32_t)rgb,
+                             pD + (uint64_t)sids[k] * dstr + (uint64_t)r0 * rgb, bytes, full);
                 }
             }
         }
